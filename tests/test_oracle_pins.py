@@ -1,0 +1,280 @@
+"""Pins of the fp64 oracle against things other than itself.
+
+Each test checks the oracle against what the DeltaKV summary (gist.science,
+section 3 "Metodologia") and plain mathematics fix: brute force on tiny
+inputs, exact invariants, special cases that reduce to textbook routines,
+printed normal-CDF values and a worked example computed by hand
+(tests/golden/hand_example.json).  No GPU is used.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+# --------------------------------------------------------------- selection
+
+@pytest.mark.parametrize("T,s,k", [(17, 1, 1), (23, 2, 3), (31, 3, 2), (64, 8, 5), (40, 5, 8)])
+def test_select_matches_brute_force_sort(oracle_mod, T, s, k):
+    """Step 1 ("Processo di Compressione"): the k nearest earlier strided
+    references by L2 over K||V.  Brute force: list every slot j with j*s < t by
+    the definition, sort all (distance, slot) pairs, take the first k."""
+    rng = _rng(T * 100 + s * 10 + k)
+    d_h = 3
+    K = rng.integers(-3, 4, size=(T, d_h)).astype(np.float64)  # many exact ties
+    V = rng.integers(-3, 4, size=(T, d_h)).astype(np.float64)
+    for t in range(1, T):
+        if t % s == 0:
+            continue
+        cands = [j for j in range(T) if j * s < t]
+        assert len(cands) == math.ceil(t / s)
+        pairs = sorted((sum((K[t] - K[j * s]) ** 2) + sum((V[t] - V[j * s]) ** 2), j) for j in cands)
+        idx, dk, dk1, k_eff = oracle_mod.select(t, K, V, s, k)
+        want = [j for _, j in pairs[:k]] + [-1] * max(0, k - len(pairs))
+        assert list(idx) == want, (t, list(idx), want)
+        assert k_eff == min(k, len(pairs))
+        assert dk == pairs[min(k, len(pairs)) - 1][0]
+        assert dk1 == (pairs[k][0] if len(pairs) > k else math.inf)
+
+
+def test_select_exact_ties_take_lower_slot(oracle_mod):
+    """Duplicated reference rows give exactly equal distances; the lower slot
+    must come first (the tie rule of the selection)."""
+    T, s, d_h = 40, 4, 2
+    K = np.zeros((T, d_h))
+    V = np.zeros((T, d_h))
+    for j in range(T // s):
+        K[j * s] = [5.0 + j, 1.0]
+    for j in (2, 5, 7):                     # three identical references
+        K[j * s] = [1.0, 1.0]
+    K[37] = [1.0, 1.0]                      # token equal to all three
+    idx, dk, dk1, _ = oracle_mod.select(37, K, V, s, 2)
+    assert list(idx) == [2, 5]
+    assert dk == 0.0 and dk1 == 0.0
+
+
+def test_select_token_before_second_reference(oracle_mod):
+    """Tokens 1..s-1 have only slot 0 (token 0) as candidate."""
+    T, s = 10, 8
+    K = _rng(1).normal(size=(T, 4))
+    V = _rng(2).normal(size=(T, 4))
+    for t in range(1, 8):
+        idx, dk, dk1, k_eff = oracle_mod.select(t, K, V, s, 3)
+        assert list(idx) == [0, -1, -1] and k_eff == 1 and dk1 == math.inf
+
+
+# -------------------------------------------------------------- rounding
+
+def test_round_bf16_ties_to_even(oracle_mod):
+    r = lambda v: oracle_mod.round_to(oracle_mod.ROUND_BF16, v)
+    assert r(1.0 + 2.0 ** -8) == 1.0                     # halfway, even is 1.0
+    assert r(1.0 + 3 * 2.0 ** -8) == 1.0 + 2.0 ** -6     # halfway, even is up
+    assert r(1.0 + 2.0 ** -8 + 2.0 ** -40) == 1.0 + 2.0 ** -7  # just above halfway
+    assert r(-2.75) == -2.75 and r(0.0) == 0.0
+    assert r(3.0 * 2.0 ** -130) == 3.0 * 2.0 ** -130   # bf16 subnormal spacing 2^-133
+
+
+def test_round_matches_torch_on_float_inputs(oracle_mod):
+    """torch's float32 -> bfloat16 conversion is round-to-nearest-even; on
+    values that are exact floats the oracle must agree bit for bit."""
+    x = torch.randn(4096, generator=torch.Generator().manual_seed(3), dtype=torch.float32) * 37.0
+    want = x.to(torch.bfloat16).double().numpy()
+    got = np.array([oracle_mod.round_to(oracle_mod.ROUND_BF16, float(v)) for v in x.double().numpy()])
+    assert np.array_equal(got, want)
+    xd = torch.randn(2048, generator=torch.Generator().manual_seed(4), dtype=torch.float64)
+    want32 = xd.float().double().numpy()
+    got32 = np.array([oracle_mod.round_to(oracle_mod.ROUND_F32, float(v)) for v in xd.numpy()])
+    assert np.array_equal(got32, want32)
+
+
+# ---------------------------------------------------------------- activation
+
+def test_gelu_matches_printed_normal_cdf(oracle_mod):
+    g = json.load(open(os.path.join(GOLDEN, "normal_cdf.json")))
+    for z, phi in zip(g["z"], g["Phi"]):
+        assert oracle_mod.act(oracle_mod.ACT_GELU_ERF, z) == pytest.approx(z * phi, rel=0, abs=2e-15 * (1 + z))
+        # GELU(-z) = -z * (1 - Phi(z))
+        assert oracle_mod.act(oracle_mod.ACT_GELU_ERF, -z) == pytest.approx(-z * (1 - phi), abs=2e-15 * (1 + z))
+    assert oracle_mod.act(oracle_mod.ACT_GELU_ERF, 0.0) == 0.0
+    assert oracle_mod.act(oracle_mod.ACT_GELU_ERF, 40.0) == 40.0
+    assert oracle_mod.act(oracle_mod.ACT_GELU_ERF, -40.0) == 0.0
+    assert oracle_mod.act(oracle_mod.ACT_NONE, -1.25) == -1.25
+    # tanh form: close to exact GELU (max gap below 1e-3) but not equal
+    gt = oracle_mod.act(oracle_mod.ACT_GELU_TANH, 1.0)
+    assert abs(gt - 0.841344746068543) < 1e-3 and gt != oracle_mod.act(oracle_mod.ACT_GELU_ERF, 1.0)
+
+
+# ---------------------------------------------------------------------- MLP
+
+def test_mlp_linear_case_is_matrix_product(oracle_mod):
+    """With no nonlinearity the two layers collapse to (W2 W1) x + W2 b1 + b2,
+    evaluated here by numpy with the matrices multiplied first.  Non-square
+    weights catch a transposed operand."""
+    rng = _rng(7)
+    W1, b1 = rng.normal(size=(5, 3)), rng.normal(size=5)
+    W2, b2 = rng.normal(size=(2, 5)), rng.normal(size=2)
+    x = rng.normal(size=3)
+    y = oracle_mod.mlp(x, W1, b1, W2, b2, oracle_mod.ACT_NONE)
+    assert np.allclose(y, (W2 @ W1) @ x + W2 @ b1 + b2, rtol=1e-13, atol=1e-13)
+
+
+def test_mlp_one_hot_weights_route_elements(oracle_mod):
+    """One-hot weights pick single entries: checks row/column roles and that
+    the nonlinearity is applied between the layers, not after them."""
+    W1 = np.zeros((4, 3)); W1[2, 1] = 1.0          # h[2] = x[1]
+    W2 = np.zeros((2, 4)); W2[1, 2] = 1.0          # y[1] = act(h[2])
+    x = np.array([9.0, 1.0, -7.0])
+    y = oracle_mod.mlp(x, W1, None, W2, None, oracle_mod.ACT_GELU_ERF)
+    assert y[0] == 0.0 and y[1] == pytest.approx(0.841344746068543, abs=1e-15)
+
+
+# --------------------------------------------------------- worked example
+
+def test_hand_worked_example(oracle_mod):
+    g = json.load(open(os.path.join(GOLDEN, "hand_example.json")))
+    K = np.array(g["K"], dtype=np.float64)[:, None]
+    V = np.array(g["V"], dtype=np.float64)[:, None]
+    arr = lambda v: None if v is None else np.array(v, dtype=np.float64)
+    idx, code, dk, dk1 = oracle_mod.compress(K, V, arr(g["W1"]), arr(g["b1"]), arr(g["W2"]), arr(g["b2"]),
+                                             g["s"], g["k"], oracle_mod.ACT_NONE, oracle_mod.ROUND_BF16)
+    assert idx.tolist() == g["expect_idx"]
+    assert code.tolist() == g["expect_code"]
+    for t, want in enumerate(g["expect_d_k"]):
+        if want is None:
+            assert math.isnan(dk[t])
+        else:
+            assert dk[t] == want
+    Kh, Vh = oracle_mod.reconstruct(K, V, idx, code, arr(g["W3"]), arr(g["b3"]), arr(g["W4"]), arr(g["b4"]),
+                                    g["s"], oracle_mod.ACT_NONE)
+    assert Kh[:, 0].tolist() == g["expect_K_hat"]
+    assert Vh[:, 0].tolist() == g["expect_V_hat"]
+    out = oracle_mod.attention(np.array([g["q"]]), Kh, Vh)
+    lg = g["expect_logits"]
+    w = [math.exp(v - max(lg)) for v in lg]
+    want = sum(wi * vi for wi, vi in zip(w, g["expect_V_hat"])) / sum(w)
+    assert out[0, 0] == pytest.approx(want, rel=1e-15)
+
+
+# ---------------------------------------------------------- invariants
+
+def _tokens(T, d_h, n_lat, seed=0, dtype=torch.float32):
+    from decode_attention_strided_b200 import synth
+    x = synth.head_tokens(seed, 0, 0, 0, T, d_h, n_lat, dtype=dtype).double().numpy()
+    return x[:, :d_h].copy(), x[:, d_h:].copy()
+
+
+def test_reference_rows_reconstruct_exactly(oracle_mod):
+    from decode_attention_strided_b200 import synth
+    T, d_h, s, k = 200, 16, 8, 2
+    K, V = _tokens(T, d_h, 4)
+    w = {n: t.double().numpy() for n, t in synth.codec_weights(0, d_h, 8, 32, dtype=torch.float32).items()}
+    idx, code, _, _ = oracle_mod.compress(K, V, w["W1"], None, w["W2"], None, s, k)
+    Kh, Vh = oracle_mod.reconstruct(K, V, idx, code, w["W3"], None, w["W4"], None, s)
+    refs = np.arange(0, T, s)
+    assert np.array_equal(Kh[refs], K[refs]) and np.array_equal(Vh[refs], V[refs])
+    assert (idx[refs] == -1).all() and (code[refs] == 0).all()
+
+
+@pytest.mark.parametrize("k", [1, 2, 4])
+def test_identity_codec_reconstructs_every_token(oracle_mod, k):
+    """Identity compressor/decompressor (d_c = hidden = 2 d_h, W = I, no
+    nonlinearity) with fp64 codes: the residual passes through unchanged, so
+    every token comes back exactly (sums of a power-of-two count of float32
+    values and their differences are exact in double)."""
+    from decode_attention_strided_b200 import synth
+    T, d_h, s = 300, 8, 4
+    K, V = _tokens(T, d_h, 4, seed=5)
+    w = {n: t.double().numpy() for n, t in synth.identity_codec(d_h).items()}
+    idx, code, _, _ = oracle_mod.compress(K, V, w["W1"], None, w["W2"], None, s, k,
+                                          oracle_mod.ACT_NONE, oracle_mod.ROUND_NONE)
+    Kh, Vh = oracle_mod.reconstruct(K, V, idx, code, w["W3"], None, w["W4"], None, s, oracle_mod.ACT_NONE)
+    k_eff = (idx >= 0).sum(axis=1)
+    exact = (k_eff & (k_eff - 1)) == 0      # refs (0) and power-of-two counts
+    assert np.array_equal(Kh[exact], K[exact]) and np.array_equal(Vh[exact], V[exact])
+    # a count of 3 makes the mean inexact: then only the last bits may move
+    assert np.allclose(Kh, K, rtol=2.0 ** -50, atol=0) and np.allclose(Vh, V, rtol=2.0 ** -50, atol=0)
+    assert exact.sum() > 0.9 * T
+
+
+def test_token_equal_to_its_references_has_zero_residual(oracle_mod):
+    """If the k chosen references all equal x_t, the residual and (with no
+    biases, GELU(0) = 0) the code are exactly zero and x_t comes back."""
+    from decode_attention_strided_b200 import synth
+    T, d_h, s, k = 64, 4, 4, 3
+    K, V = _tokens(T, d_h, 2, seed=9)
+    row_k, row_v = K[5].copy() * 0 + 0.75, V[5].copy() * 0 - 1.5
+    for j in (1, 6, 11):                   # three references equal to the token
+        K[j * s], V[j * s] = row_k, row_v
+    t = 50
+    K[t], V[t] = row_k, row_v
+    w = {n: t_.double().numpy() for n, t_ in synth.codec_weights(0, d_h, 4, 16, dtype=torch.float32).items()}
+    idx, code, dk, _ = oracle_mod.compress(K, V, w["W1"], None, w["W2"], None, s, k)
+    assert sorted(idx[t].tolist()) == [1, 6, 11] and dk[t] == 0.0
+    assert (code[t] == 0.0).all()
+    Kh, Vh = oracle_mod.reconstruct(K, V, idx, code, w["W3"], None, w["W4"], None, s)
+    assert np.array_equal(Kh[t], K[t]) and np.array_equal(Vh[t], V[t])
+
+
+# --------------------------------------------------------------- attention
+
+def _sdpa(q, K, V):
+    qt = torch.from_numpy(q)[None, :, None, :]             # [1, G, 1, d]
+    Kt = torch.from_numpy(K)[None, None].expand(1, q.shape[0], -1, -1)
+    Vt = torch.from_numpy(V)[None, None].expand(1, q.shape[0], -1, -1)
+    return torch.nn.functional.scaled_dot_product_attention(qt, Kt, Vt)[0, :, 0, :].numpy()
+
+
+def test_stride_one_is_plain_attention(oracle_mod):
+    """s = 1 makes every token a reference: decode is ordinary attention,
+    here torch's scaled_dot_product_attention in float64."""
+    from decode_attention_strided_b200 import synth
+    T, d_h = 120, 16
+    K, V = _tokens(T, d_h, 4, seed=11)
+    w = {n: t.double().numpy() for n, t in synth.codec_weights(0, d_h, 8, 32, dtype=torch.float32).items()}
+    idx, code, _, _ = oracle_mod.compress(K, V, w["W1"], None, w["W2"], None, 1, 2)
+    assert (idx == -1).all()
+    Kh, Vh = oracle_mod.reconstruct(K, V, idx, code, w["W3"], None, w["W4"], None, 1)
+    q = _rng(3).normal(size=(4, d_h))
+    assert np.allclose(oracle_mod.attention(q, Kh, Vh), _sdpa(q, K, V), rtol=1e-12, atol=1e-12)
+
+
+def test_identity_codec_attention_is_full_cache_attention(oracle_mod):
+    from decode_attention_strided_b200 import synth
+    T, d_h, s = 256, 8, 8
+    K, V = _tokens(T, d_h, 4, seed=12)
+    w = {n: t.double().numpy() for n, t in synth.identity_codec(d_h).items()}
+    idx, code, _, _ = oracle_mod.compress(K, V, w["W1"], None, w["W2"], None, s, 2,
+                                          oracle_mod.ACT_NONE, oracle_mod.ROUND_NONE)
+    Kh, Vh = oracle_mod.reconstruct(K, V, idx, code, w["W3"], None, w["W4"], None, s, oracle_mod.ACT_NONE)
+    q = _rng(4).normal(size=(2, d_h))
+    assert np.allclose(oracle_mod.attention(q, Kh, Vh), _sdpa(q, K, V), rtol=1e-12, atol=1e-12)
+
+
+def test_attention_closed_forms(oracle_mod):
+    rng = _rng(5)
+    V = rng.normal(size=(7, 3))
+    K = rng.normal(size=(7, 3))
+    # single token: the output is that token's value
+    assert np.array_equal(oracle_mod.attention(np.ones((1, 3)), K[:1], V[:1])[0], V[0])
+    # zero query: equal weights, the output is the mean value row
+    assert np.allclose(oracle_mod.attention(np.zeros((1, 3)), K, V)[0], V.mean(axis=0), rtol=1e-14, atol=1e-15)
+    # two tokens whose scaled logits differ by delta: weights 1 : e^delta
+    K2 = np.array([[0.0, 0, 0], [3.0, 0, 0]])
+    q = np.array([[1.0, 0, 0]])
+    delta = 3.0 / math.sqrt(3.0)
+    want = (V[0] + math.exp(delta) * V[1]) / (1 + math.exp(delta))
+    assert np.allclose(oracle_mod.attention(q, K2, V[:2])[0], want, rtol=1e-14)
+    # head order: permuting the query heads permutes the outputs
+    Q = rng.normal(size=(3, 3))
+    o = oracle_mod.attention(Q, K, V)
+    assert np.array_equal(oracle_mod.attention(Q[::-1].copy(), K, V), o[::-1])
