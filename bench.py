@@ -1,0 +1,455 @@
+#!/usr/bin/env python3
+"""Benchmark of the DeltaKV hot path on B200: compression at 128k context
+and decode attention over the compressed cache.
+
+One step = the whole path over one batch of synthetic input:
+  * compress: 32 layers of one 131072-token sequence, 8 kv-heads x d_h 128,
+    stride 16, k 4, d_c 32, hidden 256, bfloat16 (reference packing, nearest
+    reference search, encode);
+  * decode: one query per sequence for a batch of 8 sequences of 131072
+    cached tokens, 32 layers, 32 query heads / 8 kv-heads, over caches
+    compressed (untimed) before the run.
+`value` is compressed tokens per second over the whole step (Mtok/s);
+`decode_attn` reports the decode phase in GB/s of algorithmic bytes.
+
+Prints one JSON line (rank 0).  `--impl reference` times the fp64 CPU oracle
+on a bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "compress Mtok/s (% tensor peak); decode-attn GB/s vs HBM peak at 128k ctx"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP32_LANES_PER_SM, NUM_SMS, SM_MAX_MHZ = 128, 148, 1965.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="deltakv", choices=["deltakv", "reference"])
+    ap.add_argument("--layers", type=int, default=32)
+    ap.add_argument("--T", type=int, default=131072)
+    ap.add_argument("--decode-batch", type=int, default=8)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ workload
+
+class Shape:
+    def __init__(self, a):
+        self.L = a.layers
+        self.T = a.T
+        self.H, self.Hq, self.d_h = 8, 32, 128
+        self.s, self.k, self.d_c, self.hidden = 16, 4, 32, 256
+        self.Bc, self.Bd = 1, a.decode_batch
+        self.n_lat = 8
+        self.n_ref = math.ceil(self.T / self.s)
+        self.n_code = self.T - self.n_ref
+
+    def cand_flops_per_layer(self, B):
+        # 2 D sum_{t non-ref} ceil(t / s) per (sequence, kv-head)
+        T, s = self.T, self.s
+        tot = 0
+        full_blocks = T // s
+        # tokens t = j*s + r, r = 1..s-1: ceil(t/s) = j + 1
+        tot += (s - 1) * full_blocks * (full_blocks + 1) // 2
+        for t in range(full_blocks * s + 1, T):
+            tot += math.ceil(t / s)
+        return 2 * (2 * self.d_h) * tot * self.H * B
+
+    def mlp_flops_per_layer(self, B):
+        D = 2 * self.d_h
+        return 2 * (D * self.hidden + self.hidden * self.d_c) * self.n_code * self.H * B
+
+    def decode_bytes_per_layer(self):
+        es = 2
+        per_head = self.n_ref * 2 * self.d_h * es + self.n_code * (self.d_c * es + self.k * 4)
+        weights = (self.hidden * self.d_c + 2 * self.d_h * self.hidden) * es
+        return per_head * self.Bd * self.H + self.Bd * self.Hq * self.d_h * (es + 4) + weights
+
+
+def build_workload(sh, dev):
+    from decode_attention_strided_b200 import deltakv as dkv
+    from decode_attention_strided_b200 import synth
+
+    def layer_kv(layer, B):
+        K = torch.empty((B, sh.H, sh.T, sh.d_h), dtype=torch.bfloat16, device=dev)
+        V = torch.empty_like(K)
+        for b in range(B):
+            for h in range(sh.H):
+                x = synth.head_tokens(layer, layer, b, h, sh.T, sh.d_h, sh.n_lat, torch.bfloat16, dev)
+                K[b, h].copy_(x[:, :sh.d_h])
+                V[b, h].copy_(x[:, sh.d_h:])
+        return K, V
+
+    cc = dkv.Config(batch=sh.Bc, kv_heads=sh.H, q_heads=sh.Hq, d_h=sh.d_h, max_T=sh.T, stride_s=sh.s, k=sh.k,
+                    d_c=sh.d_c, hidden=sh.hidden, layers=sh.L)
+    cd = dkv.Config(batch=sh.Bd, kv_heads=sh.H, q_heads=sh.Hq, d_h=sh.d_h, max_T=sh.T, stride_s=sh.s, k=sh.k,
+                    d_c=sh.d_c, hidden=sh.hidden, layers=sh.L)
+    pc, pd = dkv.plan(cc), dkv.plan(cd)
+    W = [{n: t.to(dev) for n, t in synth.codec_weights(l, sh.d_h, sh.d_c, sh.hidden, device="cpu").items()}
+         for l in range(sh.L)]
+    comp_in = [layer_kv(l, sh.Bc) for l in range(sh.L)]
+    comp_cache = [pc.alloc_cache(dev) for _ in range(sh.L)]
+    ws_c = pc.alloc_workspace(dev)
+    ws_d = pd.alloc_workspace(dev)
+    dec_cache = []
+    for l in range(sh.L):
+        K, V = layer_kv(100 + l, sh.Bd)
+        c = pd.alloc_cache(dev)
+        dkv.compress(pd, sh.T, K, V, W[l]["W1"], None, W[l]["W2"], None, c, ws_d)
+        dec_cache.append(c)
+        del K, V
+    torch.cuda.synchronize()
+    q = [synth.queries(l, sh.Bd, sh.Hq, sh.d_h, device=dev) for l in range(sh.L)]
+    out = [torch.empty((sh.Bd, sh.Hq, sh.d_h), dtype=torch.float32, device=dev) for _ in range(sh.L)]
+    return dict(pc=pc, pd=pd, W=W, comp_in=comp_in, comp_cache=comp_cache, ws_c=ws_c, ws_d=ws_d,
+                dec_cache=dec_cache, q=q, out=out)
+
+
+def compress_phase(sh, w):
+    from decode_attention_strided_b200 import deltakv as dkv
+    for l in range(sh.L):
+        K, V = w["comp_in"][l]
+        dkv.compress(w["pc"], sh.T, K, V, w["W"][l]["W1"], None, w["W"][l]["W2"], None, w["comp_cache"][l], w["ws_c"])
+
+
+def decode_phase(sh, w):
+    from decode_attention_strided_b200 import deltakv as dkv
+    for l in range(sh.L):
+        dkv.decode_attention(w["pd"], sh.T, w["q"][l], w["dec_cache"][l], w["W"][l]["W3"], None,
+                             w["W"][l]["W4"], None, w["out"][l], w["ws_d"])
+
+
+# ------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------ reference arm
+
+def oracle_sample(sh, budget_s=12.0, threads=0):
+    """Time the fp64 oracle on a bounded sample of the workload and
+    extrapolate one full step.  Returns (seconds per full step, description,
+    threads used)."""
+    import numpy as np
+    import oracle
+    from decode_attention_strided_b200 import synth
+    oracle.build()
+    x = synth.head_tokens(0, 0, 0, 0, sh.T, sh.d_h, sh.n_lat, torch.bfloat16, "cpu").double().numpy()
+    K, V = x[:, :sh.d_h].copy(), x[:, sh.d_h:].copy()
+    W = {n: t.double().numpy() for n, t in synth.codec_weights(0, sh.d_h, sh.d_c, sh.hidden).items()}
+    nthreads = threads or os.cpu_count() or 1
+    rng = np.random.default_rng(0)
+    # compress: rows drawn uniformly over the sequence (their cost grows with t)
+    n_rows, t_c = 64, 0.0
+    while True:
+        rows = rng.integers(1, sh.T, size=n_rows).astype(np.int32)
+        t0 = time.perf_counter()
+        oracle.compress_rows(K, V, W["W1"], None, W["W2"], None, sh.s, sh.k, rows, n_threads=nthreads)
+        t_c = time.perf_counter() - t0
+        if t_c > budget_s / 4 or n_rows >= 1 << 16:
+            break
+        n_rows *= 4
+    per_row_c = t_c / n_rows
+    # decode: reconstruct a prefix of the cache and attend over it
+    Tp = min(sh.T, 16384)
+    idx, code, _, _ = oracle.compress(K[:Tp], V[:Tp], W["W1"], None, W["W2"], None, sh.s, sh.k, n_threads=nthreads)
+    t0 = time.perf_counter()
+    Kh, Vh = oracle.reconstruct(K[:Tp], V[:Tp], idx, code, W["W3"], None, W["W4"], None, sh.s, n_threads=nthreads)
+    q = np.random.default_rng(1).normal(size=(sh.Hq // sh.H, sh.d_h))
+    oracle.attention(q, Kh, Vh)
+    per_row_d = (time.perf_counter() - t0) / Tp
+    step_s = sh.L * (per_row_c * sh.T * sh.H * sh.Bc + per_row_d * sh.T * sh.H * sh.Bd)
+    desc = (f"oracle compress_rows on {n_rows} uniformly drawn rows of one (layer, kv-head) at T={sh.T} "
+            f"({t_c:.2f}s) + reconstruct/attend over a {Tp}-token prefix; extrapolated to the full step "
+            f"({sh.L} layers x {sh.H} heads compress, {sh.Bd} x {sh.H} heads decode)")
+    return step_s, desc, nthreads
+
+
+def run_reference(a, rank):
+    sh = Shape(a)
+    if rank != 0:
+        return
+    per_step = []
+    desc, nthreads = "", 0
+    for i in range(a.warmup + a.steps):
+        step_s, desc, nthreads = oracle_sample(sh, budget_s=8.0)
+        if i >= a.warmup:
+            per_step.append(step_s)
+    step_s = statistics.median(per_step)
+    value = sh.T * sh.Bc / step_s / 1e6
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "Mtok/s", "n_gpus": a.gpus,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(sh),
+        "cpu_baseline": {"value": value, "unit": "Mtok/s", "cores": nthreads, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "Mtok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(sh):
+    return {"workload": f"deltakv-{sh.T // 1024}k: compress {sh.L} layers x {sh.Bc} seq x {sh.H} kv-heads, "
+                        f"decode {sh.L} layers x batch {sh.Bd} x {sh.Hq} q-heads",
+            "T": sh.T, "layers": sh.L, "compress_batch": sh.Bc, "decode_batch": sh.Bd, "kv_heads": sh.H,
+            "q_heads": sh.Hq, "d_h": sh.d_h, "stride_s": sh.s, "k": sh.k, "d_c": sh.d_c, "hidden": sh.hidden,
+            "global_batch": sh.Bd, "seq_len": sh.T, "parallelism": "replicas",
+            "l2": "inputs larger than L2 (per step: 17 GB raw K/V compressed, 28.7 GB cache read)"}
+
+
+# ------------------------------------------------------------------- main
+
+def main():
+    a = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl" if a.impl == "deltakv" else "gloo",
+                                             timeout=datetime.timedelta(seconds=600))
+    if a.impl == "reference":
+        run_reference(a, rank)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+    assert torch.cuda.is_available(), "bench.py needs a CUDA device"
+    torch.cuda.set_device(local)
+    dev = f"cuda:{local}"
+    from decode_attention_strided_b200 import deltakv as dkv
+    dkv.load_library()  # fails loudly if the CUDA library is not built
+
+    sh = Shape(a)
+    t_setup = time.perf_counter()
+    w = build_workload(sh, dev)
+    setup_s = time.perf_counter() - t_setup
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    for _ in range(a.warmup):
+        compress_phase(sh, w)
+        decode_phase(sh, w)
+    torch.cuda.synchronize()
+    for p in (w["pc"], w["pd"]):
+        dkv.set_profiling(p, True)
+        dkv.profile_collect(p)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(a.steps)]
+    clocks = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    wall0 = time.perf_counter()
+    for i in range(a.steps):
+        ev[i][0].record()
+        compress_phase(sh, w)
+        ev[i][1].record()
+        decode_phase(sh, w)
+        ev[i][2].record()
+    torch.cuda.synchronize()
+    barrier()
+    wall = time.perf_counter() - wall0
+    clk = clocks.stop()
+    prof_c = dkv.profile_collect(w["pc"])
+    prof_d = dkv.profile_collect(w["pd"])
+    for p in (w["pc"], w["pd"]):
+        dkv.set_profiling(p, False)
+    status = max(dkv.device_status(w["pc"], w["ws_c"]), dkv.device_status(w["pd"], w["ws_d"]))
+    step_ms = [e[0].elapsed_time(e[2]) for e in ev]
+    comp_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    dec_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    tot_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([tot_ms, sum(comp_ms), sum(dec_ms)], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        tot_ms, sc, sd = t.tolist()
+    else:
+        sc, sd = sum(comp_ms), sum(dec_ms)
+    ms_step = tot_ms / a.steps
+    value = world * sh.T * sh.Bc * a.steps / (tot_ms / 1e3) / 1e6
+
+    peaks, peak_kind = load_peaks()
+    # dominant kernel of the step
+    prof = {}
+    for d in (prof_c, prof_d):
+        for k_, (n, ms) in d.items():
+            pn, pm = prof.get(k_, (0, 0.0))
+            prof[k_] = (pn + n, pm + ms)
+    launches = sum(n for n, _ in prof.values())
+    dom = max(prof.items(), key=lambda kv: kv[1][1])[0] if prof else None
+    roof = None
+    if dom in ("candidates_tc", "candidates_simt"):
+        n, ms = prof[dom]
+        per_launch_s = ms / n / 1e3
+        if dom == "candidates_tc":
+            fl = sh.cand_flops_per_layer(sh.Bc)
+            peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+            roof = {"kernel": dom, "bound": "tensor", "achieved": fl / per_launch_s / 1e12, "peak": peak,
+                    "unit": "TFLOP/s", "peak_source": f"{peak_kind} bf16 sustained"}
+        else:
+            fl = sh.cand_flops_per_layer(sh.Bc) * 3 / 2  # sub + fma per element and dim
+            peak = NUM_SMS * FP32_LANES_PER_SM * 2 * SM_MAX_MHZ * 1e6 / 1e12
+            roof = {"kernel": dom, "bound": "alu", "achieved": fl / per_launch_s / 1e12, "peak": peak,
+                    "unit": "TFLOP/s", "peak_source": "fp32 lanes x 2 x max SM clock"}
+        roof["frac"] = roof["achieved"] / roof["peak"]
+        roof["traffic"] = None
+        roof["algorithmic_per_launch"] = fl
+    dbytes = sh.decode_bytes_per_layer()
+    dec_ms_layer = sd / a.steps / sh.L
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    decode_attn = {"value": dbytes / (dec_ms_layer / 1e3) / 1e9, "unit": "GB/s", "peak": hbm,
+                   "peak_source": peak_kind, "frac": dbytes / (dec_ms_layer / 1e3) / 1e9 / hbm,
+                   "ms_per_layer": dec_ms_layer, "bytes_per_layer": dbytes}
+    if "decode_stream" in prof:
+        n, ms = prof["decode_stream"]
+        decode_attn["stream_kernel_ms_per_launch"] = ms / n
+    comp_fl = sh.cand_flops_per_layer(sh.Bc) + sh.mlp_flops_per_layer(sh.Bc)
+    compress = {"value": sh.T * sh.Bc / (sc / a.steps / 1e3) / 1e6, "unit": "Mtok/s",
+                "ms": sc / a.steps,
+                "tensor_frac": comp_fl * sh.L / (sc / a.steps / 1e3) / 1e12 /
+                peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])}
+
+    e2e = None
+    if not a.no_e2e:
+        e2e = run_e2e(sh, w, dev, a)
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        step_s, desc, nthreads = oracle_sample(sh, budget_s=12.0)
+        cpu = {"value": sh.T * sh.Bc / step_s / 1e6, "unit": "Mtok/s", "cores": nthreads, "kind": "oracle",
+               "sample": desc}
+    line = {
+        "metric": METRIC, "value": value, "unit": "Mtok/s", "n_gpus": world, "steps": a.steps,
+        "warmup": a.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(sh),
+        "compress": compress, "decode_attn": decode_attn, "roofline": roof, "cpu_baseline": cpu,
+        "e2e": e2e, "gpu_launches": launches, "kernels": {k_: {"launches": n, "ms": ms} for k_, (n, ms) in prof.items()},
+        "clocks": clk, "device_status": status, "setup_s": setup_s, "wall_s": wall,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def run_e2e(sh, w, dev, a):
+    """Same step through the public API with host buffers: every layer's K/V
+    is copied from pinned host memory before its compress call, and every
+    decode copies its queries in and its output back."""
+    from decode_attention_strided_b200 import deltakv as dkv
+    K0, V0 = w["comp_in"][0]
+    hK = torch.empty(K0.shape, dtype=K0.dtype, pin_memory=True)
+    hV = torch.empty(V0.shape, dtype=V0.dtype, pin_memory=True)
+    hK.copy_(K0)
+    hV.copy_(V0)
+    hq = [q.cpu().pin_memory() for q in w["q"]]
+    ho = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in w["out"]]
+    dK, dV = torch.empty_like(K0), torch.empty_like(V0)
+    dq = torch.empty_like(w["q"][0])
+    h2d = d2h = 0
+    steps = max(1, min(a.steps, 3))
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        for l in range(sh.L):
+            dK.copy_(hK, non_blocking=True)
+            dV.copy_(hV, non_blocking=True)
+            dkv.compress(w["pc"], sh.T, dK, dV, w["W"][l]["W1"], None, w["W"][l]["W2"], None,
+                         w["comp_cache"][l], w["ws_c"])
+        for l in range(sh.L):
+            dq.copy_(hq[l], non_blocking=True)
+            dkv.decode_attention(w["pd"], sh.T, dq, w["dec_cache"][l], w["W"][l]["W3"], None, w["W"][l]["W4"],
+                                 None, w["out"][l], w["ws_d"])
+            ho[l].copy_(w["out"][l], non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    h2d = sh.L * (hK.numel() * 2 + hV.numel() * 2 + hq[0].numel() * 2)
+    d2h = sh.L * ho[0].numel() * 4
+    return {"value": sh.T * sh.Bc / (ms / 1e3) / 1e6, "unit": "Mtok/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps}
+
+
+if __name__ == "__main__":
+    main()

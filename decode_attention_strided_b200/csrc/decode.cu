@@ -1,0 +1,475 @@
+// decode.cu -- split-K decode attention over the compressed cache, with every
+// non-reference token rebuilt on demand ("Ricostruzione" of the DeltaKV
+// summary; on-demand reconstruction inside attention, section 4).
+//
+// For query head g of kv-head h, with c = log2(e) / sqrt(d_h):
+//   reference slot j :  l_j = c q.K_ref_j                       = S_j
+//   other token t    :  l_t = c q.(KV_R + W4_K u_t + b4_K)
+//                           = (1/k_eff) sum_i S_{idx_ti} + a.u_t + c q.b4_K
+//   with u_t = act(W3 code_t + b3) and a = c W4_K^T q.
+// The output  sum_t 2^(l_t - M) V_hat_t / sum_t 2^(l_t - M)  splits as
+//   sum_j w_j V_ref_j + W4_V (sum_t p_t u_t) + b4_V sum_t p_t,
+//   w_j = 2^(S_j - M) + sum_{t : j in idx_t} p_t / k_eff_t,
+// so K_hat and V_hat are never formed: K_R enters through the gathered S
+// values, V_R through the per-slot weight table w, and W4 through one GEMV
+// per kv-head before (a) and after (W4_V U) the token loop.  This is the same
+// arithmetic as rebuilding every token, reassociated.
+//
+// Kernels, in stream order:
+//   decode_ref      S_j for every slot (reads K_ref), per-block maxima
+//   decode_prep     a = c W4_K^T q and c q.b4_K per query head
+//   decode_stream   per split of the compressed rows: u_t, logits, online
+//                   softmax partials (m, l, U = sum p u) and the split's w table
+//   decode_combine  per 256-slot chunk: sum_j w_j V_ref_j (reads V_ref)
+//   decode_final    merge everything, add W4_V U and b4_V, normalise
+#include <cfloat>
+
+#include "common.cuh"
+
+namespace dkv {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kRefBlockSlots = 64;
+
+// ------------------------------------------------------------ decode_ref
+template <typename T>
+__global__ void __launch_bounds__(256)
+    decode_ref_kernel(int64_t n_ref, int64_t n_ref_cap, int d_h, int H, int G, float c,
+                      const T* __restrict__ q, int64_t qsb, int64_t qsh,
+                      const T* __restrict__ refk, float* __restrict__ S,
+                      float* __restrict__ Smax, int n_refblk_cap) {
+  __shared__ float qs[kMaxG][128];
+  __shared__ float wmax[8][kMaxG];
+  const int b = blockIdx.z, h = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t bh = (int64_t)b * H + h;
+  for (int i = threadIdx.x; i < G * d_h; i += blockDim.x) {
+    int g = i / d_h, e = i - g * d_h;
+    qs[g][e] = c * to_f(q[b * qsb + (int64_t)(h * G + g) * qsh + e]);
+  }
+  __syncthreads();
+  float mx[kMaxG];
+#pragma unroll
+  for (int g = 0; g < kMaxG; ++g) mx[g] = -INFINITY;
+  for (int i = 0; i < kRefBlockSlots / 8; ++i) {
+    int64_t j = (int64_t)blockIdx.x * kRefBlockSlots + warp * (kRefBlockSlots / 8) + i;
+    if (j >= n_ref) break;
+    const T* kr = refk + (bh * n_ref_cap + j) * d_h;
+    float kv[4];
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) {
+      int e = lane + 32 * q4;
+      kv[q4] = e < d_h ? to_f(kr[e]) : 0.f;
+    }
+#pragma unroll
+    for (int g = 0; g < kMaxG; ++g) {
+      if (g < G) {
+        float acc = 0.f;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          int e = lane + 32 * q4;
+          if (e < d_h) acc = fmaf(qs[g][e], kv[q4], acc);
+        }
+        acc = warp_sum(acc);
+        mx[g] = fmaxf(mx[g], acc);
+        if (lane == 0) S[(bh * n_ref_cap + j) * G + g] = acc;
+      }
+    }
+  }
+  if (lane == 0)
+#pragma unroll
+    for (int g = 0; g < kMaxG; ++g) wmax[warp][g] = mx[g];
+  __syncthreads();
+  if (threadIdx.x < G) {
+    float m = -INFINITY;
+    for (int w = 0; w < 8; ++w) m = fmaxf(m, wmax[w][threadIdx.x]);
+    Smax[(bh * n_refblk_cap + blockIdx.x) * G + threadIdx.x] = m;
+  }
+}
+
+// ----------------------------------------------------------- decode_prep
+template <typename T>
+__global__ void __launch_bounds__(256)
+    decode_prep_kernel(int d_h, int H, int G, int hidden, float c, const T* __restrict__ q,
+                       int64_t qsb, int64_t qsh, const T* __restrict__ W4,
+                       const float* __restrict__ b4, float* __restrict__ a,
+                       float* __restrict__ cterm) {
+  __shared__ float qs[kMaxG][128];
+  const int b = blockIdx.z, h = blockIdx.y;
+  const int64_t bh = (int64_t)b * H + h;
+  for (int i = threadIdx.x; i < G * d_h; i += blockDim.x) {
+    int g = i / d_h, e = i - g * d_h;
+    qs[g][e] = c * to_f(q[b * qsb + (int64_t)(h * G + g) * qsh + e]);
+  }
+  __syncthreads();
+  for (int n = threadIdx.x; n < hidden; n += blockDim.x) {
+    float acc[kMaxG];
+#pragma unroll
+    for (int g = 0; g < kMaxG; ++g) acc[g] = 0.f;
+    for (int e = 0; e < d_h; ++e) {
+      float w = to_f(W4[(int64_t)e * hidden + n]);
+#pragma unroll
+      for (int g = 0; g < kMaxG; ++g)
+        if (g < G) acc[g] = fmaf(w, qs[g][e], acc[g]);
+    }
+    for (int g = 0; g < G; ++g) a[(bh * G + g) * hidden + n] = acc[g];
+  }
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    for (int g = 0; g < G; ++g) {
+      float acc = 0.f;
+      if (b4)
+        for (int e = lane; e < d_h; e += 32) acc = fmaf(b4[e], qs[g][e], acc);
+      acc = warp_sum(acc);
+      if (lane == 0) cterm[bh * G + g] = acc;
+    }
+  }
+}
+
+// --------------------------------------------------------- decode_stream
+// One block per (split, kv-head, sequence), 8 warps, one compressed token per
+// warp at a time.  The split's slot-weight table lives in shared memory when
+// it fits (`wt_in_smem`), else in the split's own region of the workspace.
+// Weights added to it are relative to m_ref = max_j S_j, fixed for the call;
+// U and l use a per-warp running maximum.
+template <typename T>
+__global__ void __launch_bounds__(256)
+    decode_stream_kernel(int T_, int s, int d_h, int H, int G, int k, int d_c, int hidden,
+                         int act, int ns, int64_t n_ref_cap, int64_t n_code_cap,
+                         int n_refblk, int n_refblk_cap, const T* __restrict__ code,
+                         const int32_t* __restrict__ idx, const T* __restrict__ W3,
+                         const float* __restrict__ b3, const float* __restrict__ a,
+                         const float* __restrict__ cterm, const float* __restrict__ S,
+                         const float* __restrict__ Smax, float* __restrict__ wtab_g,
+                         float* __restrict__ part, float* __restrict__ Upart, int wt_in_smem,
+                         uint32_t* __restrict__ err) {
+  extern __shared__ float smem[];
+  float* W3s = smem;                         // [d_c][hidden]
+  float* As = W3s + d_c * hidden;            // [G][hidden]
+  float* Ured = As + G * hidden;             // [G][hidden]
+  float* misc = Ured + G * hidden;           // m_ref[G], m_cta[G], l[G], cterm[G]
+  float* cw = misc + 4 * kMaxG;              // [8 warps][d_c] code rows
+  float* wt = cw + 8 * d_c;                  // [n_ref][G] when in smem
+  const int b = blockIdx.z, h = blockIdx.y, split = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
+  const int64_t bh = (int64_t)b * H + h;
+  const int64_t n_ref = (T_ + s - 1) / s;
+  const int64_t n_code = T_ - n_ref;
+  const int64_t c0 = n_code * split / ns, c1 = n_code * (split + 1) / ns;
+  float* wtab = wt_in_smem ? wt : wtab_g + ((bh * ns) + split) * n_ref_cap * G;
+
+  for (int i = tid; i < d_c * hidden; i += blockDim.x) {
+    int n = i / d_c, e = i - n * d_c;
+    W3s[e * hidden + n] = to_f(W3[i]);
+  }
+  for (int i = tid; i < G * hidden; i += blockDim.x) {
+    As[i] = a[bh * G * hidden + i];
+    Ured[i] = 0.f;
+  }
+  for (int64_t i = tid; i < n_ref * G; i += blockDim.x) wtab[i] = 0.f;
+  if (tid < G) {
+    float m = -INFINITY;
+    for (int r = 0; r < n_refblk; ++r) m = fmaxf(m, Smax[(bh * n_refblk_cap + r) * G + tid]);
+    misc[tid] = m;                        // m_ref
+    misc[kMaxG + tid] = -INFINITY;        // block max (after the loop)
+    misc[2 * kMaxG + tid] = 0.f;          // block l
+    misc[3 * kMaxG + tid] = cterm[bh * G + tid];
+  }
+  __syncthreads();
+  if (!wt_in_smem) __threadfence_block();
+
+  const int per_lane = hidden / 32;  // hidden is a multiple of 32 here
+  float mw[kMaxG], lw[kMaxG], Uw[kMaxG][8];
+  float mref[kMaxG], ct[kMaxG];
+#pragma unroll
+  for (int g = 0; g < kMaxG; ++g) {
+    mw[g] = -INFINITY;
+    lw[g] = 0.f;
+    mref[g] = g < G ? misc[g] : 0.f;
+    ct[g] = g < G ? misc[3 * kMaxG + g] : 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) Uw[g][i] = 0.f;
+  }
+  const T* cb = code + bh * n_code_cap * d_c;
+  const int32_t* ib = idx + bh * n_code_cap * k;
+  const float* Sb = S + bh * n_ref_cap * G;
+
+  for (int64_t row = c0 + warp; row < c1; row += 8) {
+    // the code row, staged in this warp's slice of shared memory
+    float* cr = cw + warp * d_c;
+    for (int e = lane; e < d_c; e += 32) cr[e] = to_f(cb[row * d_c + e]);
+    __syncwarp();
+    float u[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+      u[m] = 0.f;
+      if (m < per_lane) {
+        int n = lane + 32 * m;
+        float acc = b3 ? b3[n] : 0.f;
+        for (int e = 0; e < d_c; ++e) acc = fmaf(W3s[e * hidden + n], cr[e], acc);
+        u[m] = act_eval(act, acc);
+      }
+    }
+    __syncwarp();
+    // reference part of the logits
+    int j = lane < k ? ib[row * k + lane] : -1;
+    if (j >= n_ref) { latch_error(err, DELTAKV_ERR_DEVICE_BOUNDS, (uint32_t)j); j = -1; }
+    const unsigned valid = __ballot_sync(0xffffffffu, j >= 0);
+    const int k_eff = __popc(valid);
+    const float inv_k = 1.0f / (float)max(k_eff, 1);
+    float lg[kMaxG];
+#pragma unroll
+    for (int g = 0; g < kMaxG; ++g) {
+      if (g < G) {
+        float part_ = 0.f;
+#pragma unroll
+        for (int m = 0; m < 8; ++m)
+          if (m < per_lane) part_ = fmaf(As[g * hidden + lane + 32 * m], u[m], part_);
+        float sr = j >= 0 ? Sb[(int64_t)j * G + g] : 0.f;
+        lg[g] = warp_sum(part_) + warp_sum(sr) * inv_k + ct[g];
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < kMaxG; ++g) {
+      if (g < G) {
+        if (lg[g] > mw[g]) {
+          float sc = exp2f(mw[g] - lg[g]);
+          lw[g] *= sc;
+#pragma unroll
+          for (int m = 0; m < 8; ++m) Uw[g][m] *= sc;
+          mw[g] = lg[g];
+        }
+        float p = exp2f(lg[g] - mw[g]);
+        lw[g] += p;
+#pragma unroll
+        for (int m = 0; m < 8; ++m) Uw[g][m] = fmaf(p, u[m], Uw[g][m]);
+        float dl = lg[g] - mref[g];
+        if (dl > 100.f) latch_error(err, DELTAKV_ERR_DEVICE_BOUNDS, 0xFFFFFFFFu);
+        float pr = exp2f(fminf(dl, 100.f)) * inv_k;
+        if (j >= 0) atomicAdd(&wtab[(int64_t)j * G + g], pr);
+      }
+    }
+  }
+  // merge the warps: block max, then rescale and sum l and U
+  __shared__ float mws[8][kMaxG];
+  if (lane == 0)
+#pragma unroll
+    for (int g = 0; g < kMaxG; ++g) mws[warp][g] = mw[g];
+  __syncthreads();
+  float mb[kMaxG];
+#pragma unroll
+  for (int g = 0; g < kMaxG; ++g) {
+    mb[g] = -INFINITY;
+    for (int w = 0; w < 8; ++w) mb[g] = fmaxf(mb[g], mws[w][g]);
+  }
+#pragma unroll
+  for (int g = 0; g < kMaxG; ++g) {
+    if (g < G) {
+      float sc = mw[g] == -INFINITY ? 0.f : exp2f(mw[g] - mb[g]);
+#pragma unroll
+      for (int m = 0; m < 8; ++m)
+        if (m < per_lane) atomicAdd(&Ured[g * hidden + lane + 32 * m], Uw[g][m] * sc);
+      if (lane == 0) atomicAdd(&misc[2 * kMaxG + g], lw[g] * sc);
+    }
+  }
+  __syncthreads();
+  const int64_t pb = bh * ns + split;
+  if (tid < G) {
+    part[(pb * G + tid) * 2 + 0] = mb[tid];
+    part[(pb * G + tid) * 2 + 1] = misc[2 * kMaxG + tid];
+  }
+  for (int i = tid; i < G * hidden; i += blockDim.x) Upart[pb * G * hidden + i] = Ured[i];
+  if (wt_in_smem) {
+    float* dst = wtab_g + pb * n_ref_cap * G;
+    for (int64_t i = tid; i < n_ref * G; i += blockDim.x) dst[i] = wt[i];
+  }
+}
+
+// -------------------------------------------------------- decode_combine
+// M_g = max(m_ref, split maxima).  For 256 slots: weights
+// w_j = 2^(S_j - M) + 2^(m_ref - M) sum_splits wtab, then sum_j w_j V_ref_j.
+template <typename T>
+__global__ void __launch_bounds__(256)
+    decode_combine_kernel(int T_, int s, int d_h, int H, int G, int ns, int64_t n_ref_cap,
+                          int n_refblk, int n_refblk_cap, int n_chunk_cap,
+                          const T* __restrict__ refv, const float* __restrict__ S,
+                          const float* __restrict__ Smax, const float* __restrict__ wtab_g,
+                          const float* __restrict__ part, float* __restrict__ ochunk) {
+  __shared__ float wts[kCombineSlots][kMaxG];
+  __shared__ float Mg[kMaxG], mrefg[kMaxG], lref[kMaxG];
+  const int b = blockIdx.z, h = blockIdx.y, ch = blockIdx.x, tid = threadIdx.x;
+  const int64_t bh = (int64_t)b * H + h;
+  const int64_t n_ref = (T_ + s - 1) / s;
+  const int64_t j0 = (int64_t)ch * kCombineSlots;
+  if (tid < G) {
+    float m = -INFINITY;
+    for (int r = 0; r < n_refblk; ++r) m = fmaxf(m, Smax[(bh * n_refblk_cap + r) * G + tid]);
+    mrefg[tid] = m;
+    float M = m;
+    for (int sp = 0; sp < ns; ++sp) M = fmaxf(M, part[((bh * ns + sp) * G + tid) * 2]);
+    Mg[tid] = M;
+    lref[tid] = 0.f;
+  }
+  __syncthreads();
+  for (int i = tid; i < kCombineSlots * G; i += blockDim.x) {
+    int jj = i / G, g = i - jj * G;
+    int64_t j = j0 + jj;
+    float w = 0.f;
+    if (j < n_ref) {
+      float own = exp2f(S[(bh * n_ref_cap + j) * G + g] - Mg[g]);
+      float acc = 0.f;
+      for (int sp = 0; sp < ns; ++sp) acc += wtab_g[((bh * ns + sp) * n_ref_cap + j) * G + g];
+      w = own + acc * exp2f(mrefg[g] - Mg[g]);
+      atomicAdd(&lref[g], own);
+    }
+    wts[jj][g] = w;
+  }
+  __syncthreads();
+  const T* vb = refv + bh * n_ref_cap * d_h;
+  for (int o = tid; o < G * d_h; o += blockDim.x) {
+    int g = o / d_h, e = o - g * d_h;
+    float acc = 0.f;
+    for (int jj = 0; jj < kCombineSlots; ++jj) {
+      int64_t j = j0 + jj;
+      if (j >= n_ref) break;
+      acc = fmaf(wts[jj][g], to_f(vb[j * d_h + e]), acc);
+    }
+    ochunk[((bh * n_chunk_cap + ch) * G + g) * (d_h + 1) + e] = acc;
+  }
+  if (tid < G) ochunk[((bh * n_chunk_cap + ch) * G + tid) * (d_h + 1) + d_h] = lref[tid];
+}
+
+// ---------------------------------------------------------- decode_final
+template <typename T>
+__global__ void __launch_bounds__(256)
+    decode_final_kernel(int T_, int s, int d_h, int H, int G, int hidden, int ns, int n_chunk,
+                        int n_chunk_cap, int n_refblk, int n_refblk_cap,
+                        const T* __restrict__ W4, const float* __restrict__ b4,
+                        const float* __restrict__ Smax, const float* __restrict__ part,
+                        const float* __restrict__ Upart, const float* __restrict__ ochunk,
+                        float* __restrict__ out, int64_t osb, int64_t osh) {
+  __shared__ float Ut[kMaxG][kMaxHidden];
+  __shared__ float Mg[kMaxG], Lnr[kMaxG], Lall[kMaxG];
+  const int b = blockIdx.z, h = blockIdx.y, tid = threadIdx.x;
+  const int64_t bh = (int64_t)b * H + h;
+  if (tid < G) {
+    float M = -INFINITY;
+    for (int r = 0; r < n_refblk; ++r) M = fmaxf(M, Smax[(bh * n_refblk_cap + r) * G + tid]);
+    for (int sp = 0; sp < ns; ++sp) M = fmaxf(M, part[((bh * ns + sp) * G + tid) * 2]);
+    float lnr = 0.f;
+    for (int sp = 0; sp < ns; ++sp) {
+      float m = part[((bh * ns + sp) * G + tid) * 2];
+      float l = part[((bh * ns + sp) * G + tid) * 2 + 1];
+      if (m != -INFINITY) lnr += l * exp2f(m - M);
+    }
+    float lr = 0.f;
+    for (int c = 0; c < n_chunk; ++c) lr += ochunk[((bh * n_chunk_cap + c) * G + tid) * (d_h + 1) + d_h];
+    Mg[tid] = M;
+    Lnr[tid] = lnr;
+    Lall[tid] = lnr + lr;
+  }
+  __syncthreads();
+  for (int i = tid; i < G * hidden; i += blockDim.x) {
+    int g = i / hidden, n = i - g * hidden;
+    float acc = 0.f;
+    for (int sp = 0; sp < ns; ++sp) {
+      float m = part[((bh * ns + sp) * G + g) * 2];
+      if (m != -INFINITY) acc += Upart[((bh * ns + sp) * G + g) * hidden + n] * exp2f(m - Mg[g]);
+    }
+    Ut[g][n] = acc;
+  }
+  __syncthreads();
+  for (int o = tid; o < G * d_h; o += blockDim.x) {
+    int g = o / d_h, e = o - g * d_h;
+    float acc = 0.f;
+    for (int c = 0; c < n_chunk; ++c) acc += ochunk[((bh * n_chunk_cap + c) * G + g) * (d_h + 1) + e];
+    const T* w4 = W4 + (int64_t)(d_h + e) * hidden;
+    float y = 0.f;
+    for (int n = 0; n < hidden; ++n) y = fmaf(to_f(w4[n]), Ut[g][n], y);
+    acc += y + (b4 ? b4[d_h + e] * Lnr[g] : 0.f);
+    out[b * osb + (int64_t)(h * G + g) * osh + e] = acc / Lall[g];
+  }
+}
+
+// ------------------------------------------------------------- launcher
+template <typename E>
+static cudaError_t decode_launch(const Plan& p, int T, const void* q, int64_t qsb, int64_t qsh,
+                                 const void* cache, const void* W3, const float* b3,
+                                 const void* W4, const float* b4, float* out, int64_t osb,
+                                 int64_t osh, void* ws, cudaStream_t st) {
+  const auto& c = p.cfg;
+  const int H = c.kv_heads, B = c.batch, G = p.G;
+  const int64_t n_ref = n_ref_of(T, c.stride_s);
+  const int64_t n_code = n_code_of(T, c.stride_s);
+  const float cs = kLog2e / sqrtf((float)c.d_h);
+  const char* cb = (const char*)cache;
+  char* w = (char*)ws;
+  const E* refk = (const E*)(cb + p.off_refk);
+  const E* refv = (const E*)(cb + p.off_refv);
+  const E* code = (const E*)(cb + p.off_code);
+  const int32_t* idx = (const int32_t*)(cb + p.off_idx);
+  float* S = (float*)(w + p.ws_S);
+  float* Smax = (float*)(w + p.ws_Smax);
+  float* a = (float*)(w + p.ws_a);
+  float* cterm = (float*)(w + p.ws_cterm);
+  float* wtab = (float*)(w + p.ws_wtab);
+  float* part = (float*)(w + p.ws_part);
+  float* Upart = (float*)(w + p.ws_U);
+  float* ochunk = (float*)(w + p.ws_ochunk);
+  const int n_refblk = (int)ceil_div64(n_ref, kRefBlockSlots);
+  const int n_refblk_cap = (int)ceil_div64(p.n_ref_cap, kRefBlockSlots);
+  const int n_chunk = (int)ceil_div64(n_ref, kCombineSlots);
+
+  {
+    ProfScope ps(p, st, KID_DEC_REF);
+    decode_ref_kernel<E><<<dim3(n_refblk, H, B), 256, 0, st>>>(
+      n_ref, p.n_ref_cap, c.d_h, H, G, cs, (const E*)q, qsb, qsh, refk, S, Smax, n_refblk_cap);
+  }
+  {
+    ProfScope ps(p, st, KID_DEC_PREP);
+    decode_prep_kernel<E><<<dim3(1, H, B), 256, 0, st>>>(c.d_h, H, G, c.hidden, cs, (const E*)q, qsb,
+                                                       qsh, (const E*)W4, b4, a, cterm);
+  }
+  // splits: enough blocks for about two waves, never more rows than splits
+  int ns = (int)ceil_div64(2 * kNumSMs, (int64_t)B * H);
+  ns = (int)std::min<int64_t>(std::min<int64_t>(ns, p.ns_max), std::max<int64_t>(1, n_code / 64));
+  size_t base = sizeof(float) * (size_t)(c.d_c * c.hidden + 2 * G * c.hidden + 4 * kMaxG + 8 * c.d_c);
+  size_t wt_bytes = sizeof(float) * (size_t)(n_ref * G);
+  int wt_in_smem = base + wt_bytes <= 200 * 1024;
+  size_t smem = base + (wt_in_smem ? wt_bytes : 0);
+  auto ks = decode_stream_kernel<E>;
+  cudaError_t e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  {
+  ProfScope ps(p, st, KID_DEC_STREAM);
+  ks<<<dim3(ns, H, B), 256, smem, st>>>(T, c.stride_s, c.d_h, H, G, c.k, c.d_c, c.hidden,
+                                        (int)c.act, ns, p.n_ref_cap, p.n_code_cap, n_refblk,
+                                        n_refblk_cap, code, idx, (const E*)W3, b3, a, cterm, S,
+                                        Smax, wtab, part, Upart, wt_in_smem, (uint32_t*)ws);
+  }
+  {
+    ProfScope ps(p, st, KID_DEC_COMBINE);
+    decode_combine_kernel<E><<<dim3(n_chunk, H, B), 256, 0, st>>>(
+      T, c.stride_s, c.d_h, H, G, ns, p.n_ref_cap, n_refblk, n_refblk_cap, p.n_chunk_cap, refv, S,
+      Smax, wtab, part, ochunk);
+  }
+  {
+    ProfScope ps(p, st, KID_DEC_FINAL);
+    decode_final_kernel<E><<<dim3(1, H, B), 256, 0, st>>>(
+      T, c.stride_s, c.d_h, H, G, c.hidden, ns, n_chunk, p.n_chunk_cap, n_refblk, n_refblk_cap,
+      (const E*)W4, b4, Smax, part, Upart, ochunk, out, osb, osh);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode(const Plan& p, int T, const void* q, int64_t qsb, int64_t qsh,
+                          const void* cache, const void* W3, const float* b3, const void* W4,
+                          const float* b4, float* out, int64_t osb, int64_t osh, void* ws,
+                          cudaStream_t st) {
+  if (p.cfg.dtype == DELTAKV_BF16)
+    return decode_launch<__nv_bfloat16>(p, T, q, qsb, qsh, cache, W3, b3, W4, b4, out, osb, osh,
+                                        ws, st);
+  return decode_launch<float>(p, T, q, qsb, qsh, cache, W3, b3, W4, b4, out, osb, osh, ws, st);
+}
+
+}  // namespace dkv

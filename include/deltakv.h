@@ -1,0 +1,195 @@
+/*
+ * deltakv.h -- C ABI of the B200 (sm_100a) DeltaKV residual KV-cache library.
+ *
+ * Method: "DeltaKV: Residual-Based KV Cache Compression via Long-Range
+ * Similarity" (gist.science summary, section 3 "Metodologia").  A few tokens,
+ * picked with a fixed stride, are kept whole as references ("Struttura della
+ * Compressione"); every other token stores only a low-dimensional code of its
+ * residual against the mean of its k most similar earlier references
+ * ("Processo di Compressione", steps 1-4); decode rebuilds tokens from the
+ * references and the decoded residual ("Ricostruzione") on demand inside the
+ * attention that reads the cache (section 4, "Ottimizza i Kernel").
+ *
+ * Conventions shared by every entry point:
+ *  - The caller owns all memory.  Device pointers are plain CUDA device
+ *    addresses on the current device; nothing here allocates device memory.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream).  The returned status covers host-side validation and launch
+ *    errors only.  Errors the kernels detect (a bounded wait that ran out, an
+ *    out-of-range index) are latched in the first 16 bytes of the workspace and
+ *    reported by deltakv_device_status().
+ *  - Inputs are const and are never written.
+ *  - Every device pointer must be 16-byte aligned and innermost dimensions
+ *    must be contiguous, else DELTAKV_ERR_ALIGNMENT; nothing is launched on any
+ *    error.
+ *  - One call processes one layer; a model loops over its layers and passes
+ *    each layer's weights and cache.
+ *
+ * Notation: B sequences, H kv-heads, Hq query heads (G = Hq / H, consecutive
+ * query heads share a kv-head), d_h head size, D = 2 d_h, stride s, k
+ * references per token, d_c code width, `hidden` MLP width, T tokens.  Token
+ * t is a reference iff t mod s == 0; reference slot j is token j s.
+ */
+#ifndef DELTAKV_H
+#define DELTAKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DELTAKV_OK = 0,
+    DELTAKV_ERR_INVALID_ARG = 1,    /* NULL, negative or inconsistent argument */
+    DELTAKV_ERR_UNSUPPORTED = 2,    /* valid but not built (see deltakv_plan) */
+    DELTAKV_ERR_ALIGNMENT = 3,      /* pointer or stride breaks the 16-byte rule */
+    DELTAKV_ERR_WORKSPACE = 4,      /* workspace smaller than deltakv_plan said */
+    DELTAKV_ERR_CUDA = 5,           /* a CUDA runtime call failed */
+    DELTAKV_ERR_DEVICE_TIMEOUT = 6, /* a kernel's bounded wait ran out */
+    DELTAKV_ERR_DEVICE_BOUNDS = 7   /* a kernel met an out-of-range index */
+} deltakv_status;
+
+typedef enum { DELTAKV_BF16 = 0, DELTAKV_F32 = 1 } deltakv_dtype;
+
+/* Nonlinearity between the two linear layers of the compressor and of the
+ * decompressor.  GELU_ERF is x * Phi(x). */
+typedef enum {
+    DELTAKV_ACT_GELU_ERF = 0,
+    DELTAKV_ACT_GELU_TANH = 1,
+    DELTAKV_ACT_NONE = 2
+} deltakv_act;
+
+/* The problem as the DeltaKV summary states it (section 3): layers,
+ * kv-heads, head size, stride, k, code width, MLP width.
+ * Supported: d_h in {64, 128}; 1 <= s; 1 <= k <= 8; d_c in {16, 32, 64} or
+ * d_c == hidden == 2 d_h with d_h = 64 (identity codec); 32 <= hidden <= 256, hidden a
+ * multiple of 32; q_heads a multiple of kv_heads with G <= 8. */
+typedef struct {
+    int32_t layers;    /* informational: the model holds `layers` caches */
+    int32_t batch;     /* B */
+    int32_t kv_heads;  /* H */
+    int32_t q_heads;   /* Hq */
+    int32_t d_h;
+    int32_t max_T;     /* token capacity of one cache */
+    int32_t stride_s;  /* s */
+    int32_t k;
+    int32_t d_c;
+    int32_t hidden;
+    deltakv_dtype dtype; /* element type of K, V, q, weights, stored refs and codes */
+    deltakv_act act;
+} deltakv_config;
+
+typedef struct deltakv_plan_s* deltakv_plan_t; /* opaque, host memory only */
+typedef struct CUstream_st* deltakv_stream_t;  /* same type as cudaStream_t */
+
+/* Packed compressed cache of one layer, offsets in bytes from its base.
+ * Four planes, each [B][H][rows][cols] row-major:
+ *   ref_k, ref_v : [B][H][n_ref_cap][d_h]  dtype  -- reference rows, stored
+ *                  whole (slot j = token j s);
+ *   code         : [B][H][n_code_cap][d_c] dtype  -- one row per non-reference
+ *                  token, in token order: token t (t mod s != 0) is row
+ *                  t - floor(t / s) - 1;
+ *   idx          : [B][H][n_code_cap][k]   int32  -- its reference slots in
+ *                  ascending (distance, slot) order, -1 where fewer than k
+ *                  earlier references exist.
+ * For a cache holding T tokens the first ceil(T/s) reference rows and the
+ * first T - ceil(T/s) code/idx rows of each (b, head) are used. */
+typedef struct {
+    size_t ref_k_offset, ref_v_offset, code_offset, idx_offset;
+    size_t total_bytes;
+    int64_t n_ref_cap;
+    int64_t n_code_cap;
+} deltakv_cache_layout;
+
+/* Validate `cfg`, build a host-side plan, and report the bytes of one layer's
+ * packed cache and of the device workspace that compress, decode and
+ * reconstruct need (both 256-byte aligned sizes).  No device work.
+ * Errors: INVALID_ARG, UNSUPPORTED. */
+deltakv_status deltakv_plan(const deltakv_config* cfg, deltakv_plan_t* plan_out,
+                            size_t* cache_bytes_per_layer, size_t* workspace_bytes);
+
+deltakv_status deltakv_plan_destroy(deltakv_plan_t plan);
+
+deltakv_status deltakv_get_cache_layout(deltakv_plan_t plan, deltakv_cache_layout* out);
+
+/* Compress one layer ("Processo di Compressione" steps 1-4): for every
+ * non-reference token, choose its k nearest earlier references by squared
+ * L2 distance over [K_t ; V_t] (ties to the lower slot), subtract their mean,
+ * and encode the residual with code = W2 act(W1 r + b1) + b2; write the
+ * reference rows, codes and slots into `cache`.
+ *   T          : 0 <= T <= max_T tokens (T = 0 launches nothing)
+ *   K, V       : device, element (b, h, t, e) at base + b*strides[0] +
+ *                h*strides[1] + t*strides[2] + e (strides in elements)
+ *   W1 [hidden][D], W2 [d_c][hidden]: device, dtype, row-major
+ *   b1 [hidden], b2 [d_c]: device float32 or NULL (zero)
+ *   cache      : device, cache_bytes_per_layer bytes (overwritten)
+ *   workspace  : device, workspace_bytes bytes, contents scratch. */
+deltakv_status deltakv_compress(deltakv_plan_t plan, int32_t T,
+                                const void* K, const void* V, const int64_t kv_strides[3],
+                                const void* W1, const float* b1,
+                                const void* W2, const float* b2,
+                                void* cache, void* workspace, size_t workspace_bytes,
+                                deltakv_stream_t stream);
+
+/* Decode attention over one layer's compressed cache ("Ricostruzione" and
+ * section 4): for query head hq (kv-head hq / G),
+ *   out = sum_t softmax_t(q . K_hat_t / sqrt(d_h)) V_hat_t over the T cached
+ * tokens, where reference rows are used as stored and every other token is
+ * KV_R + W4 act(W3 code + b3) + b4 (first d_h entries K, last d_h V),
+ * rebuilt on the fly and never written out.
+ *   T >= 1; q: device [B][Hq][d_h] dtype with element strides
+ *   q_strides = {batch, head}; W3 [hidden][d_c], W4 [D][hidden] dtype;
+ *   b3 [hidden], b4 [D] float32 or NULL; out: device float32 [B][Hq][d_h]
+ *   with element strides out_strides = {batch, head}. */
+deltakv_status deltakv_decode_attention(deltakv_plan_t plan, int32_t T,
+                                        const void* q, const int64_t q_strides[2],
+                                        const void* cache,
+                                        const void* W3, const float* b3,
+                                        const void* W4, const float* b4,
+                                        float* out, const int64_t out_strides[2],
+                                        void* workspace, size_t workspace_bytes,
+                                        deltakv_stream_t stream);
+
+/* Rebuild every token of one layer ("Ricostruzione") into dense float32
+ * K_out, V_out [B][H][T][d_h] (contiguous).  For tests and debugging; the
+ * decode path never materialises these. */
+deltakv_status deltakv_reconstruct(deltakv_plan_t plan, int32_t T, const void* cache,
+                                   const void* W3, const float* b3,
+                                   const void* W4, const float* b4,
+                                   float* K_out, float* V_out,
+                                   void* workspace, size_t workspace_bytes,
+                                   deltakv_stream_t stream);
+
+/* Synchronise `stream`, read and clear the error word that the kernels latch
+ * in `workspace`, and return DELTAKV_OK, DEVICE_TIMEOUT or DEVICE_BOUNDS. */
+deltakv_status deltakv_device_status(deltakv_plan_t plan, void* workspace,
+                                     deltakv_stream_t stream);
+
+/* Benchmark support: per-kernel device time.  While profiling is on for a
+ * plan, every kernel its calls launch is bracketed by two CUDA events
+ * recorded on the call's own stream (host-side bookkeeping only; the kernels
+ * are unchanged).  deltakv_profile_collect waits for the recorded events,
+ * writes one entry per kernel that ran (up to n_max) with its launch count
+ * and summed time, and forgets the records. */
+typedef struct {
+    char name[32];
+    int32_t launches;
+    double total_ms;
+} deltakv_kernel_time;
+
+deltakv_status deltakv_set_profiling(deltakv_plan_t plan, int32_t enable);
+deltakv_status deltakv_profile_collect(deltakv_plan_t plan, deltakv_kernel_time* out,
+                                       int32_t n_max, int32_t* n_out);
+
+/* Static description of a status code. */
+const char* deltakv_status_string(deltakv_status status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int32_t deltakv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DELTAKV_H */

@@ -24,6 +24,7 @@ from .oracle import (  # noqa: F401
     attention,
     build,
     compress,
+    compress_rows,
     lib_path,
     mlp,
     reconstruct,

@@ -193,12 +193,73 @@ void deltakv_oracle_mlp(int n_in, int hid, int n_out, int act,
     free(h);
 }
 
-/* Compress one (sequence, kv-head): K, V are [T][d_h].  Outputs
- *   idx  [T][k]   chosen slots (-1 for reference tokens and padding),
- *   code [T][d_c] the stored code, rounded per round_mode (0 for refs),
- *   d_k, d_k1 [T] the k-th and (k+1)-th smallest distances (NAN for refs).
- * Tokens are independent, so the loop over them may run on several threads
- * (n_threads <= 0 keeps the library default). */
+/* Compress one non-reference or reference token t of a (sequence, kv-head):
+ * idx row [k], code row [d_c], and the k-th / (k+1)-th smallest distances.
+ * r and c are caller scratch of 2*d_h and d_c doubles. */
+static void compress_token(int t, int d_h, int s, int k, int d_c, int hidden, int act,
+                           int round_mode, const double* K, const double* V,
+                           const double* W1, const double* b1,
+                           const double* W2, const double* b2,
+                           int32_t* it, double* ct, double* dk, double* dk1,
+                           double* r, double* c)
+{
+    if (t % s == 0) { /* reference token: stored as it is */
+        for (int i = 0; i < k; ++i) it[i] = -1;
+        for (int o = 0; o < d_c; ++o) ct[o] = 0.0;
+        if (dk) *dk = NAN;
+        if (dk1) *dk1 = NAN;
+        return;
+    }
+    double a, b;
+    deltakv_oracle_select(t, d_h, s, k, K, V, it, &a, &b);
+    if (dk) *dk = a;
+    if (dk1) *dk1 = b;
+    residual(t, d_h, s, k, K, V, it, r);
+    deltakv_oracle_mlp(2 * d_h, hidden, d_c, act, W1, b1, W2, b2, r, c);
+    for (int o = 0; o < d_c; ++o) ct[o] = deltakv_oracle_round(round_mode, c[o]);
+}
+
+/* Compress the tokens listed in rows[0..n_rows) of one (sequence, kv-head)
+ * whose K, V are [T][d_h].  Output row i belongs to token rows[i]:
+ *   idx  [n_rows][k]   chosen slots (-1 for reference tokens and padding),
+ *   code [n_rows][d_c] the stored code, rounded per round_mode (0 for refs),
+ *   d_k, d_k1 [n_rows] the k-th and (k+1)-th smallest distances (NAN for
+ *   references).  Tokens are independent, so the loop may run on several
+ *   threads (n_threads <= 0 keeps the library default). */
+int deltakv_oracle_compress_rows(int T, int d_h, int s, int k, int d_c, int hidden,
+                                 int act, int round_mode,
+                                 const double* K, const double* V,
+                                 const double* W1, const double* b1,
+                                 const double* W2, const double* b2,
+                                 int n_rows, const int32_t* rows,
+                                 int32_t* idx, double* code, double* d_k, double* d_k1,
+                                 int n_threads)
+{
+    if (T < 0 || d_h <= 0 || s <= 0 || k <= 0 || d_c <= 0 || hidden <= 0 || n_rows < 0)
+        return -1;
+    for (int i = 0; i < n_rows; ++i)
+        if (rows[i] < 0 || rows[i] >= T) return -1;
+#ifdef _OPENMP
+    if (n_threads > 0) omp_set_num_threads(n_threads);
+#else
+    (void)n_threads;
+#endif
+#pragma omp parallel
+    {
+        double* r = (double*)malloc(sizeof(double) * (size_t)(2 * d_h));
+        double* c = (double*)malloc(sizeof(double) * (size_t)d_c);
+#pragma omp for schedule(dynamic, 16)
+        for (int i = 0; i < n_rows; ++i)
+            compress_token(rows[i], d_h, s, k, d_c, hidden, act, round_mode, K, V, W1, b1, W2, b2,
+                           idx + (size_t)i * k, code + (size_t)i * d_c,
+                           d_k ? d_k + i : NULL, d_k1 ? d_k1 + i : NULL, r, c);
+        free(r);
+        free(c);
+    }
+    return 0;
+}
+
+/* Compress every token 0..T-1 (rows = 0, 1, ..., T-1). */
 int deltakv_oracle_compress(int T, int d_h, int s, int k, int d_c, int hidden,
                             int act, int round_mode,
                             const double* K, const double* V,
@@ -207,41 +268,14 @@ int deltakv_oracle_compress(int T, int d_h, int s, int k, int d_c, int hidden,
                             int32_t* idx, double* code, double* d_k, double* d_k1,
                             int n_threads)
 {
-    if (T < 0 || d_h <= 0 || s <= 0 || k <= 0 || d_c <= 0 || hidden <= 0)
-        return -1;
-    int D = 2 * d_h;
-#ifdef _OPENMP
-    if (n_threads > 0) omp_set_num_threads(n_threads);
-#else
-    (void)n_threads;
-#endif
-#pragma omp parallel
-    {
-        double* r = (double*)malloc(sizeof(double) * (size_t)D);
-        double* c = (double*)malloc(sizeof(double) * (size_t)d_c);
-#pragma omp for schedule(dynamic, 16)
-        for (int t = 0; t < T; ++t) {
-            int32_t* it = idx + (size_t)t * k;
-            double* ct = code + (size_t)t * d_c;
-            if (t % s == 0) { /* reference token: stored as it is */
-                for (int i = 0; i < k; ++i) it[i] = -1;
-                for (int o = 0; o < d_c; ++o) ct[o] = 0.0;
-                if (d_k) d_k[t] = NAN;
-                if (d_k1) d_k1[t] = NAN;
-                continue;
-            }
-            double a, b;
-            deltakv_oracle_select(t, d_h, s, k, K, V, it, &a, &b);
-            if (d_k) d_k[t] = a;
-            if (d_k1) d_k1[t] = b;
-            residual(t, d_h, s, k, K, V, it, r);
-            deltakv_oracle_mlp(D, hidden, d_c, act, W1, b1, W2, b2, r, c);
-            for (int o = 0; o < d_c; ++o) ct[o] = deltakv_oracle_round(round_mode, c[o]);
-        }
-        free(r);
-        free(c);
-    }
-    return 0;
+    if (T < 0) return -1;
+    int32_t* rows = (int32_t*)malloc(sizeof(int32_t) * (size_t)(T > 0 ? T : 1));
+    for (int t = 0; t < T; ++t) rows[t] = t;
+    int rc = deltakv_oracle_compress_rows(T, d_h, s, k, d_c, hidden, act, round_mode, K, V,
+                                          W1, b1, W2, b2, T, rows, idx, code, d_k, d_k1,
+                                          n_threads);
+    free(rows);
+    return rc;
 }
 
 /* ------------------------------------------------------- reconstruction */

@@ -57,6 +57,8 @@ def _load():
             lib.deltakv_oracle_mlp.restype = None
             lib.deltakv_oracle_mlp.argtypes = [
                 ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _dp, _dp, _dp, _dp, _dp, _dp]
+            lib.deltakv_oracle_compress_rows.restype = ctypes.c_int
+            lib.deltakv_oracle_compress_rows.argtypes = [ctypes.c_int] * 8 + [_dp] * 6 + [ctypes.c_int, _ip, _ip, _dp, _dp, _dp, ctypes.c_int]
             lib.deltakv_oracle_compress.restype = ctypes.c_int
             lib.deltakv_oracle_compress.argtypes = [ctypes.c_int] * 8 + [_dp] * 6 + [_ip, _dp, _dp, _dp, ctypes.c_int]
             lib.deltakv_oracle_reconstruct.restype = ctypes.c_int
@@ -126,6 +128,30 @@ def compress(K, V, W1, b1, W2, b2, s: int, k: int, act_kind: int = ACT_GELU_ERF,
                                          _ptr(idx, _ip), _ptr(code), _ptr(dk), _ptr(dk1), int(n_threads))
     if rc != 0:
         raise ValueError("oracle compress: invalid arguments")
+    return idx, code, dk, dk1
+
+
+def compress_rows(K, V, W1, b1, W2, b2, s: int, k: int, rows, act_kind: int = ACT_GELU_ERF,
+                  round_mode: int = ROUND_BF16, n_threads: int = 0):
+    """Compress only the tokens in `rows` of one (sequence, kv-head).
+
+    Returns (idx [n,k] int32, code [n,d_c], d_k [n], d_k1 [n]) for those rows."""
+    K, V, W1, b1, W2, b2 = _f64(K), _f64(V), _f64(W1), _f64(b1), _f64(W2), _f64(b2)
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int32))
+    T, d_h = K.shape
+    hidden = W1.shape[0]
+    d_c = W2.shape[0]
+    n = rows.shape[0]
+    idx = np.empty((n, k), dtype=np.int32)
+    code = np.empty((n, d_c), dtype=np.float64)
+    dk = np.empty(n, dtype=np.float64)
+    dk1 = np.empty(n, dtype=np.float64)
+    rc = _load().deltakv_oracle_compress_rows(T, d_h, int(s), int(k), d_c, hidden, int(act_kind), int(round_mode),
+                                              _ptr(K), _ptr(V), _ptr(W1), _ptr(b1), _ptr(W2), _ptr(b2),
+                                              n, _ptr(rows, _ip), _ptr(idx, _ip), _ptr(code), _ptr(dk), _ptr(dk1),
+                                              int(n_threads))
+    if rc != 0:
+        raise ValueError("oracle compress_rows: invalid arguments")
     return idx, code, dk, dk1
 
 

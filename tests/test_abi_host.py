@@ -1,0 +1,108 @@
+"""Host-side checks of the C ABI (no GPU): the library loads, exports every
+entry point include/deltakv.h declares, validates configurations, reports the
+packed-cache layout, and rejects bad arguments before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from decode_attention_strided_b200 import build as dkv_build
+from decode_attention_strided_b200 import deltakv as dkv
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    dkv_build.build()
+    return dkv.load_library()
+
+
+def _declared_symbols():
+    text = open(os.path.join(ROOT, "include", "deltakv.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(deltakv_[a-z_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    declared = _declared_symbols()
+    assert "deltakv_plan" in declared and "deltakv_compress" in declared
+    assert "deltakv_decode_attention" in declared
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert set(declared) == set(dkv.SYMBOLS)
+
+
+def test_version_and_status_strings(lib):
+    assert dkv.version() >= 10000
+    for code in range(8):
+        assert lib.deltakv_status_string(code)
+
+
+def _cfg(**kw):
+    base = dict(batch=8, kv_heads=8, q_heads=32, d_h=128, max_T=131072, stride_s=16, k=4, d_c=32,
+                hidden=256, dtype=dkv.BF16, act=dkv.ACT_GELU_ERF, layers=32)
+    base.update(kw)
+    return dkv.Config(**base)
+
+
+def test_layout_of_the_128k_decode_configuration(lib):
+    p = dkv.plan(_cfg())
+    L = p.layout
+    assert L["n_ref_cap"] == 8192 and L["n_code_cap"] == 131072 - 8192
+    B, H = 8, 8
+    # refs: 2 planes of d_h bf16; codes d_c bf16; idx k int32
+    assert L["ref_v_offset"] - L["ref_k_offset"] == B * H * 8192 * 128 * 2
+    assert L["idx_offset"] - L["code_offset"] == B * H * (131072 - 8192) * 32 * 2
+    assert L["total_bytes"] == p.cache_bytes
+    used = B * H * (8192 * 512 + (131072 - 8192) * (64 + 16))
+    assert p.cache_bytes >= used and p.cache_bytes < used + 4096
+    # 20.9% of a full bf16 cache of the same tokens
+    full = B * H * 131072 * 2 * 128 * 2
+    assert abs(used / full - 0.2090) < 1e-3
+    for off in ("ref_k_offset", "ref_v_offset", "code_offset", "idx_offset"):
+        assert L[off] % 256 == 0
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(batch=0), 1), (dict(q_heads=12), 1), (dict(stride_s=0), 1), (dict(k=0), 1),
+    (dict(d_h=96), 2), (dict(k=9), 2), (dict(d_c=24), 2), (dict(hidden=48), 2),
+    (dict(q_heads=8 * 16), 2), (dict(dtype=7), 1), (dict(act=9), 1),
+])
+def test_plan_rejects(lib, bad, code):
+    with pytest.raises(dkv.DeltaKVError) as ei:
+        dkv.plan(_cfg(**bad))
+    assert ei.value.code == code
+
+
+def test_identity_codec_shape_is_accepted(lib):
+    p = dkv.plan(_cfg(d_h=64, d_c=128, hidden=128, dtype=dkv.F32, act=dkv.ACT_NONE))
+    assert p.cache_bytes > 0
+
+
+def test_calls_reject_bad_arguments_before_any_launch(lib):
+    p = dkv.plan(_cfg(batch=1, kv_heads=1, q_heads=4, max_T=1024))
+    vp = ctypes.c_void_p
+    strides = (ctypes.c_int64 * 3)(1024 * 128, 1024 * 128, 128)
+    fake = vp(1 << 20)  # never dereferenced: validation fails first
+    ws = p.workspace_bytes
+    # T out of range
+    assert lib.deltakv_compress(p.handle, 2048, fake, fake, strides, fake, None, fake, None, fake, fake, ws, None) == 1
+    # T = 0 is a no-op
+    assert lib.deltakv_compress(p.handle, 0, None, None, None, None, None, None, None, None, None, 0, None) == 0
+    # workspace too small
+    assert lib.deltakv_compress(p.handle, 512, fake, fake, strides, fake, None, fake, None, fake, fake, ws - 1, None) == 4
+    # misaligned pointer
+    assert lib.deltakv_compress(p.handle, 512, vp((1 << 20) + 2), fake, strides, fake, None, fake, None, fake, fake, ws, None) == 3
+    # stride that is not a multiple of 16 bytes
+    bad = (ctypes.c_int64 * 3)(1024 * 128, 1024 * 128, 129)
+    assert lib.deltakv_compress(p.handle, 512, fake, fake, bad, fake, None, fake, None, fake, fake, ws, None) == 3
+    # NULL weights
+    assert lib.deltakv_compress(p.handle, 512, fake, fake, strides, None, None, fake, None, fake, fake, ws, None) == 1
+    qs = (ctypes.c_int64 * 2)(4 * 128, 128)
+    # decode needs T >= 1
+    assert lib.deltakv_decode_attention(p.handle, 0, fake, qs, fake, fake, None, fake, None, fake, qs, fake, ws, None) == 1
+    assert lib.deltakv_decode_attention(p.handle, 100, fake, qs, fake, fake, None, fake, None, vp((1 << 20) + 4), qs, fake, ws, None) == 3
+    assert lib.deltakv_reconstruct(p.handle, -1, fake, fake, None, fake, None, fake, fake, fake, ws, None) == 1
+    assert lib.deltakv_plan_destroy(None) == 0
