@@ -14,12 +14,9 @@ void profiler_destroy(Profiler* p);
 int profiler_collect(Profiler* p, deltakv_kernel_time* out, int n_max);
 }  // namespace dkv
 
-struct deltakv_plan_s {
-  Plan p;
-  ~deltakv_plan_s() {
-    if (p.prof) profiler_destroy(p.prof);
-  }
-};
+deltakv_plan_s::~deltakv_plan_s() {
+  if (p.prof) profiler_destroy(p.prof);
+}
 
 namespace {
 

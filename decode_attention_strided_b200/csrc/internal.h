@@ -97,3 +97,9 @@ cudaError_t launch_decode(const Plan& p, int T, const void* q, int64_t qsb, int6
                           cudaStream_t st);
 
 }  // namespace dkv
+
+// The opaque plan handle of the C ABI.
+struct deltakv_plan_s {
+  dkv::Plan p;
+  ~deltakv_plan_s();
+};

@@ -27,7 +27,7 @@ STATUS = {
 
 SYMBOLS = ("deltakv_plan", "deltakv_plan_destroy", "deltakv_get_cache_layout", "deltakv_compress",
            "deltakv_decode_attention", "deltakv_reconstruct", "deltakv_device_status",
-           "deltakv_set_profiling", "deltakv_profile_collect",
+           "deltakv_decode_attention_noalloc", "deltakv_set_profiling", "deltakv_profile_collect",
            "deltakv_status_string", "deltakv_version")
 
 
@@ -76,6 +76,8 @@ def load_library(path: str = LIB_PATH):
     lib.deltakv_compress.restype = ctypes.c_int
     lib.deltakv_decode_attention.argtypes = [vp, i32, vp, i64p, vp, vp, vp, vp, vp, vp, i64p, vp, sz, vp]
     lib.deltakv_decode_attention.restype = ctypes.c_int
+    lib.deltakv_decode_attention_noalloc.argtypes = [vp, i32, vp, i64p, vp, vp, vp, vp, vp, vp, i64p, vp]
+    lib.deltakv_decode_attention_noalloc.restype = ctypes.c_int
     lib.deltakv_reconstruct.argtypes = [vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.deltakv_reconstruct.restype = ctypes.c_int
     lib.deltakv_device_status.argtypes = [vp, vp, vp]
@@ -209,6 +211,18 @@ def decode_attention(p: Plan, T: int, q, cache, W3, b3, W4, b4, out, workspace, 
     _check("deltakv_decode_attention", lib.deltakv_decode_attention(
         p.handle, int(T), _ptr(q), qs, _ptr(cache), _ptr(W3), _ptr(b3), _ptr(W4), _ptr(b4), _ptr(out), os_,
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def decode_attention_noalloc(p: Plan, T: int, q, cache, W3, b3, W4, b4, out, stream=None):
+    """deltakv_decode_attention_noalloc: decode attention without a caller
+    workspace, for callers that cannot allocate device memory (the library's
+    own 16 MiB static scratch is used; larger plans raise ERR_WORKSPACE)."""
+    lib = load_library()
+    qs = (ctypes.c_int64 * 2)(q.stride(0), q.stride(1))
+    os_ = (ctypes.c_int64 * 2)(out.stride(0), out.stride(1))
+    _check("deltakv_decode_attention_noalloc", lib.deltakv_decode_attention_noalloc(
+        p.handle, int(T), _ptr(q), qs, _ptr(cache), _ptr(W3), _ptr(b3), _ptr(W4), _ptr(b4), _ptr(out), os_,
+        _stream(stream)))
 
 
 def reconstruct(p: Plan, T: int, cache, W3, b3, W4, b4, K_out, V_out, workspace, stream=None):

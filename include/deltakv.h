@@ -162,6 +162,31 @@ deltakv_status deltakv_reconstruct(deltakv_plan_t plan, int32_t T, const void* c
                                    void* workspace, size_t workspace_bytes,
                                    deltakv_stream_t stream);
 
+/* Decode attention for callers that cannot allocate device memory: code
+ * running inside a memory budget fixed at start-up, plugins hosted by an
+ * engine that owns every allocation, or steps where an allocation could block
+ * or fail.  Same computation and arguments as deltakv_decode_attention, minus
+ * the workspace: scratch comes from a 16 MiB array that the library holds in
+ * device memory (every GPU that loads this part of the library keeps it until
+ * the process exits).  The paper has no counterpart to this entry point.
+ *  - Plans whose workspace_bytes exceeds 16 MiB: DELTAKV_ERR_WORKSPACE,
+ *    nothing launched.
+ *  - Nothing is allocated: no cudaMalloc, no cudaFree, no allocating library
+ *    call.  The first call on a device looks up the array's device address
+ *    (once per device); make that first call before any stream capture.
+ *  - All calls share the one array and it keeps the last call's contents;
+ *    the call clears what must start at zero.  Calls that overlap on the GPU
+ *    race on the array: order them on one stream.
+ *  - Device-side range checks latch into the shared array, which has no
+ *    status read-back; use deltakv_decode_attention to diagnose. */
+deltakv_status deltakv_decode_attention_noalloc(deltakv_plan_t plan, int32_t T,
+                                                const void* q, const int64_t q_strides[2],
+                                                const void* cache,
+                                                const void* W3, const float* b3,
+                                                const void* W4, const float* b4,
+                                                float* out, const int64_t out_strides[2],
+                                                deltakv_stream_t stream);
+
 /* Synchronise `stream`, read and clear the error word that the kernels latch
  * in `workspace`, and return DELTAKV_OK, DEVICE_TIMEOUT or DEVICE_BOUNDS. */
 deltakv_status deltakv_device_status(deltakv_plan_t plan, void* workspace,
