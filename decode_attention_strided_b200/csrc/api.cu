@@ -171,10 +171,11 @@ deltakv_status deltakv_compress(deltakv_plan_t plan, int32_t T, const void* K, c
   KVView kv{K, V, kv_strides[0], kv_strides[1], kv_strides[2]};
   cudaError_t e = launch_refpack(p, T, kv, cache, workspace, st);
   if (e == cudaSuccess) {
-    if (candidates_tc_supported(p))
-      e = launch_candidates_tc(p, T, kv, cache, workspace, st);
-    else
-      e = launch_candidates_simt(p, T, kv, cache, workspace, st);
+    // tensor-core search for bf16; CUDA cores for float32 caches and for K/V
+    // layouts a TMA descriptor cannot describe (reported before any launch)
+    cudaError_t t = cudaErrorNotSupported;
+    if (candidates_tc_supported(p)) t = launch_candidates_tc(p, T, kv, cache, workspace, st);
+    e = t == cudaErrorNotSupported ? launch_candidates_simt(p, T, kv, cache, workspace, st) : t;
   }
   if (e == cudaSuccess) e = launch_encode(p, T, kv, W1, b1, W2, b2, cache, workspace, st);
   return from_cuda(e);

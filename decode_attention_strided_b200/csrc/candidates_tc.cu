@@ -1,14 +1,442 @@
-// candidates_tc.cu -- tensor-core (tcgen05) nearest-reference search.
-#include "internal.h"
+// candidates_tc.cu -- nearest strided references on the 5th-generation
+// tensor cores (tcgen05 + TMEM + TMA), with a fused running top-k.
+//
+// DeltaKV summary, section 3, "Processo di Compressione" step 1: for every
+// non-reference token the k most similar earlier references by L2 distance
+// over [K ; V].  Ranking by |x_t - r_j|^2 equals ranking by
+//     e(t, j) = |r_j|^2 / 2 - <x_t, r_j>
+// (the token's own norm is common to the row), so the hot loop is the causal
+// contraction X[T x D] . R[n_ref x D]^T with a per-column bias.  It runs as
+// bf16 x bf16 -> fp32 MMAs; the epilogue keeps, per token, the KC = k + 4
+// smallest e in registers (ties to the lower slot).  The GEMM form loses
+// precision to cancellation when x_t is close to r_j, so the encode kernel
+// re-ranks these KC candidates with exact fp32 distances before choosing k.
+//
+// Work unit: two 128-token tiles of one (sequence, kv-head) -- M = 256 rows
+// share every reference tile that is staged in shared memory.
+// Warp roles (320 threads, one CTA per SM, persistent):
+//   warps 0-7  epilogue: warp w owns token tile w / 4, TMEM lanes 32 (w % 4)..
+//   warp 8     TMA producer: A tiles (tokens) and B stages (references)
+//   warp 9     MMA issuer: M=128, N=64, K=16 tcgen05.mma, fp32 in TMEM
+// TMEM: 512 columns = 4 buffers x 2 token tiles x 64 reference columns, so
+// the MMAs run up to three reference tiles ahead of the epilogue.
+// A and B live in shared memory in the 128-byte-swizzled K-major layout the
+// TMA writes; a 64-element column of a 128-row token tile is one 16 KB atom,
+// of a 64-row reference tile one 8 KB atom.
+//
+// Epilogue: each thread owns one token row, so a warp carries 32 unrelated
+// running top-k lists.  Per 32 columns it builds a bitmask of the values below
+// its current k-th best; only if some lane has a candidate are the values
+// parked in the warp's shared-memory slot, and then every lane inserts its
+// own candidates in one short loop, so a warp pays for the busiest lane, not
+// for the sum over lanes.
+#include <cfloat>
+#include <climits>
+#include <mutex>
+
+#include "common.cuh"
+#include "sm100.cuh"
 
 namespace dkv {
+using namespace sm100;
 
-bool candidates_tc_supported(const Plan& p) { (void)p; return false; }
+namespace tcc {
+constexpr int TM = 128;                     // tokens per tile (MMA M)
+constexpr int TPU = 2;                      // token tiles per unit
+constexpr int RN = 64;                      // references per tile (MMA N)
+constexpr int NBUF = 4;                     // TMEM accumulator buffers
+constexpr int STAGES = 8;                   // reference pipeline depth (atoms)
+constexpr int ATOM = TM * 128;              // bytes: 128 token rows x 128 B
+constexpr int BATOM = RN * 128;             // bytes: 64 reference rows x 128 B
+constexpr int SPILL = 32 * 32 * 4;          // bytes per warp: 32 lanes x 32 floats
+constexpr int EPI_WARPS = 8;
+constexpr int THREADS = (EPI_WARPS + 2) * 32;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr int PRODUCER_WARP = EPI_WARPS;
+constexpr int MMA_WARP = EPI_WARPS + 1;
+}  // namespace tcc
 
-cudaError_t launch_candidates_tc(const Plan& p, int T, const KVView& kv, const void* cache,
-                                 void* ws, cudaStream_t st) {
-  (void)p; (void)T; (void)kv; (void)cache; (void)ws; (void)st;
-  return cudaErrorNotSupported;
+struct TcParams {
+  int T, s, H, BH, n_units, n_pairs;
+  int n_ref;
+  int64_t n_ref_cap, n_code_cap;
+  const float* hnorm;
+  int32_t* cand;
+  uint32_t* err;
+};
+
+struct UnitInfo {
+  int p, bh, t0;
+  int R[tcc::TPU];
+  int Rmax;
+};
+
+// Static schedule: units sorted by decreasing cost (later token pairs see more
+// references), dealt to the persistent CTAs in a zig-zag.
+__device__ __forceinline__ bool unit_of(const TcParams& P, int round, UnitInfo& u) {
+  const int G = gridDim.x, c = blockIdx.x;
+  const int idx = round * G + ((round & 1) ? (G - 1 - c) : c);
+  if (idx >= P.n_units) return false;
+  u.p = P.n_pairs - 1 - idx / P.BH;
+  u.bh = idx % P.BH;
+  u.t0 = u.p * tcc::TM * tcc::TPU;
+  u.Rmax = 0;
+#pragma unroll
+  for (int i = 0; i < tcc::TPU; ++i) {
+    const int lo = u.t0 + i * tcc::TM;
+    const int hi = min(lo + tcc::TM, P.T) - 1;  // last token of the tile
+    int R = 0;
+    if (hi >= lo && hi >= 1) {
+      const int ns = min((hi + P.s - 1) / P.s, P.n_ref);  // slots seen by the tile's last token
+      R = (ns + tcc::RN - 1) / tcc::RN;
+    }
+    u.R[i] = R;
+    u.Rmax = max(u.Rmax, R);
+  }
+  return true;
+}
+
+template <int NKC, int KC>
+__global__ void __launch_bounds__(tcc::THREADS, 1)
+    cand_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
+                   const __grid_constant__ CUtensorMap mapRK, const __grid_constant__ CUtensorMap mapRV,
+                   const TcParams P) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  unsigned char* sA = smem;                                     // [TPU][NKC] atoms
+  unsigned char* sB = sA + tcc::TPU * NKC * tcc::ATOM;          // [STAGES] atoms
+  float* spill = (float*)(sB + tcc::STAGES * tcc::BATOM);       // [EPI_WARPS][32][32]
+  uint64_t* a_full = (uint64_t*)((unsigned char*)spill + tcc::EPI_WARPS * tcc::SPILL);  // [NKC]
+  uint64_t* a_empty = a_full + NKC;                             // [NKC]
+  uint64_t* b_full = a_empty + NKC;                             // [STAGES]
+  uint64_t* b_empty = b_full + tcc::STAGES;                     // [STAGES]
+  uint64_t* acc_full = b_empty + tcc::STAGES;                   // [NBUF]
+  uint64_t* acc_empty = acc_full + tcc::NBUF;                   // [NBUF]
+  uint32_t* tmem_slot = (uint32_t*)(acc_empty + tcc::NBUF);
+  volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int HALF = NKC / 2;  // atoms per d_h (K part, then V part)
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NKC; ++i) {
+      mbar_init(&a_full[i], 1);
+      mbar_init(&a_empty[i], 1);
+    }
+    for (int i = 0; i < tcc::STAGES; ++i) {
+      mbar_init(&b_full[i], 1);
+      mbar_init(&b_empty[i], 1);
+    }
+    for (int i = 0; i < tcc::NBUF; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], tcc::EPI_WARPS);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == tcc::PRODUCER_WARP && lane == 0) {
+    prefetch_tensormap(&mapK);
+    prefetch_tensormap(&mapV);
+    prefetch_tensormap(&mapRK);
+    prefetch_tensormap(&mapRV);
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, tcc::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == tcc::PRODUCER_WARP) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t a_it = 0, b_it = 0;
+      bool ok = true;
+      UnitInfo u;
+      for (int round = 0; ok && unit_of(P, round, u); ++round) {
+        if (u.Rmax == 0) continue;
+        const int h = u.bh % P.H, b = u.bh / P.H;
+        for (int kc = 0; kc < NKC && ok; ++kc) {
+          if (!mbar_wait(&a_empty[kc], (a_it & 1) ^ 1, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(&a_full[kc], tcc::TPU * tcc::ATOM);
+#pragma unroll
+          for (int i = 0; i < tcc::TPU; ++i) {
+            unsigned char* dst = sA + (i * NKC + kc) * tcc::ATOM;
+            const int y = u.t0 + i * tcc::TM;
+            if (kc < HALF)
+              tma_load_4d(&mapK, &a_full[kc], dst, kc * 64, y, h, b);
+            else
+              tma_load_4d(&mapV, &a_full[kc], dst, (kc - HALF) * 64, y, h, b);
+          }
+        }
+        ++a_it;
+        for (int r = 0; r < u.Rmax && ok; ++r) {
+          for (int kc = 0; kc < NKC; ++kc, ++b_it) {
+            const int st = b_it % tcc::STAGES;
+            const uint32_t ph = (b_it / tcc::STAGES) & 1;
+            if (!mbar_wait(&b_empty[st], ph ^ 1, abort_flag)) { ok = false; break; }
+            mbar_arrive_expect_tx(&b_full[st], tcc::BATOM);
+            unsigned char* dst = sB + st * tcc::BATOM;
+            if (kc < HALF)
+              tma_load_3d(&mapRK, &b_full[st], dst, kc * 64, r * tcc::RN, u.bh);
+            else
+              tma_load_3d(&mapRV, &b_full[st], dst, (kc - HALF) * 64, r * tcc::RN, u.bh);
+          }
+        }
+      }
+      if (!ok) {
+        latch_error(P.err, DELTAKV_ERR_DEVICE_TIMEOUT, 1);
+        *abort_flag = 1;
+      } else {
+        // let the last reference loads land before the block can finish
+        for (int i = 0; i < tcc::STAGES && b_it > (uint32_t)i; ++i) {
+          const uint32_t it = b_it - 1 - i;
+          mbar_wait(&b_full[it % tcc::STAGES], (it / tcc::STAGES) & 1, abort_flag);
+        }
+      }
+    }
+  } else if (warp == tcc::MMA_WARP) {
+    // ----------------------------------------------------------------- MMA
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(tcc::TM, tcc::RN);
+      const uint32_t a_base = smem_u32(sA), b_base = smem_u32(sB);
+      uint32_t a_it = 0, b_it = 0, acc_it = 0;
+      bool ok = true;
+      UnitInfo u;
+      for (int round = 0; ok && unit_of(P, round, u); ++round) {
+        if (u.Rmax == 0) continue;
+        for (int r = 0; r < u.Rmax && ok; ++r, ++acc_it) {
+          const uint32_t buf = acc_it % tcc::NBUF;
+          if (!mbar_wait(&acc_empty[buf], ((acc_it / tcc::NBUF) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          for (int kc = 0; kc < NKC; ++kc, ++b_it) {
+            const int st = b_it % tcc::STAGES;
+            if (!mbar_wait(&b_full[st], (b_it / tcc::STAGES) & 1, abort_flag)) { ok = false; break; }
+            if (r == 0 && !mbar_wait(&a_full[kc], a_it & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+#pragma unroll
+            for (int i = 0; i < tcc::TPU; ++i) {
+              if (r >= u.R[i]) continue;
+              const uint32_t d = tmem + buf * (tcc::TPU * tcc::RN) + i * tcc::RN;
+#pragma unroll
+              for (int k16 = 0; k16 < 4; ++k16) {
+                const uint64_t ad = desc_kmajor_sw128(a_base + (i * NKC + kc) * tcc::ATOM + k16 * 32);
+                const uint64_t bd = desc_kmajor_sw128(b_base + st * tcc::BATOM + k16 * 32);
+                umma_bf16(d, ad, bd, idesc, (kc | k16) != 0);
+              }
+            }
+            umma_commit(&b_empty[st]);
+            if (r == u.Rmax - 1) umma_commit(&a_empty[kc]);
+          }
+          if (ok) umma_commit(&acc_full[buf]);
+        }
+        ++a_it;
+      }
+      if (!ok) {
+        latch_error(P.err, DELTAKV_ERR_DEVICE_TIMEOUT, 2);
+        *abort_flag = 1;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int ti = warp / 4, q = warp % 4, row = q * 32 + lane;
+    float* sp = spill + warp * (32 * 32) + lane * 32;  // this lane's 32 floats
+    const int sw = lane & 7;                            // float4 swizzle of the slot
+    uint32_t acc_it = 0;
+    bool ok = true;
+    UnitInfo u;
+    for (int round = 0; ok && unit_of(P, round, u); ++round) {
+      if (u.Rmax == 0) continue;
+      const int t = u.t0 + ti * tcc::TM + row;
+      const int first = u.t0 + ti * tcc::TM;
+      const int cnt = t < P.T ? min((t + P.s - 1) / P.s, P.n_ref) : 0;  // valid slots j < cnt
+      const int cnt_lo = min((first + P.s - 1) / P.s, P.n_ref);         // smallest cnt in the tile
+      const float* hn = P.hnorm + (int64_t)u.bh * P.n_ref_cap;
+      float bd[KC];
+      int bi[KC];
+#pragma unroll
+      for (int x = 0; x < KC; ++x) { bd[x] = FLT_MAX; bi[x] = INT_MAX; }
+      for (int r = 0; r < u.Rmax; ++r, ++acc_it) {
+        const uint32_t buf = acc_it % tcc::NBUF;
+        const bool mine = r < u.R[ti];
+        const int jb = r * tcc::RN;
+        float v[tcc::RN];
+        if (!mbar_wait(&acc_full[buf], (acc_it / tcc::NBUF) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        if (mine)
+          tmem_ld64(tmem + ((uint32_t)(q * 32) << 16) + buf * (tcc::TPU * tcc::RN) + ti * tcc::RN, v);
+        // the accumulator is in registers: hand the buffer back to the MMA warp
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        if (!mine) continue;
+        const bool need_mask = jb + tcc::RN > cnt_lo;
+        // e = |r_j|^2 / 2 - <x_t, r_j>
+        const float4* h4 = reinterpret_cast<const float4*>(hn + jb);
+#pragma unroll
+        for (int x4 = 0; x4 < tcc::RN / 4; ++x4) {
+          const float4 t4 = __ldg(h4 + x4);
+          v[4 * x4] = t4.x - v[4 * x4];
+          v[4 * x4 + 1] = t4.y - v[4 * x4 + 1];
+          v[4 * x4 + 2] = t4.z - v[4 * x4 + 2];
+          v[4 * x4 + 3] = t4.w - v[4 * x4 + 3];
+        }
+        if (need_mask) {
+#pragma unroll
+          for (int x = 0; x < tcc::RN; ++x)
+            if (jb + x >= cnt) v[x] = FLT_MAX;
+        }
+#pragma unroll
+        for (int c = 0; c < tcc::RN / 32; ++c) {
+          const float thr = bd[KC - 1];
+          uint32_t m = 0;
+#pragma unroll
+          for (int x = 0; x < 32; ++x) m |= (v[c * 32 + x] < thr ? 1u : 0u) << x;
+          if (__any_sync(0xffffffffu, m != 0)) {
+            if (m) {
+#pragma unroll
+              for (int i4 = 0; i4 < 8; ++i4)
+                reinterpret_cast<float4*>(sp)[i4 ^ sw] =
+                    make_float4(v[c * 32 + 4 * i4], v[c * 32 + 4 * i4 + 1], v[c * 32 + 4 * i4 + 2],
+                                v[c * 32 + 4 * i4 + 3]);
+            }
+            __syncwarp();
+            while (m) {
+              const int x = __ffs(m) - 1;
+              m &= m - 1;
+              const float vx = sp[(((x >> 2) ^ sw) << 2) | (x & 3)];
+              if (vx < bd[KC - 1]) topk_insert<KC>(bd, bi, vx, jb + c * 32 + x);
+            }
+            __syncwarp();
+          }
+        }
+      }
+      if (ok && t < P.T && (t % P.s) != 0) {
+        int32_t* o = P.cand + ((int64_t)u.bh * P.n_code_cap + (t - t / P.s - 1)) * KC;
+#pragma unroll
+        for (int x = 0; x < KC; ++x) o[x] = bi[x] == INT_MAX ? -1 : bi[x];
+      }
+    }
+    if (!ok) {
+      latch_error(P.err, DELTAKV_ERR_DEVICE_TIMEOUT, 3);
+      *abort_flag = 1;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, tcc::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ host
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)p;
+  });
+  return fn;
+}
+
+// bf16 tensor map with a 64 x rows box in the 128-byte swizzle layout.
+bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
+              cuuint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint32_t box[5] = {64, box_rows, 1, 1, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  int dev = 0, n = kNumSMs;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : kNumSMs;
+}
+
+template <int NKC>
+size_t smem_bytes() {
+  return 1024 + (size_t)tcc::TPU * NKC * tcc::ATOM + (size_t)tcc::STAGES * tcc::BATOM +
+         (size_t)tcc::EPI_WARPS * tcc::SPILL + 512;
+}
+
+template <int NKC, int KC>
+cudaError_t launch_tc(const CUtensorMap& mK, const CUtensorMap& mV, const CUtensorMap& mRK,
+                      const CUtensorMap& mRV, const TcParams& P, int grid, cudaStream_t st) {
+  auto kern = cand_tc_kernel<NKC, KC>;
+  const size_t smem = smem_bytes<NKC>();
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, tcc::THREADS, smem, st>>>(mK, mV, mRK, mRV, P);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool candidates_tc_supported(const Plan& p) {
+  return p.cfg.dtype == DELTAKV_BF16 && (p.cfg.d_h == 64 || p.cfg.d_h == 128) && encode_fn() != nullptr;
+}
+
+cudaError_t launch_candidates_tc(const Plan& p, int T, const KVView& kv, const void* cache, void* ws,
+                                 cudaStream_t st) {
+  const auto& c = p.cfg;
+  const int64_t n_code = n_code_of(T, c.stride_s);
+  if (n_code == 0) return cudaSuccess;
+  const int n_ref = (int)n_ref_of(T, c.stride_s);
+  const int d_h = c.d_h;
+  CUtensorMap mK, mV, mRK, mRV;
+  {
+    cuuint64_t dims[4] = {(cuuint64_t)d_h, (cuuint64_t)T, (cuuint64_t)c.kv_heads, (cuuint64_t)c.batch};
+    cuuint64_t str[3] = {(cuuint64_t)kv.st * 2, (cuuint64_t)kv.sh * 2, (cuuint64_t)kv.sb * 2};
+    if (!make_map(&mK, kv.K, 4, dims, str, tcc::TM) || !make_map(&mV, kv.V, 4, dims, str, tcc::TM))
+      return cudaErrorNotSupported;  // nothing launched; the caller uses the CUDA-core kernel
+  }
+  {
+    const char* cb = (const char*)cache;
+    cuuint64_t dims[3] = {(cuuint64_t)d_h, (cuuint64_t)n_ref, (cuuint64_t)c.batch * c.kv_heads};
+    cuuint64_t str[2] = {(cuuint64_t)d_h * 2, (cuuint64_t)p.n_ref_cap * d_h * 2};
+    if (!make_map(&mRK, cb + p.off_refk, 3, dims, str, tcc::RN) ||
+        !make_map(&mRV, cb + p.off_refv, 3, dims, str, tcc::RN))
+      return cudaErrorNotSupported;
+  }
+  TcParams P;
+  P.T = T;
+  P.s = c.stride_s;
+  P.H = c.kv_heads;
+  P.BH = c.batch * c.kv_heads;
+  P.n_pairs = (int)ceil_div64(T, tcc::TM * tcc::TPU);
+  P.n_units = P.n_pairs * P.BH;
+  P.n_ref = n_ref;
+  P.n_ref_cap = p.n_ref_cap;
+  P.n_code_cap = p.n_code_cap;
+  P.hnorm = (const float*)((const char*)ws + p.ws_hnorm);
+  P.cand = (int32_t*)((char*)ws + p.ws_cand);
+  P.err = (uint32_t*)ws;
+  const int grid = std::min(P.n_units, sm_count());
+  ProfScope ps(p, st, KID_CAND_TC);
+  if (d_h == 128)
+    return p.KC == 8 ? launch_tc<4, 8>(mK, mV, mRK, mRV, P, grid, st)
+                     : launch_tc<4, 12>(mK, mV, mRK, mRV, P, grid, st);
+  return p.KC == 8 ? launch_tc<2, 8>(mK, mV, mRK, mRV, P, grid, st)
+                   : launch_tc<2, 12>(mK, mV, mRK, mRV, P, grid, st);
 }
 
 }  // namespace dkv
