@@ -74,7 +74,7 @@ void build_plan(const deltakv_config& c, Plan& p) {
   w = align256(w + (size_t)(BH * p.n_code_cap * p.KC) * 4);
   const size_t compress_end = w;
   w = kErrBytes;
-  p.ns_max = kMaxSplit;
+  p.nslot_cap = (int)std::max<int64_t>(kMaxSplit, ceil_div64(kNumSMs, BH) + 1);
   const int64_t n_refblk_cap = ceil_div64(p.n_ref_cap, 64);
   p.n_chunk_cap = (int)ceil_div64(p.n_ref_cap, kCombineSlots);
   p.ws_S = w;
@@ -86,11 +86,11 @@ void build_plan(const deltakv_config& c, Plan& p) {
   p.ws_cterm = w;
   w = align256(w + (size_t)(BH * p.G) * 4);
   p.ws_wtab = w;
-  w = align256(w + (size_t)(BH * p.ns_max * p.n_ref_cap * p.G) * 4);
+  w = align256(w + (size_t)(BH * p.n_ref_cap * p.G) * 4);
   p.ws_part = w;
-  w = align256(w + (size_t)(BH * p.ns_max * p.G * 2) * 4);
+  w = align256(w + (size_t)(BH * p.nslot_cap * p.G * 2) * 4);
   p.ws_U = w;
-  w = align256(w + (size_t)(BH * p.ns_max * p.G * c.hidden) * 4);
+  w = align256(w + (size_t)(BH * p.nslot_cap * p.G * c.hidden) * 4);
   p.ws_ochunk = w;
   w = align256(w + (size_t)(BH * p.n_chunk_cap * p.G * (c.d_h + 1)) * 4);
   p.ws_bytes = std::max(compress_end, w);
@@ -177,7 +177,9 @@ deltakv_status deltakv_compress(deltakv_plan_t plan, int32_t T, const void* K, c
     if (candidates_tc_supported(p)) t = launch_candidates_tc(p, T, kv, cache, workspace, st);
     e = t == cudaErrorNotSupported ? launch_candidates_simt(p, T, kv, cache, workspace, st) : t;
   }
-  if (e == cudaSuccess) e = launch_encode(p, T, kv, W1, b1, W2, b2, cache, workspace, st);
+  if (e == cudaSuccess)
+    e = encode_tc_supported(p) ? launch_encode_tc(p, T, kv, W1, b1, W2, b2, cache, workspace, st)
+                               : launch_encode(p, T, kv, W1, b1, W2, b2, cache, workspace, st);
   return from_cuda(e);
 }
 

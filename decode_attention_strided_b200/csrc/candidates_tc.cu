@@ -224,7 +224,7 @@ __global__ void __launch_bounds__(tcc::THREADS, 1)
               for (int k16 = 0; k16 < 4; ++k16) {
                 const uint64_t ad = desc_kmajor_sw128(a_base + (i * NKC + kc) * tcc::ATOM + k16 * 32);
                 const uint64_t bd = desc_kmajor_sw128(b_base + st * tcc::BATOM + k16 * 32);
-                umma_bf16(d, ad, bd, idesc, (kc | k16) != 0);
+                umma_f16(d, ad, bd, idesc, (kc | k16) != 0);
               }
             }
             umma_commit(&b_empty[st]);

@@ -37,7 +37,7 @@ __global__ void __launch_bounds__(256)
     decode_ref_kernel(int64_t n_ref, int64_t n_ref_cap, int d_h, int H, int G, float c,
                       const T* __restrict__ q, int64_t qsb, int64_t qsh,
                       const T* __restrict__ refk, float* __restrict__ S,
-                      float* __restrict__ Smax, int n_refblk_cap) {
+                      float* __restrict__ Smax, int n_refblk_cap, float* __restrict__ wtab) {
   __shared__ float qs[kMaxG][128];
   __shared__ float wmax[8][kMaxG];
   const int b = blockIdx.z, h = blockIdx.y;
@@ -72,7 +72,10 @@ __global__ void __launch_bounds__(256)
         }
         acc = warp_sum(acc);
         mx[g] = fmaxf(mx[g], acc);
-        if (lane == 0) S[(bh * n_ref_cap + j) * G + g] = acc;
+        if (lane == 0) {
+          S[(bh * n_ref_cap + j) * G + g] = acc;
+          wtab[(bh * n_ref_cap + j) * G + g] = 0.f;
+        }
       }
     }
   }
@@ -142,7 +145,7 @@ __global__ void __launch_bounds__(256)
                          const float* __restrict__ cterm, const float* __restrict__ S,
                          const float* __restrict__ Smax, float* __restrict__ wtab_g,
                          float* __restrict__ part, float* __restrict__ Upart, int wt_in_smem,
-                         uint32_t* __restrict__ err) {
+                         int nslot_cap, uint32_t* __restrict__ err) {
   extern __shared__ float smem[];
   float* W3s = smem;                         // [d_c][hidden]
   float* As = W3s + d_c * hidden;            // [G][hidden]
@@ -156,7 +159,9 @@ __global__ void __launch_bounds__(256)
   const int64_t n_ref = (T_ + s - 1) / s;
   const int64_t n_code = T_ - n_ref;
   const int64_t c0 = n_code * split / ns, c1 = n_code * (split + 1) / ns;
-  float* wtab = wt_in_smem ? wt : wtab_g + ((bh * ns) + split) * n_ref_cap * G;
+  // the kv-head's slot-weight table (zeroed by decode_ref), relative to
+  // m_ref; with room in shared memory the block sums into a private copy first
+  float* wtab = wt_in_smem ? wt : wtab_g + bh * n_ref_cap * G;
 
   for (int i = tid; i < d_c * hidden; i += blockDim.x) {
     int n = i / d_c, e = i - n * d_c;
@@ -166,7 +171,8 @@ __global__ void __launch_bounds__(256)
     As[i] = a[bh * G * hidden + i];
     Ured[i] = 0.f;
   }
-  for (int64_t i = tid; i < n_ref * G; i += blockDim.x) wtab[i] = 0.f;
+  if (wt_in_smem)
+    for (int64_t i = tid; i < n_ref * G; i += blockDim.x) wtab[i] = 0.f;
   if (tid < G) {
     float m = -INFINITY;
     for (int r = 0; r < n_refblk; ++r) m = fmaxf(m, Smax[(bh * n_refblk_cap + r) * G + tid]);
@@ -273,16 +279,32 @@ __global__ void __launch_bounds__(256)
     }
   }
   __syncthreads();
-  const int64_t pb = bh * ns + split;
+  const int64_t pb = bh * nslot_cap + split;
   if (tid < G) {
     part[(pb * G + tid) * 2 + 0] = mb[tid];
     part[(pb * G + tid) * 2 + 1] = misc[2 * kMaxG + tid];
   }
   for (int i = tid; i < G * hidden; i += blockDim.x) Upart[pb * G * hidden + i] = Ured[i];
   if (wt_in_smem) {
-    float* dst = wtab_g + pb * n_ref_cap * G;
-    for (int64_t i = tid; i < n_ref * G; i += blockDim.x) dst[i] = wt[i];
+    float* dst = wtab_g + bh * n_ref_cap * G;
+    for (int64_t i = tid; i < n_ref * G; i += blockDim.x)
+      if (wt[i] != 0.f) atomicAdd(dst + i, wt[i]);
   }
+}
+
+// Partial (m, l, U) slots per kv-head: a fixed count for the CUDA-core
+// stream kernel, the CTAs of the even chunk split for the tensor-core one.
+struct SlotInfo {
+  int tc, ns, n_ch, grid, nslot_cap;
+  int64_t N;
+};
+
+__device__ __forceinline__ int slots_of(const SlotInfo& si, int64_t bh) {
+  if (!si.tc) return si.ns;
+  if (si.n_ch == 0) return 0;
+  const int64_t first = (bh * si.n_ch * si.grid) / si.N;
+  const int64_t last = (((bh + 1) * si.n_ch - 1) * si.grid) / si.N;
+  return (int)(last - first + 1);
 }
 
 // -------------------------------------------------------- decode_combine
@@ -290,7 +312,7 @@ __global__ void __launch_bounds__(256)
 // w_j = 2^(S_j - M) + 2^(m_ref - M) sum_splits wtab, then sum_j w_j V_ref_j.
 template <typename T>
 __global__ void __launch_bounds__(256)
-    decode_combine_kernel(int T_, int s, int d_h, int H, int G, int ns, int64_t n_ref_cap,
+    decode_combine_kernel(int T_, int s, int d_h, int H, int G, SlotInfo si, int64_t n_ref_cap,
                           int n_refblk, int n_refblk_cap, int n_chunk_cap,
                           const T* __restrict__ refv, const float* __restrict__ S,
                           const float* __restrict__ Smax, const float* __restrict__ wtab_g,
@@ -306,7 +328,8 @@ __global__ void __launch_bounds__(256)
     for (int r = 0; r < n_refblk; ++r) m = fmaxf(m, Smax[(bh * n_refblk_cap + r) * G + tid]);
     mrefg[tid] = m;
     float M = m;
-    for (int sp = 0; sp < ns; ++sp) M = fmaxf(M, part[((bh * ns + sp) * G + tid) * 2]);
+    const int ns = slots_of(si, bh);
+    for (int sp = 0; sp < ns; ++sp) M = fmaxf(M, part[((bh * si.nslot_cap + sp) * G + tid) * 2]);
     Mg[tid] = M;
     lref[tid] = 0.f;
   }
@@ -317,9 +340,7 @@ __global__ void __launch_bounds__(256)
     float w = 0.f;
     if (j < n_ref) {
       float own = exp2f(S[(bh * n_ref_cap + j) * G + g] - Mg[g]);
-      float acc = 0.f;
-      for (int sp = 0; sp < ns; ++sp) acc += wtab_g[((bh * ns + sp) * n_ref_cap + j) * G + g];
-      w = own + acc * exp2f(mrefg[g] - Mg[g]);
+      w = own + wtab_g[(bh * n_ref_cap + j) * G + g] * exp2f(mrefg[g] - Mg[g]);
       atomicAdd(&lref[g], own);
     }
     wts[jj][g] = w;
@@ -342,7 +363,7 @@ __global__ void __launch_bounds__(256)
 // ---------------------------------------------------------- decode_final
 template <typename T>
 __global__ void __launch_bounds__(256)
-    decode_final_kernel(int T_, int s, int d_h, int H, int G, int hidden, int ns, int n_chunk,
+    decode_final_kernel(int T_, int s, int d_h, int H, int G, int hidden, SlotInfo si, int n_chunk,
                         int n_chunk_cap, int n_refblk, int n_refblk_cap,
                         const T* __restrict__ W4, const float* __restrict__ b4,
                         const float* __restrict__ Smax, const float* __restrict__ part,
@@ -352,14 +373,16 @@ __global__ void __launch_bounds__(256)
   __shared__ float Mg[kMaxG], Lnr[kMaxG], Lall[kMaxG];
   const int b = blockIdx.z, h = blockIdx.y, tid = threadIdx.x;
   const int64_t bh = (int64_t)b * H + h;
+  const int ns = slots_of(si, bh);
+  const int64_t pb0 = bh * si.nslot_cap;
   if (tid < G) {
     float M = -INFINITY;
     for (int r = 0; r < n_refblk; ++r) M = fmaxf(M, Smax[(bh * n_refblk_cap + r) * G + tid]);
-    for (int sp = 0; sp < ns; ++sp) M = fmaxf(M, part[((bh * ns + sp) * G + tid) * 2]);
+    for (int sp = 0; sp < ns; ++sp) M = fmaxf(M, part[((pb0 + sp) * G + tid) * 2]);
     float lnr = 0.f;
     for (int sp = 0; sp < ns; ++sp) {
-      float m = part[((bh * ns + sp) * G + tid) * 2];
-      float l = part[((bh * ns + sp) * G + tid) * 2 + 1];
+      float m = part[((pb0 + sp) * G + tid) * 2];
+      float l = part[((pb0 + sp) * G + tid) * 2 + 1];
       if (m != -INFINITY) lnr += l * exp2f(m - M);
     }
     float lr = 0.f;
@@ -373,8 +396,8 @@ __global__ void __launch_bounds__(256)
     int g = i / hidden, n = i - g * hidden;
     float acc = 0.f;
     for (int sp = 0; sp < ns; ++sp) {
-      float m = part[((bh * ns + sp) * G + g) * 2];
-      if (m != -INFINITY) acc += Upart[((bh * ns + sp) * G + g) * hidden + n] * exp2f(m - Mg[g]);
+      float m = part[((pb0 + sp) * G + g) * 2];
+      if (m != -INFINITY) acc += Upart[((pb0 + sp) * G + g) * hidden + n] * exp2f(m - Mg[g]);
     }
     Ut[g][n] = acc;
   }
@@ -423,41 +446,57 @@ static cudaError_t decode_launch(const Plan& p, int T, const void* q, int64_t qs
   {
     ProfScope ps(p, st, KID_DEC_REF);
     decode_ref_kernel<E><<<dim3(n_refblk, H, B), 256, 0, st>>>(
-      n_ref, p.n_ref_cap, c.d_h, H, G, cs, (const E*)q, qsb, qsh, refk, S, Smax, n_refblk_cap);
+        n_ref, p.n_ref_cap, c.d_h, H, G, cs, (const E*)q, qsb, qsh, refk, S, Smax, n_refblk_cap, wtab);
   }
   {
     ProfScope ps(p, st, KID_DEC_PREP);
     decode_prep_kernel<E><<<dim3(1, H, B), 256, 0, st>>>(c.d_h, H, G, c.hidden, cs, (const E*)q, qsb,
-                                                       qsh, (const E*)W4, b4, a, cterm);
+                                                         qsh, (const E*)W4, b4, a, cterm);
   }
-  // splits: enough blocks for about two waves, never more rows than splits
-  int ns = (int)ceil_div64(2 * kNumSMs, (int64_t)B * H);
-  ns = (int)std::min<int64_t>(std::min<int64_t>(ns, p.ns_max), std::max<int64_t>(1, n_code / 64));
-  size_t base = sizeof(float) * (size_t)(c.d_c * c.hidden + 2 * G * c.hidden + 4 * kMaxG + 8 * c.d_c);
-  size_t wt_bytes = sizeof(float) * (size_t)(n_ref * G);
-  int wt_in_smem = base + wt_bytes <= 200 * 1024;
-  size_t smem = base + (wt_in_smem ? wt_bytes : 0);
-  auto ks = decode_stream_kernel<E>;
-  cudaError_t e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  SlotInfo si{};
+  si.nslot_cap = p.nslot_cap;
+  cudaError_t e = cudaErrorNotSupported;
+  if (decode_tc_supported(p)) {
+    e = launch_decode_tc(p, T, cache, W3, b3, ws, st);
+    if (e == cudaSuccess) {
+      si.tc = 1;
+      si.n_ch = (int)ceil_div64(n_code, 128);
+      si.N = (int64_t)si.n_ch * B * H;
+      si.grid = decode_tc_grid(p, si.N);
+    }
+  }
+  if (e == cudaErrorNotSupported) {
+    // splits: enough blocks for about two waves, never more rows than splits
+    int ns = (int)ceil_div64(2 * kNumSMs, (int64_t)B * H);
+    ns = (int)std::min<int64_t>(std::min<int64_t>(ns, p.nslot_cap), std::max<int64_t>(1, n_code / 64));
+    size_t base = sizeof(float) * (size_t)(c.d_c * c.hidden + 2 * G * c.hidden + 4 * kMaxG + 8 * c.d_c);
+    size_t wt_bytes = sizeof(float) * (size_t)(n_ref * G);
+    int wt_in_smem = base + wt_bytes <= 200 * 1024;
+    size_t smem = base + (wt_in_smem ? wt_bytes : 0);
+    auto ks = decode_stream_kernel<E>;
+    e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    ProfScope ps(p, st, KID_DEC_STREAM);
+    ks<<<dim3(ns, H, B), 256, smem, st>>>(T, c.stride_s, c.d_h, H, G, c.k, c.d_c, c.hidden, (int)c.act, ns,
+                                          p.n_ref_cap, p.n_code_cap, n_refblk, n_refblk_cap, code, idx,
+                                          (const E*)W3, b3, a, cterm, S, Smax, wtab, part, Upart,
+                                          wt_in_smem, p.nslot_cap, (uint32_t*)ws);
+    e = cudaGetLastError();
+    si.tc = 0;
+    si.ns = ns;
+  }
   if (e != cudaSuccess) return e;
-  {
-  ProfScope ps(p, st, KID_DEC_STREAM);
-  ks<<<dim3(ns, H, B), 256, smem, st>>>(T, c.stride_s, c.d_h, H, G, c.k, c.d_c, c.hidden,
-                                        (int)c.act, ns, p.n_ref_cap, p.n_code_cap, n_refblk,
-                                        n_refblk_cap, code, idx, (const E*)W3, b3, a, cterm, S,
-                                        Smax, wtab, part, Upart, wt_in_smem, (uint32_t*)ws);
-  }
   {
     ProfScope ps(p, st, KID_DEC_COMBINE);
     decode_combine_kernel<E><<<dim3(n_chunk, H, B), 256, 0, st>>>(
-      T, c.stride_s, c.d_h, H, G, ns, p.n_ref_cap, n_refblk, n_refblk_cap, p.n_chunk_cap, refv, S,
-      Smax, wtab, part, ochunk);
+        T, c.stride_s, c.d_h, H, G, si, p.n_ref_cap, n_refblk, n_refblk_cap, p.n_chunk_cap, refv, S,
+        Smax, wtab, part, ochunk);
   }
   {
     ProfScope ps(p, st, KID_DEC_FINAL);
     decode_final_kernel<E><<<dim3(1, H, B), 256, 0, st>>>(
-      T, c.stride_s, c.d_h, H, G, c.hidden, ns, n_chunk, p.n_chunk_cap, n_refblk, n_refblk_cap,
-      (const E*)W4, b4, Smax, part, Upart, ochunk, out, osb, osh);
+        T, c.stride_s, c.d_h, H, G, c.hidden, si, n_chunk, p.n_chunk_cap, n_refblk, n_refblk_cap,
+        (const E*)W4, b4, Smax, part, Upart, ochunk, out, osb, osh);
   }
   return cudaGetLastError();
 }

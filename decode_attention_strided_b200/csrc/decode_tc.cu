@@ -1,0 +1,661 @@
+// decode_tc.cu -- the token loop of decode attention over the compressed cache
+// on the 5th-generation tensor cores (bf16 caches).
+//
+// DeltaKV summary, section 3 "Ricostruzione" and section 4 (reconstruction
+// on demand inside the attention that reads the cache).  For query head g of
+// kv-head h and compressed token t (logits in log2 units, c = log2 e/sqrt d_h):
+//   u_t  = act(W3 code_t + b3)                       GEMM1 + act, per token
+//   l_tg = a_g . u_t + c q_g.b4_K + mean_i S[idx_ti][g]
+//          (a_g = c W4_K^T q_g,  S[j][g] = c q_g . K_ref_j)
+//   p_tg = 2^(l_tg - m)   with m a running maximum
+//   U_g += sum_t p_tg u_t         (W4_V U_g is applied once per kv-head later)
+//   w[j][g] += p_tg / k_eff for j in idx_t   (V_ref side, per-slot weights)
+// so no token's K or V is ever materialised.  Per 128-token chunk:
+//   producer warp  TMA: the chunk's codes (zero-filled past the last row)
+//                  and slots into a 2-stage ring
+//   MMA warp       D1 = codes . W3^T  (M=128, N=hidden, K=d_c; bf16, exact
+//                  products), z = u . [a_hi; a_lo]^T (M=128, N=16, K=hidden),
+//                  U_chunk = u^T . P  (M=128 hidden units, N=16, K=128 tokens;
+//                  the u tile read through an MN-major descriptor)
+//   epilogue       8 warps: act(D1 + b3) -> fp16 u tile (double-buffered);
+//                  warps 2-5 also do the softmax step (S gathers, per-chunk
+//                  maximum, P tile, slot-weight reductions into the global
+//                  table); both groups fold U_chunk into register
+//                  accumulators with the online-softmax rescale.
+// A persistent grid splits the flattened (kv-head, chunk) list evenly; each
+// CTA writes one partial (m, l, U) per kv-head segment it touches.
+#include <cfloat>
+#include <climits>
+#include <mutex>
+
+#include <cuda_fp16.h>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace dkv {
+using namespace sm100;
+
+namespace dtc {
+constexpr int CH = 128;                 // tokens per chunk (MMA M)
+constexpr int EPI = 8;                  // epilogue warps: group A = 2..5, B = 6..9
+constexpr int THREADS = (EPI + 2) * 32;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t COL_D1 = 0, COL_Z = 256, COL_U = 288;
+constexpr int PRODUCER = 0, MMA = 1;
+}  // namespace dtc
+
+// Even split of N chunks over `grid` CTAs: CTA c owns chunks x with
+// floor(x grid / N) == c.
+__host__ __device__ inline int64_t dtc_begin(int64_t c, int64_t N, int grid) {
+  return (c * N + grid - 1) / grid;
+}
+__host__ __device__ inline int64_t dtc_owner(int64_t x, int64_t N, int grid) { return (x * grid) / N; }
+
+struct DecTcParams {
+  int s, d_h, G, k, d_c, hidden, act, H, BH;
+  int64_t n_code, n_ref, n_ref_cap, n_code_cap;
+  int n_ch;
+  int64_t N;
+  int grid, nslot_cap, n_refblk, n_refblk_cap;
+  int code_swz;        // 32, 64 or 128: bytes per swizzled row of the code tile
+  int code_atoms;      // 64-column atoms of the code tile (2 when d_c = 128)
+  const int32_t* idx;
+  const __nv_bfloat16* W3;
+  const float* b3;
+  const float* a;
+  const float* cterm;
+  const float* S;
+  const float* Smax;
+  float* wtab;
+  float* part;
+  float* Upart;
+  uint32_t* err;
+};
+
+// K-major smem descriptor for 32-, 64- or 128-byte swizzled rows.
+__device__ __forceinline__ uint64_t desc_kmajor(uint32_t saddr, int swz) {
+  const uint64_t type = swz == 128 ? 2 : (swz == 64 ? 4 : 6);
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFF);
+  d |= (uint64_t)1 << 16;
+  d |= (uint64_t)((8 * swz) >> 4) << 32;  // 8-row groups
+  d |= (uint64_t)1 << 46;
+  d |= type << 61;
+  return d;
+}
+
+// MN-major, 128-byte swizzle: 64 contiguous M-elements per 128-byte row,
+// K rows 128 bytes apart (8-row groups `sbo` apart), M blocks `lbo` apart.
+__device__ __forceinline__ uint64_t desc_mnmajor_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFF);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+// kind::f16 instruction descriptors.
+__host__ __device__ constexpr uint32_t idesc_kind_f16(bool bf16, int M, int N, bool a_mn) {
+  return (1u << 4) | (bf16 ? (1u << 7) | (1u << 10) : 0u) | (a_mn ? (1u << 15) : 0u) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Byte offset of byte `bo` of row `row` in a K-major tile with `swz`-byte rows.
+__device__ __forceinline__ uint32_t swz_off(int row, int bo, int swz) {
+  const int mask = swz / 16 - 1;
+  const int chunk = (bo >> 4) ^ (((row * swz) >> 7) & mask);
+  return (uint32_t)(row * swz + (chunk << 4) + (bo & 15));
+}
+
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void named_bar(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16f(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                 "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]),
+                 "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+               :
+               : "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__host__ __device__ inline size_t dtc_align(size_t x) { return (x + 1023) & ~size_t(1023); }
+
+// Offsets of the shared-memory regions (from a 1024-aligned base).
+struct DecLayout {
+  size_t code, idx, w3, az, u, p, fl, bar, total;
+  __host__ __device__ DecLayout(int d_c, int k, int hidden) {
+    const size_t code_b = (size_t)dtc::CH * d_c * 2, idx_b = (size_t)dtc::CH * k * 4;
+    const size_t w3_b = (size_t)hidden * d_c * 2, az_b = (size_t)(hidden / 64) * 16 * 128;
+    const size_t u_b = (size_t)(hidden / 64) * dtc::CH * 128, p_b = 2 * 16 * 128;
+    size_t o = 0;
+    code = o; o = dtc_align(o + 2 * dtc_align(code_b));
+    idx = o;  o = dtc_align(o + 2 * dtc_align(idx_b));
+    w3 = o;   o = dtc_align(o + w3_b);
+    az = o;   o = dtc_align(o + 2 * dtc_align(az_b));
+    u = o;    o = dtc_align(o + 2 * u_b);
+    p = o;    o = dtc_align(o + p_b);
+    fl = o;   o += 256 * sizeof(float);
+    bar = o;  o += 32 * 8 + 16;
+    total = o;
+  }
+};
+
+__global__ void __launch_bounds__(dtc::THREADS, 1)
+    decode_tc_kernel(const __grid_constant__ CUtensorMap mapC, const DecTcParams P) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* base = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const DecLayout L(P.d_c, P.k, P.hidden);
+  const size_t code_b = dtc_align((size_t)dtc::CH * P.d_c * 2), idx_b = dtc_align((size_t)dtc::CH * P.k * 4);
+  const size_t az_b = dtc_align((size_t)(P.hidden / 64) * 16 * 128), u_b = (size_t)(P.hidden / 64) * dtc::CH * 128;
+  auto sCode = [&](int i) { return base + L.code + i * code_b; };
+  auto sIdx = [&](int i) { return (int32_t*)(base + L.idx + i * idx_b); };
+  unsigned char* sW3 = base + L.w3;
+  auto sAz = [&](int i) { return base + L.az + i * az_b; };
+  auto sU = [&](int i) { return base + L.u + i * u_b; };
+  unsigned char* sP = base + L.p;
+  float* fl = (float*)(base + L.fl);
+  float* m_run = fl;         // [8]
+  float* l_run = fl + 8;     // [8]
+  float* alpha = fl + 16;    // [8]
+  float* m_ref = fl + 24;    // [8]
+  float* ctv = fl + 32;      // [8]
+  float* mred = fl + 40;     // [4][8]
+  float* lred = fl + 72;     // [4][8]
+  uint64_t* bar = (uint64_t*)(base + L.bar);
+  uint64_t* in_full = bar + 0;    // [2]
+  uint64_t* in_empty = bar + 2;   // [2]
+  uint64_t* d1_full = bar + 4;
+  uint64_t* u_full = bar + 5;     // [2]
+  uint64_t* u_empty = bar + 7;    // [2]
+  uint64_t* z_full = bar + 9;
+  uint64_t* z_empty = bar + 10;
+  uint64_t* p_full = bar + 11;
+  uint64_t* p_empty = bar + 12;
+  uint64_t* ua_full = bar + 13;
+  uint64_t* ua_empty = bar + 14;
+  uint32_t* tmem_slot = (uint32_t*)(bar + 16);
+  volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
+  const int G = P.G, hidden = P.hidden, half = hidden / 2;
+  const int64_t x_begin = dtc_begin(blockIdx.x, P.N, P.grid), x_end = dtc_begin(blockIdx.x + 1, P.N, P.grid);
+  const int n_local = (int)(x_end - x_begin);
+
+  // ---- one-time set-up: W3 (bf16, K-major, swizzled like the code tile),
+  // zero rows of the P and a tiles, barriers, TMEM
+  {
+    const int swz = P.code_swz;
+    const int row_elems = swz / 2;  // bf16 per swizzled row
+    for (int i = tid; i < hidden * P.d_c / 8; i += blockDim.x) {
+      const int n = i / (P.d_c / 8), c8 = (i % (P.d_c / 8)) * 8;  // hidden unit, code column
+      const uint4 v = *reinterpret_cast<const uint4*>(P.W3 + (int64_t)n * P.d_c + c8);
+      const int atom = c8 / row_elems, col = c8 % row_elems;
+      *reinterpret_cast<uint4*>(sW3 + (size_t)atom * hidden * swz + swz_off(n, col * 2, swz)) = v;
+    }
+    for (int i = tid; i < 2 * 16 * 128 / 4; i += blockDim.x) reinterpret_cast<uint32_t*>(sP)[i] = 0u;
+    for (int i = tid; i < 2 * (int)az_b / 4; i += blockDim.x) reinterpret_cast<uint32_t*>(sAz(0))[i] = 0u;
+  }
+  if (tid == 0) {
+    mbar_init(&in_full[0], 1);
+    mbar_init(&in_full[1], 1);
+    mbar_init(&in_empty[0], 2);
+    mbar_init(&in_empty[1], 2);
+    mbar_init(d1_full, 1);
+    mbar_init(&u_full[0], dtc::EPI);
+    mbar_init(&u_full[1], dtc::EPI);
+    mbar_init(&u_empty[0], 1);
+    mbar_init(&u_empty[1], 1);
+    mbar_init(z_full, 1);
+    mbar_init(z_empty, 4);
+    mbar_init(p_full, 1);
+    mbar_init(p_empty, 1);
+    mbar_init(ua_full, 1);
+    mbar_init(ua_empty, dtc::EPI);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == dtc::MMA) {
+    tmem_alloc(tmem_slot, dtc::TMEM_COLS);
+    tmem_relinquish();
+  }
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == dtc::PRODUCER) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && n_local > 0) {
+      const uint32_t code_bytes = (uint32_t)(dtc::CH * P.d_c * 2), idx_bytes = (uint32_t)(dtc::CH * P.k * 4);
+      bool ok = true;
+      for (int it = 0; it < n_local && ok; ++it) {
+        const int64_t x = x_begin + it;
+        const int bh = (int)(x / P.n_ch);
+        const int64_t row0 = (x % P.n_ch) * dtc::CH;
+        const int st = it & 1;
+        if (!mbar_wait(&in_empty[st], ((it >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+        mbar_arrive_expect_tx(&in_full[st], code_bytes + idx_bytes);
+        for (int a = 0; a < P.code_atoms; ++a)
+          tma_load_3d(&mapC, &in_full[st], sCode(st) + (size_t)a * dtc::CH * 128, a * 64, (int)row0, bh);
+        bulk_load(sIdx(st), P.idx + ((int64_t)bh * P.n_code_cap + row0) * P.k, idx_bytes, &in_full[st]);
+      }
+      if (!ok) {
+        latch_error(P.err, DELTAKV_ERR_DEVICE_TIMEOUT, 20);
+        *abort_flag = 1;
+      }
+    }
+  } else if (warp == dtc::MMA) {
+    // ----------------------------------------------------------------- MMA
+    if (lane == 0 && n_local > 0) {
+      const uint32_t id_g1 = idesc_kind_f16(true, dtc::CH, hidden, false);
+      const uint32_t id_z = idesc_kind_f16(false, dtc::CH, 16, false);
+      const uint32_t id_u = idesc_kind_f16(false, 128, 16, true);
+      const int swz = P.code_swz;
+      auto gemm1 = [&](int st) {
+        const uint32_t c0 = smem_u32(sCode(st)), w0 = smem_u32(sW3);
+        for (int k16 = 0; k16 < P.d_c / 16; ++k16) {
+          const int per_row = swz / 32;  // k16 steps per swizzled row
+          const int atom = k16 / per_row, off = (k16 % per_row) * 32;
+          umma_f16(tmem + dtc::COL_D1, desc_kmajor(c0 + atom * dtc::CH * swz + off, swz),
+                   desc_kmajor(w0 + atom * hidden * swz + off, swz), id_g1, k16 != 0);
+        }
+      };
+      bool ok = true;
+      int seg = -1, prev_bh = -1;
+      for (int it = 0; it < n_local && ok; ++it) {
+        const int64_t x = x_begin + it;
+        const int bh = (int)(x / P.n_ch);
+        if (bh != prev_bh) { ++seg; prev_bh = bh; }
+        const int ub = it & 1;
+        if (it == 0) {
+          if (!mbar_wait(&in_full[0], 0, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          gemm1(0);
+          umma_commit(d1_full);
+          umma_commit(&in_empty[0]);
+        }
+        // act(D1) of this chunk is in the u tile (and D1 is free again)
+        if (!mbar_wait(&u_full[ub], (it >> 1) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        if (it + 1 < n_local) {
+          const int st = (it + 1) & 1;
+          if (!mbar_wait(&in_full[st], ((it + 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          gemm1(st);
+          umma_commit(d1_full);
+          umma_commit(&in_empty[st]);
+        }
+        // z = u . [a_hi; a_lo]^T
+        if (!mbar_wait(z_empty, (it & 1) ^ 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        {
+          const uint32_t u0 = smem_u32(sU(ub)), a0 = smem_u32(sAz(seg & 1));
+          for (int k16 = 0; k16 < hidden / 16; ++k16) {
+            const int atom = k16 >> 2, off = (k16 & 3) * 32;
+            umma_f16(tmem + dtc::COL_Z, desc_kmajor(u0 + atom * dtc::CH * 128 + off, 128),
+                     desc_kmajor(a0 + atom * 16 * 128 + off, 128), id_z, k16 != 0);
+          }
+          umma_commit(z_full);
+        }
+        // U_chunk = u^T . P
+        if (!mbar_wait(p_full, it & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(ua_empty, (it & 1) ^ 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        {
+          const uint32_t u0 = smem_u32(sU(ub)), p0 = smem_u32(sP);
+          for (int h2 = 0; h2 < hidden / 128; ++h2)
+            for (int k16 = 0; k16 < dtc::CH / 16; ++k16) {
+              const uint64_t ad = desc_mnmajor_sw128(u0 + (2 * h2) * dtc::CH * 128 + k16 * 16 * 128,
+                                                     dtc::CH * 128, 1024);
+              const uint64_t bd = desc_kmajor(p0 + (k16 >> 2) * 16 * 128 + (k16 & 3) * 32, 128);
+              umma_f16(tmem + dtc::COL_U + 16 * h2, ad, bd, id_u, k16 != 0);
+            }
+          umma_commit(ua_full);
+          umma_commit(&u_empty[ub]);
+          umma_commit(p_empty);
+        }
+      }
+      if (!ok) {
+        latch_error(P.err, DELTAKV_ERR_DEVICE_TIMEOUT, 21);
+        *abort_flag = 1;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int ew = warp - 2;                  // 0..7
+    const bool groupA = ew < 4;
+    const int q = warp & 3;                   // TMEM lane quarter
+    const int n = q * 32 + lane;              // token row (D1, z) / unit in half (U)
+    const int hh = groupA ? 0 : 1;            // hidden half of this group
+    float Ureg[kMaxG];
+#pragma unroll
+    for (int g = 0; g < kMaxG; ++g) Ureg[g] = 0.f;
+    bool ok = true;
+    int prev_bh = -1, seg_count = 0;
+    for (int it = 0; it < n_local && ok; ++it) {
+      const int64_t x = x_begin + it;
+      const int bh = (int)(x / P.n_ch);
+      const int64_t row0 = (x % P.n_ch) * dtc::CH;
+      const int st = it & 1, ub = it & 1;
+      if (bh != prev_bh) {
+        // new kv-head segment: its a_hi / a_lo rows go to the a tile of this
+        // segment's parity (the z MMAs of segment - 2, the last users of that
+        // tile, completed before their softmax steps), state is reset
+        prev_bh = bh;
+        named_bar(2, dtc::EPI * 32);
+        unsigned char* az = sAz(seg_count & 1);
+        const float* ab = P.a + (int64_t)bh * G * hidden;
+        for (int i = tid - 64; i < G * hidden; i += dtc::EPI * 32) {
+          const int g = i / hidden, c = i % hidden;
+          const float v = ab[i];
+          const __half hi = __float2half_rn(v);
+          const __half lo = __float2half_rn(v - __half2float(hi));
+          const int atom = c >> 6, cc = c & 63;
+          *reinterpret_cast<__half*>(az + atom * 16 * 128 + swz_off(g, cc * 2, 128)) = hi;
+          *reinterpret_cast<__half*>(az + atom * 16 * 128 + swz_off(G + g, cc * 2, 128)) = lo;
+        }
+        if (tid - 64 < G) {
+          const int g = tid - 64;
+          float m = -INFINITY;
+          for (int r = 0; r < P.n_refblk; ++r) m = fmaxf(m, P.Smax[((int64_t)bh * P.n_refblk_cap + r) * G + g]);
+          m_ref[g] = m;
+          m_run[g] = m;
+          l_run[g] = 0.f;
+          ctv[g] = P.cterm[(int64_t)bh * G + g];
+        }
+#pragma unroll
+        for (int g = 0; g < kMaxG; ++g) Ureg[g] = 0.f;
+        fence_async_smem();
+        named_bar(2, dtc::EPI * 32);
+        ++seg_count;
+      }
+      // ------------------------------------------------------ act(D1 + b3)
+      if (!mbar_wait(d1_full, it & 1, abort_flag)) { ok = false; break; }
+      if (!mbar_wait(&u_empty[ub], ((it >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      {
+        unsigned char* ut = sU(ub);
+        for (int c0 = hh * half; c0 < (hh + 1) * half; c0 += 32) {
+          float v[32];
+          tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + dtc::COL_D1 + c0, v);
+          __align__(16) __half2 h2[16];
+#pragma unroll
+          for (int x2 = 0; x2 < 16; ++x2) {
+            const float a0 = act_eval(P.act, v[2 * x2] + (P.b3 ? P.b3[c0 + 2 * x2] : 0.f));
+            const float a1 = act_eval(P.act, v[2 * x2 + 1] + (P.b3 ? P.b3[c0 + 2 * x2 + 1] : 0.f));
+            h2[x2] = __floats2half2_rn(a0, a1);
+          }
+          const int atom = c0 >> 6, cc = c0 & 63;
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            *reinterpret_cast<uint4*>(ut + atom * dtc::CH * 128 + swz_off(n, (cc + 8 * v4) * 2, 128)) =
+                reinterpret_cast<const uint4*>(h2)[v4];
+        }
+      }
+      tc_fence_before();
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&u_full[ub]);
+
+      // ------------------------------------------------------------ softmax
+      if (groupA) {
+        if (!mbar_wait(z_full, it & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        float zz[16];
+        tmem_ld16f(tmem + ((uint32_t)(q * 32) << 16) + dtc::COL_Z, zz);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(z_empty);
+        const int64_t row = row0 + n;
+        const bool valid = row < P.n_code;
+        const int32_t* ir = sIdx(st) + n * P.k;
+        const float* Sb = P.S + (int64_t)bh * P.n_ref_cap * G;
+        float lg[kMaxG];
+        int k_eff = 0;
+#pragma unroll
+        for (int g = 0; g < kMaxG; ++g) lg[g] = 0.f;
+        if (valid) {
+          for (int i = 0; i < P.k; ++i) {
+            const int j = ir[i];
+            if (j < 0) continue;
+            if (j >= P.n_ref) {
+              latch_error(P.err, DELTAKV_ERR_DEVICE_BOUNDS, (uint32_t)j);
+              continue;
+            }
+            ++k_eff;
+            if (G == 4) {
+              const float4 s4 = *reinterpret_cast<const float4*>(Sb + (int64_t)j * 4);
+              lg[0] += s4.x; lg[1] += s4.y; lg[2] += s4.z; lg[3] += s4.w;
+            } else {
+#pragma unroll
+              for (int g = 0; g < kMaxG; ++g)
+                if (g < G) lg[g] += Sb[(int64_t)j * G + g];
+            }
+          }
+        }
+        const float inv_k = 1.0f / (float)max(k_eff, 1);
+        float mx[kMaxG];
+#pragma unroll
+        for (int g = 0; g < kMaxG; ++g) {
+          lg[g] = g < G ? zz[g] + zz[G + g] + ctv[g] + lg[g] * inv_k : 0.f;
+          mx[g] = valid && g < G ? lg[g] : -INFINITY;
+          mx[g] = warp_max(mx[g]);
+        }
+        if (lane == 0) {
+#pragma unroll
+          for (int g = 0; g < kMaxG; ++g)
+            if (g < G) mred[(ew & 3) * 8 + g] = mx[g];
+        }
+        named_bar(1, 128);
+        float mnew[kMaxG], p[kMaxG];
+#pragma unroll
+        for (int g = 0; g < kMaxG; ++g) {
+          if (g < G) {
+            float m = m_run[g];
+            for (int w = 0; w < 4; ++w) m = fmaxf(m, mred[w * 8 + g]);
+            mnew[g] = m;
+            p[g] = valid ? exp2f(lg[g] - m) : 0.f;
+          } else {
+            mnew[g] = 0.f;
+            p[g] = 0.f;
+          }
+        }
+        // P tile (B operand of the U MMA) once the previous U MMA is done
+        if (!mbar_wait(p_empty, (it & 1) ^ 1, abort_flag)) { ok = false; break; }
+        {
+          const int atom = n >> 6, cc = n & 63;
+#pragma unroll
+          for (int g = 0; g < kMaxG; ++g)
+            if (g < G)
+              *reinterpret_cast<__half*>(sP + atom * 16 * 128 + swz_off(g, cc * 2, 128)) = __float2half_rn(p[g]);
+        }
+        // slot weights relative to m_ref, into the kv-head's global table
+        if (valid && k_eff > 0) {
+          float* wt = P.wtab + (int64_t)bh * P.n_ref_cap * G;
+          float sc[kMaxG];
+#pragma unroll
+          for (int g = 0; g < kMaxG; ++g) sc[g] = g < G ? p[g] * exp2f(fminf(mnew[g] - m_ref[g], 100.f)) * inv_k : 0.f;
+          for (int i = 0; i < P.k; ++i) {
+            const int j = ir[i];
+            if (j < 0 || j >= P.n_ref) continue;
+            if (G == 4) {
+              asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(wt + (int64_t)j * 4),
+                           "f"(sc[0]), "f"(sc[1]), "f"(sc[2]), "f"(sc[3])
+                           : "memory");
+            } else {
+#pragma unroll
+              for (int g = 0; g < kMaxG; ++g)
+                if (g < G) atomicAdd(wt + (int64_t)j * G + g, sc[g]);
+            }
+          }
+        }
+        float ls[kMaxG];
+#pragma unroll
+        for (int g = 0; g < kMaxG; ++g) ls[g] = warp_sum(p[g]);
+        if (lane == 0) {
+#pragma unroll
+          for (int g = 0; g < kMaxG; ++g)
+            if (g < G) lred[(ew & 3) * 8 + g] = ls[g];
+        }
+        fence_async_smem();
+        named_bar(1, 128);
+        if (ew == 0 && lane < G) {
+          const int g = lane;
+          const float al = exp2f(m_run[g] - mnew[g]);
+          alpha[g] = al;
+          l_run[g] = l_run[g] * al + lred[g] + lred[8 + g] + lred[16 + g] + lred[24 + g];
+          m_run[g] = mnew[g];
+        }
+        named_bar(1, 128);
+        if (ew == 0 && lane == 0) {
+          mbar_arrive(p_full);
+          mbar_arrive(&in_empty[st]);
+        }
+      }
+      // --------------------------------------------- fold U_chunk into Ureg
+      if (!groupA && !mbar_wait(p_full, it & 1, abort_flag)) { ok = false; break; }
+      if (!mbar_wait(ua_full, it & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      if (hh < hidden / 128) {
+        float du[16];
+        tmem_ld16f(tmem + ((uint32_t)(q * 32) << 16) + dtc::COL_U + 16 * hh, du);
+#pragma unroll
+        for (int g = 0; g < kMaxG; ++g)
+          if (g < G) Ureg[g] = Ureg[g] * alpha[g] + du[g];
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ua_empty);
+
+      // ------------------------------------------------ segment end: flush
+      const bool seg_end = (it == n_local - 1) || ((x + 1) / P.n_ch != bh);
+      if (seg_end) {
+        // partial slot: this CTA's rank among the CTAs that cover the head
+        const int64_t pb = (int64_t)bh * P.nslot_cap + (int64_t)blockIdx.x - dtc_owner((int64_t)bh * P.n_ch, P.N, P.grid);
+        if (hh < hidden / 128) {
+          const int unit = 128 * hh + n;
+#pragma unroll
+          for (int g = 0; g < kMaxG; ++g)
+            if (g < G) P.Upart[(pb * G + g) * hidden + unit] = Ureg[g];
+        }
+        if (ew == 0 && lane < G) {
+          P.part[(pb * G + lane) * 2 + 0] = m_run[lane];
+          P.part[(pb * G + lane) * 2 + 1] = l_run[lane];
+        }
+      }
+    }
+    if (!ok) {
+      latch_error(P.err, DELTAKV_ERR_DEVICE_TIMEOUT, 22);
+      *abort_flag = 1;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == dtc::MMA) {
+    tc_fence_after();
+    tmem_dealloc(tmem, dtc::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ host
+namespace {
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_fn_dec() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)p;
+  });
+  return fn;
+}
+}  // namespace
+
+bool decode_tc_supported(const Plan& p) {
+  const auto& c = p.cfg;
+  if (c.dtype != DELTAKV_BF16 || !encode_fn_dec()) return false;
+  if (!(c.hidden == 128 || c.hidden == 256)) return false;
+  if (!(c.d_c == 16 || c.d_c == 32 || c.d_c == 64 || c.d_c == 128)) return false;
+  if (2 * p.G > 16) return false;
+  return DecLayout(c.d_c, c.k, c.hidden).total + 1024 <= 227 * 1024;
+}
+
+int decode_tc_grid(const Plan& p, int64_t N) {
+  (void)p;
+  return (int)std::min<int64_t>(N, kNumSMs);
+}
+
+cudaError_t launch_decode_tc(const Plan& p, int T, const void* cache, const void* W3, const float* b3,
+                             void* ws, cudaStream_t st) {
+  const auto& c = p.cfg;
+  const int64_t n_code = n_code_of(T, c.stride_s);
+  const int n_ch = (int)ceil_div64(n_code, dtc::CH);
+  const int BH = c.batch * c.kv_heads;
+  const int64_t N = (int64_t)n_ch * BH;
+  if (N == 0) return cudaSuccess;
+  const char* cb = (const char*)cache;
+  char* w = (char*)ws;
+  DecTcParams P;
+  P.s = c.stride_s; P.d_h = c.d_h; P.G = p.G; P.k = c.k; P.d_c = c.d_c; P.hidden = c.hidden;
+  P.act = (int)c.act; P.H = c.kv_heads; P.BH = BH;
+  P.n_code = n_code; P.n_ref = n_ref_of(T, c.stride_s); P.n_ref_cap = p.n_ref_cap; P.n_code_cap = p.n_code_cap;
+  P.n_ch = n_ch; P.N = N; P.grid = decode_tc_grid(p, N); P.nslot_cap = p.nslot_cap;
+  P.n_refblk = (int)ceil_div64(P.n_ref, 64);
+  P.n_refblk_cap = (int)ceil_div64(p.n_ref_cap, 64);
+  P.code_swz = c.d_c >= 64 ? 128 : c.d_c * 2;
+  P.code_atoms = c.d_c > 64 ? c.d_c / 64 : 1;
+  P.idx = (const int32_t*)(cb + p.off_idx);
+  P.W3 = (const __nv_bfloat16*)W3; P.b3 = b3;
+  P.a = (const float*)(w + p.ws_a); P.cterm = (const float*)(w + p.ws_cterm);
+  P.S = (const float*)(w + p.ws_S); P.Smax = (const float*)(w + p.ws_Smax);
+  P.wtab = (float*)(w + p.ws_wtab); P.part = (float*)(w + p.ws_part); P.Upart = (float*)(w + p.ws_U);
+  P.err = (uint32_t*)ws;
+  CUtensorMap mapC;
+  {
+    cuuint64_t dims[3] = {(cuuint64_t)c.d_c, (cuuint64_t)n_code, (cuuint64_t)BH};
+    cuuint64_t str[2] = {(cuuint64_t)c.d_c * 2, (cuuint64_t)p.n_code_cap * c.d_c * 2};
+    cuuint32_t box[3] = {(cuuint32_t)std::min(c.d_c, 64), (cuuint32_t)dtc::CH, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    const CUtensorMapSwizzle sw = P.code_swz == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                  : P.code_swz == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                     : CU_TENSOR_MAP_SWIZZLE_32B;
+    if (encode_fn_dec()(&mapC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<char*>(cb + p.off_code), dims,
+                        str, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorNotSupported;
+  }
+  const size_t smem = DecLayout(c.d_c, c.k, c.hidden).total + 1024;
+  cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  ProfScope ps(p, st, KID_DEC_STREAM);
+  decode_tc_kernel<<<P.grid, dtc::THREADS, smem, st>>>(mapC, P);
+  return cudaGetLastError();
+}
+
+}  // namespace dkv

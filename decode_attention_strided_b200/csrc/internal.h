@@ -45,7 +45,7 @@ struct Plan {
   // compress workspace
   size_t ws_hnorm, ws_cand;
   // decode workspace
-  int ns_max;            // decode splits per (b, head)
+  int nslot_cap;         // decode partial slots per (b, head)
   int n_chunk_cap;       // combine blocks per (b, head)
   size_t ws_S, ws_Smax, ws_a, ws_cterm, ws_wtab, ws_part, ws_U, ws_ochunk;
   size_t ws_bytes;
@@ -86,11 +86,19 @@ cudaError_t launch_candidates_tc(const Plan& p, int T, const KVView& kv, const v
 cudaError_t launch_encode(const Plan& p, int T, const KVView& kv, const void* W1, const float* b1,
                           const void* W2, const float* b2, void* cache, void* ws,
                           cudaStream_t st);
+bool encode_tc_supported(const Plan& p);
+cudaError_t launch_encode_tc(const Plan& p, int T, const KVView& kv, const void* W1, const float* b1,
+                             const void* W2, const float* b2, void* cache, void* ws,
+                             cudaStream_t st);
 // ---- reconstruct (tests / debugging) ----
 cudaError_t launch_reconstruct(const Plan& p, int T, const void* cache, const void* W3,
                                const float* b3, const void* W4, const float* b4, float* Kout,
                                float* Vout, void* ws, cudaStream_t st);
 // ---- decode ----
+bool decode_tc_supported(const Plan& p);
+int decode_tc_grid(const Plan& p, int64_t N);
+cudaError_t launch_decode_tc(const Plan& p, int T, const void* cache, const void* W3, const float* b3,
+                             void* ws, cudaStream_t st);
 cudaError_t launch_decode(const Plan& p, int T, const void* q, int64_t qsb, int64_t qsh,
                           const void* cache, const void* W3, const float* b3, const void* W4,
                           const float* b4, float* out, int64_t osb, int64_t osh, void* ws,
