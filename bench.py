@@ -96,6 +96,39 @@ class Shape:
         return per_head * self.Bd * self.H + self.Bd * self.Hq * self.d_h * (es + 4) + weights
 
 
+def kernel_rooflines(sh, prof, peaks, peak_kind):
+    """Per-kernel roofline: algorithmic work of one launch / its mean
+    CUDA-event duration, against the bound that work implies."""
+    tensor_peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    hbm_peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    out = {}
+
+    def add(name, bound, work, unit, peak, src):
+        if name not in prof:
+            return
+        n, ms = prof[name]
+        sec = ms / n / 1e3
+        scale = 1e12 if unit == "TFLOP/s" else 1e9
+        ach = work / sec / scale
+        out[name] = {"kernel": name, "bound": bound, "achieved": ach, "peak": peak, "unit": unit,
+                     "frac": ach / peak, "traffic": None, "algorithmic_per_launch": work,
+                     "peak_source": src, "ms_per_launch": ms / n}
+
+    src_t = f"{peak_kind} bf16 sustained (MEASURED_PEAKS bf16_tflops_sustained)" if peak_kind == "measured" \
+        else "fallback 1.4 PFLOP/s sustained"
+    src_h = f"{peak_kind} HBM copy (hbm_gbs)" if peak_kind == "measured" else "fallback 6.65 TB/s"
+    # nearest-reference search: 2 D sum_t ceil(t/s) per (sequence, kv-head), compress batch
+    add("candidates_tc", "tensor", sh.cand_flops_per_layer(sh.Bc), "TFLOP/s", tensor_peak, src_t)
+    add("candidates_simt", "alu", sh.cand_flops_per_layer(sh.Bc) * 1.5, "TFLOP/s",
+        NUM_SMS * FP32_LANES_PER_SM * 2 * SM_MAX_MHZ * 1e6 / 1e12, "fp32 lanes x 2 x max SM clock")
+    # encode: the two compressor GEMMs per compressed row
+    add("encode", "tensor", sh.mlp_flops_per_layer(sh.Bc), "TFLOP/s", tensor_peak, src_t)
+    # decode token loop: the code and slot planes it streams (decode batch)
+    stream_bytes = sh.Bd * sh.H * sh.n_code * (sh.d_c * 2 + sh.k * 4)
+    add("decode_stream", "hbm", stream_bytes, "GB/s", hbm_peak, src_h)
+    return out
+
+
 def build_workload(sh, dev):
     from decode_attention_strided_b200 import deltakv as dkv
     from decode_attention_strided_b200 import synth
@@ -358,23 +391,8 @@ def main():
             prof[k_] = (pn + n, pm + ms)
     launches = sum(n for n, _ in prof.values())
     dom = max(prof.items(), key=lambda kv: kv[1][1])[0] if prof else None
-    roof = None
-    if dom in ("candidates_tc", "candidates_simt"):
-        n, ms = prof[dom]
-        per_launch_s = ms / n / 1e3
-        if dom == "candidates_tc":
-            fl = sh.cand_flops_per_layer(sh.Bc)
-            peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
-            roof = {"kernel": dom, "bound": "tensor", "achieved": fl / per_launch_s / 1e12, "peak": peak,
-                    "unit": "TFLOP/s", "peak_source": f"{peak_kind} bf16 sustained"}
-        else:
-            fl = sh.cand_flops_per_layer(sh.Bc) * 3 / 2  # sub + fma per element and dim
-            peak = NUM_SMS * FP32_LANES_PER_SM * 2 * SM_MAX_MHZ * 1e6 / 1e12
-            roof = {"kernel": dom, "bound": "alu", "achieved": fl / per_launch_s / 1e12, "peak": peak,
-                    "unit": "TFLOP/s", "peak_source": "fp32 lanes x 2 x max SM clock"}
-        roof["frac"] = roof["achieved"] / roof["peak"]
-        roof["traffic"] = None
-        roof["algorithmic_per_launch"] = fl
+    rooflines = kernel_rooflines(sh, prof, peaks, peak_kind)
+    roof = rooflines.get(dom)
     dbytes = sh.decode_bytes_per_layer()
     dec_ms_layer = sd / a.steps / sh.L
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
@@ -402,7 +420,8 @@ def main():
         "metric": METRIC, "value": value, "unit": "Mtok/s", "n_gpus": world, "steps": a.steps,
         "warmup": a.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(sh),
-        "compress": compress, "decode_attn": decode_attn, "roofline": roof, "cpu_baseline": cpu,
+        "compress": compress, "decode_attn": decode_attn, "roofline": roof, "rooflines": rooflines,
+        "cpu_baseline": cpu,
         "e2e": e2e, "gpu_launches": launches, "kernels": {k_: {"launches": n, "ms": ms} for k_, (n, ms) in prof.items()},
         "clocks": clk, "device_status": status, "setup_s": setup_s, "wall_s": wall,
     }

@@ -14,14 +14,16 @@
 //   producer warp  TMA: the chunk's codes (zero-filled past the last row)
 //                  and slots into a 2-stage ring
 //   MMA warp       D1 = codes . W3^T  (M=128, N=hidden, K=d_c; bf16, exact
-//                  products), z = u . [a_hi; a_lo]^T (M=128, N=16, K=hidden),
+//                  products), z = u . [a_hi, a_lo rows]^T (M=128, N=16, K=hidden),
 //                  U_chunk = u^T . P  (M=128 hidden units, N=16, K=128 tokens;
 //                  the u tile read through an MN-major descriptor)
-//   epilogue       8 warps: act(D1 + b3) -> fp16 u tile (double-buffered);
-//                  warps 2-5 also do the softmax step (S gathers, per-chunk
-//                  maximum, P tile, slot-weight reductions into the global
-//                  table); both groups fold U_chunk into register
-//                  accumulators with the online-softmax rescale.
+//   activation     8 warps: act(D1 + b3) -> fp16 u tile (two buffers)
+//   softmax        4 warps: S gathers (issued early), per-chunk maximum,
+//                  fp16 P tile (two buffers), slot-weight reductions into the
+//                  global table, and the fold of U_chunk into register
+//                  accumulators with the online-softmax rescale
+// The MMA warp issues G1(0); then per chunk i: z(i), G1(i+1), U(i-1), so the
+// activation warps never wait on the softmax of the same chunk.
 // A persistent grid splits the flattened (kv-head, chunk) list evenly; each
 // CTA writes one partial (m, l, U) per kv-head segment it touches.
 #include <cfloat>
@@ -38,9 +40,13 @@ using namespace sm100;
 
 namespace dtc {
 constexpr int CH = 128;                 // tokens per chunk (MMA M)
-constexpr int EPI = 8;                  // epilogue warps: group A = 2..5, B = 6..9
-constexpr int THREADS = (EPI + 2) * 32;
+constexpr int ACT = 8;                  // activation warps 2..9 (two per TMEM lane quarter)
+constexpr int SMX = 4;                  // softmax warps 10..13 (one per lane quarter)
+constexpr int ACT0 = 2;
+constexpr int THREADS = (2 + ACT + SMX) * 32;
 constexpr uint32_t TMEM_COLS = 512;
+// TMEM columns: D1 [0, 256), z [256, 288) two buffers of 16, U [288, 352)
+// two buffers of 2 x 16 (hidden halves)
 constexpr uint32_t COL_D1 = 0, COL_Z = 256, COL_U = 288;
 constexpr int PRODUCER = 0, MMA = 1;
 }  // namespace dtc
@@ -145,7 +151,7 @@ struct DecLayout {
   __host__ __device__ DecLayout(int d_c, int k, int hidden) {
     const size_t code_b = (size_t)dtc::CH * d_c * 2, idx_b = (size_t)dtc::CH * k * 4;
     const size_t w3_b = (size_t)hidden * d_c * 2, az_b = (size_t)(hidden / 64) * 16 * 128;
-    const size_t u_b = (size_t)(hidden / 64) * dtc::CH * 128, p_b = 2 * 16 * 128;
+    const size_t u_b = (size_t)(hidden / 64) * dtc::CH * 128, p_b = 2 * 2 * 16 * 128;
     size_t o = 0;
     code = o; o = dtc_align(o + 2 * dtc_align(code_b));
     idx = o;  o = dtc_align(o + 2 * dtc_align(idx_b));
@@ -154,11 +160,21 @@ struct DecLayout {
     u = o;    o = dtc_align(o + 2 * u_b);
     p = o;    o = dtc_align(o + p_b);
     fl = o;   o += 256 * sizeof(float);
-    bar = o;  o += 32 * 8 + 16;
+    bar = o;  o += 24 * 8 + 16;
     total = o;
   }
 };
 
+// ACT: the codec nonlinearity (compile-time, so the activation loop has no
+// per-element branch); HAS_B3: whether b3 is added.
+template <int ACT, bool HAS_B3>
+__device__ __forceinline__ float dec_act(float v, const float* b3, int c) {
+  if (HAS_B3) v += b3[c];
+  if (ACT == DELTAKV_ACT_GELU_ERF) return gelu_fast(v);
+  return act_eval(ACT, v);
+}
+
+template <int ACT, bool HAS_B3>
 __global__ void __launch_bounds__(dtc::THREADS, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap mapC, const DecTcParams P) {
   extern __shared__ unsigned char smem_raw[];
@@ -171,28 +187,28 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
   unsigned char* sW3 = base + L.w3;
   auto sAz = [&](int i) { return base + L.az + i * az_b; };
   auto sU = [&](int i) { return base + L.u + i * u_b; };
-  unsigned char* sP = base + L.p;
+  auto sP = [&](int i) { return base + L.p + i * 2 * 16 * 128; };
   float* fl = (float*)(base + L.fl);
-  float* m_run = fl;         // [8]
-  float* l_run = fl + 8;     // [8]
-  float* alpha = fl + 16;    // [8]
-  float* m_ref = fl + 24;    // [8]
-  float* ctv = fl + 32;      // [8]
-  float* mred = fl + 40;     // [4][8]
-  float* lred = fl + 72;     // [4][8]
+  float* m_run = fl;          // [8]
+  float* l_run = fl + 8;      // [8]
+  float* alpha = fl + 16;     // [2][8] per chunk parity
+  float* m_ref = fl + 32;     // [8]
+  float* ctv = fl + 40;       // [8]
+  float* mred = fl + 48;      // [4][8]
+  float* lred = fl + 80;      // [4][8]
   uint64_t* bar = (uint64_t*)(base + L.bar);
   uint64_t* in_full = bar + 0;    // [2]
   uint64_t* in_empty = bar + 2;   // [2]
   uint64_t* d1_full = bar + 4;
   uint64_t* u_full = bar + 5;     // [2]
   uint64_t* u_empty = bar + 7;    // [2]
-  uint64_t* z_full = bar + 9;
-  uint64_t* z_empty = bar + 10;
-  uint64_t* p_full = bar + 11;
-  uint64_t* p_empty = bar + 12;
-  uint64_t* ua_full = bar + 13;
-  uint64_t* ua_empty = bar + 14;
-  uint32_t* tmem_slot = (uint32_t*)(bar + 16);
+  uint64_t* z_full = bar + 9;     // [2]
+  uint64_t* z_empty = bar + 11;   // [2]
+  uint64_t* p_full = bar + 13;    // [2]
+  uint64_t* p_empty = bar + 15;   // [2]
+  uint64_t* ua_full = bar + 17;   // [2]
+  uint64_t* ua_empty = bar + 19;  // [2]
+  uint32_t* tmem_slot = (uint32_t*)(bar + 21);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
@@ -201,35 +217,33 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
   const int n_local = (int)(x_end - x_begin);
 
   // ---- one-time set-up: W3 (bf16, K-major, swizzled like the code tile),
-  // zero rows of the P and a tiles, barriers, TMEM
+  // zero P and a tiles (their padding rows are never written), barriers, TMEM
   {
     const int swz = P.code_swz;
-    const int row_elems = swz / 2;  // bf16 per swizzled row
+    const int row_elems = swz / 2;
     for (int i = tid; i < hidden * P.d_c / 8; i += blockDim.x) {
-      const int n = i / (P.d_c / 8), c8 = (i % (P.d_c / 8)) * 8;  // hidden unit, code column
+      const int n = i / (P.d_c / 8), c8 = (i % (P.d_c / 8)) * 8;
       const uint4 v = *reinterpret_cast<const uint4*>(P.W3 + (int64_t)n * P.d_c + c8);
       const int atom = c8 / row_elems, col = c8 % row_elems;
       *reinterpret_cast<uint4*>(sW3 + (size_t)atom * hidden * swz + swz_off(n, col * 2, swz)) = v;
     }
-    for (int i = tid; i < 2 * 16 * 128 / 4; i += blockDim.x) reinterpret_cast<uint32_t*>(sP)[i] = 0u;
+    for (int i = tid; i < 2 * 2 * 16 * 128 / 4; i += blockDim.x) reinterpret_cast<uint32_t*>(sP(0))[i] = 0u;
     for (int i = tid; i < 2 * (int)az_b / 4; i += blockDim.x) reinterpret_cast<uint32_t*>(sAz(0))[i] = 0u;
   }
   if (tid == 0) {
-    mbar_init(&in_full[0], 1);
-    mbar_init(&in_full[1], 1);
-    mbar_init(&in_empty[0], 2);
-    mbar_init(&in_empty[1], 2);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&in_full[i], 1);
+      mbar_init(&in_empty[i], 2);
+      mbar_init(&u_full[i], dtc::ACT);
+      mbar_init(&u_empty[i], 1);
+      mbar_init(&z_full[i], 1);
+      mbar_init(&z_empty[i], dtc::SMX);
+      mbar_init(&p_full[i], 1);
+      mbar_init(&p_empty[i], 1);
+      mbar_init(&ua_full[i], 1);
+      mbar_init(&ua_empty[i], dtc::SMX);
+    }
     mbar_init(d1_full, 1);
-    mbar_init(&u_full[0], dtc::EPI);
-    mbar_init(&u_full[1], dtc::EPI);
-    mbar_init(&u_empty[0], 1);
-    mbar_init(&u_empty[1], 1);
-    mbar_init(z_full, 1);
-    mbar_init(z_empty, 4);
-    mbar_init(p_full, 1);
-    mbar_init(p_empty, 1);
-    mbar_init(ua_full, 1);
-    mbar_init(ua_empty, dtc::EPI);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -266,37 +280,66 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
     }
   } else if (warp == dtc::MMA) {
     // ----------------------------------------------------------------- MMA
+    // order: G1(0); for i: z(i), G1(i+1), U(i-1); U(n-1)
     if (lane == 0 && n_local > 0) {
       const uint32_t id_g1 = idesc_kind_f16(true, dtc::CH, hidden, false);
       const uint32_t id_z = idesc_kind_f16(false, dtc::CH, 16, false);
       const uint32_t id_u = idesc_kind_f16(false, 128, 16, true);
       const int swz = P.code_swz;
+      bool ok = true;
       auto gemm1 = [&](int st) {
         const uint32_t c0 = smem_u32(sCode(st)), w0 = smem_u32(sW3);
+        const int per_row = swz / 32;  // k16 steps per swizzled row
         for (int k16 = 0; k16 < P.d_c / 16; ++k16) {
-          const int per_row = swz / 32;  // k16 steps per swizzled row
           const int atom = k16 / per_row, off = (k16 % per_row) * 32;
           umma_f16(tmem + dtc::COL_D1, desc_kmajor(c0 + atom * dtc::CH * swz + off, swz),
                    desc_kmajor(w0 + atom * hidden * swz + off, swz), id_g1, k16 != 0);
         }
       };
-      bool ok = true;
+      auto issue_u = [&](int j) {
+        const int jb = j & 1;
+        if (!mbar_wait(&p_full[jb], (j >> 1) & 1, abort_flag)) return false;
+        if (!mbar_wait(&ua_empty[jb], ((j >> 1) & 1) ^ 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t u0 = smem_u32(sU(jb)), p0 = smem_u32(sP(jb));
+        for (int h2 = 0; h2 < hidden / 128; ++h2)
+          for (int k16 = 0; k16 < dtc::CH / 16; ++k16) {
+            const uint64_t ad = desc_mnmajor_sw128(u0 + (2 * h2) * dtc::CH * 128 + k16 * 16 * 128,
+                                                   dtc::CH * 128, 1024);
+            const uint64_t bd = desc_kmajor(p0 + (k16 >> 2) * 16 * 128 + (k16 & 3) * 32, 128);
+            umma_f16(tmem + dtc::COL_U + 32 * jb + 16 * h2, ad, bd, id_u, k16 != 0);
+          }
+        umma_commit(&ua_full[jb]);
+        umma_commit(&u_empty[jb]);
+        umma_commit(&p_empty[jb]);
+        return true;
+      };
       int seg = -1, prev_bh = -1;
+      if (mbar_wait(&in_full[0], 0, abort_flag)) {
+        tc_fence_after();
+        gemm1(0);
+        umma_commit(d1_full);
+        umma_commit(&in_empty[0]);
+      } else {
+        ok = false;
+      }
       for (int it = 0; it < n_local && ok; ++it) {
         const int64_t x = x_begin + it;
         const int bh = (int)(x / P.n_ch);
         if (bh != prev_bh) { ++seg; prev_bh = bh; }
         const int ub = it & 1;
-        if (it == 0) {
-          if (!mbar_wait(&in_full[0], 0, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          gemm1(0);
-          umma_commit(d1_full);
-          umma_commit(&in_empty[0]);
-        }
-        // act(D1) of this chunk is in the u tile (and D1 is free again)
         if (!mbar_wait(&u_full[ub], (it >> 1) & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(&z_empty[ub], ((it >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
+        {
+          const uint32_t u0 = smem_u32(sU(ub)), a0 = smem_u32(sAz(seg & 1));
+          for (int k16 = 0; k16 < hidden / 16; ++k16) {
+            const int atom = k16 >> 2, off = (k16 & 3) * 32;
+            umma_f16(tmem + dtc::COL_Z + 16 * ub, desc_kmajor(u0 + atom * dtc::CH * 128 + off, 128),
+                     desc_kmajor(a0 + atom * 16 * 128 + off, 128), id_z, k16 != 0);
+          }
+          umma_commit(&z_full[ub]);
+        }
         if (it + 1 < n_local) {
           const int st = (it + 1) & 1;
           if (!mbar_wait(&in_full[st], ((it + 1) >> 1) & 1, abort_flag)) { ok = false; break; }
@@ -305,77 +348,93 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
           umma_commit(d1_full);
           umma_commit(&in_empty[st]);
         }
-        // z = u . [a_hi; a_lo]^T
-        if (!mbar_wait(z_empty, (it & 1) ^ 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        {
-          const uint32_t u0 = smem_u32(sU(ub)), a0 = smem_u32(sAz(seg & 1));
-          for (int k16 = 0; k16 < hidden / 16; ++k16) {
-            const int atom = k16 >> 2, off = (k16 & 3) * 32;
-            umma_f16(tmem + dtc::COL_Z, desc_kmajor(u0 + atom * dtc::CH * 128 + off, 128),
-                     desc_kmajor(a0 + atom * 16 * 128 + off, 128), id_z, k16 != 0);
-          }
-          umma_commit(z_full);
-        }
-        // U_chunk = u^T . P
-        if (!mbar_wait(p_full, it & 1, abort_flag)) { ok = false; break; }
-        if (!mbar_wait(ua_empty, (it & 1) ^ 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        {
-          const uint32_t u0 = smem_u32(sU(ub)), p0 = smem_u32(sP);
-          for (int h2 = 0; h2 < hidden / 128; ++h2)
-            for (int k16 = 0; k16 < dtc::CH / 16; ++k16) {
-              const uint64_t ad = desc_mnmajor_sw128(u0 + (2 * h2) * dtc::CH * 128 + k16 * 16 * 128,
-                                                     dtc::CH * 128, 1024);
-              const uint64_t bd = desc_kmajor(p0 + (k16 >> 2) * 16 * 128 + (k16 & 3) * 32, 128);
-              umma_f16(tmem + dtc::COL_U + 16 * h2, ad, bd, id_u, k16 != 0);
-            }
-          umma_commit(ua_full);
-          umma_commit(&u_empty[ub]);
-          umma_commit(p_empty);
-        }
+        if (it >= 1 && !issue_u(it - 1)) { ok = false; break; }
       }
+      if (ok && !issue_u(n_local - 1)) ok = false;
       if (!ok) {
         latch_error(P.err, DELTAKV_ERR_DEVICE_TIMEOUT, 21);
         *abort_flag = 1;
       }
     }
-  } else {
-    // ------------------------------------------------------------ epilogue
-    const int ew = warp - 2;                  // 0..7
-    const bool groupA = ew < 4;
-    const int q = warp & 3;                   // TMEM lane quarter
-    const int n = q * 32 + lane;              // token row (D1, z) / unit in half (U)
-    const int hh = groupA ? 0 : 1;            // hidden half of this group
-    float Ureg[kMaxG];
-#pragma unroll
-    for (int g = 0; g < kMaxG; ++g) Ureg[g] = 0.f;
+  } else if (warp < dtc::ACT0 + dtc::ACT) {
+    // ------------------------------------------------- activation warps
+    const int aw = warp - dtc::ACT0;        // 0..7
+    const int q = warp & 3, n = q * 32 + lane;
+    const int hh = aw < 4 ? 0 : 1;          // hidden half
     bool ok = true;
     int prev_bh = -1, seg_count = 0;
     for (int it = 0; it < n_local && ok; ++it) {
       const int64_t x = x_begin + it;
       const int bh = (int)(x / P.n_ch);
-      const int64_t row0 = (x % P.n_ch) * dtc::CH;
-      const int st = it & 1, ub = it & 1;
+      const int ub = it & 1;
+      if (!mbar_wait(&u_empty[ub], ((it >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
       if (bh != prev_bh) {
-        // new kv-head segment: its a_hi / a_lo rows go to the a tile of this
-        // segment's parity (the z MMAs of segment - 2, the last users of that
-        // tile, completed before their softmax steps), state is reset
+        // a_hi / a_lo rows of this kv-head into the a tile of this segment's
+        // parity; its last users (z MMAs of two segments back) are complete
+        // because the U MMAs after them have released this u buffer
         prev_bh = bh;
-        named_bar(2, dtc::EPI * 32);
         unsigned char* az = sAz(seg_count & 1);
         const float* ab = P.a + (int64_t)bh * G * hidden;
-        for (int i = tid - 64; i < G * hidden; i += dtc::EPI * 32) {
+        for (int i = tid - dtc::ACT0 * 32; i < G * hidden; i += dtc::ACT * 32) {
           const int g = i / hidden, c = i % hidden;
           const float v = ab[i];
           const __half hi = __float2half_rn(v);
           const __half lo = __float2half_rn(v - __half2float(hi));
           const int atom = c >> 6, cc = c & 63;
-          *reinterpret_cast<__half*>(az + atom * 16 * 128 + swz_off(g, cc * 2, 128)) = hi;
-          *reinterpret_cast<__half*>(az + atom * 16 * 128 + swz_off(G + g, cc * 2, 128)) = lo;
+          *reinterpret_cast<__half*>(az + atom * 16 * 128 + swz_off(2 * g, cc * 2, 128)) = hi;
+          *reinterpret_cast<__half*>(az + atom * 16 * 128 + swz_off(2 * g + 1, cc * 2, 128)) = lo;
         }
-        if (tid - 64 < G) {
-          const int g = tid - 64;
+        fence_async_smem();
+        named_bar(2, dtc::ACT * 32);
+        ++seg_count;
+      }
+      if (!mbar_wait(d1_full, it & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      unsigned char* ut = sU(ub);
+      const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16) + dtc::COL_D1;
+#pragma unroll 1
+      for (int c0 = hh * half; c0 < (hh + 1) * half; c0 += 32) {
+        float v[32];
+        tmem_ld32(trow + c0, v);
+        __align__(16) __half2 h2[16];
+#pragma unroll
+        for (int x2 = 0; x2 < 16; ++x2)
+          h2[x2] = __floats2half2_rn(dec_act<ACT, HAS_B3>(v[2 * x2], P.b3, c0 + 2 * x2),
+                                     dec_act<ACT, HAS_B3>(v[2 * x2 + 1], P.b3, c0 + 2 * x2 + 1));
+        const int atom = c0 >> 6, cc = c0 & 63;
+#pragma unroll
+        for (int v4 = 0; v4 < 4; ++v4)
+          *reinterpret_cast<uint4*>(ut + atom * dtc::CH * 128 + swz_off(n, (cc + 8 * v4) * 2, 128)) =
+              reinterpret_cast<const uint4*>(h2)[v4];
+      }
+      tc_fence_before();
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&u_full[ub]);
+    }
+    if (!ok) {
+      latch_error(P.err, DELTAKV_ERR_DEVICE_TIMEOUT, 22);
+      *abort_flag = 1;
+    }
+  } else {
+    // ---------------------------------------------------- softmax warps
+    const int sw = warp - (dtc::ACT0 + dtc::ACT);   // 0..3
+    const int q = warp & 3, n = q * 32 + lane;      // token row / hidden unit in a half
+    float Ureg[2][kMaxG];
+#pragma unroll
+    for (int g = 0; g < kMaxG; ++g) Ureg[0][g] = Ureg[1][g] = 0.f;
+    bool ok = true;
+    int prev_bh = -1;
+    for (int it = 0; it < n_local && ok; ++it) {
+      const int64_t x = x_begin + it;
+      const int bh = (int)(x / P.n_ch);
+      const int64_t row0 = (x % P.n_ch) * dtc::CH;
+      const int st = it & 1, zb = it & 1;
+      if (bh != prev_bh) {
+        prev_bh = bh;
+        named_bar(3, dtc::SMX * 32);
+        if (sw == 0 && lane < G) {
+          const int g = lane;
           float m = -INFINITY;
           for (int r = 0; r < P.n_refblk; ++r) m = fmaxf(m, P.Smax[((int64_t)bh * P.n_refblk_cap + r) * G + g]);
           m_ref[g] = m;
@@ -384,188 +443,179 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
           ctv[g] = P.cterm[(int64_t)bh * G + g];
         }
 #pragma unroll
-        for (int g = 0; g < kMaxG; ++g) Ureg[g] = 0.f;
-        fence_async_smem();
-        named_bar(2, dtc::EPI * 32);
-        ++seg_count;
+        for (int g = 0; g < kMaxG; ++g) Ureg[0][g] = Ureg[1][g] = 0.f;
+        named_bar(3, dtc::SMX * 32);
       }
-      // ------------------------------------------------------ act(D1 + b3)
-      if (!mbar_wait(d1_full, it & 1, abort_flag)) { ok = false; break; }
-      if (!mbar_wait(&u_empty[ub], ((it >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
-      tc_fence_after();
-      {
-        unsigned char* ut = sU(ub);
-        for (int c0 = hh * half; c0 < (hh + 1) * half; c0 += 32) {
-          float v[32];
-          tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + dtc::COL_D1 + c0, v);
-          __align__(16) __half2 h2[16];
+      // reference logits S[idx]: loads issued before the wait on z
+      const int64_t row = row0 + n;
+      const bool valid = row < P.n_code;
+      if (!mbar_wait(&in_full[st], (it >> 1) & 1, abort_flag)) { ok = false; break; }
+      const int32_t* ir = sIdx(st) + n * P.k;
+      const float* Sb = P.S + (int64_t)bh * P.n_ref_cap * G;
+      float4 sv[kMaxK];
+      int k_eff = 0;
 #pragma unroll
-          for (int x2 = 0; x2 < 16; ++x2) {
-            const float a0 = act_eval(P.act, v[2 * x2] + (P.b3 ? P.b3[c0 + 2 * x2] : 0.f));
-            const float a1 = act_eval(P.act, v[2 * x2 + 1] + (P.b3 ? P.b3[c0 + 2 * x2 + 1] : 0.f));
-            h2[x2] = __floats2half2_rn(a0, a1);
-          }
-          const int atom = c0 >> 6, cc = c0 & 63;
-#pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4)
-            *reinterpret_cast<uint4*>(ut + atom * dtc::CH * 128 + swz_off(n, (cc + 8 * v4) * 2, 128)) =
-                reinterpret_cast<const uint4*>(h2)[v4];
-        }
-      }
-      tc_fence_before();
-      fence_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&u_full[ub]);
-
-      // ------------------------------------------------------------ softmax
-      if (groupA) {
-        if (!mbar_wait(z_full, it & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        float zz[16];
-        tmem_ld16f(tmem + ((uint32_t)(q * 32) << 16) + dtc::COL_Z, zz);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(z_empty);
-        const int64_t row = row0 + n;
-        const bool valid = row < P.n_code;
-        const int32_t* ir = sIdx(st) + n * P.k;
-        const float* Sb = P.S + (int64_t)bh * P.n_ref_cap * G;
-        float lg[kMaxG];
-        int k_eff = 0;
-#pragma unroll
-        for (int g = 0; g < kMaxG; ++g) lg[g] = 0.f;
-        if (valid) {
-          for (int i = 0; i < P.k; ++i) {
-            const int j = ir[i];
-            if (j < 0) continue;
-            if (j >= P.n_ref) {
-              latch_error(P.err, DELTAKV_ERR_DEVICE_BOUNDS, (uint32_t)j);
-              continue;
-            }
+      for (int i = 0; i < kMaxK; ++i) {
+        sv[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (i < P.k && valid) {
+          const int j = ir[i];
+          if (j >= 0 && j < P.n_ref) {
             ++k_eff;
-            if (G == 4) {
-              const float4 s4 = *reinterpret_cast<const float4*>(Sb + (int64_t)j * 4);
-              lg[0] += s4.x; lg[1] += s4.y; lg[2] += s4.z; lg[3] += s4.w;
-            } else {
-#pragma unroll
-              for (int g = 0; g < kMaxG; ++g)
-                if (g < G) lg[g] += Sb[(int64_t)j * G + g];
-            }
+            if (G == 4) sv[i] = __ldg(reinterpret_cast<const float4*>(Sb + (int64_t)j * 4));
+          } else if (j >= P.n_ref) {
+            latch_error(P.err, DELTAKV_ERR_DEVICE_BOUNDS, (uint32_t)j);
           }
-        }
-        const float inv_k = 1.0f / (float)max(k_eff, 1);
-        float mx[kMaxG];
-#pragma unroll
-        for (int g = 0; g < kMaxG; ++g) {
-          lg[g] = g < G ? zz[g] + zz[G + g] + ctv[g] + lg[g] * inv_k : 0.f;
-          mx[g] = valid && g < G ? lg[g] : -INFINITY;
-          mx[g] = warp_max(mx[g]);
-        }
-        if (lane == 0) {
-#pragma unroll
-          for (int g = 0; g < kMaxG; ++g)
-            if (g < G) mred[(ew & 3) * 8 + g] = mx[g];
-        }
-        named_bar(1, 128);
-        float mnew[kMaxG], p[kMaxG];
-#pragma unroll
-        for (int g = 0; g < kMaxG; ++g) {
-          if (g < G) {
-            float m = m_run[g];
-            for (int w = 0; w < 4; ++w) m = fmaxf(m, mred[w * 8 + g]);
-            mnew[g] = m;
-            p[g] = valid ? exp2f(lg[g] - m) : 0.f;
-          } else {
-            mnew[g] = 0.f;
-            p[g] = 0.f;
-          }
-        }
-        // P tile (B operand of the U MMA) once the previous U MMA is done
-        if (!mbar_wait(p_empty, (it & 1) ^ 1, abort_flag)) { ok = false; break; }
-        {
-          const int atom = n >> 6, cc = n & 63;
-#pragma unroll
-          for (int g = 0; g < kMaxG; ++g)
-            if (g < G)
-              *reinterpret_cast<__half*>(sP + atom * 16 * 128 + swz_off(g, cc * 2, 128)) = __float2half_rn(p[g]);
-        }
-        // slot weights relative to m_ref, into the kv-head's global table
-        if (valid && k_eff > 0) {
-          float* wt = P.wtab + (int64_t)bh * P.n_ref_cap * G;
-          float sc[kMaxG];
-#pragma unroll
-          for (int g = 0; g < kMaxG; ++g) sc[g] = g < G ? p[g] * exp2f(fminf(mnew[g] - m_ref[g], 100.f)) * inv_k : 0.f;
-          for (int i = 0; i < P.k; ++i) {
-            const int j = ir[i];
-            if (j < 0 || j >= P.n_ref) continue;
-            if (G == 4) {
-              asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(wt + (int64_t)j * 4),
-                           "f"(sc[0]), "f"(sc[1]), "f"(sc[2]), "f"(sc[3])
-                           : "memory");
-            } else {
-#pragma unroll
-              for (int g = 0; g < kMaxG; ++g)
-                if (g < G) atomicAdd(wt + (int64_t)j * G + g, sc[g]);
-            }
-          }
-        }
-        float ls[kMaxG];
-#pragma unroll
-        for (int g = 0; g < kMaxG; ++g) ls[g] = warp_sum(p[g]);
-        if (lane == 0) {
-#pragma unroll
-          for (int g = 0; g < kMaxG; ++g)
-            if (g < G) lred[(ew & 3) * 8 + g] = ls[g];
-        }
-        fence_async_smem();
-        named_bar(1, 128);
-        if (ew == 0 && lane < G) {
-          const int g = lane;
-          const float al = exp2f(m_run[g] - mnew[g]);
-          alpha[g] = al;
-          l_run[g] = l_run[g] * al + lred[g] + lred[8 + g] + lred[16 + g] + lred[24 + g];
-          m_run[g] = mnew[g];
-        }
-        named_bar(1, 128);
-        if (ew == 0 && lane == 0) {
-          mbar_arrive(p_full);
-          mbar_arrive(&in_empty[st]);
         }
       }
-      // --------------------------------------------- fold U_chunk into Ureg
-      if (!groupA && !mbar_wait(p_full, it & 1, abort_flag)) { ok = false; break; }
-      if (!mbar_wait(ua_full, it & 1, abort_flag)) { ok = false; break; }
+      float lg[kMaxG];
+#pragma unroll
+      for (int g = 0; g < kMaxG; ++g) lg[g] = 0.f;
+      if (G != 4 && valid) {
+        for (int i = 0; i < P.k; ++i) {
+          const int j = ir[i];
+          if (j < 0 || j >= P.n_ref) continue;
+#pragma unroll
+          for (int g = 0; g < kMaxG; ++g)
+            if (g < G) lg[g] += Sb[(int64_t)j * G + g];
+        }
+      }
+      if (!mbar_wait(&z_full[zb], (it >> 1) & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      if (hh < hidden / 128) {
-        float du[16];
-        tmem_ld16f(tmem + ((uint32_t)(q * 32) << 16) + dtc::COL_U + 16 * hh, du);
+      float zz[16];
+      tmem_ld16f(tmem + ((uint32_t)(q * 32) << 16) + dtc::COL_Z + 16 * zb, zz);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&z_empty[zb]);
+      if (G == 4) {
+#pragma unroll
+        for (int i = 0; i < kMaxK; ++i) {
+          lg[0] += sv[i].x; lg[1] += sv[i].y; lg[2] += sv[i].z; lg[3] += sv[i].w;
+        }
+      }
+      const float inv_k = 1.0f / (float)max(k_eff, 1);
+      float mx[kMaxG];
+#pragma unroll
+      for (int g = 0; g < kMaxG; ++g) {
+        lg[g] = g < G ? zz[2 * g] + zz[2 * g + 1] + ctv[g] + lg[g] * inv_k : 0.f;
+        mx[g] = valid && g < G ? lg[g] : -INFINITY;
+        if (g < G) mx[g] = warp_max(mx[g]);
+      }
+      if (lane == 0) {
 #pragma unroll
         for (int g = 0; g < kMaxG; ++g)
-          if (g < G) Ureg[g] = Ureg[g] * alpha[g] + du[g];
+          if (g < G) mred[sw * 8 + g] = mx[g];
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(ua_empty);
-
-      // ------------------------------------------------ segment end: flush
-      const bool seg_end = (it == n_local - 1) || ((x + 1) / P.n_ch != bh);
-      if (seg_end) {
-        // partial slot: this CTA's rank among the CTAs that cover the head
-        const int64_t pb = (int64_t)bh * P.nslot_cap + (int64_t)blockIdx.x - dtc_owner((int64_t)bh * P.n_ch, P.N, P.grid);
-        if (hh < hidden / 128) {
-          const int unit = 128 * hh + n;
+      named_bar(3, dtc::SMX * 32);
+      float mnew[kMaxG], p[kMaxG];
 #pragma unroll
-          for (int g = 0; g < kMaxG; ++g)
-            if (g < G) P.Upart[(pb * G + g) * hidden + unit] = Ureg[g];
+      for (int g = 0; g < kMaxG; ++g) {
+        if (g < G) {
+          float m = m_run[g];
+          for (int w = 0; w < dtc::SMX; ++w) m = fmaxf(m, mred[w * 8 + g]);
+          mnew[g] = m;
+          p[g] = valid ? exp2f(lg[g] - m) : 0.f;
+        } else {
+          mnew[g] = 0.f;
+          p[g] = 0.f;
         }
-        if (ew == 0 && lane < G) {
+      }
+      if (!mbar_wait(&p_empty[zb], ((it >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+      {
+        unsigned char* pt = sP(zb);
+        const int atom = n >> 6, cc = n & 63;
+#pragma unroll
+        for (int g = 0; g < kMaxG; ++g)
+          if (g < G) *reinterpret_cast<__half*>(pt + atom * 16 * 128 + swz_off(g, cc * 2, 128)) = __float2half_rn(p[g]);
+      }
+      // slot weights, relative to m_ref, into the kv-head's global table
+      if (valid && k_eff > 0) {
+        float* wt = P.wtab + (int64_t)bh * P.n_ref_cap * G;
+        float sc[kMaxG];
+#pragma unroll
+        for (int g = 0; g < kMaxG; ++g) sc[g] = g < G ? p[g] * exp2f(fminf(mnew[g] - m_ref[g], 100.f)) * inv_k : 0.f;
+        for (int i = 0; i < P.k; ++i) {
+          const int j = ir[i];
+          if (j < 0 || j >= P.n_ref) continue;
+          if (G == 4) {
+            asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(wt + (int64_t)j * 4), "f"(sc[0]),
+                         "f"(sc[1]), "f"(sc[2]), "f"(sc[3])
+                         : "memory");
+          } else {
+#pragma unroll
+            for (int g = 0; g < kMaxG; ++g)
+              if (g < G) atomicAdd(wt + (int64_t)j * G + g, sc[g]);
+          }
+        }
+      }
+      float ls[kMaxG];
+#pragma unroll
+      for (int g = 0; g < kMaxG; ++g) ls[g] = g < G ? warp_sum(p[g]) : 0.f;
+      if (lane == 0) {
+#pragma unroll
+        for (int g = 0; g < kMaxG; ++g)
+          if (g < G) lred[sw * 8 + g] = ls[g];
+      }
+      fence_async_smem();
+      named_bar(3, dtc::SMX * 32);
+      if (sw == 0 && lane < G) {
+        const int g = lane;
+        const float al = exp2f(m_run[g] - mnew[g]);
+        alpha[zb * 8 + g] = al;
+        float lc = 0.f;
+        for (int w = 0; w < dtc::SMX; ++w) lc += lred[w * 8 + g];
+        l_run[g] = l_run[g] * al + lc;
+        m_run[g] = mnew[g];
+      }
+      named_bar(3, dtc::SMX * 32);
+      if (sw == 0 && lane == 0) {
+        mbar_arrive(&p_full[zb]);
+        mbar_arrive(&in_empty[st]);
+      }
+      // fold the previous chunk's U (its MMA was issued after this chunk's z)
+      const bool seg_end = (it == n_local - 1) || ((x + 1) / P.n_ch != bh);
+      const bool prev_same = it >= 1 && (x - 1) / P.n_ch == bh;
+      // fold U_chunk j (TMEM buffer j & 1): the previous chunk, and at the
+      // end of a kv-head segment also this one
+      for (int pass = 0; pass < 2; ++pass) {
+        const int j = pass == 0 ? it - 1 : it;
+        if (pass == 0 ? !prev_same : !seg_end) continue;
+        const int jb = j & 1;
+        if (!mbar_wait(&ua_full[jb], (j >> 1) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          if (h2 < hidden / 128) {
+            float du[16];
+            tmem_ld16f(tmem + ((uint32_t)(q * 32) << 16) + dtc::COL_U + 32 * jb + 16 * h2, du);
+#pragma unroll
+            for (int g = 0; g < kMaxG; ++g)
+              if (g < G) Ureg[h2][g] = Ureg[h2][g] * alpha[jb * 8 + g] + du[g];
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ua_empty[jb]);
+      }
+      if (!ok) break;
+      if (seg_end) {
+        const int64_t pb = (int64_t)bh * P.nslot_cap + (int64_t)blockIdx.x - dtc_owner((int64_t)bh * P.n_ch, P.N, P.grid);
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          if (h2 < hidden / 128) {
+            const int unit = 128 * h2 + n;
+#pragma unroll
+            for (int g = 0; g < kMaxG; ++g)
+              if (g < G) P.Upart[(pb * G + g) * hidden + unit] = Ureg[h2][g];
+          }
+        }
+        if (sw == 0 && lane < G) {
           P.part[(pb * G + lane) * 2 + 0] = m_run[lane];
           P.part[(pb * G + lane) * 2 + 1] = l_run[lane];
         }
       }
     }
     if (!ok) {
-      latch_error(P.err, DELTAKV_ERR_DEVICE_TIMEOUT, 22);
+      latch_error(P.err, DELTAKV_ERR_DEVICE_TIMEOUT, 23);
       *abort_flag = 1;
     }
   }
@@ -651,10 +701,22 @@ cudaError_t launch_decode_tc(const Plan& p, int T, const void* cache, const void
       return cudaErrorNotSupported;
   }
   const size_t smem = DecLayout(c.d_c, c.k, c.hidden).total + 1024;
-  cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  void (*kern)(const CUtensorMap, const DecTcParams) = nullptr;
+  const bool hb = b3 != nullptr;
+  switch ((int)c.act) {
+    case DELTAKV_ACT_GELU_ERF:
+      kern = hb ? decode_tc_kernel<DELTAKV_ACT_GELU_ERF, true> : decode_tc_kernel<DELTAKV_ACT_GELU_ERF, false>;
+      break;
+    case DELTAKV_ACT_GELU_TANH:
+      kern = hb ? decode_tc_kernel<DELTAKV_ACT_GELU_TANH, true> : decode_tc_kernel<DELTAKV_ACT_GELU_TANH, false>;
+      break;
+    default:
+      kern = hb ? decode_tc_kernel<DELTAKV_ACT_NONE, true> : decode_tc_kernel<DELTAKV_ACT_NONE, false>;
+  }
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   ProfScope ps(p, st, KID_DEC_STREAM);
-  decode_tc_kernel<<<P.grid, dtc::THREADS, smem, st>>>(mapC, P);
+  kern<<<P.grid, dtc::THREADS, smem, st>>>(mapC, P);
   return cudaGetLastError();
 }
 

@@ -342,8 +342,8 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
         __half2 hi2[8], lo2[8];
 #pragma unroll
         for (int x = 0; x < 8; ++x) {
-          const float a = act_eval(P.act, v[2 * x] + (P.b1 ? P.b1[c0 + 2 * x] : 0.f));
-          const float bq = act_eval(P.act, v[2 * x + 1] + (P.b1 ? P.b1[c0 + 2 * x + 1] : 0.f));
+          const float a = act_fast(P.act, v[2 * x] + (P.b1 ? P.b1[c0 + 2 * x] : 0.f));
+          const float bq = act_fast(P.act, v[2 * x + 1] + (P.b1 ? P.b1[c0 + 2 * x + 1] : 0.f));
           split_half2(a, bq, hi2[x], lo2[x]);
         }
         const uint32_t o0 = sw128_offset(n, c0, enc::ROWS), o1 = sw128_offset(n, c0 + 8, enc::ROWS);
