@@ -122,10 +122,11 @@ def kernel_rooflines(sh, prof, peaks, peak_kind):
     add("candidates_simt", "alu", sh.cand_flops_per_layer(sh.Bc) * 1.5, "TFLOP/s",
         NUM_SMS * FP32_LANES_PER_SM * 2 * SM_MAX_MHZ * 1e6 / 1e12, "fp32 lanes x 2 x max SM clock")
     # encode: the two compressor GEMMs per compressed row
-    add("encode", "tensor", sh.mlp_flops_per_layer(sh.Bc), "TFLOP/s", tensor_peak, src_t)
+    add("encode_tc", "tensor", sh.mlp_flops_per_layer(sh.Bc), "TFLOP/s", tensor_peak, src_t)
     # decode token loop: the code and slot planes it streams (decode batch)
     stream_bytes = sh.Bd * sh.H * sh.n_code * (sh.d_c * 2 + sh.k * 4)
-    add("decode_stream", "hbm", stream_bytes, "GB/s", hbm_peak, src_h)
+    add("decode_stream_tc", "hbm", stream_bytes, "GB/s", hbm_peak, src_h)
+    add("decode_stream_simt", "hbm", stream_bytes, "GB/s", hbm_peak, src_h)
     return out
 
 
@@ -399,9 +400,10 @@ def main():
     decode_attn = {"value": dbytes / (dec_ms_layer / 1e3) / 1e9, "unit": "GB/s", "peak": hbm,
                    "peak_source": peak_kind, "frac": dbytes / (dec_ms_layer / 1e3) / 1e9 / hbm,
                    "ms_per_layer": dec_ms_layer, "bytes_per_layer": dbytes}
-    if "decode_stream" in prof:
-        n, ms = prof["decode_stream"]
-        decode_attn["stream_kernel_ms_per_launch"] = ms / n
+    for k_ in ("decode_stream_tc", "decode_stream_simt"):
+        if k_ in prof:
+            n, ms = prof[k_]
+            decode_attn["stream_kernel_ms_per_launch"] = ms / n
     comp_fl = sh.cand_flops_per_layer(sh.Bc) + sh.mlp_flops_per_layer(sh.Bc)
     compress = {"value": sh.T * sh.Bc / (sc / a.steps / 1e3) / 1e6, "unit": "Mtok/s",
                 "ms": sc / a.steps,

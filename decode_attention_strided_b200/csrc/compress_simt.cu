@@ -356,7 +356,7 @@ static cudaError_t encode_launch(const Plan& p, int T, const KVView& kv, const v
   char* cb = (char*)cache;
   int64_t n_code = n_code_of(T, c.stride_s);
   dim3 grid((unsigned)ceil_div64(n_code, kEncTile), c.kv_heads, c.batch);
-  ProfScope ps(p, st, KID_ENCODE);
+  ProfScope ps(p, st, KID_ENCODE_SIMT);
   kern<<<grid, 256, smem, st>>>(T, c.stride_s, c.d_h, c.kv_heads, c.k, c.d_c, c.hidden, (int)c.act,
                                 p.n_ref_cap, p.n_code_cap, (const E*)kv.K, (const E*)kv.V, kv.sb,
                                 kv.sh, kv.st, (const E*)W1, b1, (const E*)W2, b2,

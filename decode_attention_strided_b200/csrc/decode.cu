@@ -476,7 +476,7 @@ static cudaError_t decode_launch(const Plan& p, int T, const void* q, int64_t qs
     auto ks = decode_stream_kernel<E>;
     e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    ProfScope ps(p, st, KID_DEC_STREAM);
+    ProfScope ps(p, st, KID_DEC_STREAM_SIMT);
     ks<<<dim3(ns, H, B), 256, smem, st>>>(T, c.stride_s, c.d_h, H, G, c.k, c.d_c, c.hidden, (int)c.act, ns,
                                           p.n_ref_cap, p.n_code_cap, n_refblk, n_refblk_cap, code, idx,
                                           (const E*)W3, b3, a, cterm, S, Smax, wtab, part, Upart,

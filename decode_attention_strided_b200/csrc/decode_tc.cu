@@ -650,6 +650,11 @@ EncodeTiledFn encode_fn_dec() {
 bool decode_tc_supported(const Plan& p) {
   const auto& c = p.cfg;
   if (c.dtype != DELTAKV_BF16 || !encode_fn_dec()) return false;
+  // u = act(W3 c + b3) enters the logit MMA as one fp16 term, so each logit
+  // carries an error of up to 2^-12 sum_h |a_h u_h|.  With a nonlinear codec
+  // that stays far inside the attention tolerance; a linear codec (no
+  // activation) feeds larger, unsquashed u and takes the fp32 token loop.
+  if (c.act == DELTAKV_ACT_NONE) return false;
   if (!(c.hidden == 128 || c.hidden == 256)) return false;
   if (!(c.d_c == 16 || c.d_c == 32 || c.d_c == 64 || c.d_c == 128)) return false;
   if (2 * p.G > 16) return false;
@@ -711,11 +716,11 @@ cudaError_t launch_decode_tc(const Plan& p, int T, const void* cache, const void
       kern = hb ? decode_tc_kernel<DELTAKV_ACT_GELU_TANH, true> : decode_tc_kernel<DELTAKV_ACT_GELU_TANH, false>;
       break;
     default:
-      kern = hb ? decode_tc_kernel<DELTAKV_ACT_NONE, true> : decode_tc_kernel<DELTAKV_ACT_NONE, false>;
+      return cudaErrorNotSupported;  // decode_tc_supported excludes the linear codec
   }
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  ProfScope ps(p, st, KID_DEC_STREAM);
+  ProfScope ps(p, st, KID_DEC_STREAM_TC);
   kern<<<P.grid, dtc::THREADS, smem, st>>>(mapC, P);
   return cudaGetLastError();
 }

@@ -12,10 +12,15 @@
 // One persistent CTA per SM, 8 warps.  W1 [hidden x D] and W2 [d_c x hidden]
 // stay in shared memory as fp16 for the whole launch (bf16 values are exact
 // in fp16); per 64-row tile:
-//   phase 1  warp per token: gather, re-rank, mean, residual r -> A tiles
-//   phase 2  tcgen05.mma  D1 = R . W1^T                   (fp32 in TMEM)
-//   phase 3  TMEM -> + b1 -> act -> H tiles (alias the A tiles)
-//   phase 4  tcgen05.mma  D2 = H . W2^T
+//   phase 1  8 lanes per token, 32 tokens in flight: gather the k + 4
+//            candidate rows, exact distances, choose k, reload them for the
+//            mean, residual r -> R tile (64 tokens x D, K-major)
+//   phase 2  tcgen05.mma  D1^T = W1 . R^T  (M = 128 hidden units per half,
+//            N = 64 tokens; fp32 in TMEM): TMEM lanes are hidden units
+//   phase 3  all 8 warps: thread = hidden unit, act(D1 + b1) over its 64
+//            tokens -> H tile stored as hidden rows of 64 tokens, which is
+//            the MN-major A operand of
+//   phase 4  tcgen05.mma  codes = H . W2^T  (M = 128 with 64 tokens, N = d_c)
 //   phase 5  TMEM -> + b2 -> bf16 codes
 // Precision: every MMA operand that is not a weight is split into two fp16
 // terms, hi = fp16(v) and lo = fp16(v - hi), and multiplied twice, so r and
@@ -23,9 +28,6 @@
 // term the unrounded codes would differ from exact ones by enough to flip
 // the final bf16 rounding of a code element often, and each flip moves the
 // decoded token.
-// The MMA is M = 128; a tile uses only its first 64 rows, the other 64 read
-// the neighbouring operand atom (in-bounds shared memory) and their results
-// are never read, which halves the A footprint so the weights fit.
 #include <cfloat>
 #include <climits>
 
@@ -40,7 +42,6 @@ using namespace sm100;
 namespace enc {
 constexpr int ROWS = 64;       // compressed rows per tile (the MMA runs M = 128)
 constexpr int MMA_M = 128;
-constexpr int ATOM = ROWS * 128;  // bytes of one 64-row x 64-column fp16 atom
 constexpr int THREADS = 256;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t D2_COL = 256;  // TMEM column of the second accumulator
@@ -56,6 +57,17 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
 __device__ __forceinline__ uint32_t sw128_offset(int row, int col, int rows_per_atom) {
   const int atom = col >> 6, c = col & 63;
   return (uint32_t)(atom * rows_per_atom * 128 + row * 128 + ((((c >> 3) ^ (row & 7))) << 4) + (c & 7) * 2);
+}
+
+// MN-major, 128-byte swizzle descriptor: 64 contiguous M-elements per 128-byte
+// row, 8-row K groups `sbo` bytes apart, 64-element M blocks `lbo` apart.
+__device__ __forceinline__ uint64_t desc_mnmajor_sw128_enc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFF);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
 }
 
 // v = hi + lo with hi = fp16(v), lo = fp16(v - hi), for two values at once.
@@ -88,23 +100,6 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// EPL bf16 (or fp16) values in one vector register group.
-template <int EPL> struct PackT;
-template <> struct PackT<8> { using type = uint4; };
-template <> struct PackT<4> { using type = uint2; };
-template <int EPL> using Pack = typename PackT<EPL>::type;
-
-template <int EPL>
-__device__ __forceinline__ void unpack(const Pack<EPL>& p, float (&f)[EPL]) {
-  const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&p);
-#pragma unroll
-  for (int q = 0; q < EPL / 2; ++q) {
-    const float2 v = __bfloat1622float2(p2[q]);
-    f[2 * q] = v.x;
-    f[2 * q + 1] = v.y;
-  }
-}
-
 struct EncParams {
   int T, s, d_h, H, k, d_c, hidden, act, BH;
   int64_t n_code, n_ref, n_ref_cap, n_code_cap;
@@ -124,26 +119,70 @@ struct EncParams {
   int n_tiles, tiles_per_bh;
 };
 
-// EPL: bf16 elements of x each lane holds (D / 32); KC: candidates per token.
-template <int EPL, int KC>
+// EPL: elements of [K ; V] per lane with 8 lanes per row (D / 8);
+// KC: candidates per token; ACT: activation; HAS_B: biases present.
+template <int EPL> struct RowPack;
+template <> struct RowPack<32> { static constexpr int V4 = 4; };  // 4 x 16 B
+template <> struct RowPack<16> { static constexpr int V4 = 2; };  // 2 x 16 B
+
+template <int EPL>
+__device__ __forceinline__ void load_row(const __nv_bfloat16* src, uint4 (&r)[RowPack<EPL>::V4]) {
+#pragma unroll
+  for (int i = 0; i < RowPack<EPL>::V4; ++i) r[i] = __ldg(reinterpret_cast<const uint4*>(src) + i);
+}
+
+template <int EPL>
+__device__ __forceinline__ void unpack_row(const uint4 (&r)[RowPack<EPL>::V4], float (&f)[EPL]) {
+#pragma unroll
+  for (int i = 0; i < RowPack<EPL>::V4; ++i) {
+    const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&r[i]);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 v = __bfloat1622float2(p2[q]);
+      f[8 * i + 2 * q] = v.x;
+      f[8 * i + 2 * q + 1] = v.y;
+    }
+  }
+}
+
+__device__ __forceinline__ float group8_sum(float v) {
+  v += __shfl_xor_sync(0xffffffffu, v, 4, 8);
+  v += __shfl_xor_sync(0xffffffffu, v, 2, 8);
+  v += __shfl_xor_sync(0xffffffffu, v, 1, 8);
+  return v;
+}
+
+template <int ACT>
+__device__ __forceinline__ float enc_act(float v) {
+  if (ACT == DELTAKV_ACT_GELU_ERF) return gelu_fast(v);
+  return act_eval(ACT, v);
+}
+
+template <int EPL, int KC, int ACT>
 __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncParams P) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  constexpr int D = EPL * 32;
-  const int hid_atoms = (P.hidden + 63) / 64;
-  const int rh_atoms = max(D / 64, hid_atoms);
-  unsigned char* sW1 = smem;                                        // [D/64][hidden][128 B]
-  unsigned char* sRH = sW1 + (D / 64) * P.hidden * 128;             // hi atoms, then lo atoms
-  unsigned char* sLo = sRH + rh_atoms * enc::ATOM;                  //   [rh_atoms][64][128 B] each
-  unsigned char* sW2 = sLo + rh_atoms * enc::ATOM;                  // [hid_atoms][d_c][128 B]
-  uint64_t* mma_bar = (uint64_t*)(sW2 + ((hid_atoms * P.d_c * 128 + 1023) & ~1023));
+  constexpr int D = EPL * 8;
+  constexpr int KA = D / 64;                       // 64-column atoms along D
+  const int hidden = P.hidden, hid_atoms = (hidden + 63) / 64;
+  // shared memory: W1 [hidden rows][D] K-major (A of GEMM1^T), then the
+  // R tile (B of GEMM1^T: 64 token rows x D, hi atoms then lo atoms) which
+  // the H tile (A of GEMM2, MN-major: hidden rows x 64 tokens, hi then lo)
+  // later overwrites, then W2 [d_c rows][hidden] K-major (B of GEMM2)
+  unsigned char* sW1 = smem;
+  unsigned char* sR = sW1 + (size_t)KA * hidden * 128;
+  const size_t r_part = (size_t)KA * enc::ROWS * 128;          // one of hi / lo
+  const size_t h_part = (size_t)hidden * 128;                  // one of hi / lo
+  const size_t rh_b = r_part > h_part ? 2 * r_part : 2 * h_part;
+  unsigned char* sW2 = sR + rh_b;
+  uint64_t* mma_bar = (uint64_t*)(sW2 + (((size_t)hid_atoms * P.d_c * 128 + 1023) & ~size_t(1023)));
   uint32_t* tmem_slot = (uint32_t*)(mma_bar + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
 
-  // ---- weights -> fp16, 128-byte swizzled K-major atoms (once per CTA)
-  for (int i = tid; i < P.hidden * D / 8; i += blockDim.x) {
+  // ---- weights -> fp16 (bf16 values are exact in fp16), swizzled K-major
+  for (int i = tid; i < hidden * D / 8; i += blockDim.x) {
     const int n = i / (D / 8), c8 = (i % (D / 8)) * 8;
     const uint4 raw = *reinterpret_cast<const uint4*>(P.W1 + (int64_t)n * D + c8);
     const __nv_bfloat162* b2v = reinterpret_cast<const __nv_bfloat162*>(&raw);
@@ -151,13 +190,13 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
     __half2* o2 = reinterpret_cast<__half2*>(&out);
 #pragma unroll
     for (int q = 0; q < 4; ++q) o2[q] = __float22half2_rn(__bfloat1622float2(b2v[q]));
-    *reinterpret_cast<uint4*>(sW1 + sw128_offset(n, c8, P.hidden)) = out;
+    *reinterpret_cast<uint4*>(sW1 + sw128_offset(n, c8, hidden)) = out;
   }
   for (int i = tid; i < P.d_c * hid_atoms * 8; i += blockDim.x) {
     const int o = i / (hid_atoms * 8), c8 = (i % (hid_atoms * 8)) * 8;
     uint4 out = make_uint4(0, 0, 0, 0);
-    if (c8 < P.hidden) {
-      const uint4 raw = *reinterpret_cast<const uint4*>(P.W2 + (int64_t)o * P.hidden + c8);
+    if (c8 < hidden) {
+      const uint4 raw = *reinterpret_cast<const uint4*>(P.W2 + (int64_t)o * hidden + c8);
       const __nv_bfloat162* b2v = reinterpret_cast<const __nv_bfloat162*>(&raw);
       __half2* o2 = reinterpret_cast<__half2*>(&out);
 #pragma unroll
@@ -182,6 +221,10 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
   uint32_t mma_phase = 0;
   bool ok = true;
 
+  const int grp = lane >> 3, s8 = lane & 7;   // row within the warp's 4, lane within the row
+  const int e0 = s8 * EPL;                     // this lane's first element of [K ; V]
+  const bool inK = e0 < P.d_h;
+
   for (int tile = blockIdx.x; tile < P.n_tiles && ok; tile += gridDim.x) {
     const int bh = tile / P.tiles_per_bh;
     const int64_t row0 = (int64_t)(tile % P.tiles_per_bh) * enc::ROWS;
@@ -190,119 +233,114 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
     const __nv_bfloat16* Vb = P.V + b * P.sb + h * P.sh;
     const __nv_bfloat16* rk = P.refk + (int64_t)bh * P.n_ref_cap * P.d_h;
     const __nv_bfloat16* rv = P.refv + (int64_t)bh * P.n_ref_cap * P.d_h;
-    const int e0 = lane * EPL;  // this lane's first element of [K ; V]
-    const bool inK = e0 < P.d_h;
 
-    // ------------------------------------------ phase 1: re-rank, mean, residual
-    // Two rows per warp at a time; every gather of a row pair is issued before
-    // any of them is used, so the L2 round trips overlap.
-    for (int n0 = warp * 2; n0 < enc::ROWS; n0 += 16) {
-      constexpr int NR = 2;
-      Pack<EPL> xr[NR], rr[NR][KC];
-      int jj[NR][KC];
-      int64_t tt[NR];
-      bool live[NR];
+    // ------------------------------- phase 1: re-rank, mean, residual (8 lanes / row)
+    for (int n = warp * 4 + grp; n < enc::ROWS; n += 32) {
+      const int64_t row = row0 + n;
+      const bool live = row < P.n_code;
+      const int64_t t = live ? (row / (P.s - 1)) * P.s + (row % (P.s - 1)) + 1 : 0;
+      const int32_t* cr = P.cand + ((int64_t)bh * P.n_code_cap + row) * KC;
+      const int myc0 = (live && s8 < KC) ? cr[s8] : -1;
+      const int myc1 = (live && s8 + 8 < KC) ? cr[s8 + 8] : -1;
+      float xv[EPL];
+      {
+        uint4 xr[RowPack<EPL>::V4];
+        if (live) load_row<EPL>(inK ? Kb + t * P.st + e0 : Vb + t * P.st + (e0 - P.d_h), xr);
+        else
 #pragma unroll
-      for (int u = 0; u < NR; ++u) {
-        const int64_t row = row0 + n0 + u;
-        live[u] = row < P.n_code;
-        tt[u] = live[u] ? (row / (P.s - 1)) * P.s + (row % (P.s - 1)) + 1 : 0;
-        const int my_c = (live[u] && lane < KC) ? P.cand[((int64_t)bh * P.n_code_cap + row) * KC + lane] : -1;
-        if (live[u]) {
-          const __nv_bfloat16* src = inK ? Kb + tt[u] * P.st + e0 : Vb + tt[u] * P.st + (e0 - P.d_h);
-          xr[u] = *reinterpret_cast<const Pack<EPL>*>(src);
+          for (int i = 0; i < RowPack<EPL>::V4; ++i) xr[i] = make_uint4(0, 0, 0, 0);
+        unpack_row<EPL>(xr, xv);
+      }
+      int cj[KC];
+      float cd[KC];
+#pragma unroll
+      for (int c = 0; c < KC; ++c) {
+        int j = c < 8 ? __shfl_sync(0xffffffffu, myc0, c, 8) : __shfl_sync(0xffffffffu, myc1, c - 8, 8);
+        if (j >= 0 && (int64_t)j * P.s >= t) {  // not an earlier reference: drop it
+          if (s8 == 0) latch_error(P.err, DELTAKV_ERR_DEVICE_BOUNDS, (uint32_t)j);
+          j = -1;
+        }
+        cj[c] = j;
+      }
+      // exact distances, 4 candidate rows in flight at a time
+#pragma unroll
+      for (int c0 = 0; c0 < KC; c0 += 4) {
+        uint4 rr[4][RowPack<EPL>::V4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int j = cj[c0 + u];
+          if (j >= 0) load_row<EPL>(inK ? rk + (int64_t)j * P.d_h + e0 : rv + (int64_t)j * P.d_h + (e0 - P.d_h), rr[u]);
         }
 #pragma unroll
-        for (int c = 0; c < KC; ++c) {
-          int j = __shfl_sync(0xffffffffu, my_c, c);
-          if (j >= 0 && (int64_t)j * P.s >= tt[u]) {  // not an earlier reference: drop it
-            if (lane == 0) latch_error(P.err, DELTAKV_ERR_DEVICE_BOUNDS, (uint32_t)j);
-            j = -1;
+        for (int u = 0; u < 4; ++u) {
+          float part = 0.f;
+          if (cj[c0 + u] >= 0) {
+            float rf[EPL];
+            unpack_row<EPL>(rr[u], rf);
+#pragma unroll
+            for (int q = 0; q < EPL; ++q) {
+              const float df = xv[q] - rf[q];
+              part = fmaf(df, df, part);
+            }
           }
-          jj[u][c] = j;
+          part = group8_sum(part);
+          cd[c0 + u] = cj[c0 + u] >= 0 ? part : FLT_MAX;
         }
       }
+      // the k smallest (distance, slot), ascending
+      uint32_t chosen = 0;
+      int k_eff = 0, my_sel = -1;
+      for (int qk = 0; qk < P.k; ++qk) {
+        int best = -1;
+        float bdv = FLT_MAX;
+        int bj = INT_MAX;
 #pragma unroll
-      for (int u = 0; u < NR; ++u)
-#pragma unroll
-        for (int c = 0; c < KC; ++c)
-          if (jj[u][c] >= 0) {
-            const int j = jj[u][c];
-            const __nv_bfloat16* src = inK ? rk + (int64_t)j * P.d_h + e0 : rv + (int64_t)j * P.d_h + (e0 - P.d_h);
-            rr[u][c] = *reinterpret_cast<const Pack<EPL>*>(src);
+        for (int c = 0; c < KC; ++c) {
+          const bool avail = cj[c] >= 0 && !(chosen & (1u << c));
+          if (avail && (cd[c] < bdv || (cd[c] == bdv && cj[c] < bj))) {
+            best = c;
+            bdv = cd[c];
+            bj = cj[c];
           }
-#pragma unroll
-      for (int u = 0; u < NR; ++u) {
-        const int n = n0 + u;
-        const int64_t row = row0 + n;
-        float rres[EPL];
-        if (live[u]) {
-          float xv[EPL];
-          unpack<EPL>(xr[u], xv);
-          float cd[KC];
-#pragma unroll
-          for (int c = 0; c < KC; ++c) {
-            float part = 0.f;
-            if (jj[u][c] >= 0) {
-              float rf[EPL];
-              unpack<EPL>(rr[u][c], rf);
-#pragma unroll
-              for (int q = 0; q < EPL; ++q) {
-                const float df = xv[q] - rf[q];
-                part = fmaf(df, df, part);
-              }
-            }
-            part = warp_sum(part);
-            cd[c] = jj[u][c] >= 0 ? part : FLT_MAX;
-          }
-          // the k smallest (distance, slot) of the candidates, ascending
-          uint32_t chosen = 0;
-          int k_eff = 0, my_sel = -1;
-          for (int q = 0; q < P.k; ++q) {
-            int best = -1;
-            float bdv = FLT_MAX;
-            int bj = INT_MAX;
-#pragma unroll
-            for (int c = 0; c < KC; ++c) {
-              const bool avail = jj[u][c] >= 0 && !(chosen & (1u << c));
-              if (avail && (cd[c] < bdv || (cd[c] == bdv && jj[u][c] < bj))) {
-                best = c;
-                bdv = cd[c];
-                bj = jj[u][c];
-              }
-            }
-            if (best >= 0) {
-              chosen |= 1u << best;
-              ++k_eff;
-            }
-            if (lane == q) my_sel = best >= 0 ? bj : -1;
-          }
-          if (lane < P.k) P.idx[((int64_t)bh * P.n_code_cap + row) * P.k + lane] = my_sel;
-          const float inv = 1.0f / (float)max(k_eff, 1);
-          float m[EPL];
-#pragma unroll
-          for (int q = 0; q < EPL; ++q) m[q] = 0.f;
-#pragma unroll
-          for (int c = 0; c < KC; ++c)
-            if (chosen & (1u << c)) {
-              float rf[EPL];
-              unpack<EPL>(rr[u][c], rf);
-#pragma unroll
-              for (int q = 0; q < EPL; ++q) m[q] += rf[q];
-            }
-#pragma unroll
-          for (int q = 0; q < EPL; ++q) rres[q] = xv[q] - m[q] * inv;
-        } else {
-#pragma unroll
-          for (int q = 0; q < EPL; ++q) rres[q] = 0.f;
         }
-        // r = hi + lo in fp16, into the swizzled A tiles
-        __half2 hi2[EPL / 2], lo2[EPL / 2];
+        if (best >= 0) {
+          chosen |= 1u << best;
+          ++k_eff;
+        }
+        if (s8 == qk) my_sel = best >= 0 ? bj : -1;
+      }
+      if (live && s8 < P.k) P.idx[((int64_t)bh * P.n_code_cap + row) * P.k + s8] = my_sel;
+      // mean of the chosen rows (reloaded: they are in L2), residual
+      float m[EPL];
 #pragma unroll
-        for (int q = 0; q < EPL / 2; ++q) split_half2(rres[2 * q], rres[2 * q + 1], hi2[q], lo2[q]);
-        const uint32_t off = sw128_offset(n, e0, enc::ROWS);
-        *reinterpret_cast<Pack<EPL>*>(sRH + off) = *reinterpret_cast<const Pack<EPL>*>(hi2);
-        *reinterpret_cast<Pack<EPL>*>(sLo + off) = *reinterpret_cast<const Pack<EPL>*>(lo2);
+      for (int q = 0; q < EPL; ++q) m[q] = 0.f;
+#pragma unroll
+      for (int c = 0; c < KC; ++c) {
+        if (chosen & (1u << c)) {
+          const int j = cj[c];
+          uint4 rr[RowPack<EPL>::V4];
+          load_row<EPL>(inK ? rk + (int64_t)j * P.d_h + e0 : rv + (int64_t)j * P.d_h + (e0 - P.d_h), rr);
+          float rf[EPL];
+          unpack_row<EPL>(rr, rf);
+#pragma unroll
+          for (int q = 0; q < EPL; ++q) m[q] += rf[q];
+        }
+      }
+      const float inv = 1.0f / (float)max(k_eff, 1);
+      // r = hi + lo (fp16) into the R tile: row n, columns e0 .. e0 + EPL
+#pragma unroll
+      for (int v = 0; v < EPL / 8; ++v) {
+        __half2 hi2[4], lo2[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int i = 8 * v + 2 * q;
+          const float r0 = live ? xv[i] - m[i] * inv : 0.f;
+          const float r1 = live ? xv[i + 1] - m[i + 1] * inv : 0.f;
+          split_half2(r0, r1, hi2[q], lo2[q]);
+        }
+        const uint32_t off = sw128_offset(n, e0 + 8 * v, enc::ROWS);
+        *reinterpret_cast<uint4*>(sR + off) = *reinterpret_cast<const uint4*>(hi2);
+        *reinterpret_cast<uint4*>(sR + r_part + off) = *reinterpret_cast<const uint4*>(lo2);
       }
     }
     fence_proxy_async_smem();
@@ -310,47 +348,46 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
     __syncthreads();
     tc_fence_after();
 
-    // --------------------------------------------------- phase 2: GEMM1
+    // ------------------------------ phase 2: D1^T = W1 . R^T (hidden x tokens)
     if (tid == 0) {
-      const uint32_t w0 = smem_u32(sW1);
-      const uint32_t idesc = idesc_f16_f32(enc::MMA_M, P.hidden);
+      const uint32_t w0 = smem_u32(sW1), r0 = smem_u32(sR);
+      const uint32_t idesc = idesc_f16_f32(128, enc::ROWS);
 #pragma unroll 1
-      for (int part = 0; part < 2; ++part) {
-        const uint32_t a0 = smem_u32(part == 0 ? sRH : sLo);
+      for (int hh = 0; hh < hidden / 128; ++hh)
 #pragma unroll 1
-        for (int k16 = 0; k16 < D / 16; ++k16) {
-          const int atom = k16 >> 2, off = (k16 & 3) * 32;
-          umma_f16(tmem, desc_kmajor_sw128(a0 + atom * enc::ATOM + off),
-                   desc_kmajor_sw128(w0 + atom * P.hidden * 128 + off), idesc, (part | k16) != 0);
-        }
-      }
+        for (int part = 0; part < 2; ++part)
+#pragma unroll 1
+          for (int k16 = 0; k16 < D / 16; ++k16) {
+            const int atom = k16 >> 2, off = (k16 & 3) * 32;
+            umma_f16(tmem + enc::ROWS * hh,
+                     desc_kmajor_sw128(w0 + atom * hidden * 128 + hh * 128 * 128 + off),
+                     desc_kmajor_sw128(r0 + part * (uint32_t)r_part + atom * enc::ROWS * 128 + off), idesc,
+                     (part | k16) != 0);
+          }
       umma_commit(mma_bar);
     }
     if (!mbar_wait(mma_bar, mma_phase, abort_flag)) { ok = false; break; }
     mma_phase ^= 1;
     tc_fence_after();
 
-    // ------------------------------------------- phase 3: act(D1 + b1) -> H
-    // rows 0..63 live in TMEM lanes 0..63: warps 0, 1 (columns of the first
-    // half) and 4, 5 (second half) read them
-    if ((warp & 3) < 2) {
-      const int q = warp & 3, half = warp >> 2, n = q * 32 + lane;
-      const int cols = P.hidden / 2;
-      for (int c0 = half * cols; c0 < (half + 1) * cols; c0 += 16) {
-        float v[16];
-        tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + c0, v);
-        __half2 hi2[8], lo2[8];
+    // ---------------- phase 3: H = act(D1 + b1), hidden rows x 64 tokens (all 8 warps)
+    if (warp < 4 * (hidden / 128)) {
+      const int q = warp & 3, hh = warp >> 2;
+      const int unit = 128 * hh + 32 * q + lane;
+      const float bias = P.b1 ? P.b1[unit] : 0.f;
+      float v[64];
+      tmem_ld64(tmem + ((uint32_t)(32 * q) << 16) + enc::ROWS * hh, v);
 #pragma unroll
-        for (int x = 0; x < 8; ++x) {
-          const float a = act_fast(P.act, v[2 * x] + (P.b1 ? P.b1[c0 + 2 * x] : 0.f));
-          const float bq = act_fast(P.act, v[2 * x + 1] + (P.b1 ? P.b1[c0 + 2 * x + 1] : 0.f));
-          split_half2(a, bq, hi2[x], lo2[x]);
-        }
-        const uint32_t o0 = sw128_offset(n, c0, enc::ROWS), o1 = sw128_offset(n, c0 + 8, enc::ROWS);
-        *reinterpret_cast<uint4*>(sRH + o0) = *reinterpret_cast<const uint4*>(&hi2[0]);
-        *reinterpret_cast<uint4*>(sRH + o1) = *reinterpret_cast<const uint4*>(&hi2[4]);
-        *reinterpret_cast<uint4*>(sLo + o0) = *reinterpret_cast<const uint4*>(&lo2[0]);
-        *reinterpret_cast<uint4*>(sLo + o1) = *reinterpret_cast<const uint4*>(&lo2[4]);
+      for (int c8 = 0; c8 < 8; ++c8) {
+        __half2 hi2[4], lo2[4];
+#pragma unroll
+        for (int x = 0; x < 4; ++x)
+          split_half2(enc_act<ACT>(v[8 * c8 + 2 * x] + bias), enc_act<ACT>(v[8 * c8 + 2 * x + 1] + bias), hi2[x],
+                      lo2[x]);
+        // MN-major row `unit` of 64 tokens: 16-byte chunk c8, swizzled by row
+        const uint32_t off = (uint32_t)unit * 128 + (((c8 ^ (unit & 7))) << 4);
+        *reinterpret_cast<uint4*>(sR + off) = *reinterpret_cast<const uint4*>(hi2);
+        *reinterpret_cast<uint4*>(sR + h_part + off) = *reinterpret_cast<const uint4*>(lo2);
       }
     }
     fence_proxy_async_smem();
@@ -358,20 +395,20 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
     __syncthreads();
     tc_fence_after();
 
-    // --------------------------------------------------- phase 4: GEMM2
+    // --------------------------- phase 4: codes = H . W2^T (tokens x d_c)
     if (tid == 0) {
-      const uint32_t w0 = smem_u32(sW2);
-      const uint32_t idesc = idesc_f16_f32(enc::MMA_M, P.d_c);
+      const uint32_t w0 = smem_u32(sW2), h0 = smem_u32(sR);
+      const uint32_t idesc = idesc_f16_f32(enc::MMA_M, P.d_c) | (1u << 15);  // A MN-major
 #pragma unroll 1
-      for (int part = 0; part < 2; ++part) {
-        const uint32_t h0 = smem_u32(part == 0 ? sRH : sLo);
+      for (int part = 0; part < 2; ++part)
 #pragma unroll 1
-        for (int k16 = 0; k16 < P.hidden / 16; ++k16) {
-          const int atom = k16 >> 2, off = (k16 & 3) * 32;
-          umma_f16(tmem + enc::D2_COL, desc_kmajor_sw128(h0 + atom * enc::ATOM + off),
-                   desc_kmajor_sw128(w0 + atom * P.d_c * 128 + off), idesc, (part | k16) != 0);
+        for (int k16 = 0; k16 < hidden / 16; ++k16) {
+          // A: 16 hidden rows per step; the second 64-token block (rows of the
+          // M = 128 MMA that no token owns) reads the same rows again
+          const uint64_t ad = desc_mnmajor_sw128_enc(h0 + part * (uint32_t)h_part + k16 * 16 * 128, 0, 1024);
+          const uint64_t bd = desc_kmajor_sw128(w0 + (k16 >> 2) * P.d_c * 128 + (k16 & 3) * 32);
+          umma_f16(tmem + enc::D2_COL, ad, bd, idesc, (part | k16) != 0);
         }
-      }
       umma_commit(mma_bar);
     }
     if (!mbar_wait(mma_bar, mma_phase, abort_flag)) { ok = false; break; }
@@ -418,28 +455,31 @@ size_t encode_tc_smem(const Plan& p) {
   const int D = p.D, hidden = p.cfg.hidden, d_c = p.cfg.d_c;
   const int hid_atoms = (hidden + 63) / 64;
   const size_t w1 = (size_t)(D / 64) * hidden * 128;
+  const size_t rh = std::max(2 * (size_t)(D / 64) * enc::ROWS * 128, 2 * (size_t)hidden * 128);
   const size_t w2 = ((size_t)hid_atoms * d_c * 128 + 1023) & ~size_t(1023);
-  const size_t rh = 2 * (size_t)std::max(D / 64, hid_atoms) * enc::ATOM;
-  // the M = 128 reads of the last lo atom run 8 KB past it: W2 (and, when W2
-  // is shorter than that, the padding below) keeps them inside the block
-  const size_t tail = w2 < (size_t)enc::ATOM ? (size_t)enc::ATOM - w2 : 0;
-  return 1024 + w1 + rh + w2 + tail + 64;
+  return 1024 + w1 + rh + w2 + 64;
 }
 
 bool encode_tc_supported(const Plan& p) {
   const auto& c = p.cfg;
-  return c.dtype == DELTAKV_BF16 && (c.d_h == 64 || c.d_h == 128) && c.hidden % 32 == 0 &&
-         c.hidden <= 256 && c.d_c % 16 == 0 && c.d_c <= 256 && encode_tc_smem(p) <= 227 * 1024;
+  return c.dtype == DELTAKV_BF16 && (c.d_h == 64 || c.d_h == 128) && (c.hidden == 128 || c.hidden == 256) &&
+         c.d_c % 16 == 0 && c.d_c <= 256 && encode_tc_smem(p) <= 227 * 1024;
 }
 
 namespace {
-template <int EPL, int KC>
-cudaError_t encode_tc_launch(const EncParams& P, size_t smem, int grid, cudaStream_t st) {
-  auto kern = encode_tc_kernel<EPL, KC>;
+template <int EPL, int KC, int ACT>
+cudaError_t encode_tc_launch3(const EncParams& P, size_t smem, int grid, cudaStream_t st) {
+  auto kern = encode_tc_kernel<EPL, KC, ACT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   kern<<<grid, enc::THREADS, smem, st>>>(P);
   return cudaGetLastError();
+}
+template <int EPL, int KC>
+cudaError_t encode_tc_launch(const EncParams& P, size_t smem, int grid, cudaStream_t st) {
+  if (P.act == DELTAKV_ACT_GELU_ERF) return encode_tc_launch3<EPL, KC, DELTAKV_ACT_GELU_ERF>(P, smem, grid, st);
+  if (P.act == DELTAKV_ACT_GELU_TANH) return encode_tc_launch3<EPL, KC, DELTAKV_ACT_GELU_TANH>(P, smem, grid, st);
+  return encode_tc_launch3<EPL, KC, DELTAKV_ACT_NONE>(P, smem, grid, st);
 }
 }  // namespace
 
@@ -484,10 +524,10 @@ cudaError_t launch_encode_tc(const Plan& p, int T, const KVView& kv, const void*
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = std::min(P.n_tiles, sms);
   const size_t smem = encode_tc_smem(p);
-  ProfScope ps(p, st, KID_ENCODE);
+  ProfScope ps(p, st, KID_ENCODE_TC);
   if (c.d_h == 128)
-    return p.KC == 8 ? encode_tc_launch<8, 8>(P, smem, grid, st) : encode_tc_launch<8, 12>(P, smem, grid, st);
-  return p.KC == 8 ? encode_tc_launch<4, 8>(P, smem, grid, st) : encode_tc_launch<4, 12>(P, smem, grid, st);
+    return p.KC == 8 ? encode_tc_launch<32, 8>(P, smem, grid, st) : encode_tc_launch<32, 12>(P, smem, grid, st);
+  return p.KC == 8 ? encode_tc_launch<16, 8>(P, smem, grid, st) : encode_tc_launch<16, 12>(P, smem, grid, st);
 }
 
 }  // namespace dkv

@@ -24,8 +24,8 @@ constexpr size_t kErrBytes = 256;
 
 // Kernels the library launches (profiling ids).
 enum KernelId {
-  KID_REFPACK = 0, KID_CAND_SIMT, KID_CAND_TC, KID_ENCODE, KID_RECONSTRUCT, KID_DEC_REF,
-  KID_DEC_PREP, KID_DEC_STREAM, KID_DEC_COMBINE, KID_DEC_FINAL, KID_COUNT
+  KID_REFPACK = 0, KID_CAND_SIMT, KID_CAND_TC, KID_ENCODE_SIMT, KID_ENCODE_TC, KID_RECONSTRUCT, KID_DEC_REF,
+  KID_DEC_PREP, KID_DEC_STREAM_SIMT, KID_DEC_STREAM_TC, KID_DEC_COMBINE, KID_DEC_FINAL, KID_COUNT
 };
 const char* kernel_name(int id);
 

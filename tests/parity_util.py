@@ -88,6 +88,7 @@ class GpuResult:
     V_hat: np.ndarray
     out: np.ndarray      # [B,Hq,d_h] float64
     status: int
+    kernels: frozenset   # names of the library kernels that ran
 
 
 def run_gpu(c: Case, inp: Inputs, decode=True) -> GpuResult:
@@ -95,6 +96,7 @@ def run_gpu(c: Case, inp: Inputs, decode=True) -> GpuResult:
     cfg = dkv.Config(batch=c.B, kv_heads=c.H, q_heads=c.Hq, d_h=c.d_h, max_T=c.max_T or c.T,
                      stride_s=c.s, k=c.k, d_c=c.d_c, hidden=c.hidden, dtype=c.dtype, act=c.act)
     p = dkv.plan(cfg)
+    dkv.set_profiling(p, True)
     if c.strided:
         # K and V interleaved in one buffer [B, T+3, H, 2, d_h]: non-contiguous
         # batch/head/token strides
@@ -120,13 +122,14 @@ def run_gpu(c: Case, inp: Inputs, decode=True) -> GpuResult:
         dkv.decode_attention(p, c.T, q, cache, W["W3"], bias["b3"], W["W4"], bias["b4"], out, ws)
     status = dkv.device_status(p, ws)
     torch.cuda.synchronize()
+    kernels = frozenset(dkv.profile_collect(p))
     planes = p.cache_planes(cache)
     n_code = c.T - math.ceil(c.T / c.s)
     return GpuResult(
         idx=planes["idx"][:, :, :n_code].cpu().numpy(),
         code=planes["code"][:, :, :n_code].float().cpu().double().numpy(),
         K_hat=Kh.cpu().double().numpy(), V_hat=Vh.cpu().double().numpy(),
-        out=out.cpu().double().numpy(), status=status)
+        out=out.cpu().double().numpy(), status=status, kernels=kernels)
 
 
 @dataclasses.dataclass
@@ -201,7 +204,7 @@ def check_case(c: Case, decode=True, heads=None):
     assert g.status == 0, dkv.STATUS.get(g.status, g.status)
     tokens = non_ref_tokens(c.T, c.s)
     G = c.Hq // c.H
-    worst = {"recon_rel_l2": 0.0, "attn_max_abs": 0.0, "flagged": 0, "rows": 0}
+    worst = {"recon_rel_l2": 0.0, "attn_max_abs": 0.0, "flagged": 0, "rows": 0, "kernels": g.kernels}
     for b in range(c.B):
         for h in range(c.H):
             if heads is not None and (b, h) not in heads:

@@ -63,12 +63,30 @@ BF16_CASES = [
     ("ragged_capacity", Case(B=1, H=1, Hq=4, d_h=128, T=2500, s=32, k=4, d_c=32, hidden=256, dtype=dkv.BF16,
                              max_T=5000)),
     ("fp32_biases", Case(B=1, H=1, Hq=2, d_h=64, T=640, s=8, k=3, d_c=32, hidden=64, dtype=dkv.F32, biases=True)),
+    # shapes that take the tensor-core compressor and token loop
+    ("d_h64_tc", Case(B=1, H=2, Hq=4, d_h=64, T=3001, s=8, k=4, d_c=64, hidden=256, dtype=dkv.BF16)),
+    ("biases_tanh_tc", Case(B=1, H=2, Hq=8, d_h=128, T=2600, s=16, k=3, d_c=16, hidden=128, dtype=dkv.BF16,
+                            act=dkv.ACT_GELU_TANH, biases=True)),
+    ("identity_act_tc", Case(B=1, H=1, Hq=2, d_h=64, T=1800, s=4, k=2, d_c=32, hidden=128, dtype=dkv.BF16,
+                             act=dkv.ACT_NONE, biases=True)),
 ]
+
+# kernels each case must have run: the tensor-core paths where the shape allows
+TC_EXPECT = {
+    "base": {"candidates_tc", "encode_tc", "decode_stream_tc"},
+    "k8_dc64": {"encode_tc"},
+    "ragged_capacity": {"candidates_tc", "encode_tc", "decode_stream_tc"},
+    "d_h64_tc": {"candidates_tc", "encode_tc", "decode_stream_tc"},
+    "biases_tanh_tc": {"candidates_tc", "encode_tc", "decode_stream_tc"},
+    "identity_act_tc": {"encode_tc", "decode_stream_simt"},
+}
 
 
 @pytest.mark.parametrize("name,case", BF16_CASES, ids=[n for n, _ in BF16_CASES])
 def test_variants(name, case):
-    check_case(case)
+    w = check_case(case)
+    missing = TC_EXPECT.get(name, set()) - w["kernels"]
+    assert not missing, f"{name}: expected kernels did not run: {sorted(missing)} (ran {sorted(w['kernels'])})"
 
 
 def test_t1_output_is_the_single_value():
