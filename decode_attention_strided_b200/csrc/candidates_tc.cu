@@ -17,12 +17,16 @@
 // Warp roles (320 threads, one CTA per SM, persistent):
 //   warps 0-7  epilogue: warp w owns token tile w / 4, TMEM lanes 32 (w % 4)..
 //   warp 8     TMA producer: A tiles (tokens) and B stages (references)
-//   warp 9     MMA issuer: M=128, N=64, K=16 tcgen05.mma, fp32 in TMEM
-// TMEM: 512 columns = 4 buffers x 2 token tiles x 64 reference columns, so
-// the MMAs run up to three reference tiles ahead of the epilogue.
+//   warp 9     MMA issuer: M=128, N=128, K=16 tcgen05.mma, fp32 in TMEM
+// TMEM: 512 columns = 2 buffers x 2 token tiles x 128 reference columns, so
+// the MMAs fill one reference tile while the epilogue drains the other.
+// Shape choice: an M = 128 MMA occupies the tensor pipe for at least about
+// 58 cycles whatever its N, and a commit costs a pipeline drain unless the
+// MMAs before it cover it; N = 128 (64 cycles of math per MMA) and one commit
+// per 8 MMAs (512 cycles) keep the pipe math-bound.
 // A and B live in shared memory in the 128-byte-swizzled K-major layout the
 // TMA writes; a 64-element column of a 128-row token tile is one 16 KB atom,
-// of a 64-row reference tile one 8 KB atom.
+// and so is one of a 128-row reference tile.
 //
 // Epilogue: each thread owns one token row, so a warp carries 32 unrelated
 // running top-k lists.  Per 32 columns it builds a bitmask of the values below
@@ -42,13 +46,14 @@ using namespace sm100;
 
 namespace tcc {
 constexpr int TM = 128;                     // tokens per tile (MMA M)
-constexpr int TPU = 2;                      // token tiles per unit
-constexpr int RN = 64;                      // references per tile (MMA N)
-constexpr int NBUF = 4;                     // TMEM accumulator buffers
-constexpr int STAGES = 8;                   // reference pipeline depth (atoms)
+constexpr int TPU = 2;                      // token tiles per unit (the epilogue selects between the two)
+constexpr int RN = 128;                     // references per tile (MMA N)
+constexpr int NBUF = 2;                     // TMEM accumulator buffers
+constexpr int STAGES = 5;                   // reference pipeline depth (atoms)
 constexpr int ATOM = TM * 128;              // bytes: 128 token rows x 128 B
 constexpr int BATOM = RN * 128;             // bytes: 64 reference rows x 128 B
-constexpr int SPILL = 32 * 32 * 4;          // bytes per warp: 32 lanes x 32 floats
+constexpr int CHUNK = 16;                   // columns per slow-path chunk
+constexpr int SPILL = 32 * CHUNK * 4;       // bytes per warp: 32 lanes x CHUNK floats
 constexpr int EPI_WARPS = 8;
 constexpr int THREADS = (EPI_WARPS + 2) * 32;
 constexpr uint32_t TMEM_COLS = 512;
@@ -216,17 +221,18 @@ __global__ void __launch_bounds__(tcc::THREADS, 1)
             if (!mbar_wait(&b_full[st], (b_it / tcc::STAGES) & 1, abort_flag)) { ok = false; break; }
             if (r == 0 && !mbar_wait(&a_full[kc], a_it & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
+            // the two token tiles alternate, so consecutive MMAs never chain
+            // on one accumulator
 #pragma unroll
-            for (int i = 0; i < tcc::TPU; ++i) {
-              if (r >= u.R[i]) continue;
-              const uint32_t d = tmem + buf * (tcc::TPU * tcc::RN) + i * tcc::RN;
+            for (int k16 = 0; k16 < 4; ++k16)
 #pragma unroll
-              for (int k16 = 0; k16 < 4; ++k16) {
+              for (int i = 0; i < tcc::TPU; ++i) {
+                if (r >= u.R[i]) continue;
+                const uint32_t d = tmem + buf * (tcc::TPU * tcc::RN) + i * tcc::RN;
                 const uint64_t ad = desc_kmajor_sw128(a_base + (i * NKC + kc) * tcc::ATOM + k16 * 32);
                 const uint64_t bd = desc_kmajor_sw128(b_base + st * tcc::BATOM + k16 * 32);
                 umma_f16(d, ad, bd, idesc, (kc | k16) != 0);
               }
-            }
             umma_commit(&b_empty[st]);
             if (r == u.Rmax - 1) umma_commit(&a_empty[kc]);
           }
@@ -242,8 +248,8 @@ __global__ void __launch_bounds__(tcc::THREADS, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int ti = warp / 4, q = warp % 4, row = q * 32 + lane;
-    float* sp = spill + warp * (32 * 32) + lane * 32;  // this lane's 32 floats
-    const int sw = lane & 7;                            // float4 swizzle of the slot
+    float* sp = spill + warp * (32 * tcc::CHUNK) + lane * tcc::CHUNK;  // this lane's CHUNK floats
+    const int sw = (lane >> 1) & 3;  // float4 swizzle: 8 lanes of a phase hit 8 distinct bank groups
     uint32_t acc_it = 0;
     bool ok = true;
     UnitInfo u;
@@ -254,64 +260,84 @@ __global__ void __launch_bounds__(tcc::THREADS, 1)
       const int cnt = t < P.T ? min((t + P.s - 1) / P.s, P.n_ref) : 0;  // valid slots j < cnt
       const int cnt_lo = min((first + P.s - 1) / P.s, P.n_ref);         // smallest cnt in the tile
       const float* hn = P.hnorm + (int64_t)u.bh * P.n_ref_cap;
+      const int R_mine = ti == 0 ? u.R[0] : u.R[1];
       float bd[KC];
       int bi[KC];
 #pragma unroll
       for (int x = 0; x < KC; ++x) { bd[x] = FLT_MAX; bi[x] = INT_MAX; }
       for (int r = 0; r < u.Rmax; ++r, ++acc_it) {
         const uint32_t buf = acc_it % tcc::NBUF;
-        const bool mine = r < u.R[ti];
-        const int jb = r * tcc::RN;
-        float v[tcc::RN];
         if (!mbar_wait(&acc_full[buf], (acc_it / tcc::NBUF) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        if (mine)
-          tmem_ld64(tmem + ((uint32_t)(q * 32) << 16) + buf * (tcc::TPU * tcc::RN) + ti * tcc::RN, v);
-        // the accumulator is in registers: hand the buffer back to the MMA warp
+        if (r < R_mine) {
+#pragma unroll 1
+          for (int hf = 0; hf < tcc::RN / 64; ++hf) {
+            const int jb = r * tcc::RN + hf * 64;
+            float v[64];
+            tmem_ld64(tmem + ((uint32_t)(q * 32) << 16) + buf * (tcc::TPU * tcc::RN) + ti * tcc::RN + hf * 64, v);
+            // e = |r_j|^2 / 2 - <x_t, r_j>
+            const float4* h4 = reinterpret_cast<const float4*>(hn + jb);
+#pragma unroll
+            for (int x4 = 0; x4 < 16; ++x4) {
+              const float4 t4 = __ldg(h4 + x4);
+              v[4 * x4] = t4.x - v[4 * x4];
+              v[4 * x4 + 1] = t4.y - v[4 * x4 + 1];
+              v[4 * x4 + 2] = t4.z - v[4 * x4 + 2];
+              v[4 * x4 + 3] = t4.w - v[4 * x4 + 3];
+            }
+            if (jb + 64 > cnt_lo) {
+#pragma unroll
+              for (int x = 0; x < 64; ++x)
+                if (jb + x >= cnt) v[x] = FLT_MAX;
+            }
+            if (r == 0 && hf == 0) {
+              // first block of the unit: every list is empty, so every lane
+              // takes every value -- insert them all without branching
+#pragma unroll
+              for (int x = 0; x < 64; ++x) topk_insert_inorder<KC>(bd, bi, v[x], jb + x);
+              continue;
+            }
+            // fast path: most blocks hold nothing below any lane's k-th best
+            float mn[32];
+#pragma unroll
+            for (int x = 0; x < 32; ++x) mn[x] = fminf(v[x], v[x + 32]);
+#pragma unroll
+            for (int w = 16; w >= 1; w >>= 1)
+#pragma unroll
+              for (int x = 0; x < w; ++x) mn[x] = fminf(mn[x], mn[x + w]);
+            if (!__any_sync(0xffffffffu, mn[0] < bd[KC - 1])) continue;
+#pragma unroll
+            for (int c = 0; c < 64 / tcc::CHUNK; ++c) {
+              const float thr = bd[KC - 1];
+              // four independent partial masks keep the dependency chains short
+              uint32_t mp[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+              for (int x = 0; x < tcc::CHUNK; ++x) mp[x & 3] |= (v[c * tcc::CHUNK + x] < thr ? 1u : 0u) << x;
+              uint32_t m = (mp[0] | mp[1]) | (mp[2] | mp[3]);
+              if (__any_sync(0xffffffffu, m != 0)) {
+                if (m) {
+#pragma unroll
+                  for (int i4 = 0; i4 < tcc::CHUNK / 4; ++i4)
+                    reinterpret_cast<float4*>(sp)[i4 ^ sw] =
+                        make_float4(v[c * tcc::CHUNK + 4 * i4], v[c * tcc::CHUNK + 4 * i4 + 1],
+                                    v[c * tcc::CHUNK + 4 * i4 + 2], v[c * tcc::CHUNK + 4 * i4 + 3]);
+                }
+                __syncwarp();
+                while (m) {
+                  const int x = __ffs(m) - 1;
+                  m &= m - 1;
+                  const float vx = sp[(((x >> 2) ^ sw) << 2) | (x & 3)];
+                  topk_insert_inorder<KC>(bd, bi, vx, jb + c * tcc::CHUNK + x);
+                }
+                __syncwarp();
+              }
+            }
+          }
+        }
+        // the buffer is drained: hand it back to the MMA warp
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[buf]);
-        if (!mine) continue;
-        const bool need_mask = jb + tcc::RN > cnt_lo;
-        // e = |r_j|^2 / 2 - <x_t, r_j>
-        const float4* h4 = reinterpret_cast<const float4*>(hn + jb);
-#pragma unroll
-        for (int x4 = 0; x4 < tcc::RN / 4; ++x4) {
-          const float4 t4 = __ldg(h4 + x4);
-          v[4 * x4] = t4.x - v[4 * x4];
-          v[4 * x4 + 1] = t4.y - v[4 * x4 + 1];
-          v[4 * x4 + 2] = t4.z - v[4 * x4 + 2];
-          v[4 * x4 + 3] = t4.w - v[4 * x4 + 3];
-        }
-        if (need_mask) {
-#pragma unroll
-          for (int x = 0; x < tcc::RN; ++x)
-            if (jb + x >= cnt) v[x] = FLT_MAX;
-        }
-#pragma unroll
-        for (int c = 0; c < tcc::RN / 32; ++c) {
-          const float thr = bd[KC - 1];
-          uint32_t m = 0;
-#pragma unroll
-          for (int x = 0; x < 32; ++x) m |= (v[c * 32 + x] < thr ? 1u : 0u) << x;
-          if (__any_sync(0xffffffffu, m != 0)) {
-            if (m) {
-#pragma unroll
-              for (int i4 = 0; i4 < 8; ++i4)
-                reinterpret_cast<float4*>(sp)[i4 ^ sw] =
-                    make_float4(v[c * 32 + 4 * i4], v[c * 32 + 4 * i4 + 1], v[c * 32 + 4 * i4 + 2],
-                                v[c * 32 + 4 * i4 + 3]);
-            }
-            __syncwarp();
-            while (m) {
-              const int x = __ffs(m) - 1;
-              m &= m - 1;
-              const float vx = sp[(((x >> 2) ^ sw) << 2) | (x & 3)];
-              if (vx < bd[KC - 1]) topk_insert<KC>(bd, bi, vx, jb + c * 32 + x);
-            }
-            __syncwarp();
-          }
-        }
       }
       if (ok && t < P.T && (t % P.s) != 0) {
         int32_t* o = P.cand + ((int64_t)u.bh * P.n_code_cap + (t - t / P.s - 1)) * KC;

@@ -82,6 +82,26 @@ __device__ __forceinline__ void topk_insert(float (&bd)[KC], int (&bi)[KC], floa
   }
 }
 
+// Insert (d, j) into a list kept in ascending order, for a caller that offers
+// slots in increasing order (so an equal distance ranks after every entry
+// already held).  Each new entry is computed from the old list directly --
+// eight comparisons and selects with no chain between positions -- so the
+// insertion has a short dependency depth.  No-op when d is not below the
+// last entry.
+template <int KC>
+__device__ __forceinline__ void topk_insert_inorder(float (&bd)[KC], int (&bi)[KC], float d, int j) {
+  bool lt[KC];
+#pragma unroll
+  for (int i = 0; i < KC; ++i) lt[i] = d < bd[i];
+#pragma unroll
+  for (int i = KC - 1; i > 0; --i) {
+    bd[i] = lt[i - 1] ? bd[i - 1] : (lt[i] ? d : bd[i]);
+    bi[i] = lt[i - 1] ? bi[i - 1] : (lt[i] ? j : bi[i]);
+  }
+  bd[0] = lt[0] ? d : bd[0];
+  bi[0] = lt[0] ? j : bi[0];
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
