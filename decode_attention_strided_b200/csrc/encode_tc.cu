@@ -40,11 +40,17 @@ namespace dkv {
 using namespace sm100;
 
 namespace enc {
-constexpr int ROWS = 64;       // compressed rows per tile (the MMA runs M = 128)
+constexpr int ROWS = 64;          // compressed rows per tile (GEMM1^T N; GEMM2 runs M = 128)
 constexpr int MMA_M = 128;
-constexpr int THREADS = 256;
+constexpr int GATHER_WARPS = 8;   // warps 0-7: re-rank, mean, residual
+constexpr int ACT0 = 8;           // warps 8-11: activation and code store (one per TMEM lane quarter)
+constexpr int ACT_WARPS = 4;
+constexpr int MMA_WARP = 12;      // warp 12: TMEM allocation and MMA issue
+constexpr int THREADS = 13 * 32;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t D2_COL = 256;  // TMEM column of the second accumulator
+constexpr uint32_t W1_COL = 0;    // W1 halves, D/2 packed columns each
+constexpr uint32_t D1_COL = 256;  // GEMM1^T accumulators, 64 columns per half
+constexpr uint32_t D2_COL = 384;  // GEMM2 accumulator, d_c columns
 }  // namespace enc
 
 // tcgen05 kind::f16 instruction descriptor, fp16 A/B, fp32 D, K-major.
@@ -119,11 +125,10 @@ struct EncParams {
   int n_tiles, tiles_per_bh;
 };
 
-// EPL: elements of [K ; V] per lane with 8 lanes per row (D / 8);
-// KC: candidates per token; ACT: activation; HAS_B: biases present.
+// EPL: elements of [K ; V] per lane with 16 lanes per row (D / 16).
 template <int EPL> struct RowPack;
-template <> struct RowPack<32> { static constexpr int V4 = 4; };  // 4 x 16 B
 template <> struct RowPack<16> { static constexpr int V4 = 2; };  // 2 x 16 B
+template <> struct RowPack<8> { static constexpr int V4 = 1; };   // 1 x 16 B
 
 template <int EPL>
 __device__ __forceinline__ void load_row(const __nv_bfloat16* src, uint4 (&r)[RowPack<EPL>::V4]) {
@@ -145,12 +150,16 @@ __device__ __forceinline__ void unpack_row(const uint4 (&r)[RowPack<EPL>::V4], f
   }
 }
 
-__device__ __forceinline__ float group8_sum(float v) {
-  v += __shfl_xor_sync(0xffffffffu, v, 4, 8);
-  v += __shfl_xor_sync(0xffffffffu, v, 2, 8);
-  v += __shfl_xor_sync(0xffffffffu, v, 1, 8);
+__device__ __forceinline__ float group16_sum(float v) {
+  v += __shfl_xor_sync(0xffffffffu, v, 8, 16);
+  v += __shfl_xor_sync(0xffffffffu, v, 4, 16);
+  v += __shfl_xor_sync(0xffffffffu, v, 2, 16);
+  v += __shfl_xor_sync(0xffffffffu, v, 1, 16);
   return v;
 }
+
+// Candidate rows loaded together: all of them when there are 8, else 4.
+template <int KC> struct CandBatch { static constexpr int N = KC == 8 ? 8 : 4; };
 
 template <int ACT>
 __device__ __forceinline__ float enc_act(float v) {
@@ -158,58 +167,116 @@ __device__ __forceinline__ float enc_act(float v) {
   return act_eval(ACT, v);
 }
 
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// D[tmem] (+)= A[tmem] * B[smem desc]^T, kind::f16, A read from tensor memory
+// (lane m = row m; 32-bit column c holds K elements 2c (low half) and 2c + 1).
+__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Row n of a 64-row tile: its code row, token and this lane's x slice.
+struct GatherRow {
+  int64_t row, t;
+  const __nv_bfloat16* x;  // this lane's slice of x_t (valid when live)
+  const int32_t* cand;     // the row's candidate slots
+  bool live;
+};
+
+template <int KC>
+__device__ __forceinline__ GatherRow gather_row(const EncParams& P, int tile, int n, bool inK, int e0) {
+  GatherRow g;
+  const int bh = tile / P.tiles_per_bh;
+  g.row = (int64_t)(tile % P.tiles_per_bh) * enc::ROWS + n;
+  g.live = g.row < P.n_code;
+  g.t = g.live ? (g.row / (P.s - 1)) * P.s + (g.row % (P.s - 1)) + 1 : 0;
+  const int b = bh / P.H, h = bh % P.H;
+  g.x = (inK ? P.K + e0 : P.V + (e0 - P.d_h)) + b * P.sb + h * P.sh + g.t * P.st;
+  g.cand = P.cand + ((int64_t)bh * P.n_code_cap + g.row) * KC;
+  return g;
+}
+
+template <int EPL, int KC>
+__device__ __forceinline__ void gather_prefetch(const EncParams& P, const GatherRow& g, int s16,
+                                                uint4 (&x)[RowPack<EPL>::V4], int& c) {
+  if (g.live) {
+    load_row<EPL>(g.x, x);
+  } else {
+#pragma unroll
+    for (int i = 0; i < RowPack<EPL>::V4; ++i) x[i] = make_uint4(0, 0, 0, 0);
+  }
+  c = (g.live && s16 < KC) ? g.cand[s16] : -1;
+}
+
+struct EncBars {
+  uint64_t r_full[2], r_empty[2], d1_full, d1_empty, h_full, h_empty, d2_full, d2_empty;
+};
+
 template <int EPL, int KC, int ACT>
 __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncParams P) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  constexpr int D = EPL * 8;
+  constexpr int D = EPL * 16;
   constexpr int KA = D / 64;                       // 64-column atoms along D
-  const int hidden = P.hidden, hid_atoms = (hidden + 63) / 64;
-  // shared memory: W1 [hidden rows][D] K-major (A of GEMM1^T), then the
-  // R tile (B of GEMM1^T: 64 token rows x D, hi atoms then lo atoms) which
-  // the H tile (A of GEMM2, MN-major: hidden rows x 64 tokens, hi then lo)
-  // later overwrites, then W2 [d_c rows][hidden] K-major (B of GEMM2)
-  unsigned char* sW1 = smem;
-  unsigned char* sR = sW1 + (size_t)KA * hidden * 128;
+  const int hidden = P.hidden, nh = hidden / 128, hid_atoms = hidden / 64;
+  // shared memory: two R tiles (B of GEMM1^T: 64 token rows x D, K-major,
+  // hi atoms then lo atoms), the H tile (A of GEMM2, MN-major: hidden rows x
+  // 64 tokens, hi then lo), W2 [d_c rows][hidden] K-major (B of GEMM2)
   const size_t r_part = (size_t)KA * enc::ROWS * 128;          // one of hi / lo
   const size_t h_part = (size_t)hidden * 128;                  // one of hi / lo
-  const size_t rh_b = r_part > h_part ? 2 * r_part : 2 * h_part;
-  unsigned char* sW2 = sR + rh_b;
-  uint64_t* mma_bar = (uint64_t*)(sW2 + (((size_t)hid_atoms * P.d_c * 128 + 1023) & ~size_t(1023)));
-  uint32_t* tmem_slot = (uint32_t*)(mma_bar + 1);
+  unsigned char* sR = smem;                                    // [2][hi, lo]
+  unsigned char* sH = sR + 4 * r_part;
+  unsigned char* sW2 = sH + 2 * h_part;
+  EncBars* bars = (EncBars*)(sW2 + (((size_t)hid_atoms * P.d_c * 128 + 1023) & ~size_t(1023)));
+  uint32_t* tmem_slot = (uint32_t*)(bars + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
 
-  // ---- weights -> fp16 (bf16 values are exact in fp16), swizzled K-major
-  for (int i = tid; i < hidden * D / 8; i += blockDim.x) {
-    const int n = i / (D / 8), c8 = (i % (D / 8)) * 8;
-    const uint4 raw = *reinterpret_cast<const uint4*>(P.W1 + (int64_t)n * D + c8);
+  // W2 -> fp16, swizzled K-major (bf16 values of normal range are exact in fp16)
+  for (int i = tid; i < P.d_c * hid_atoms * 8; i += blockDim.x) {
+    const int o = i / (hid_atoms * 8), c8 = (i % (hid_atoms * 8)) * 8;
+    const uint4 raw = *reinterpret_cast<const uint4*>(P.W2 + (int64_t)o * hidden + c8);
     const __nv_bfloat162* b2v = reinterpret_cast<const __nv_bfloat162*>(&raw);
     uint4 out;
     __half2* o2 = reinterpret_cast<__half2*>(&out);
 #pragma unroll
     for (int q = 0; q < 4; ++q) o2[q] = __float22half2_rn(__bfloat1622float2(b2v[q]));
-    *reinterpret_cast<uint4*>(sW1 + sw128_offset(n, c8, hidden)) = out;
-  }
-  for (int i = tid; i < P.d_c * hid_atoms * 8; i += blockDim.x) {
-    const int o = i / (hid_atoms * 8), c8 = (i % (hid_atoms * 8)) * 8;
-    uint4 out = make_uint4(0, 0, 0, 0);
-    if (c8 < hidden) {
-      const uint4 raw = *reinterpret_cast<const uint4*>(P.W2 + (int64_t)o * hidden + c8);
-      const __nv_bfloat162* b2v = reinterpret_cast<const __nv_bfloat162*>(&raw);
-      __half2* o2 = reinterpret_cast<__half2*>(&out);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) o2[q] = __float22half2_rn(__bfloat1622float2(b2v[q]));
-    }
     *reinterpret_cast<uint4*>(sW2 + sw128_offset(o, c8, P.d_c)) = out;
   }
   if (tid == 0) {
-    mbar_init(mma_bar, 1);
+    mbar_init(&bars->r_full[0], enc::GATHER_WARPS);
+    mbar_init(&bars->r_full[1], enc::GATHER_WARPS);
+    mbar_init(&bars->r_empty[0], 1);
+    mbar_init(&bars->r_empty[1], 1);
+    mbar_init(&bars->d1_full, 1);
+    mbar_init(&bars->d1_empty, enc::ACT_WARPS);
+    mbar_init(&bars->h_full, enc::ACT_WARPS);
+    mbar_init(&bars->h_empty, 1);
+    mbar_init(&bars->d2_full, 1);
+    mbar_init(&bars->d2_empty, enc::ACT_WARPS);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0) {
+  if (warp == enc::MMA_WARP) {
     tmem_alloc(tmem_slot, enc::TMEM_COLS);
     tmem_relinquish();
   }
@@ -218,234 +285,311 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  uint32_t mma_phase = 0;
-  bool ok = true;
 
-  const int grp = lane >> 3, s8 = lane & 7;   // row within the warp's 4, lane within the row
-  const int e0 = s8 * EPL;                     // this lane's first element of [K ; V]
-  const bool inK = e0 < P.d_h;
+  // tiles of this CTA: blockIdx.x, blockIdx.x + gridDim.x, ...
+  const int n_local = P.n_tiles > (int)blockIdx.x ? (P.n_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
 
-  for (int tile = blockIdx.x; tile < P.n_tiles && ok; tile += gridDim.x) {
-    const int bh = tile / P.tiles_per_bh;
-    const int64_t row0 = (int64_t)(tile % P.tiles_per_bh) * enc::ROWS;
-    const int b = bh / P.H, h = bh % P.H;
-    const __nv_bfloat16* Kb = P.K + b * P.sb + h * P.sh;
-    const __nv_bfloat16* Vb = P.V + b * P.sb + h * P.sh;
-    const __nv_bfloat16* rk = P.refk + (int64_t)bh * P.n_ref_cap * P.d_h;
-    const __nv_bfloat16* rv = P.refv + (int64_t)bh * P.n_ref_cap * P.d_h;
-
-    // ------------------------------- phase 1: re-rank, mean, residual (8 lanes / row)
-    for (int n = warp * 4 + grp; n < enc::ROWS; n += 32) {
-      const int64_t row = row0 + n;
-      const bool live = row < P.n_code;
-      const int64_t t = live ? (row / (P.s - 1)) * P.s + (row % (P.s - 1)) + 1 : 0;
-      const int32_t* cr = P.cand + ((int64_t)bh * P.n_code_cap + row) * KC;
-      const int myc0 = (live && s8 < KC) ? cr[s8] : -1;
-      const int myc1 = (live && s8 + 8 < KC) ? cr[s8 + 8] : -1;
-      float xv[EPL];
-      {
-        uint4 xr[RowPack<EPL>::V4];
-        if (live) load_row<EPL>(inK ? Kb + t * P.st + e0 : Vb + t * P.st + (e0 - P.d_h), xr);
-        else
+  if (warp >= enc::ACT0 && warp < enc::ACT0 + enc::ACT_WARPS) {
+    // W1 -> tensor memory, fp16: A of GEMM1^T, half hh at columns
+    // W1_COL + hh D/2, lane = hidden unit within the half
+    const int q = warp - enc::ACT0;
+    for (int hh = 0; hh < nh; ++hh) {
+      const __nv_bfloat16* wrow = P.W1 + (int64_t)(hh * 128 + q * 32 + lane) * D;
+#pragma unroll 1
+      for (int c0 = 0; c0 < D / 2; c0 += 32) {
+        uint32_t r[32];
 #pragma unroll
-          for (int i = 0; i < RowPack<EPL>::V4; ++i) xr[i] = make_uint4(0, 0, 0, 0);
-        unpack_row<EPL>(xr, xv);
-      }
-      int cj[KC];
-      float cd[KC];
+        for (int v = 0; v < 8; ++v) {
+          const uint4 raw = __ldg(reinterpret_cast<const uint4*>(wrow + 2 * c0) + v);
+          const __nv_bfloat162* b2v = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
-      for (int c = 0; c < KC; ++c) {
-        int j = c < 8 ? __shfl_sync(0xffffffffu, myc0, c, 8) : __shfl_sync(0xffffffffu, myc1, c - 8, 8);
-        if (j >= 0 && (int64_t)j * P.s >= t) {  // not an earlier reference: drop it
-          if (s8 == 0) latch_error(P.err, DELTAKV_ERR_DEVICE_BOUNDS, (uint32_t)j);
-          j = -1;
-        }
-        cj[c] = j;
-      }
-      // exact distances, 4 candidate rows in flight at a time
-#pragma unroll
-      for (int c0 = 0; c0 < KC; c0 += 4) {
-        uint4 rr[4][RowPack<EPL>::V4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int j = cj[c0 + u];
-          if (j >= 0) load_row<EPL>(inK ? rk + (int64_t)j * P.d_h + e0 : rv + (int64_t)j * P.d_h + (e0 - P.d_h), rr[u]);
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          float part = 0.f;
-          if (cj[c0 + u] >= 0) {
-            float rf[EPL];
-            unpack_row<EPL>(rr[u], rf);
-#pragma unroll
-            for (int q = 0; q < EPL; ++q) {
-              const float df = xv[q] - rf[q];
-              part = fmaf(df, df, part);
-            }
-          }
-          part = group8_sum(part);
-          cd[c0 + u] = cj[c0 + u] >= 0 ? part : FLT_MAX;
-        }
-      }
-      // the k smallest (distance, slot), ascending
-      uint32_t chosen = 0;
-      int k_eff = 0, my_sel = -1;
-      for (int qk = 0; qk < P.k; ++qk) {
-        int best = -1;
-        float bdv = FLT_MAX;
-        int bj = INT_MAX;
-#pragma unroll
-        for (int c = 0; c < KC; ++c) {
-          const bool avail = cj[c] >= 0 && !(chosen & (1u << c));
-          if (avail && (cd[c] < bdv || (cd[c] == bdv && cj[c] < bj))) {
-            best = c;
-            bdv = cd[c];
-            bj = cj[c];
+          for (int x = 0; x < 4; ++x) {
+            __half2 h2 = __float22half2_rn(__bfloat1622float2(b2v[x]));
+            r[4 * v + x] = *reinterpret_cast<uint32_t*>(&h2);
           }
         }
-        if (best >= 0) {
-          chosen |= 1u << best;
-          ++k_eff;
-        }
-        if (s8 == qk) my_sel = best >= 0 ? bj : -1;
-      }
-      if (live && s8 < P.k) P.idx[((int64_t)bh * P.n_code_cap + row) * P.k + s8] = my_sel;
-      // mean of the chosen rows (reloaded: they are in L2), residual
-      float m[EPL];
-#pragma unroll
-      for (int q = 0; q < EPL; ++q) m[q] = 0.f;
-#pragma unroll
-      for (int c = 0; c < KC; ++c) {
-        if (chosen & (1u << c)) {
-          const int j = cj[c];
-          uint4 rr[RowPack<EPL>::V4];
-          load_row<EPL>(inK ? rk + (int64_t)j * P.d_h + e0 : rv + (int64_t)j * P.d_h + (e0 - P.d_h), rr);
-          float rf[EPL];
-          unpack_row<EPL>(rr, rf);
-#pragma unroll
-          for (int q = 0; q < EPL; ++q) m[q] += rf[q];
-        }
-      }
-      const float inv = 1.0f / (float)max(k_eff, 1);
-      // r = hi + lo (fp16) into the R tile: row n, columns e0 .. e0 + EPL
-#pragma unroll
-      for (int v = 0; v < EPL / 8; ++v) {
-        __half2 hi2[4], lo2[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int i = 8 * v + 2 * q;
-          const float r0 = live ? xv[i] - m[i] * inv : 0.f;
-          const float r1 = live ? xv[i + 1] - m[i + 1] * inv : 0.f;
-          split_half2(r0, r1, hi2[q], lo2[q]);
-        }
-        const uint32_t off = sw128_offset(n, e0 + 8 * v, enc::ROWS);
-        *reinterpret_cast<uint4*>(sR + off) = *reinterpret_cast<const uint4*>(hi2);
-        *reinterpret_cast<uint4*>(sR + r_part + off) = *reinterpret_cast<const uint4*>(lo2);
+        tmem_st32(tmem + ((uint32_t)(q * 32) << 16) + enc::W1_COL + hh * (D / 2) + c0, r);
       }
     }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-
-    // ------------------------------ phase 2: D1^T = W1 . R^T (hidden x tokens)
-    if (tid == 0) {
-      const uint32_t w0 = smem_u32(sW1), r0 = smem_u32(sR);
-      const uint32_t idesc = idesc_f16_f32(128, enc::ROWS);
-#pragma unroll 1
-      for (int hh = 0; hh < hidden / 128; ++hh)
-#pragma unroll 1
-        for (int part = 0; part < 2; ++part)
-#pragma unroll 1
-          for (int k16 = 0; k16 < D / 16; ++k16) {
-            const int atom = k16 >> 2, off = (k16 & 3) * 32;
-            umma_f16(tmem + enc::ROWS * hh,
-                     desc_kmajor_sw128(w0 + atom * hidden * 128 + hh * 128 * 128 + off),
-                     desc_kmajor_sw128(r0 + part * (uint32_t)r_part + atom * enc::ROWS * 128 + off), idesc,
-                     (part | k16) != 0);
-          }
-      umma_commit(mma_bar);
-    }
-    if (!mbar_wait(mma_bar, mma_phase, abort_flag)) { ok = false; break; }
-    mma_phase ^= 1;
-    tc_fence_after();
-
-    // ---------------- phase 3: H = act(D1 + b1), hidden rows x 64 tokens (all 8 warps)
-    if (warp < 4 * (hidden / 128)) {
-      const int q = warp & 3, hh = warp >> 2;
-      const int unit = 128 * hh + 32 * q + lane;
-      const float bias = P.b1 ? P.b1[unit] : 0.f;
-      float v[64];
-      tmem_ld64(tmem + ((uint32_t)(32 * q) << 16) + enc::ROWS * hh, v);
-#pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8) {
-        __half2 hi2[4], lo2[4];
-#pragma unroll
-        for (int x = 0; x < 4; ++x)
-          split_half2(enc_act<ACT>(v[8 * c8 + 2 * x] + bias), enc_act<ACT>(v[8 * c8 + 2 * x + 1] + bias), hi2[x],
-                      lo2[x]);
-        // MN-major row `unit` of 64 tokens: 16-byte chunk c8, swizzled by row
-        const uint32_t off = (uint32_t)unit * 128 + (((c8 ^ (unit & 7))) << 4);
-        *reinterpret_cast<uint4*>(sR + off) = *reinterpret_cast<const uint4*>(hi2);
-        *reinterpret_cast<uint4*>(sR + h_part + off) = *reinterpret_cast<const uint4*>(lo2);
-      }
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-
-    // --------------------------- phase 4: codes = H . W2^T (tokens x d_c)
-    if (tid == 0) {
-      const uint32_t w0 = smem_u32(sW2), h0 = smem_u32(sR);
-      const uint32_t idesc = idesc_f16_f32(enc::MMA_M, P.d_c) | (1u << 15);  // A MN-major
-#pragma unroll 1
-      for (int part = 0; part < 2; ++part)
-#pragma unroll 1
-        for (int k16 = 0; k16 < hidden / 16; ++k16) {
-          // A: 16 hidden rows per step; the second 64-token block (rows of the
-          // M = 128 MMA that no token owns) reads the same rows again
-          const uint64_t ad = desc_mnmajor_sw128_enc(h0 + part * (uint32_t)h_part + k16 * 16 * 128, 0, 1024);
-          const uint64_t bd = desc_kmajor_sw128(w0 + (k16 >> 2) * P.d_c * 128 + (k16 & 3) * 32);
-          umma_f16(tmem + enc::D2_COL, ad, bd, idesc, (part | k16) != 0);
-        }
-      umma_commit(mma_bar);
-    }
-    if (!mbar_wait(mma_bar, mma_phase, abort_flag)) { ok = false; break; }
-    mma_phase ^= 1;
-    tc_fence_after();
-
-    // ----------------------------------------- phase 5: codes = D2 + b2
-    if (warp < 2) {
-      const int n = warp * 32 + lane;
-      const int64_t row = row0 + n;
-      for (int c0 = 0; c0 < P.d_c; c0 += 16) {
-        float v[16];
-        tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + enc::D2_COL + c0, v);
-        if (row < P.n_code) {
-          uint4 o[2];
-          __nv_bfloat162* o2 = reinterpret_cast<__nv_bfloat162*>(o);
-#pragma unroll
-          for (int x = 0; x < 8; ++x)
-            o2[x] = __floats2bfloat162_rn(v[2 * x] + (P.b2 ? P.b2[c0 + 2 * x] : 0.f),
-                                          v[2 * x + 1] + (P.b2 ? P.b2[c0 + 2 * x + 1] : 0.f));
-          uint4* dst = reinterpret_cast<uint4*>(P.code + ((int64_t)bh * P.n_code_cap + row) * P.d_c + c0);
-          dst[0] = o[0];
-          dst[1] = o[1];
-        }
-      }
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-  }
-  if (!ok) {
-    if (lane == 0) latch_error(P.err, DELTAKV_ERR_DEVICE_TIMEOUT, 10);
-    *abort_flag = 1;
+    tmem_st_wait();
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  tc_fence_after();
+
+  if (warp < enc::GATHER_WARPS) {
+    // ------------------------------------ gather: re-rank, mean, residual
+    const int grp = lane >> 4, s16 = lane & 15;  // row within the warp's 2, lane within the row
+    const int e0 = s16 * EPL;                      // this lane's first element of [K ; V]
+    const bool inK = e0 < P.d_h;
+    constexpr int NB = CandBatch<KC>::N;
+    constexpr int PASSES = enc::ROWS / (2 * enc::GATHER_WARPS);
+    bool ok = true;
+    // The x slice and candidate slot of the next row pass are loaded one pass
+    // ahead, so only the candidate rows' latency sits on a pass's path.
+    uint4 pf_x[RowPack<EPL>::V4];
+    int pf_c = -1;
+    if (n_local > 0) gather_prefetch<EPL, KC>(P, gather_row<KC>(P, blockIdx.x, warp * 2 + grp, inK, e0), s16, pf_x, pf_c);
+    for (int it = 0; it < n_local && ok; ++it) {
+      const int tile = blockIdx.x + it * gridDim.x, rb = it & 1;
+      const int bh = tile / P.tiles_per_bh;
+      // this lane's slice of reference row j: rs + j d_h
+      const __nv_bfloat16* rs = (inK ? P.refk + e0 : P.refv + (e0 - P.d_h)) + (int64_t)bh * P.n_ref_cap * P.d_h;
+      unsigned char* sRb = sR + rb * 2 * r_part;
+      if (it >= 2 && !mbar_wait(&bars->r_empty[rb], ((it >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
+#pragma unroll 1
+      for (int pass = 0; pass < PASSES; ++pass) {
+        const int n = pass * 2 * enc::GATHER_WARPS + warp * 2 + grp;
+        const GatherRow g = gather_row<KC>(P, tile, n, inK, e0);
+        float xr[EPL];
+        unpack_row<EPL>(pf_x, xr);
+        const int myc = pf_c;
+        {
+          const int ntile = pass + 1 < PASSES ? tile : tile + gridDim.x;
+          const int nn = pass + 1 < PASSES ? n + 2 * enc::GATHER_WARPS : warp * 2 + grp;
+          if (ntile < P.n_tiles) gather_prefetch<EPL, KC>(P, gather_row<KC>(P, ntile, nn, inK, e0), s16, pf_x, pf_c);
+        }
+        int cj[KC];
+        float cd[KC];
+#pragma unroll
+        for (int c = 0; c < KC; ++c) {
+          int j = __shfl_sync(0xffffffffu, myc, c, 16);
+          if (j >= 0 && (int64_t)j * P.s >= g.t) {  // not an earlier reference: drop it
+            if (s16 == 0) latch_error(P.err, DELTAKV_ERR_DEVICE_BOUNDS, (uint32_t)j);
+            j = -1;
+          }
+          cj[c] = j;
+        }
+        // exact distances, NB candidate rows in flight at a time; with
+        // NB == KC the rows stay in registers for the mean
+        uint4 rr[NB][RowPack<EPL>::V4];
+#pragma unroll
+        for (int c0 = 0; c0 < KC; c0 += NB) {
+#pragma unroll
+          for (int u = 0; u < NB; ++u) {
+            const int j = cj[c0 + u];
+            if (j >= 0) load_row<EPL>(rs + (int64_t)j * P.d_h, rr[u]);
+          }
+#pragma unroll
+          for (int u = 0; u < NB; ++u) {
+            float part = 0.f;
+            if (cj[c0 + u] >= 0) {
+#pragma unroll
+              for (int i = 0; i < RowPack<EPL>::V4; ++i) {
+                const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&rr[u][i]);
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                  const float2 v = __bfloat1622float2(p2[x]);
+                  const float d0 = xr[8 * i + 2 * x] - v.x, d1 = xr[8 * i + 2 * x + 1] - v.y;
+                  part = fmaf(d0, d0, part);
+                  part = fmaf(d1, d1, part);
+                }
+              }
+            }
+            part = group16_sum(part);
+            cd[c0 + u] = cj[c0 + u] >= 0 ? part : FLT_MAX;
+          }
+        }
+        // the k smallest (distance, slot), ascending
+        uint32_t chosen = 0;
+        int k_eff = 0, my_sel = -1;
+        for (int qk = 0; qk < P.k; ++qk) {
+          int best = -1;
+          float bdv = FLT_MAX;
+          int bj = INT_MAX;
+#pragma unroll
+          for (int c = 0; c < KC; ++c) {
+            const bool avail = cj[c] >= 0 && !(chosen & (1u << c));
+            if (avail && (cd[c] < bdv || (cd[c] == bdv && cj[c] < bj))) {
+              best = c;
+              bdv = cd[c];
+              bj = cj[c];
+            }
+          }
+          if (best >= 0) {
+            chosen |= 1u << best;
+            ++k_eff;
+          }
+          if (s16 == qk) my_sel = best >= 0 ? bj : -1;
+        }
+        if (g.live && s16 < P.k) P.idx[((int64_t)bh * P.n_code_cap + g.row) * P.k + s16] = my_sel;
+        // r = x - mean of the chosen rows, formed in place as x - sum_c inv r_c
+        const float inv = 1.0f / (float)max(k_eff, 1);
+#pragma unroll
+        for (int c = 0; c < KC; ++c) {
+          if (chosen & (1u << c)) {
+            uint4 rc[RowPack<EPL>::V4];
+            if constexpr (NB == KC) {
+#pragma unroll
+              for (int i = 0; i < RowPack<EPL>::V4; ++i) rc[i] = rr[c][i];
+            } else {
+              load_row<EPL>(rs + (int64_t)cj[c] * P.d_h, rc);  // reloaded: it is in L2
+            }
+#pragma unroll
+            for (int i = 0; i < RowPack<EPL>::V4; ++i) {
+              const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&rc[i]);
+#pragma unroll
+              for (int x = 0; x < 4; ++x) {
+                const float2 v = __bfloat1622float2(p2[x]);
+                xr[8 * i + 2 * x] = fmaf(-inv, v.x, xr[8 * i + 2 * x]);
+                xr[8 * i + 2 * x + 1] = fmaf(-inv, v.y, xr[8 * i + 2 * x + 1]);
+              }
+            }
+          }
+        }
+        // r = hi + lo (fp16) into the R tile: row n, columns e0 .. e0 + EPL
+#pragma unroll
+        for (int v = 0; v < EPL / 8; ++v) {
+          __half2 hi2[4], lo2[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int i = 8 * v + 2 * q;
+            split_half2(g.live ? xr[i] : 0.f, g.live ? xr[i + 1] : 0.f, hi2[q], lo2[q]);
+          }
+          const uint32_t off = sw128_offset(n, e0 + 8 * v, enc::ROWS);
+          *reinterpret_cast<uint4*>(sRb + off) = *reinterpret_cast<const uint4*>(hi2);
+          *reinterpret_cast<uint4*>(sRb + r_part + off) = *reinterpret_cast<const uint4*>(lo2);
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->r_full[rb]);
+    }
+    if (!ok) {
+      if (lane == 0) latch_error(P.err, DELTAKV_ERR_DEVICE_TIMEOUT, 10);
+      *abort_flag = 1;
+    }
+  } else if (warp == enc::MMA_WARP) {
+    // ---------------------------------------------------------- MMA issue
+    if (lane == 0) {
+      const uint32_t r_base = smem_u32(sR), h0 = smem_u32(sH), w0 = smem_u32(sW2);
+      const uint32_t id1 = idesc_f16_f32(128, enc::ROWS);
+      const uint32_t id2 = idesc_f16_f32(enc::MMA_M, P.d_c) | (1u << 15);  // A MN-major
+      bool ok = true;
+      for (int it = 0; it <= n_local && ok; ++it) {
+        if (it < n_local) {
+          // GEMM1^T of tile it: D1[hh] = W1[hh] . R^T  (hidden x tokens)
+          const int rb = it & 1;
+          if (!mbar_wait(&bars->r_full[rb], (it >> 1) & 1, abort_flag)) { ok = false; break; }
+          if (it >= 1 && !mbar_wait(&bars->d1_empty, (it - 1) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t rt = r_base + rb * 2 * (uint32_t)r_part;
+          for (int hh = 0; hh < nh; ++hh)
+#pragma unroll 1
+            for (int part = 0; part < 2; ++part)
+#pragma unroll
+              for (int k16 = 0; k16 < D / 16; ++k16)
+                umma_f16_ts(tmem + enc::D1_COL + enc::ROWS * hh, tmem + enc::W1_COL + hh * (D / 2) + k16 * 8,
+                            desc_kmajor_sw128(rt + part * (uint32_t)r_part + (k16 >> 2) * enc::ROWS * 128 +
+                                              (k16 & 3) * 32),
+                            id1, (part | k16) != 0);
+          umma_commit(&bars->r_empty[rb]);
+          umma_commit(&bars->d1_full);
+        }
+        if (it >= 1) {
+          // GEMM2 of tile it - 1: codes = H . W2^T (tokens x d_c)
+          const int pt = it - 1;
+          if (!mbar_wait(&bars->h_full, pt & 1, abort_flag)) { ok = false; break; }
+          if (pt >= 1 && !mbar_wait(&bars->d2_empty, (pt - 1) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll 1
+          for (int part = 0; part < 2; ++part)
+#pragma unroll 1
+            for (int k16 = 0; k16 < hidden / 16; ++k16) {
+              // A: 16 hidden rows per step; the second 64-token block (rows of
+              // the M = 128 MMA that no token owns) reads the same rows again
+              const uint64_t ad = desc_mnmajor_sw128_enc(h0 + part * (uint32_t)h_part + k16 * 16 * 128, 0, 1024);
+              const uint64_t bd = desc_kmajor_sw128(w0 + (k16 >> 2) * P.d_c * 128 + (k16 & 3) * 32);
+              umma_f16(tmem + enc::D2_COL, ad, bd, id2, (part | k16) != 0);
+            }
+          umma_commit(&bars->h_empty);
+          umma_commit(&bars->d2_full);
+        }
+      }
+      if (!ok) {
+        latch_error(P.err, DELTAKV_ERR_DEVICE_TIMEOUT, 11);
+        *abort_flag = 1;
+      }
+    }
+  } else if (warp >= enc::ACT0 && warp < enc::ACT0 + enc::ACT_WARPS) {
+    // ------------------- activation H = act(D1 + b1), then the code store
+    const int q = warp - enc::ACT0;
+    bool ok = true;
+    for (int it = 0; it < n_local && ok; ++it) {
+      const int tile = blockIdx.x + it * gridDim.x;
+      if (!mbar_wait(&bars->d1_full, it & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      for (int hh = 0; hh < nh; ++hh) {
+        const int unit = 128 * hh + 32 * q + lane;
+        const float bias = P.b1 ? P.b1[unit] : 0.f;
+#pragma unroll 1
+        for (int cc = 0; cc < 2; ++cc) {
+          float v[32];
+          tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + enc::D1_COL + enc::ROWS * hh + 32 * cc, v);
+          if (hh == nh - 1 && cc == 1) {
+            // the accumulator is in registers: GEMM1 of the next tile may start
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->d1_empty);
+          }
+          if (hh == 0 && cc == 0 && it >= 1 && !mbar_wait(&bars->h_empty, (it - 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) {
+            __half2 hi2[4], lo2[4];
+#pragma unroll
+            for (int x = 0; x < 4; ++x)
+              split_half2(enc_act<ACT>(v[8 * c4 + 2 * x] + bias), enc_act<ACT>(v[8 * c4 + 2 * x + 1] + bias),
+                          hi2[x], lo2[x]);
+            // MN-major row `unit` of 64 tokens: 16-byte chunk c8, swizzled by row
+            const int c8 = 4 * cc + c4;
+            const uint32_t off = (uint32_t)unit * 128 + (((c8 ^ (unit & 7))) << 4);
+            *reinterpret_cast<uint4*>(sH + off) = *reinterpret_cast<const uint4*>(hi2);
+            *reinterpret_cast<uint4*>(sH + h_part + off) = *reinterpret_cast<const uint4*>(lo2);
+          }
+        }
+        if (!ok) break;
+      }
+      if (!ok) break;
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->h_full);
+      // codes = D2 + b2 (TMEM lanes 0-63: the first two activation warps)
+      if (!mbar_wait(&bars->d2_full, it & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      if (q < 2) {
+        const int bh = tile / P.tiles_per_bh;
+        const int64_t row = (int64_t)(tile % P.tiles_per_bh) * enc::ROWS + q * 32 + lane;
+        for (int c0 = 0; c0 < P.d_c; c0 += 16) {
+          float v[16];
+          tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + enc::D2_COL + c0, v);
+          if (row < P.n_code) {
+            uint4 o[2];
+            __nv_bfloat162* o2 = reinterpret_cast<__nv_bfloat162*>(o);
+#pragma unroll
+            for (int x = 0; x < 8; ++x)
+              o2[x] = __floats2bfloat162_rn(v[2 * x] + (P.b2 ? P.b2[c0 + 2 * x] : 0.f),
+                                            v[2 * x + 1] + (P.b2 ? P.b2[c0 + 2 * x + 1] : 0.f));
+            uint4* dst = reinterpret_cast<uint4*>(P.code + ((int64_t)bh * P.n_code_cap + row) * P.d_c + c0);
+            dst[0] = o[0];
+            dst[1] = o[1];
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->d2_empty);
+    }
+    if (!ok) {
+      if (lane == 0) latch_error(P.err, DELTAKV_ERR_DEVICE_TIMEOUT, 12);
+      *abort_flag = 1;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == enc::MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, enc::TMEM_COLS);
   }
@@ -453,17 +597,16 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
 
 size_t encode_tc_smem(const Plan& p) {
   const int D = p.D, hidden = p.cfg.hidden, d_c = p.cfg.d_c;
-  const int hid_atoms = (hidden + 63) / 64;
-  const size_t w1 = (size_t)(D / 64) * hidden * 128;
-  const size_t rh = std::max(2 * (size_t)(D / 64) * enc::ROWS * 128, 2 * (size_t)hidden * 128);
-  const size_t w2 = ((size_t)hid_atoms * d_c * 128 + 1023) & ~size_t(1023);
-  return 1024 + w1 + rh + w2 + 64;
+  const size_t r = 4 * (size_t)(D / 64) * enc::ROWS * 128;   // two tiles, hi and lo
+  const size_t h = 2 * (size_t)hidden * 128;                 // hi and lo
+  const size_t w2 = ((size_t)(hidden / 64) * d_c * 128 + 1023) & ~size_t(1023);
+  return 1024 + r + h + w2 + sizeof(EncBars) + 64;
 }
 
 bool encode_tc_supported(const Plan& p) {
   const auto& c = p.cfg;
   return c.dtype == DELTAKV_BF16 && (c.d_h == 64 || c.d_h == 128) && (c.hidden == 128 || c.hidden == 256) &&
-         c.d_c % 16 == 0 && c.d_c <= 256 && encode_tc_smem(p) <= 227 * 1024;
+         c.d_c % 16 == 0 && c.d_c <= 64 && encode_tc_smem(p) <= 227 * 1024;
 }
 
 namespace {
@@ -526,8 +669,8 @@ cudaError_t launch_encode_tc(const Plan& p, int T, const KVView& kv, const void*
   const size_t smem = encode_tc_smem(p);
   ProfScope ps(p, st, KID_ENCODE_TC);
   if (c.d_h == 128)
-    return p.KC == 8 ? encode_tc_launch<32, 8>(P, smem, grid, st) : encode_tc_launch<32, 12>(P, smem, grid, st);
-  return p.KC == 8 ? encode_tc_launch<16, 8>(P, smem, grid, st) : encode_tc_launch<16, 12>(P, smem, grid, st);
+    return p.KC == 8 ? encode_tc_launch<16, 8>(P, smem, grid, st) : encode_tc_launch<16, 12>(P, smem, grid, st);
+  return p.KC == 8 ? encode_tc_launch<8, 8>(P, smem, grid, st) : encode_tc_launch<8, 12>(P, smem, grid, st);
 }
 
 }  // namespace dkv
