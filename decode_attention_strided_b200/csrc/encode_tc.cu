@@ -42,11 +42,11 @@ using namespace sm100;
 namespace enc {
 constexpr int ROWS = 64;          // compressed rows per tile (GEMM1^T N; GEMM2 runs M = 128)
 constexpr int MMA_M = 128;
-constexpr int GATHER_WARPS = 8;   // warps 0-7: re-rank, mean, residual
-constexpr int ACT0 = 8;           // warps 8-11: activation and code store (one per TMEM lane quarter)
+constexpr int GATHER_WARPS = 11;  // warps 0-10: re-rank, mean, residual
+constexpr int MMA_WARP = 11;      // warp 11: TMEM allocation and MMA issue
+constexpr int ACT0 = 12;          // warps 12-15: activation and code store; warp w reads TMEM lanes 32 (w % 4)..
 constexpr int ACT_WARPS = 4;
-constexpr int MMA_WARP = 12;      // warp 12: TMEM allocation and MMA issue
-constexpr int THREADS = 13 * 32;
+constexpr int THREADS = 16 * 32;  // four warps per scheduler: 128 registers a thread
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t W1_COL = 0;    // W1 halves, D/2 packed columns each
 constexpr uint32_t D1_COL = 256;  // GEMM1^T accumulators, 64 columns per half
@@ -196,6 +196,7 @@ __device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
 // Row n of a 64-row tile: its code row, token and this lane's x slice.
 struct GatherRow {
   int64_t row, t;
+  bool inrow;              // n < ROWS (the last pass of a tile may run past it)
   const __nv_bfloat16* x;  // this lane's slice of x_t (valid when live)
   const int32_t* cand;     // the row's candidate slots
   bool live;
@@ -206,7 +207,8 @@ __device__ __forceinline__ GatherRow gather_row(const EncParams& P, int tile, in
   GatherRow g;
   const int bh = tile / P.tiles_per_bh;
   g.row = (int64_t)(tile % P.tiles_per_bh) * enc::ROWS + n;
-  g.live = g.row < P.n_code;
+  g.inrow = n < enc::ROWS;
+  g.live = g.inrow && g.row < P.n_code;
   g.t = g.live ? (g.row / (P.s - 1)) * P.s + (g.row % (P.s - 1)) + 1 : 0;
   const int b = bh / P.H, h = bh % P.H;
   g.x = (inK ? P.K + e0 : P.V + (e0 - P.d_h)) + b * P.sb + h * P.sh + g.t * P.st;
@@ -292,7 +294,7 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
   if (warp >= enc::ACT0 && warp < enc::ACT0 + enc::ACT_WARPS) {
     // W1 -> tensor memory, fp16: A of GEMM1^T, half hh at columns
     // W1_COL + hh D/2, lane = hidden unit within the half
-    const int q = warp - enc::ACT0;
+    const int q = warp & 3;
     for (int hh = 0; hh < nh; ++hh) {
       const __nv_bfloat16* wrow = P.W1 + (int64_t)(hh * 128 + q * 32 + lane) * D;
 #pragma unroll 1
@@ -323,7 +325,7 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
     const int e0 = s16 * EPL;                      // this lane's first element of [K ; V]
     const bool inK = e0 < P.d_h;
     constexpr int NB = CandBatch<KC>::N;
-    constexpr int PASSES = enc::ROWS / (2 * enc::GATHER_WARPS);
+    constexpr int PASSES = (enc::ROWS + 2 * enc::GATHER_WARPS - 1) / (2 * enc::GATHER_WARPS);
     bool ok = true;
     // The x slice and candidate slot of the next row pass are loaded one pass
     // ahead, so only the candidate rows' latency sits on a pass's path.
@@ -346,7 +348,7 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
         const int myc = pf_c;
         {
           const int ntile = pass + 1 < PASSES ? tile : tile + gridDim.x;
-          const int nn = pass + 1 < PASSES ? n + 2 * enc::GATHER_WARPS : warp * 2 + grp;
+          const int nn = pass + 1 < PASSES ? n + 2 * enc::GATHER_WARPS : warp * 2 + grp;  // may pass ROWS: not live
           if (ntile < P.n_tiles) gather_prefetch<EPL, KC>(P, gather_row<KC>(P, ntile, nn, inK, e0), s16, pf_x, pf_c);
         }
         int cj[KC];
@@ -390,29 +392,30 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
             cd[c0 + u] = cj[c0 + u] >= 0 ? part : FLT_MAX;
           }
         }
-        // the k smallest (distance, slot), ascending
-        uint32_t chosen = 0;
-        int k_eff = 0, my_sel = -1;
-        for (int qk = 0; qk < P.k; ++qk) {
-          int best = -1;
-          float bdv = FLT_MAX;
-          int bj = INT_MAX;
+        // the k smallest (distance, slot), ascending: lane c of the row ranks
+        // candidate c against the others; ranks below k are the references
+        float my_d = FLT_MAX;
+        int my_j = -1, n_valid = 0;
 #pragma unroll
-          for (int c = 0; c < KC; ++c) {
-            const bool avail = cj[c] >= 0 && !(chosen & (1u << c));
-            if (avail && (cd[c] < bdv || (cd[c] == bdv && cj[c] < bj))) {
-              best = c;
-              bdv = cd[c];
-              bj = cj[c];
-            }
+        for (int c = 0; c < KC; ++c) {
+          if (s16 == c) {
+            my_d = cd[c];
+            my_j = cj[c];
           }
-          if (best >= 0) {
-            chosen |= 1u << best;
-            ++k_eff;
-          }
-          if (s16 == qk) my_sel = best >= 0 ? bj : -1;
+          n_valid += cj[c] >= 0 ? 1 : 0;
         }
-        if (g.live && s16 < P.k) P.idx[((int64_t)bh * P.n_code_cap + g.row) * P.k + s16] = my_sel;
+        int rank = 0;
+#pragma unroll
+        for (int c = 0; c < KC; ++c)
+          rank += (cj[c] >= 0 && (cd[c] < my_d || (cd[c] == my_d && cj[c] < my_j))) ? 1 : 0;
+        const bool pick = s16 < KC && my_j >= 0 && rank < P.k;
+        const uint32_t chosen = (__ballot_sync(0xffffffffu, pick) >> (16 * grp)) & 0xFFFFu;
+        const int k_eff = min(P.k, n_valid);
+        if (g.live) {
+          int32_t* idx_row = P.idx + ((int64_t)bh * P.n_code_cap + g.row) * P.k;
+          if (pick) idx_row[rank] = my_j;
+          if (s16 >= k_eff && s16 < P.k) idx_row[s16] = -1;
+        }
         // r = x - mean of the chosen rows, formed in place as x - sum_c inv r_c
         const float inv = 1.0f / (float)max(k_eff, 1);
 #pragma unroll
@@ -446,9 +449,11 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
             const int i = 8 * v + 2 * q;
             split_half2(g.live ? xr[i] : 0.f, g.live ? xr[i + 1] : 0.f, hi2[q], lo2[q]);
           }
-          const uint32_t off = sw128_offset(n, e0 + 8 * v, enc::ROWS);
-          *reinterpret_cast<uint4*>(sRb + off) = *reinterpret_cast<const uint4*>(hi2);
-          *reinterpret_cast<uint4*>(sRb + r_part + off) = *reinterpret_cast<const uint4*>(lo2);
+          if (g.inrow) {
+            const uint32_t off = sw128_offset(n, e0 + 8 * v, enc::ROWS);
+            *reinterpret_cast<uint4*>(sRb + off) = *reinterpret_cast<const uint4*>(hi2);
+            *reinterpret_cast<uint4*>(sRb + r_part + off) = *reinterpret_cast<const uint4*>(lo2);
+          }
         }
       }
       fence_proxy_async_smem();
@@ -513,7 +518,7 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
     }
   } else if (warp >= enc::ACT0 && warp < enc::ACT0 + enc::ACT_WARPS) {
     // ------------------- activation H = act(D1 + b1), then the code store
-    const int q = warp - enc::ACT0;
+    const int q = warp & 3;
     bool ok = true;
     for (int it = 0; it < n_local && ok; ++it) {
       const int tile = blockIdx.x + it * gridDim.x;
