@@ -22,8 +22,8 @@
 //                  fp16 P tile (two buffers), slot-weight reductions into the
 //                  global table, and the fold of U_chunk into register
 //                  accumulators with the online-softmax rescale
-// The MMA warp issues G1(0); then per chunk i: z(i), G1(i+1), U(i-1), so the
-// activation warps never wait on the softmax of the same chunk.
+// The MMA warp issues G1(0); then per chunk i: G1(i+1), z(i), U(i-1), so the
+// activation warps wait only for the next GEMM1, never for z or the softmax.
 // A persistent grid splits the flattened (kv-head, chunk) list evenly; each
 // CTA writes one partial (m, l, U) per kv-head segment it touches.
 #include <cfloat>
@@ -280,7 +280,7 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
     }
   } else if (warp == dtc::MMA) {
     // ----------------------------------------------------------------- MMA
-    // order: G1(0); for i: z(i), G1(i+1), U(i-1); U(n-1)
+    // order: G1(0); for i: G1(i+1), z(i), U(i-1); U(n-1)
     if (lane == 0 && n_local > 0) {
       const uint32_t id_g1 = idesc_kind_f16(true, dtc::CH, hidden, false);
       const uint32_t id_z = idesc_kind_f16(false, dtc::CH, 16, false);
@@ -329,6 +329,17 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
         if (bh != prev_bh) { ++seg; prev_bh = bh; }
         const int ub = it & 1;
         if (!mbar_wait(&u_full[ub], (it >> 1) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        // the activation warps have read D1(it): start the next chunk's GEMM1
+        // first, so they wait only for it and not for z(it) as well
+        if (it + 1 < n_local) {
+          const int st = (it + 1) & 1;
+          if (!mbar_wait(&in_full[st], ((it + 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          gemm1(st);
+          umma_commit(d1_full);
+          umma_commit(&in_empty[st]);
+        }
         if (!mbar_wait(&z_empty[ub], ((it >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         {
@@ -339,14 +350,6 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
                      desc_kmajor(a0 + atom * 16 * 128 + off, 128), id_z, k16 != 0);
           }
           umma_commit(&z_full[ub]);
-        }
-        if (it + 1 < n_local) {
-          const int st = (it + 1) & 1;
-          if (!mbar_wait(&in_full[st], ((it + 1) >> 1) & 1, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          gemm1(st);
-          umma_commit(d1_full);
-          umma_commit(&in_empty[st]);
         }
         if (it >= 1 && !issue_u(it - 1)) { ok = false; break; }
       }
