@@ -12,28 +12,25 @@
 // precision to cancellation when x_t is close to r_j, so the encode kernel
 // re-ranks these KC candidates with exact fp32 distances before choosing k.
 //
-// Work unit: two 128-token tiles of one (sequence, kv-head) -- M = 256 rows
+// Work unit: two 128-token tiles of one (sequence, kv-head) -- 256 tokens
 // share every reference tile that is staged in shared memory.
 // Warp roles (320 threads, one CTA per SM, persistent):
-//   warps 0-7  epilogue: warp w owns token tile w / 4, TMEM lanes 32 (w % 4)..
-//   warp 8     TMA producer: A tiles (tokens) and B stages (references)
-//   warp 9     MMA issuer: M=128, N=128, K=16 tcgen05.mma, fp32 in TMEM
-// TMEM: 512 columns = 2 buffers x 2 token tiles x 128 reference columns, so
-// the MMAs fill one reference tile while the epilogue drains the other.
-// Shape choice: an M = 128 MMA occupies the tensor pipe for at least about
-// 58 cycles whatever its N, and a commit costs a pipeline drain unless the
-// MMAs before it cover it; N = 128 (64 cycles of math per MMA) and one commit
-// per 8 MMAs (512 cycles) keep the pipe math-bound.
-// A and B live in shared memory in the 128-byte-swizzled K-major layout the
-// TMA writes; a 64-element column of a 128-row token tile is one 16 KB atom,
-// and so is one of a 128-row reference tile.
-//
-// Epilogue: each thread owns one token row, so a warp carries 32 unrelated
-// running top-k lists.  Per 32 columns it builds a bitmask of the values below
-// its current k-th best; only if some lane has a candidate are the values
-// parked in the warp's shared-memory slot, and then every lane inserts its
-// own candidates in one short loop, so a warp pays for the busiest lane, not
-// for the sum over lanes.
+//   warps 0-7  warp w owns token tile w / 4, TMEM lanes 32 (w % 4)..: at the
+//              start of a unit it writes its token rows into tensor memory
+//              (the A operand), then drains that tile's accumulator into the
+//              rows' running top-k lists
+//   warp 8     TMA producer: whole reference tiles (128 rows x D) into a
+//              3-slot ring
+//   warp 9     MMA issuer: M=128, N=128, K=16 tcgen05.mma with A in tensor
+//              memory and B in shared memory, fp32 accumulators in TMEM
+// TMEM (512 columns): A of token tile 0 and 1 (D/2 columns each, two bf16
+// per column), then one 128-column accumulator per token tile.  The MMAs of
+// tile 1 run while the epilogue drains tile 0 and the other way round.
+// Shape choices: an M = 128 MMA occupies the tensor pipe for at least about
+// 58 cycles whatever its N, so N = 128 (64 cycles of math) keeps it math-bound;
+// with A in tensor memory each MMA reads only its 4 KB of B from shared
+// memory, which leaves shared-memory bandwidth for the TMA writes and the
+// epilogue.
 #include <cfloat>
 #include <climits>
 #include <mutex>
@@ -46,25 +43,29 @@ using namespace sm100;
 
 namespace tcc {
 constexpr int TM = 128;                     // tokens per tile (MMA M)
-constexpr int TPU = 2;                      // token tiles per unit (the epilogue selects between the two)
+constexpr int TPU = 2;                      // token tiles per unit
 constexpr int RN = 128;                     // references per tile (MMA N)
-constexpr int NBUF = 2;                     // TMEM accumulator buffers
-constexpr int STAGES = 5;                   // reference pipeline depth (atoms)
-constexpr int ATOM = TM * 128;              // bytes: 128 token rows x 128 B
-constexpr int BATOM = RN * 128;             // bytes: 64 reference rows x 128 B
+constexpr int NSLOT = 3;                    // reference tiles in flight
+constexpr int BATOM = RN * 128;             // bytes: 128 reference rows x 128 B
 constexpr int CHUNK = 16;                   // columns per slow-path chunk
 constexpr int SPILL = 32 * CHUNK * 4;       // bytes per warp: 32 lanes x CHUNK floats
 constexpr int EPI_WARPS = 8;
 constexpr int THREADS = (EPI_WARPS + 2) * 32;
 constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t A_COL = 0;               // A of tile i at A_COL + i * 128
+constexpr uint32_t D_COL = 256;             // accumulator of tile i at D_COL + i * RN
 constexpr int PRODUCER_WARP = EPI_WARPS;
 constexpr int MMA_WARP = EPI_WARPS + 1;
+__host__ __device__ constexpr int spill_bytes(int) { return EPI_WARPS * SPILL; }
 }  // namespace tcc
 
 struct TcParams {
-  int T, s, H, BH, n_units, n_pairs;
+  int T, s, H, BH, n_units, n_pairs, d_h;
   int n_ref;
   int64_t n_ref_cap, n_code_cap;
+  const __nv_bfloat16* K;
+  const __nv_bfloat16* V;
+  int64_t sb, sh, st;
   const float* hnorm;
   int32_t* cand;
   uint32_t* err;
@@ -101,51 +102,107 @@ __device__ __forceinline__ bool unit_of(const TcParams& P, int round, UnitInfo& 
   return true;
 }
 
+// One 64-column block of one token row's accumulator: e = |r_j|^2 / 2 -
+// <x_t, r_j> for slots jb .. jb + 63, folded into the row's running list.
+template <int KC>
+__device__ __forceinline__ void cand_block(float (&v)[64], const float* hn, int jb, int cnt, int cnt_lo,
+                                           bool first, float (&bd)[KC], int (&bi)[KC], float* sp, int sw) {
+  const float4* h4 = reinterpret_cast<const float4*>(hn + jb);
+#pragma unroll
+  for (int x4 = 0; x4 < 16; ++x4) {
+    const float4 t4 = __ldg(h4 + x4);
+    v[4 * x4] = t4.x - v[4 * x4];
+    v[4 * x4 + 1] = t4.y - v[4 * x4 + 1];
+    v[4 * x4 + 2] = t4.z - v[4 * x4 + 2];
+    v[4 * x4 + 3] = t4.w - v[4 * x4 + 3];
+  }
+  if (jb + 64 > cnt_lo) {
+#pragma unroll
+    for (int x = 0; x < 64; ++x)
+      if (jb + x >= cnt) v[x] = FLT_MAX;
+  }
+  if (first) {
+    // the list is empty: every value is taken, without branching
+#pragma unroll
+    for (int x = 0; x < 64; ++x) topk_insert_inorder<KC>(bd, bi, v[x], jb + x);
+    return;
+  }
+  // fast path: most blocks hold nothing below any lane's k-th best
+  float mn[32];
+#pragma unroll
+  for (int x = 0; x < 32; ++x) mn[x] = fminf(v[x], v[x + 32]);
+#pragma unroll
+  for (int w = 16; w >= 1; w >>= 1)
+#pragma unroll
+    for (int x = 0; x < w; ++x) mn[x] = fminf(mn[x], mn[x + w]);
+  if (!__any_sync(0xffffffffu, mn[0] < bd[KC - 1])) return;
+#pragma unroll
+  for (int c = 0; c < 64 / tcc::CHUNK; ++c) {
+    const float thr = bd[KC - 1];
+    // four independent partial masks keep the dependency chains short
+    uint32_t mp[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int x = 0; x < tcc::CHUNK; ++x) mp[x & 3] |= (v[c * tcc::CHUNK + x] < thr ? 1u : 0u) << x;
+    uint32_t m = (mp[0] | mp[1]) | (mp[2] | mp[3]);
+    if (__any_sync(0xffffffffu, m != 0)) {
+      if (m) {
+#pragma unroll
+        for (int i4 = 0; i4 < tcc::CHUNK / 4; ++i4)
+          reinterpret_cast<float4*>(sp)[i4 ^ sw] =
+              make_float4(v[c * tcc::CHUNK + 4 * i4], v[c * tcc::CHUNK + 4 * i4 + 1], v[c * tcc::CHUNK + 4 * i4 + 2],
+                          v[c * tcc::CHUNK + 4 * i4 + 3]);
+      }
+      __syncwarp();
+      while (m) {
+        const int x = __ffs(m) - 1;
+        m &= m - 1;
+        const float vx = sp[(((x >> 2) ^ sw) << 2) | (x & 3)];
+        topk_insert_inorder<KC>(bd, bi, vx, jb + c * tcc::CHUNK + x);
+      }
+      __syncwarp();
+    }
+  }
+}
+
 template <int NKC, int KC>
 __global__ void __launch_bounds__(tcc::THREADS, 1)
-    cand_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
-                   const __grid_constant__ CUtensorMap mapRK, const __grid_constant__ CUtensorMap mapRV,
+    cand_tc_kernel(const __grid_constant__ CUtensorMap mapRK, const __grid_constant__ CUtensorMap mapRV,
                    const TcParams P) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  unsigned char* sA = smem;                                     // [TPU][NKC] atoms
-  unsigned char* sB = sA + tcc::TPU * NKC * tcc::ATOM;          // [STAGES] atoms
-  float* spill = (float*)(sB + tcc::STAGES * tcc::BATOM);       // [EPI_WARPS][32][32]
-  uint64_t* a_full = (uint64_t*)((unsigned char*)spill + tcc::EPI_WARPS * tcc::SPILL);  // [NKC]
-  uint64_t* a_empty = a_full + NKC;                             // [NKC]
-  uint64_t* b_full = a_empty + NKC;                             // [STAGES]
-  uint64_t* b_empty = b_full + tcc::STAGES;                     // [STAGES]
-  uint64_t* acc_full = b_empty + tcc::STAGES;                   // [NBUF]
-  uint64_t* acc_empty = acc_full + tcc::NBUF;                   // [NBUF]
-  uint32_t* tmem_slot = (uint32_t*)(acc_empty + tcc::NBUF);
+  constexpr int D = NKC * 64;
+  constexpr int SLOT = NKC * tcc::BATOM;                        // bytes of one reference tile
+  unsigned char* sB = smem;                                     // [NSLOT][NKC] atoms
+  float* spill = (float*)(sB + tcc::NSLOT * SLOT);              // [EPI_WARPS][32][CHUNK]
+  uint64_t* b_full = (uint64_t*)((unsigned char*)spill + tcc::spill_bytes(KC));  // [NSLOT]
+  uint64_t* b_empty = b_full + tcc::NSLOT;                      // [NSLOT]
+  uint64_t* a_full = b_empty + tcc::NSLOT;                      // [1]
+  uint64_t* d_full = a_full + 1;                                // [TPU]
+  uint64_t* d_empty = d_full + tcc::TPU;                        // [TPU]
+  uint32_t* tmem_slot = (uint32_t*)(d_empty + tcc::TPU);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int HALF = NKC / 2;  // atoms per d_h (K part, then V part)
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NKC; ++i) {
-      mbar_init(&a_full[i], 1);
-      mbar_init(&a_empty[i], 1);
-    }
-    for (int i = 0; i < tcc::STAGES; ++i) {
+    for (int i = 0; i < tcc::NSLOT; ++i) {
       mbar_init(&b_full[i], 1);
       mbar_init(&b_empty[i], 1);
     }
-    for (int i = 0; i < tcc::NBUF; ++i) {
-      mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], tcc::EPI_WARPS);
+    mbar_init(a_full, tcc::EPI_WARPS);
+    for (int i = 0; i < tcc::TPU; ++i) {
+      mbar_init(&d_full[i], 1);
+      mbar_init(&d_empty[i], tcc::EPI_WARPS / tcc::TPU);  // the warps of token tile i
     }
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == tcc::PRODUCER_WARP && lane == 0) {
-    prefetch_tensormap(&mapK);
-    prefetch_tensormap(&mapV);
     prefetch_tensormap(&mapRK);
     prefetch_tensormap(&mapRV);
   }
-  if (warp == 0) {
+  if (warp == tcc::MMA_WARP) {
     tmem_alloc(tmem_slot, tcc::TMEM_COLS);
     tmem_relinquish();
   }
@@ -157,37 +214,21 @@ __global__ void __launch_bounds__(tcc::THREADS, 1)
   if (warp == tcc::PRODUCER_WARP) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      uint32_t a_it = 0, b_it = 0;
+      uint32_t b_it = 0;
       bool ok = true;
       UnitInfo u;
       for (int round = 0; ok && unit_of(P, round, u); ++round) {
-        if (u.Rmax == 0) continue;
-        const int h = u.bh % P.H, b = u.bh / P.H;
-        for (int kc = 0; kc < NKC && ok; ++kc) {
-          if (!mbar_wait(&a_empty[kc], (a_it & 1) ^ 1, abort_flag)) { ok = false; break; }
-          mbar_arrive_expect_tx(&a_full[kc], tcc::TPU * tcc::ATOM);
-#pragma unroll
-          for (int i = 0; i < tcc::TPU; ++i) {
-            unsigned char* dst = sA + (i * NKC + kc) * tcc::ATOM;
-            const int y = u.t0 + i * tcc::TM;
+        for (int r = 0; r < u.Rmax && ok; ++r, ++b_it) {
+          const int sl = b_it % tcc::NSLOT;
+          const uint32_t ph = (b_it / tcc::NSLOT) & 1;
+          if (!mbar_wait(&b_empty[sl], ph ^ 1, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(&b_full[sl], SLOT);
+          unsigned char* dst = sB + sl * SLOT;
+          for (int kc = 0; kc < NKC; ++kc) {
             if (kc < HALF)
-              tma_load_4d(&mapK, &a_full[kc], dst, kc * 64, y, h, b);
+              tma_load_3d(&mapRK, &b_full[sl], dst + kc * tcc::BATOM, kc * 64, r * tcc::RN, u.bh);
             else
-              tma_load_4d(&mapV, &a_full[kc], dst, (kc - HALF) * 64, y, h, b);
-          }
-        }
-        ++a_it;
-        for (int r = 0; r < u.Rmax && ok; ++r) {
-          for (int kc = 0; kc < NKC; ++kc, ++b_it) {
-            const int st = b_it % tcc::STAGES;
-            const uint32_t ph = (b_it / tcc::STAGES) & 1;
-            if (!mbar_wait(&b_empty[st], ph ^ 1, abort_flag)) { ok = false; break; }
-            mbar_arrive_expect_tx(&b_full[st], tcc::BATOM);
-            unsigned char* dst = sB + st * tcc::BATOM;
-            if (kc < HALF)
-              tma_load_3d(&mapRK, &b_full[st], dst, kc * 64, r * tcc::RN, u.bh);
-            else
-              tma_load_3d(&mapRV, &b_full[st], dst, (kc - HALF) * 64, r * tcc::RN, u.bh);
+              tma_load_3d(&mapRV, &b_full[sl], dst + kc * tcc::BATOM, (kc - HALF) * 64, r * tcc::RN, u.bh);
           }
         }
       }
@@ -196,9 +237,9 @@ __global__ void __launch_bounds__(tcc::THREADS, 1)
         *abort_flag = 1;
       } else {
         // let the last reference loads land before the block can finish
-        for (int i = 0; i < tcc::STAGES && b_it > (uint32_t)i; ++i) {
+        for (int i = 0; i < tcc::NSLOT && b_it > (uint32_t)i; ++i) {
           const uint32_t it = b_it - 1 - i;
-          mbar_wait(&b_full[it % tcc::STAGES], (it / tcc::STAGES) & 1, abort_flag);
+          mbar_wait(&b_full[it % tcc::NSLOT], (it / tcc::NSLOT) & 1, abort_flag);
         }
       }
     }
@@ -206,39 +247,33 @@ __global__ void __launch_bounds__(tcc::THREADS, 1)
     // ----------------------------------------------------------------- MMA
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(tcc::TM, tcc::RN);
-      const uint32_t a_base = smem_u32(sA), b_base = smem_u32(sB);
-      uint32_t a_it = 0, b_it = 0, acc_it = 0;
+      const uint32_t b_base = smem_u32(sB);
+      uint32_t b_it = 0, acc_it = 0, unit_it = 0;
       bool ok = true;
       UnitInfo u;
       for (int round = 0; ok && unit_of(P, round, u); ++round) {
         if (u.Rmax == 0) continue;
-        for (int r = 0; r < u.Rmax && ok; ++r, ++acc_it) {
-          const uint32_t buf = acc_it % tcc::NBUF;
-          if (!mbar_wait(&acc_empty[buf], ((acc_it / tcc::NBUF) & 1) ^ 1, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          for (int kc = 0; kc < NKC; ++kc, ++b_it) {
-            const int st = b_it % tcc::STAGES;
-            if (!mbar_wait(&b_full[st], (b_it / tcc::STAGES) & 1, abort_flag)) { ok = false; break; }
-            if (r == 0 && !mbar_wait(&a_full[kc], a_it & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(a_full, unit_it & 1, abort_flag)) { ok = false; break; }
+        ++unit_it;
+        for (int r = 0; r < u.Rmax && ok; ++r, ++acc_it, ++b_it) {
+          const int sl = b_it % tcc::NSLOT;
+          if (!mbar_wait(&b_full[sl], (b_it / tcc::NSLOT) & 1, abort_flag)) { ok = false; break; }
+#pragma unroll
+          for (int i = 0; i < tcc::TPU; ++i) {
+            if (acc_it >= 1 && !mbar_wait(&d_empty[i], (acc_it - 1) & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            // the two token tiles alternate, so consecutive MMAs never chain
-            // on one accumulator
+            const uint32_t d = tmem + tcc::D_COL + i * tcc::RN;
+            const uint32_t a = tmem + tcc::A_COL + i * 128;
 #pragma unroll
-            for (int k16 = 0; k16 < 4; ++k16)
-#pragma unroll
-              for (int i = 0; i < tcc::TPU; ++i) {
-                if (r >= u.R[i]) continue;
-                const uint32_t d = tmem + buf * (tcc::TPU * tcc::RN) + i * tcc::RN;
-                const uint64_t ad = desc_kmajor_sw128(a_base + (i * NKC + kc) * tcc::ATOM + k16 * 32);
-                const uint64_t bd = desc_kmajor_sw128(b_base + st * tcc::BATOM + k16 * 32);
-                umma_f16(d, ad, bd, idesc, (kc | k16) != 0);
-              }
-            umma_commit(&b_empty[st]);
-            if (r == u.Rmax - 1) umma_commit(&a_empty[kc]);
+            for (int k16 = 0; k16 < D / 16; ++k16)
+              umma_f16_ts(d, a + k16 * 8,
+                           desc_kmajor_sw128(b_base + sl * SLOT + (k16 >> 2) * tcc::BATOM + (k16 & 3) * 32), idesc,
+                           k16 != 0);
+            umma_commit(&d_full[i]);
           }
-          if (ok) umma_commit(&acc_full[buf]);
+          if (!ok) break;
+          umma_commit(&b_empty[sl]);
         }
-        ++a_it;
       }
       if (!ok) {
         latch_error(P.err, DELTAKV_ERR_DEVICE_TIMEOUT, 2);
@@ -246,8 +281,8 @@ __global__ void __launch_bounds__(tcc::THREADS, 1)
       }
     }
   } else {
-    // ------------------------------------------------------------ epilogue
-    const int ti = warp / 4, q = warp % 4, row = q * 32 + lane;
+    // ------------------------------------------------ token rows + epilogue
+    const int q = warp & 3, ti = warp >> 2, row = q * 32 + lane;
     float* sp = spill + warp * (32 * tcc::CHUNK) + lane * tcc::CHUNK;  // this lane's CHUNK floats
     const int sw = (lane >> 1) & 3;  // float4 swizzle: 8 lanes of a phase hit 8 distinct bank groups
     uint32_t acc_it = 0;
@@ -256,90 +291,65 @@ __global__ void __launch_bounds__(tcc::THREADS, 1)
     for (int round = 0; ok && unit_of(P, round, u); ++round) {
       if (u.Rmax == 0) continue;
       const int t = u.t0 + ti * tcc::TM + row;
+      // A of token tile ti: this thread's token row, [K ; V] as bf16 pairs.
+      // Every MMA that read it in the previous unit is complete: this warp
+      // consumed that unit's last accumulator of tile ti.
+      {
+        const int b = u.bh / P.H, h = u.bh % P.H;
+        const __nv_bfloat16* kr = P.K + b * P.sb + h * P.sh + (int64_t)t * P.st;
+        const __nv_bfloat16* vr = P.V + b * P.sb + h * P.sh + (int64_t)t * P.st;
+        const uint32_t ta = tmem + ((uint32_t)(q * 32) << 16) + tcc::A_COL + ti * 128;
+#pragma unroll 1
+        for (int c0 = 0; c0 < D / 2; c0 += 32) {
+          // columns c0 .. c0 + 31 hold elements 2 c0 .. 2 c0 + 63 of [K ; V]
+          const int e = 2 * c0;
+          const __nv_bfloat16* src = e < P.d_h ? kr + e : vr + (e - P.d_h);
+          uint32_t w[32];
+#pragma unroll
+          for (int v4 = 0; v4 < 8; ++v4) {
+            const uint4 x = t < P.T ? __ldg(reinterpret_cast<const uint4*>(src) + v4) : make_uint4(0, 0, 0, 0);
+            w[4 * v4] = x.x;
+            w[4 * v4 + 1] = x.y;
+            w[4 * v4 + 2] = x.z;
+            w[4 * v4 + 3] = x.w;
+          }
+          tmem_st32(ta + c0, w);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(a_full);
+      }
       const int first = u.t0 + ti * tcc::TM;
       const int cnt = t < P.T ? min((t + P.s - 1) / P.s, P.n_ref) : 0;  // valid slots j < cnt
       const int cnt_lo = min((first + P.s - 1) / P.s, P.n_ref);         // smallest cnt in the tile
       const float* hn = P.hnorm + (int64_t)u.bh * P.n_ref_cap;
-      const int R_mine = ti == 0 ? u.R[0] : u.R[1];
       float bd[KC];
       int bi[KC];
 #pragma unroll
-      for (int x = 0; x < KC; ++x) { bd[x] = FLT_MAX; bi[x] = INT_MAX; }
-      for (int r = 0; r < u.Rmax; ++r, ++acc_it) {
-        const uint32_t buf = acc_it % tcc::NBUF;
-        if (!mbar_wait(&acc_full[buf], (acc_it / tcc::NBUF) & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        if (r < R_mine) {
-#pragma unroll 1
-          for (int hf = 0; hf < tcc::RN / 64; ++hf) {
-            const int jb = r * tcc::RN + hf * 64;
-            float v[64];
-            tmem_ld64(tmem + ((uint32_t)(q * 32) << 16) + buf * (tcc::TPU * tcc::RN) + ti * tcc::RN + hf * 64, v);
-            // e = |r_j|^2 / 2 - <x_t, r_j>
-            const float4* h4 = reinterpret_cast<const float4*>(hn + jb);
-#pragma unroll
-            for (int x4 = 0; x4 < 16; ++x4) {
-              const float4 t4 = __ldg(h4 + x4);
-              v[4 * x4] = t4.x - v[4 * x4];
-              v[4 * x4 + 1] = t4.y - v[4 * x4 + 1];
-              v[4 * x4 + 2] = t4.z - v[4 * x4 + 2];
-              v[4 * x4 + 3] = t4.w - v[4 * x4 + 3];
-            }
-            if (jb + 64 > cnt_lo) {
-#pragma unroll
-              for (int x = 0; x < 64; ++x)
-                if (jb + x >= cnt) v[x] = FLT_MAX;
-            }
-            if (r == 0 && hf == 0) {
-              // first block of the unit: every list is empty, so every lane
-              // takes every value -- insert them all without branching
-#pragma unroll
-              for (int x = 0; x < 64; ++x) topk_insert_inorder<KC>(bd, bi, v[x], jb + x);
-              continue;
-            }
-            // fast path: most blocks hold nothing below any lane's k-th best
-            float mn[32];
-#pragma unroll
-            for (int x = 0; x < 32; ++x) mn[x] = fminf(v[x], v[x + 32]);
-#pragma unroll
-            for (int w = 16; w >= 1; w >>= 1)
-#pragma unroll
-              for (int x = 0; x < w; ++x) mn[x] = fminf(mn[x], mn[x + w]);
-            if (!__any_sync(0xffffffffu, mn[0] < bd[KC - 1])) continue;
-#pragma unroll
-            for (int c = 0; c < 64 / tcc::CHUNK; ++c) {
-              const float thr = bd[KC - 1];
-              // four independent partial masks keep the dependency chains short
-              uint32_t mp[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-              for (int x = 0; x < tcc::CHUNK; ++x) mp[x & 3] |= (v[c * tcc::CHUNK + x] < thr ? 1u : 0u) << x;
-              uint32_t m = (mp[0] | mp[1]) | (mp[2] | mp[3]);
-              if (__any_sync(0xffffffffu, m != 0)) {
-                if (m) {
-#pragma unroll
-                  for (int i4 = 0; i4 < tcc::CHUNK / 4; ++i4)
-                    reinterpret_cast<float4*>(sp)[i4 ^ sw] =
-                        make_float4(v[c * tcc::CHUNK + 4 * i4], v[c * tcc::CHUNK + 4 * i4 + 1],
-                                    v[c * tcc::CHUNK + 4 * i4 + 2], v[c * tcc::CHUNK + 4 * i4 + 3]);
-                }
-                __syncwarp();
-                while (m) {
-                  const int x = __ffs(m) - 1;
-                  m &= m - 1;
-                  const float vx = sp[(((x >> 2) ^ sw) << 2) | (x & 3)];
-                  topk_insert_inorder<KC>(bd, bi, vx, jb + c * tcc::CHUNK + x);
-                }
-                __syncwarp();
-              }
-            }
-          }
-        }
-        // the buffer is drained: hand it back to the MMA warp
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      for (int x = 0; x < KC; ++x) {
+        bd[x] = FLT_MAX;
+        bi[x] = INT_MAX;
       }
-      if (ok && t < P.T && (t % P.s) != 0) {
+      for (int r = 0; r < u.Rmax; ++r, ++acc_it) {
+        if (!mbar_wait(&d_full[ti], acc_it & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t dcol = tmem + ((uint32_t)(q * 32) << 16) + tcc::D_COL + ti * tcc::RN;
+#pragma unroll 1
+        for (int hf = 0; hf < tcc::RN / 64; ++hf) {
+          float v[64];
+          tmem_ld64(dcol + hf * 64, v);
+          if (hf == tcc::RN / 64 - 1) {
+            // the accumulator is in registers: the next MMAs may reuse it
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&d_empty[ti]);
+          }
+          cand_block<KC>(v, hn, r * tcc::RN + hf * 64, cnt, cnt_lo, r == 0 && hf == 0, bd, bi, sp, sw);
+        }
+      }
+      if (!ok) break;
+      if (t < P.T && (t % P.s) != 0) {
         int32_t* o = P.cand + ((int64_t)u.bh * P.n_code_cap + (t - t / P.s - 1)) * KC;
 #pragma unroll
         for (int x = 0; x < KC; ++x) o[x] = bi[x] == INT_MAX ? -1 : bi[x];
@@ -352,7 +362,7 @@ __global__ void __launch_bounds__(tcc::THREADS, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == tcc::MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, tcc::TMEM_COLS);
   }
@@ -398,20 +408,19 @@ int sm_count() {
   return n > 0 ? n : kNumSMs;
 }
 
-template <int NKC>
+template <int NKC, int KC>
 size_t smem_bytes() {
-  return 1024 + (size_t)tcc::TPU * NKC * tcc::ATOM + (size_t)tcc::STAGES * tcc::BATOM +
-         (size_t)tcc::EPI_WARPS * tcc::SPILL + 512;
+  return 1024 + (size_t)tcc::NSLOT * NKC * tcc::BATOM + (size_t)tcc::spill_bytes(KC) + 256;
 }
 
 template <int NKC, int KC>
-cudaError_t launch_tc(const CUtensorMap& mK, const CUtensorMap& mV, const CUtensorMap& mRK,
-                      const CUtensorMap& mRV, const TcParams& P, int grid, cudaStream_t st) {
+cudaError_t launch_tc(const CUtensorMap& mRK, const CUtensorMap& mRV, const TcParams& P, int grid,
+                      cudaStream_t st) {
   auto kern = cand_tc_kernel<NKC, KC>;
-  const size_t smem = smem_bytes<NKC>();
+  const size_t smem = smem_bytes<NKC, KC>();
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, tcc::THREADS, smem, st>>>(mK, mV, mRK, mRV, P);
+  kern<<<grid, tcc::THREADS, smem, st>>>(mRK, mRV, P);
   return cudaGetLastError();
 }
 
@@ -428,13 +437,7 @@ cudaError_t launch_candidates_tc(const Plan& p, int T, const KVView& kv, const v
   if (n_code == 0) return cudaSuccess;
   const int n_ref = (int)n_ref_of(T, c.stride_s);
   const int d_h = c.d_h;
-  CUtensorMap mK, mV, mRK, mRV;
-  {
-    cuuint64_t dims[4] = {(cuuint64_t)d_h, (cuuint64_t)T, (cuuint64_t)c.kv_heads, (cuuint64_t)c.batch};
-    cuuint64_t str[3] = {(cuuint64_t)kv.st * 2, (cuuint64_t)kv.sh * 2, (cuuint64_t)kv.sb * 2};
-    if (!make_map(&mK, kv.K, 4, dims, str, tcc::TM) || !make_map(&mV, kv.V, 4, dims, str, tcc::TM))
-      return cudaErrorNotSupported;  // nothing launched; the caller uses the CUDA-core kernel
-  }
+  CUtensorMap mRK, mRV;
   {
     const char* cb = (const char*)cache;
     cuuint64_t dims[3] = {(cuuint64_t)d_h, (cuuint64_t)n_ref, (cuuint64_t)c.batch * c.kv_heads};
@@ -448,6 +451,12 @@ cudaError_t launch_candidates_tc(const Plan& p, int T, const KVView& kv, const v
   P.s = c.stride_s;
   P.H = c.kv_heads;
   P.BH = c.batch * c.kv_heads;
+  P.d_h = d_h;
+  P.K = (const __nv_bfloat16*)kv.K;
+  P.V = (const __nv_bfloat16*)kv.V;
+  P.sb = kv.sb;
+  P.sh = kv.sh;
+  P.st = kv.st;
   P.n_pairs = (int)ceil_div64(T, tcc::TM * tcc::TPU);
   P.n_units = P.n_pairs * P.BH;
   P.n_ref = n_ref;
@@ -459,10 +468,8 @@ cudaError_t launch_candidates_tc(const Plan& p, int T, const KVView& kv, const v
   const int grid = std::min(P.n_units, sm_count());
   ProfScope ps(p, st, KID_CAND_TC);
   if (d_h == 128)
-    return p.KC == 8 ? launch_tc<4, 8>(mK, mV, mRK, mRV, P, grid, st)
-                     : launch_tc<4, 12>(mK, mV, mRK, mRV, P, grid, st);
-  return p.KC == 8 ? launch_tc<2, 8>(mK, mV, mRK, mRV, P, grid, st)
-                   : launch_tc<2, 12>(mK, mV, mRK, mRV, P, grid, st);
+    return p.KC == 8 ? launch_tc<4, 8>(mRK, mRV, P, grid, st) : launch_tc<4, 12>(mRK, mRV, P, grid, st);
+  return p.KC == 8 ? launch_tc<2, 8>(mRK, mRV, P, grid, st) : launch_tc<2, 12>(mRK, mRV, P, grid, st);
 }
 
 }  // namespace dkv
