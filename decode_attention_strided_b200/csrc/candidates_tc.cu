@@ -102,6 +102,28 @@ __device__ __forceinline__ bool unit_of(const TcParams& P, int round, UnitInfo& 
   return true;
 }
 
+// (a0, a1) - (b0, b1) as one packed fp32x2 subtraction.
+__device__ __forceinline__ void sub_f32x2(float& o0, float& o1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 x, y, z;\n\t"
+      "mov.b64 x, {%2, %3};\n\tmov.b64 y, {%4, %5};\n\t"
+      "sub.rn.f32x2 z, x, y;\n\tmov.b64 {%0, %1}, z;\n\t}"
+      : "=f"(o0), "=f"(o1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+__device__ __forceinline__ float min3f(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Minimum of 16 consecutive values (eight three-input minima).
+__device__ __forceinline__ float min16(const float* v) {
+  const float a0 = min3f(v[0], v[1], v[2]), a1 = min3f(v[3], v[4], v[5]), a2 = min3f(v[6], v[7], v[8]);
+  const float a3 = min3f(v[9], v[10], v[11]), a4 = min3f(v[12], v[13], v[14]);
+  return fminf(min3f(a0, a1, a2), min3f(a3, a4, v[15]));
+}
+
 // One 64-column block of one token row's accumulator: e = |r_j|^2 / 2 -
 // <x_t, r_j> for slots jb .. jb + 63, folded into the row's running list.
 template <int KC>
@@ -111,10 +133,8 @@ __device__ __forceinline__ void cand_block(float (&v)[64], const float* hn, int 
 #pragma unroll
   for (int x4 = 0; x4 < 16; ++x4) {
     const float4 t4 = __ldg(h4 + x4);
-    v[4 * x4] = t4.x - v[4 * x4];
-    v[4 * x4 + 1] = t4.y - v[4 * x4 + 1];
-    v[4 * x4 + 2] = t4.z - v[4 * x4 + 2];
-    v[4 * x4 + 3] = t4.w - v[4 * x4 + 3];
+    sub_f32x2(v[4 * x4], v[4 * x4 + 1], t4.x, t4.y, v[4 * x4], v[4 * x4 + 1]);
+    sub_f32x2(v[4 * x4 + 2], v[4 * x4 + 3], t4.z, t4.w, v[4 * x4 + 2], v[4 * x4 + 3]);
   }
   if (jb + 64 > cnt_lo) {
 #pragma unroll
@@ -127,40 +147,36 @@ __device__ __forceinline__ void cand_block(float (&v)[64], const float* hn, int 
     for (int x = 0; x < 64; ++x) topk_insert_inorder<KC>(bd, bi, v[x], jb + x);
     return;
   }
-  // fast path: most blocks hold nothing below any lane's k-th best
-  float mn[32];
+  // fast path: most blocks hold nothing below any lane's k-th best; the
+  // per-chunk minima also let the slow path skip chunks without a candidate
+  float cm[64 / tcc::CHUNK];
 #pragma unroll
-  for (int x = 0; x < 32; ++x) mn[x] = fminf(v[x], v[x + 32]);
-#pragma unroll
-  for (int w = 16; w >= 1; w >>= 1)
-#pragma unroll
-    for (int x = 0; x < w; ++x) mn[x] = fminf(mn[x], mn[x + w]);
-  if (!__any_sync(0xffffffffu, mn[0] < bd[KC - 1])) return;
+  for (int c = 0; c < 64 / tcc::CHUNK; ++c) cm[c] = min16(v + c * tcc::CHUNK);
+  if (!__any_sync(0xffffffffu, fminf(min3f(cm[0], cm[1], cm[2]), cm[3]) < bd[KC - 1])) return;
 #pragma unroll
   for (int c = 0; c < 64 / tcc::CHUNK; ++c) {
     const float thr = bd[KC - 1];
+    if (!__any_sync(0xffffffffu, cm[c] < thr)) continue;
     // four independent partial masks keep the dependency chains short
     uint32_t mp[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
     for (int x = 0; x < tcc::CHUNK; ++x) mp[x & 3] |= (v[c * tcc::CHUNK + x] < thr ? 1u : 0u) << x;
     uint32_t m = (mp[0] | mp[1]) | (mp[2] | mp[3]);
-    if (__any_sync(0xffffffffu, m != 0)) {
-      if (m) {
+    if (m) {
 #pragma unroll
-        for (int i4 = 0; i4 < tcc::CHUNK / 4; ++i4)
-          reinterpret_cast<float4*>(sp)[i4 ^ sw] =
-              make_float4(v[c * tcc::CHUNK + 4 * i4], v[c * tcc::CHUNK + 4 * i4 + 1], v[c * tcc::CHUNK + 4 * i4 + 2],
-                          v[c * tcc::CHUNK + 4 * i4 + 3]);
-      }
-      __syncwarp();
-      while (m) {
-        const int x = __ffs(m) - 1;
-        m &= m - 1;
-        const float vx = sp[(((x >> 2) ^ sw) << 2) | (x & 3)];
-        topk_insert_inorder<KC>(bd, bi, vx, jb + c * tcc::CHUNK + x);
-      }
-      __syncwarp();
+      for (int i4 = 0; i4 < tcc::CHUNK / 4; ++i4)
+        reinterpret_cast<float4*>(sp)[i4 ^ sw] =
+            make_float4(v[c * tcc::CHUNK + 4 * i4], v[c * tcc::CHUNK + 4 * i4 + 1], v[c * tcc::CHUNK + 4 * i4 + 2],
+                        v[c * tcc::CHUNK + 4 * i4 + 3]);
     }
+    __syncwarp();
+    while (m) {
+      const int x = __ffs(m) - 1;
+      m &= m - 1;
+      const float vx = sp[(((x >> 2) ^ sw) << 2) | (x & 3)];
+      topk_insert_inorder<KC>(bd, bi, vx, jb + c * tcc::CHUNK + x);
+    }
+    __syncwarp();
   }
 }
 

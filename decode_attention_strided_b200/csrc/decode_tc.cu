@@ -188,13 +188,10 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
   auto sU = [&](int i) { return base + L.u + i * u_b; };
   auto sP = [&](int i) { return base + L.p + i * 2 * 16 * 128; };
   float* fl = (float*)(base + L.fl);
-  float* m_run = fl;          // [8]
-  float* l_run = fl + 8;      // [8]
-  float* alpha = fl + 16;     // [2][8] per chunk parity
-  float* m_ref = fl + 32;     // [8]
-  float* ctv = fl + 40;       // [8]
-  float* mred = fl + 48;      // [4][8]
-  float* lred = fl + 80;      // [4][8]
+  float* m_ref = fl;          // [8]     segment's reference-logit maximum
+  float* ctv = fl + 8;        // [8]     segment's constant logit term
+  float* lred = fl + 16;      // [4][8]  per-warp denominators at a segment end
+  float* mred = fl + 48;      // [2][4][8] per-warp chunk maxima, by chunk parity
   uint64_t* bar = (uint64_t*)(base + L.bar);
   uint64_t* in_full = bar + 0;    // [2]
   uint64_t* in_empty = bar + 2;   // [2]
@@ -232,12 +229,12 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&in_full[i], 1);
-      mbar_init(&in_empty[i], 2);
+      mbar_init(&in_empty[i], 1 + dtc::SMX);  // the GEMM1 commit and the softmax warps
       mbar_init(&u_full[i], dtc::ACT);
       mbar_init(&u_empty[i], 1);
       mbar_init(&z_full[i], 1);
       mbar_init(&z_empty[i], dtc::SMX);
-      mbar_init(&p_full[i], 1);
+      mbar_init(&p_full[i], dtc::SMX);
       mbar_init(&p_empty[i], 1);
       mbar_init(&ua_full[i], 1);
       mbar_init(&ua_empty[i], dtc::SMX);
@@ -422,9 +419,16 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
     // ---------------------------------------------------- softmax warps
     const int sw = warp - (dtc::ACT0 + dtc::ACT);   // 0..3
     const int q = warp & 3, n = q * 32 + lane;      // token row / hidden unit in a half
-    float Ureg[2][kMaxG];
+    // per-thread copies of the segment state (identical in every thread,
+    // except lt: this thread's own share of the softmax denominator)
+    // (the segment's reference maximum and constant term stay in shared memory)
+    float Ureg[2][kMaxG], m_run[kMaxG], lt[kMaxG], alpha_prev[kMaxG];
 #pragma unroll
-    for (int g = 0; g < kMaxG; ++g) Ureg[0][g] = Ureg[1][g] = 0.f;
+    for (int g = 0; g < kMaxG; ++g) {
+      Ureg[0][g] = Ureg[1][g] = 0.f;
+      m_run[g] = lt[g] = 0.f;
+      alpha_prev[g] = 1.f;
+    }
     bool ok = true;
     int prev_bh = -1;
     for (int it = 0; it < n_local && ok; ++it) {
@@ -440,13 +444,15 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
           float m = -INFINITY;
           for (int r = 0; r < P.n_refblk; ++r) m = fmaxf(m, P.Smax[((int64_t)bh * P.n_refblk_cap + r) * G + g]);
           m_ref[g] = m;
-          m_run[g] = m;
-          l_run[g] = 0.f;
           ctv[g] = P.cterm[(int64_t)bh * G + g];
         }
-#pragma unroll
-        for (int g = 0; g < kMaxG; ++g) Ureg[0][g] = Ureg[1][g] = 0.f;
         named_bar(3, dtc::SMX * 32);
+#pragma unroll
+        for (int g = 0; g < kMaxG; ++g) {
+          m_run[g] = g < G ? m_ref[g] : 0.f;
+          lt[g] = 0.f;
+          Ureg[0][g] = Ureg[1][g] = 0.f;
+        }
       }
       // reference logits S[idx]: loads issued before the wait on z
       const int64_t row = row0 + n;
@@ -495,30 +501,33 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
         }
       }
       const float inv_k = 1.0f / (float)max(k_eff, 1);
-      float mx[kMaxG];
+      // chunk maximum of every head's logits: warp reduction, then across the
+      // four warps through a slot pair indexed by chunk parity
 #pragma unroll
       for (int g = 0; g < kMaxG; ++g) {
-        lg[g] = g < G ? zz[2 * g] + zz[2 * g + 1] + ctv[g] + lg[g] * inv_k : 0.f;
-        mx[g] = valid && g < G ? lg[g] : -INFINITY;
-        if (g < G) mx[g] = warp_max(mx[g]);
-      }
-      if (lane == 0) {
-#pragma unroll
-        for (int g = 0; g < kMaxG; ++g)
-          if (g < G) mred[sw * 8 + g] = mx[g];
+        if (g < G) {
+          lg[g] = zz[2 * g] + zz[2 * g + 1] + ctv[g] + lg[g] * inv_k;
+          float wm;
+          const float mv = valid ? lg[g] : -INFINITY;
+          asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(wm) : "f"(mv));
+          if (lane == 0) mred[zb * 32 + sw * 8 + g] = wm;
+        }
       }
       named_bar(3, dtc::SMX * 32);
-      float mnew[kMaxG], p[kMaxG];
+      float p[kMaxG], mnew[kMaxG], alpha[kMaxG];
 #pragma unroll
       for (int g = 0; g < kMaxG; ++g) {
         if (g < G) {
           float m = m_run[g];
-          for (int w = 0; w < dtc::SMX; ++w) m = fmaxf(m, mred[w * 8 + g]);
+#pragma unroll
+          for (int w = 0; w < dtc::SMX; ++w) m = fmaxf(m, mred[zb * 32 + w * 8 + g]);
           mnew[g] = m;
+          alpha[g] = exp2f(m_run[g] - m);
           p[g] = valid ? exp2f(lg[g] - m) : 0.f;
+          lt[g] = lt[g] * alpha[g] + p[g];
+          m_run[g] = m;
         } else {
-          mnew[g] = 0.f;
-          p[g] = 0.f;
+          mnew[g] = alpha[g] = p[g] = 0.f;
         }
       }
       if (!mbar_wait(&p_empty[zb], ((it >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
@@ -529,7 +538,11 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
         for (int g = 0; g < kMaxG; ++g)
           if (g < G) *reinterpret_cast<__half*>(pt + atom * 16 * 128 + swz_off(g, cc * 2, 128)) = __float2half_rn(p[g]);
       }
-      // slot weights, relative to m_ref, into the kv-head's global table
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[zb]);
+      // slot weights, relative to the reference maximum, into the kv-head's
+      // global table
       if (valid && k_eff > 0) {
         float* wt = P.wtab + (int64_t)bh * P.n_ref_cap * G;
         float sc[kMaxG];
@@ -549,30 +562,8 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
           }
         }
       }
-      float ls[kMaxG];
-#pragma unroll
-      for (int g = 0; g < kMaxG; ++g) ls[g] = g < G ? warp_sum(p[g]) : 0.f;
-      if (lane == 0) {
-#pragma unroll
-        for (int g = 0; g < kMaxG; ++g)
-          if (g < G) lred[sw * 8 + g] = ls[g];
-      }
-      fence_async_smem();
-      named_bar(3, dtc::SMX * 32);
-      if (sw == 0 && lane < G) {
-        const int g = lane;
-        const float al = exp2f(m_run[g] - mnew[g]);
-        alpha[zb * 8 + g] = al;
-        float lc = 0.f;
-        for (int w = 0; w < dtc::SMX; ++w) lc += lred[w * 8 + g];
-        l_run[g] = l_run[g] * al + lc;
-        m_run[g] = mnew[g];
-      }
-      named_bar(3, dtc::SMX * 32);
-      if (sw == 0 && lane == 0) {
-        mbar_arrive(&p_full[zb]);
-        mbar_arrive(&in_empty[st]);
-      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&in_empty[st]);  // this warp is done with the chunk's slots
       // fold the previous chunk's U (its MMA was issued after this chunk's z)
       const bool seg_end = (it == n_local - 1) || ((x + 1) / P.n_ch != bh);
       const bool prev_same = it >= 1 && (x - 1) / P.n_ch == bh;
@@ -591,7 +582,7 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
             tmem_ld16f(tmem + ((uint32_t)(q * 32) << 16) + dtc::COL_U + 32 * jb + 16 * h2, du);
 #pragma unroll
             for (int g = 0; g < kMaxG; ++g)
-              if (g < G) Ureg[h2][g] = Ureg[h2][g] * alpha[jb * 8 + g] + du[g];
+              if (g < G) Ureg[h2][g] = Ureg[h2][g] * (pass == 0 ? alpha_prev[g] : alpha[g]) + du[g];
           }
         }
         tc_fence_before();
@@ -599,6 +590,8 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
         if (lane == 0) mbar_arrive(&ua_empty[jb]);
       }
       if (!ok) break;
+#pragma unroll
+      for (int g = 0; g < kMaxG; ++g) alpha_prev[g] = alpha[g];
       if (seg_end) {
         const int64_t pb = (int64_t)bh * P.nslot_cap + (int64_t)blockIdx.x - dtc_owner((int64_t)bh * P.n_ch, P.N, P.grid);
 #pragma unroll
@@ -610,9 +603,24 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
               if (g < G) P.Upart[(pb * G + g) * hidden + unit] = Ureg[h2][g];
           }
         }
+        // the segment's softmax denominator: this thread's shares, summed
+#pragma unroll
+        for (int g = 0; g < kMaxG; ++g) {
+          if (g < G) {
+            const float ls = warp_sum(lt[g]);
+            if (lane == 0) lred[sw * 8 + g] = ls;
+          }
+        }
+        named_bar(3, dtc::SMX * 32);
         if (sw == 0 && lane < G) {
-          P.part[(pb * G + lane) * 2 + 0] = m_run[lane];
-          P.part[(pb * G + lane) * 2 + 1] = l_run[lane];
+          float l = 0.f;
+          for (int w = 0; w < dtc::SMX; ++w) l += lred[w * 8 + lane];
+          float mr = m_run[0];
+#pragma unroll
+          for (int g = 1; g < kMaxG; ++g)
+            if (lane == g) mr = m_run[g];
+          P.part[(pb * G + lane) * 2 + 0] = mr;
+          P.part[(pb * G + lane) * 2 + 1] = l;
         }
       }
     }
