@@ -58,6 +58,33 @@ __device__ __forceinline__ float gelu_fast(float x) {
   return fmaxf(x, 0.0f) - p;
 }
 
+// gelu_fast on two values at once: the same operations, with the polynomial
+// evaluated by packed fp32x2 FMAs (each lane rounds exactly as fmaf does, so
+// the results equal two gelu_fast calls bit for bit).
+__device__ __forceinline__ float2 gelu_fast2(float x0, float x1) {
+  unsigned long long t, p, c;
+  const float a0 = fminf(fabsf(x0), 5.0f), a1 = fminf(fabsf(x1), 5.0f);
+  asm("{\n\t.reg .b64 a, s, o;\n\t"
+      "mov.b64 a, {%1, %2};\n\t"
+      "mov.b64 s, {%3, %3};\n\t"
+      "mov.b64 o, {%4, %4};\n\t"
+      "fma.rn.f32x2 %0, a, s, o;\n\t}"
+      : "=l"(t)
+      : "f"(a0), "f"(a1), "f"(0.4f), "f"(-1.0f));
+  const float k[12] = {4.889592901e-02f,  -7.081953436e-02f, -1.480407715e-01f, 3.208711743e-01f,
+                       1.524367370e-02f,  -4.781557322e-01f, 4.370784760e-01f,  -2.034248412e-02f,
+                       -2.592293620e-01f, 2.329209447e-01f,  -9.394139796e-02f, 1.552190445e-02f};
+  asm("mov.b64 %0, {%1, %1};" : "=l"(p) : "f"(k[0]));
+#pragma unroll
+  for (int i = 1; i < 12; ++i) {
+    asm("mov.b64 %0, {%1, %1};" : "=l"(c) : "f"(k[i]));
+    asm("fma.rn.f32x2 %0, %0, %1, %2;" : "+l"(p) : "l"(t), "l"(c));
+  }
+  float p0, p1;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(p0), "=f"(p1) : "l"(p));
+  return make_float2(fmaxf(x0, 0.0f) - p0, fmaxf(x1, 0.0f) - p1);
+}
+
 // The activation inside the tensor-core kernels: exact GELU through
 // gelu_fast, the other forms as in act_eval.
 __device__ __forceinline__ float act_fast(int act, float z) {

@@ -397,9 +397,20 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
         tmem_ld32(trow + c0, v);
         __align__(16) __half2 h2[16];
 #pragma unroll
-        for (int x2 = 0; x2 < 16; ++x2)
-          h2[x2] = __floats2half2_rn(dec_act<ACT, HAS_B3>(v[2 * x2], P.b3, c0 + 2 * x2),
-                                     dec_act<ACT, HAS_B3>(v[2 * x2 + 1], P.b3, c0 + 2 * x2 + 1));
+        for (int x2 = 0; x2 < 16; ++x2) {
+          if (ACT == DELTAKV_ACT_GELU_ERF) {
+            float z0 = v[2 * x2], z1 = v[2 * x2 + 1];
+            if (HAS_B3) {
+              z0 += P.b3[c0 + 2 * x2];
+              z1 += P.b3[c0 + 2 * x2 + 1];
+            }
+            const float2 g2 = gelu_fast2(z0, z1);
+            h2[x2] = __floats2half2_rn(g2.x, g2.y);
+          } else {
+            h2[x2] = __floats2half2_rn(dec_act<ACT, HAS_B3>(v[2 * x2], P.b3, c0 + 2 * x2),
+                                       dec_act<ACT, HAS_B3>(v[2 * x2 + 1], P.b3, c0 + 2 * x2 + 1));
+          }
+        }
         const int atom = c0 >> 6, cc = c0 & 63;
 #pragma unroll
         for (int v4 = 0; v4 < 4; ++v4)

@@ -350,17 +350,25 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
           for (int u = 0; u < NB; ++u) {
             float part = 0.f;
             if (cj[c0 + u] >= 0) {
+              // even and odd elements accumulate in the two lanes of a packed
+              // fp32x2 register
+              unsigned long long acc = 0ull;
 #pragma unroll
               for (int i = 0; i < RowPack<EPL>::V4; ++i) {
                 const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&rr[u][i]);
 #pragma unroll
                 for (int x = 0; x < 4; ++x) {
                   const float2 v = __bfloat1622float2(p2[x]);
-                  const float d0 = xr[8 * i + 2 * x] - v.x, d1 = xr[8 * i + 2 * x + 1] - v.y;
-                  part = fmaf(d0, d0, part);
-                  part = fmaf(d1, d1, part);
+                  asm("{\n\t.reg .b64 a, b, d;\n\t"
+                      "mov.b64 a, {%1, %2};\n\tmov.b64 b, {%3, %4};\n\t"
+                      "sub.rn.f32x2 d, a, b;\n\tfma.rn.f32x2 %0, d, d, %0;\n\t}"
+                      : "+l"(acc)
+                      : "f"(xr[8 * i + 2 * x]), "f"(xr[8 * i + 2 * x + 1]), "f"(v.x), "f"(v.y));
                 }
               }
+              float e0, e1;
+              asm("mov.b64 {%0, %1}, %2;" : "=f"(e0), "=f"(e1) : "l"(acc));
+              part = e0 + e1;
             }
             part = group16_sum(part);
             cd[c0 + u] = cj[c0 + u] >= 0 ? part : FLT_MAX;
@@ -519,9 +527,15 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
           for (int c4 = 0; c4 < 4; ++c4) {
             __half2 hi2[4], lo2[4];
 #pragma unroll
-            for (int x = 0; x < 4; ++x)
-              split_half2(enc_act<ACT>(v[8 * c4 + 2 * x] + bias), enc_act<ACT>(v[8 * c4 + 2 * x + 1] + bias),
-                          hi2[x], lo2[x]);
+            for (int x = 0; x < 4; ++x) {
+              if (ACT == DELTAKV_ACT_GELU_ERF) {
+                const float2 g2 = gelu_fast2(v[8 * c4 + 2 * x] + bias, v[8 * c4 + 2 * x + 1] + bias);
+                split_half2(g2.x, g2.y, hi2[x], lo2[x]);
+              } else {
+                split_half2(enc_act<ACT>(v[8 * c4 + 2 * x] + bias), enc_act<ACT>(v[8 * c4 + 2 * x + 1] + bias),
+                            hi2[x], lo2[x]);
+              }
+            }
             // MN-major row `unit` of 64 tokens: 16-byte chunk c8, swizzled by row
             const int c8 = 4 * cc + c4;
             const uint32_t off = (uint32_t)unit * 128 + (((c8 ^ (unit & 7))) << 4);
