@@ -69,6 +69,16 @@ BF16_CASES = [
                             act=dkv.ACT_GELU_TANH, biases=True)),
     ("identity_act_tc", Case(B=1, H=1, Hq=2, d_h=64, T=1800, s=4, k=2, d_c=32, hidden=128, dtype=dkv.BF16,
                              act=dkv.ACT_NONE, biases=True)),
+    # points of the single-layer sweep (d_h 128, bf16, hidden 256, 8 latent
+    # directions), two kv-heads each so that the oracle covers every row
+    ("sweep_s4_k1_dc16", Case(B=1, H=2, Hq=8, d_h=128, T=4096, s=4, k=1, d_c=16, hidden=256, dtype=dkv.BF16,
+                              n_lat=8)),
+    ("sweep_s8_k2_dc64", Case(B=1, H=1, Hq=4, d_h=128, T=16384, s=8, k=2, d_c=64, hidden=256, dtype=dkv.BF16,
+                              n_lat=8)),
+    ("sweep_s32_k8_dc32", Case(B=1, H=2, Hq=8, d_h=128, T=16384, s=32, k=8, d_c=32, hidden=256, dtype=dkv.BF16,
+                               n_lat=8)),
+    ("sweep_s16_k4_dc16", Case(B=1, H=2, Hq=8, d_h=128, T=8192, s=16, k=4, d_c=16, hidden=256, dtype=dkv.BF16,
+                               n_lat=8)),
 ]
 
 # kernels each case must have run: the tensor-core paths where the shape allows
@@ -79,6 +89,10 @@ TC_EXPECT = {
     "d_h64_tc": {"candidates_tc", "encode_tc", "decode_stream_tc"},
     "biases_tanh_tc": {"candidates_tc", "encode_tc", "decode_stream_tc"},
     "identity_act_tc": {"encode_tc", "decode_stream_simt"},
+    "sweep_s4_k1_dc16": {"candidates_tc", "encode_tc", "decode_stream_tc"},
+    "sweep_s8_k2_dc64": {"candidates_tc", "encode_tc", "decode_stream_tc"},
+    "sweep_s32_k8_dc32": {"candidates_tc", "encode_tc", "decode_stream_tc"},
+    "sweep_s16_k4_dc16": {"candidates_tc", "encode_tc", "decode_stream_tc"},
 }
 
 
