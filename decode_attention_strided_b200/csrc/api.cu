@@ -85,6 +85,8 @@ void build_plan(const deltakv_config& c, Plan& p) {
   w = align256(w + (size_t)(BH * p.G * c.hidden) * 4);
   p.ws_cterm = w;
   w = align256(w + (size_t)(BH * p.G) * 4);
+  p.ws_mref = w;
+  w = align256(w + (size_t)(BH * p.G) * 4);
   p.ws_wtab = w;
   w = align256(w + (size_t)(BH * p.n_ref_cap * p.G) * 4);
   p.ws_part = w;

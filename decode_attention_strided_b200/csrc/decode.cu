@@ -96,10 +96,34 @@ __global__ void __launch_bounds__(256)
     decode_prep_kernel(int d_h, int H, int G, int hidden, float c, const T* __restrict__ q,
                        int64_t qsb, int64_t qsh, const T* __restrict__ W4,
                        const float* __restrict__ b4, float* __restrict__ a,
-                       float* __restrict__ cterm) {
+                       float* __restrict__ cterm, const float* __restrict__ Smax, int n_refblk,
+                       int n_refblk_cap, float* __restrict__ mref) {
   __shared__ float qs[kMaxG][128];
+  __shared__ float wm[8][kMaxG];
   const int b = blockIdx.z, h = blockIdx.y;
   const int64_t bh = (int64_t)b * H + h;
+  {
+    // m_ref = max_j S_j of this (sequence, kv-head), from the per-block maxima
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float m[kMaxG];
+#pragma unroll
+    for (int g = 0; g < kMaxG; ++g) m[g] = -INFINITY;
+    for (int r = threadIdx.x; r < n_refblk; r += blockDim.x)
+#pragma unroll
+      for (int g = 0; g < kMaxG; ++g)
+        if (g < G) m[g] = fmaxf(m[g], Smax[(bh * n_refblk_cap + r) * G + g]);
+#pragma unroll
+    for (int g = 0; g < kMaxG; ++g) {
+      const float wmax = warp_max(m[g]);
+      if (lane == 0 && g < G) wm[warp][g] = wmax;
+    }
+    __syncthreads();
+    if (threadIdx.x < G) {
+      float r = wm[0][threadIdx.x];
+      for (int w = 1; w < (int)(blockDim.x >> 5); ++w) r = fmaxf(r, wm[w][threadIdx.x]);
+      mref[bh * G + threadIdx.x] = r;
+    }
+  }
   for (int i = threadIdx.x; i < G * d_h; i += blockDim.x) {
     int g = i / d_h, e = i - g * d_h;
     qs[g][e] = c * to_f(q[b * qsb + (int64_t)(h * G + g) * qsh + e]);
@@ -307,66 +331,129 @@ __device__ __forceinline__ int slots_of(const SlotInfo& si, int64_t bh) {
   return (int)(last - first + 1);
 }
 
+// Eight consecutive elements as floats (16-byte aligned for bf16, 32 for fp32).
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
+  const uint4 r = __ldg(reinterpret_cast<const uint4*>(p));
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&r);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+__device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p)), b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
 // -------------------------------------------------------- decode_combine
 // M_g = max(m_ref, split maxima).  For 256 slots: weights
 // w_j = 2^(S_j - M) + 2^(m_ref - M) sum_splits wtab, then sum_j w_j V_ref_j.
 template <typename T>
 __global__ void __launch_bounds__(256)
     decode_combine_kernel(int T_, int s, int d_h, int H, int G, SlotInfo si, int64_t n_ref_cap,
-                          int n_refblk, int n_refblk_cap, int n_chunk_cap,
-                          const T* __restrict__ refv, const float* __restrict__ S,
-                          const float* __restrict__ Smax, const float* __restrict__ wtab_g,
+                          int n_chunk_cap, const T* __restrict__ refv, const float* __restrict__ S,
+                          const float* __restrict__ mref, const float* __restrict__ wtab_g,
                           const float* __restrict__ part, float* __restrict__ ochunk) {
   __shared__ float wts[kCombineSlots][kMaxG];
-  __shared__ float Mg[kMaxG], mrefg[kMaxG], lref[kMaxG];
+  __shared__ float Mg[kMaxG], mrefg[kMaxG], lw[8][kMaxG];
+  __shared__ float red[8][kMaxG][128];
   const int b = blockIdx.z, h = blockIdx.y, ch = blockIdx.x, tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
   const int64_t bh = (int64_t)b * H + h;
   const int64_t n_ref = (T_ + s - 1) / s;
   const int64_t j0 = (int64_t)ch * kCombineSlots;
   if (tid < G) {
-    float m = -INFINITY;
-    for (int r = 0; r < n_refblk; ++r) m = fmaxf(m, Smax[(bh * n_refblk_cap + r) * G + tid]);
+    const float m = mref[bh * G + tid];
     mrefg[tid] = m;
     float M = m;
     const int ns = slots_of(si, bh);
     for (int sp = 0; sp < ns; ++sp) M = fmaxf(M, part[((bh * si.nslot_cap + sp) * G + tid) * 2]);
     Mg[tid] = M;
-    lref[tid] = 0.f;
   }
   __syncthreads();
-  for (int i = tid; i < kCombineSlots * G; i += blockDim.x) {
-    int jj = i / G, g = i - jj * G;
-    int64_t j = j0 + jj;
-    float w = 0.f;
-    if (j < n_ref) {
-      float own = exp2f(S[(bh * n_ref_cap + j) * G + g] - Mg[g]);
-      w = own + wtab_g[(bh * n_ref_cap + j) * G + g] * exp2f(mrefg[g] - Mg[g]);
-      atomicAdd(&lref[g], own);
+  float lsum[kMaxG];
+#pragma unroll
+  for (int g = 0; g < kMaxG; ++g) lsum[g] = 0.f;
+  for (int jj = tid; jj < kCombineSlots; jj += blockDim.x) {
+    const int64_t j = j0 + jj;
+#pragma unroll
+    for (int g = 0; g < kMaxG; ++g) {
+      if (g < G) {
+        float w = 0.f;
+        if (j < n_ref) {
+          const float own = exp2f(S[(bh * n_ref_cap + j) * G + g] - Mg[g]);
+          w = own + wtab_g[(bh * n_ref_cap + j) * G + g] * exp2f(mrefg[g] - Mg[g]);
+          lsum[g] += own;
+        }
+        wts[jj][g] = w;
+      }
     }
-    wts[jj][g] = w;
+  }
+#pragma unroll
+  for (int g = 0; g < kMaxG; ++g) {
+    const float ls = warp_sum(lsum[g]);
+    if (lane == 0 && g < G) lw[warp][g] = ls;
   }
   __syncthreads();
+  // sum_j w_j V_ref_j: thread = (slot group, 8 consecutive elements); every
+  // V row segment is loaded once (16 bytes of bf16) for all heads of the group
   const T* vb = refv + bh * n_ref_cap * d_h;
-  for (int o = tid; o < G * d_h; o += blockDim.x) {
-    int g = o / d_h, e = o - g * d_h;
-    float acc = 0.f;
-    for (int jj = 0; jj < kCombineSlots; ++jj) {
-      int64_t j = j0 + jj;
-      if (j >= n_ref) break;
-      acc = fmaf(wts[jj][g], to_f(vb[j * d_h + e]), acc);
+  const int eg = d_h / 8, e8 = tid % eg, js = tid / eg, njs = blockDim.x / eg;
+  float acc[kMaxG][8];
+#pragma unroll
+  for (int g = 0; g < kMaxG; ++g)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[g][i] = 0.f;
+  for (int jj = js; jj < kCombineSlots; jj += njs) {
+    const int64_t j = j0 + jj;
+    if (j >= n_ref) break;
+    float v[8];
+    load8(vb + j * d_h + e8 * 8, v);
+#pragma unroll
+    for (int g = 0; g < kMaxG; ++g) {
+      if (g < G) {
+        const float w = wts[jj][g];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[g][i] = fmaf(w, v[i], acc[g][i]);
+      }
     }
-    ochunk[((bh * n_chunk_cap + ch) * G + g) * (d_h + 1) + e] = acc;
   }
-  if (tid < G) ochunk[((bh * n_chunk_cap + ch) * G + tid) * (d_h + 1) + d_h] = lref[tid];
+  // lanes that share e8 hold different slot groups: fold them, then the warps
+  for (int o = eg; o < 32; o <<= 1)
+#pragma unroll
+    for (int g = 0; g < kMaxG; ++g)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[g][i] += __shfl_xor_sync(0xffffffffu, acc[g][i], o);
+  if (lane < eg) {
+#pragma unroll
+    for (int g = 0; g < kMaxG; ++g)
+      if (g < G)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) red[warp][g][e8 * 8 + i] = acc[g][i];
+  }
+  __syncthreads();
+  for (int o = tid; o < G * d_h; o += blockDim.x) {
+    const int g = o / d_h, e = o - g * d_h;
+    float sum = 0.f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) sum += red[w][g][e];
+    ochunk[((bh * n_chunk_cap + ch) * G + g) * (d_h + 1) + e] = sum;
+  }
+  if (tid < G) {
+    float l = 0.f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) l += lw[w][tid];
+    ochunk[((bh * n_chunk_cap + ch) * G + tid) * (d_h + 1) + d_h] = l;
+  }
 }
 
 // ---------------------------------------------------------- decode_final
 template <typename T>
 __global__ void __launch_bounds__(256)
     decode_final_kernel(int T_, int s, int d_h, int H, int G, int hidden, SlotInfo si, int n_chunk,
-                        int n_chunk_cap, int n_refblk, int n_refblk_cap,
-                        const T* __restrict__ W4, const float* __restrict__ b4,
-                        const float* __restrict__ Smax, const float* __restrict__ part,
+                        int n_chunk_cap, const T* __restrict__ W4, const float* __restrict__ b4,
+                        const float* __restrict__ mref, const float* __restrict__ part,
                         const float* __restrict__ Upart, const float* __restrict__ ochunk,
                         float* __restrict__ out, int64_t osb, int64_t osh) {
   __shared__ float Ut[kMaxG][kMaxHidden];
@@ -375,21 +462,29 @@ __global__ void __launch_bounds__(256)
   const int64_t bh = (int64_t)b * H + h;
   const int ns = slots_of(si, bh);
   const int64_t pb0 = bh * si.nslot_cap;
-  if (tid < G) {
-    float M = -INFINITY;
-    for (int r = 0; r < n_refblk; ++r) M = fmaxf(M, Smax[(bh * n_refblk_cap + r) * G + tid]);
-    for (int sp = 0; sp < ns; ++sp) M = fmaxf(M, part[((pb0 + sp) * G + tid) * 2]);
-    float lnr = 0.f;
-    for (int sp = 0; sp < ns; ++sp) {
-      float m = part[((pb0 + sp) * G + tid) * 2];
-      float l = part[((pb0 + sp) * G + tid) * 2 + 1];
-      if (m != -INFINITY) lnr += l * exp2f(m - M);
+  {
+    // warp g: the maximum, the token-loop denominator and the reference
+    // denominator of head g (the chunks' sums split over the lanes)
+    const int warp = tid >> 5, lane = tid & 31;
+    for (int g = warp; g < G; g += (int)(blockDim.x >> 5)) {
+      float M = mref[bh * G + g];
+      for (int sp = 0; sp < ns; ++sp) M = fmaxf(M, part[((pb0 + sp) * G + g) * 2]);
+      float lnr = 0.f;
+      for (int sp = lane; sp < ns; sp += 32) {
+        float m = part[((pb0 + sp) * G + g) * 2];
+        float l = part[((pb0 + sp) * G + g) * 2 + 1];
+        if (m != -INFINITY) lnr += l * exp2f(m - M);
+      }
+      float lr = 0.f;
+      for (int c = lane; c < n_chunk; c += 32) lr += ochunk[((bh * n_chunk_cap + c) * G + g) * (d_h + 1) + d_h];
+      lnr = warp_sum(lnr);
+      lr = warp_sum(lr);
+      if (lane == 0) {
+        Mg[g] = M;
+        Lnr[g] = lnr;
+        Lall[g] = lnr + lr;
+      }
     }
-    float lr = 0.f;
-    for (int c = 0; c < n_chunk; ++c) lr += ochunk[((bh * n_chunk_cap + c) * G + tid) * (d_h + 1) + d_h];
-    Mg[tid] = M;
-    Lnr[tid] = lnr;
-    Lall[tid] = lnr + lr;
   }
   __syncthreads();
   for (int i = tid; i < G * hidden; i += blockDim.x) {
@@ -435,6 +530,7 @@ static cudaError_t decode_launch(const Plan& p, int T, const void* q, int64_t qs
   float* Smax = (float*)(w + p.ws_Smax);
   float* a = (float*)(w + p.ws_a);
   float* cterm = (float*)(w + p.ws_cterm);
+  float* mref = (float*)(w + p.ws_mref);
   float* wtab = (float*)(w + p.ws_wtab);
   float* part = (float*)(w + p.ws_part);
   float* Upart = (float*)(w + p.ws_U);
@@ -451,7 +547,8 @@ static cudaError_t decode_launch(const Plan& p, int T, const void* q, int64_t qs
   {
     ProfScope ps(p, st, KID_DEC_PREP);
     decode_prep_kernel<E><<<dim3(1, H, B), 256, 0, st>>>(c.d_h, H, G, c.hidden, cs, (const E*)q, qsb,
-                                                         qsh, (const E*)W4, b4, a, cterm);
+                                                         qsh, (const E*)W4, b4, a, cterm, Smax, n_refblk,
+                                                         n_refblk_cap, mref);
   }
   SlotInfo si{};
   si.nslot_cap = p.nslot_cap;
@@ -489,14 +586,13 @@ static cudaError_t decode_launch(const Plan& p, int T, const void* q, int64_t qs
   {
     ProfScope ps(p, st, KID_DEC_COMBINE);
     decode_combine_kernel<E><<<dim3(n_chunk, H, B), 256, 0, st>>>(
-        T, c.stride_s, c.d_h, H, G, si, p.n_ref_cap, n_refblk, n_refblk_cap, p.n_chunk_cap, refv, S,
-        Smax, wtab, part, ochunk);
+        T, c.stride_s, c.d_h, H, G, si, p.n_ref_cap, p.n_chunk_cap, refv, S, mref, wtab, part, ochunk);
   }
   {
     ProfScope ps(p, st, KID_DEC_FINAL);
     decode_final_kernel<E><<<dim3(1, H, B), 256, 0, st>>>(
-        T, c.stride_s, c.d_h, H, G, c.hidden, si, n_chunk, p.n_chunk_cap, n_refblk, n_refblk_cap,
-        (const E*)W4, b4, Smax, part, Upart, ochunk, out, osb, osh);
+        T, c.stride_s, c.d_h, H, G, c.hidden, si, n_chunk, p.n_chunk_cap, (const E*)W4, b4, mref, part, Upart,
+        ochunk, out, osb, osh);
   }
   return cudaGetLastError();
 }

@@ -22,8 +22,9 @@
 //                  fp16 P tile (two buffers), slot-weight reductions into the
 //                  global table, and the fold of U_chunk into register
 //                  accumulators with the online-softmax rescale
-// The MMA warp issues G1(0); then per chunk i: G1(i+1), z(i), U(i-1), so the
-// activation warps wait only for the next GEMM1, never for z or the softmax.
+// The MMA warp issues G1(0), then polls: G1(i+1) and z(i) go out when the
+// activation of chunk i is done, U(j) when the softmax of chunk j is done, so
+// neither the activation nor the softmax waits behind the other.
 // A persistent grid splits the flattened (kv-head, chunk) list evenly; each
 // CTA writes one partial (m, l, U) per kv-head segment it touches.
 #include <cfloat>
@@ -73,6 +74,7 @@ struct DecTcParams {
   const float* cterm;
   const float* S;
   const float* Smax;
+  const float* mref;  // per (sequence, kv-head, head): max_j S_j
   float* wtab;
   float* part;
   float* Upart;
@@ -276,7 +278,8 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
     }
   } else if (warp == dtc::MMA) {
     // ----------------------------------------------------------------- MMA
-    // order: G1(0); for i: G1(i+1), z(i), U(i-1); U(n-1)
+    // order: G1(0), then as they become ready: G1(i+1) and z(i) after the
+    // activation of chunk i, U(j) after the softmax of chunk j
     if (lane == 0 && n_local > 0) {
       const uint32_t id_g1 = idesc_kind_f16(true, dtc::CH, hidden, false);
       const uint32_t id_z = idesc_kind_f16(false, dtc::CH, 16, false);
@@ -294,9 +297,6 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
       };
       auto issue_u = [&](int j) {
         const int jb = j & 1;
-        if (!mbar_wait(&p_full[jb], (j >> 1) & 1, abort_flag)) return false;
-        if (!mbar_wait(&ua_empty[jb], ((j >> 1) & 1) ^ 1, abort_flag)) return false;
-        tc_fence_after();
         const uint32_t u0 = smem_u32(sU(jb)), p0 = smem_u32(sP(jb));
         for (int h2 = 0; h2 < hidden / 128; ++h2)
           for (int k16 = 0; k16 < dtc::CH / 16; ++k16) {
@@ -308,9 +308,7 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
         umma_commit(&ua_full[jb]);
         umma_commit(&u_empty[jb]);
         umma_commit(&p_empty[jb]);
-        return true;
       };
-      int seg = -1, prev_bh = -1;
       if (mbar_wait(&in_full[0], 0, abort_flag)) {
         tc_fence_after();
         gemm1(0);
@@ -319,26 +317,38 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
       } else {
         ok = false;
       }
-      for (int it = 0; it < n_local && ok; ++it) {
-        const int64_t x = x_begin + it;
-        const int bh = (int)(x / P.n_ch);
-        if (bh != prev_bh) { ++seg; prev_bh = bh; }
-        const int ub = it & 1;
-        if (!mbar_wait(&u_full[ub], (it >> 1) & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        // the activation warps have read D1(it): start the next chunk's GEMM1
-        // first, so they wait only for it and not for z(it) as well
-        if (it + 1 < n_local) {
-          const int st = (it + 1) & 1;
-          if (!mbar_wait(&in_full[st], ((it + 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+      // Event loop: U(j) goes out as soon as the softmax of chunk j is done
+      // (it frees the u buffer that the activation warps need two chunks
+      // later); GEMM1(i+1) and then z(i) as soon as the activation of chunk i
+      // is done.  Neither waits behind the other.
+      int z_next = 0, u_next = 0, seg = -1, prev_bh = -1;
+      uint64_t t_last = globaltimer();
+      uint32_t spins = 0;
+      while (ok && u_next < n_local) {
+        bool did = false;
+        if (u_next < z_next && mbar_try_wait(&p_full[u_next & 1], (u_next >> 1) & 1) &&
+            mbar_try_wait(&ua_empty[u_next & 1], ((u_next >> 1) & 1) ^ 1)) {
           tc_fence_after();
-          gemm1(st);
-          umma_commit(d1_full);
-          umma_commit(&in_empty[st]);
+          issue_u(u_next);
+          ++u_next;
+          did = true;
         }
-        if (!mbar_wait(&z_empty[ub], ((it >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        {
+        if (z_next < n_local && mbar_try_wait(&u_full[z_next & 1], (z_next >> 1) & 1)) {
+          const int it = z_next, ub = it & 1;
+          const int bh = (int)((x_begin + it) / P.n_ch);
+          if (bh != prev_bh) { ++seg; prev_bh = bh; }
+          tc_fence_after();
+          // the activation warps have read D1(it): the next chunk's GEMM1 first
+          if (it + 1 < n_local) {
+            const int st = (it + 1) & 1;
+            if (!mbar_wait(&in_full[st], ((it + 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            gemm1(st);
+            umma_commit(d1_full);
+            umma_commit(&in_empty[st]);
+          }
+          if (!mbar_wait(&z_empty[ub], ((it >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
           const uint32_t u0 = smem_u32(sU(ub)), a0 = smem_u32(sAz(seg & 1));
           for (int k16 = 0; k16 < hidden / 16; ++k16) {
             const int atom = k16 >> 2, off = (k16 & 3) * 32;
@@ -346,10 +356,17 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
                      desc_kmajor(a0 + atom * 16 * 128 + off, 128), id_z, k16 != 0);
           }
           umma_commit(&z_full[ub]);
+          ++z_next;
+          did = true;
         }
-        if (it >= 1 && !issue_u(it - 1)) { ok = false; break; }
+        if (did) {
+          spins = 0;
+        } else if ((++spins & 63) == 0) {
+          const uint64_t now = globaltimer();
+          if (spins == 64) t_last = now;  // first idle check of this stretch
+          if (*abort_flag || now - t_last > kWaitLimitNs) ok = false;
+        }
       }
-      if (ok && !issue_u(n_local - 1)) ok = false;
       if (!ok) {
         latch_error(P.err, DELTAKV_ERR_DEVICE_TIMEOUT, 21);
         *abort_flag = 1;
@@ -452,9 +469,7 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
         named_bar(3, dtc::SMX * 32);
         if (sw == 0 && lane < G) {
           const int g = lane;
-          float m = -INFINITY;
-          for (int r = 0; r < P.n_refblk; ++r) m = fmaxf(m, P.Smax[((int64_t)bh * P.n_refblk_cap + r) * G + g]);
-          m_ref[g] = m;
+          m_ref[g] = P.mref[(int64_t)bh * G + g];
           ctv[g] = P.cterm[(int64_t)bh * G + g];
         }
         named_bar(3, dtc::SMX * 32);
@@ -710,6 +725,7 @@ cudaError_t launch_decode_tc(const Plan& p, int T, const void* cache, const void
   P.W3 = (const __nv_bfloat16*)W3; P.b3 = b3;
   P.a = (const float*)(w + p.ws_a); P.cterm = (const float*)(w + p.ws_cterm);
   P.S = (const float*)(w + p.ws_S); P.Smax = (const float*)(w + p.ws_Smax);
+  P.mref = (const float*)(w + p.ws_mref);
   P.wtab = (float*)(w + p.ws_wtab); P.part = (float*)(w + p.ws_part); P.Upart = (float*)(w + p.ws_U);
   P.err = (uint32_t*)ws;
   CUtensorMap mapC;

@@ -47,7 +47,7 @@ struct Plan {
   // decode workspace
   int nslot_cap;         // decode partial slots per (b, head)
   int n_chunk_cap;       // combine blocks per (b, head)
-  size_t ws_S, ws_Smax, ws_a, ws_cterm, ws_wtab, ws_part, ws_U, ws_ochunk;
+  size_t ws_S, ws_Smax, ws_mref, ws_a, ws_cterm, ws_wtab, ws_part, ws_U, ws_ochunk;
   size_t ws_bytes;
 };
 
