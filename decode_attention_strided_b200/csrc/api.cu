@@ -70,6 +70,8 @@ void build_plan(const deltakv_config& c, Plan& p) {
   size_t w = kErrBytes;
   p.ws_hnorm = w;
   w = align256(w + (size_t)(BH * p.n_ref_cap) * 4);
+  p.ws_hsplit = w;  // 0.5 |x_j|^2 as three bf16 terms in a 16-element row (bf16 caches)
+  w = align256(w + (size_t)(BH * p.n_ref_cap) * 32);
   p.ws_cand = w;
   w = align256(w + (size_t)(BH * p.n_code_cap * p.KC) * 4);
   const size_t compress_end = w;

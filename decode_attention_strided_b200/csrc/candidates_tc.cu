@@ -26,6 +26,9 @@
 // TMEM (512 columns): A of token tile 0 and 1 (D/2 columns each, two bf16
 // per column), then one 128-column accumulator per token tile.  The MMAs of
 // tile 1 run while the epilogue drains tile 0 and the other way round.
+// The ranking key e is formed inside the accumulator: A holds -x_t, and one
+// more K = 16 MMA per tile adds a ones row times the bf16 split of h_j (three
+// terms, 24 significant bits), so the epilogue reads e directly.
 // Shape choices: an M = 128 MMA occupies the tensor pipe for at least about
 // 58 cycles whatever its N, so N = 128 (64 cycles of math) keeps it math-bound;
 // with A in tensor memory each MMA reads only its 4 KB of B from shared
@@ -47,6 +50,7 @@ constexpr int TPU = 2;                      // token tiles per unit
 constexpr int RN = 128;                     // references per tile (MMA N)
 constexpr int NSLOT = 3;                    // reference tiles in flight
 constexpr int BATOM = RN * 128;             // bytes: 128 reference rows x 128 B
+constexpr int HATOM = RN * 32;              // bytes: 128 rows x 16 bf16 (32-byte swizzle)
 constexpr int CHUNK = 16;                   // columns per slow-path chunk
 constexpr int SPILL = 32 * CHUNK * 4;       // bytes per warp: 32 lanes x CHUNK floats
 constexpr int EPI_WARPS = 8;
@@ -102,15 +106,6 @@ __device__ __forceinline__ bool unit_of(const TcParams& P, int round, UnitInfo& 
   return true;
 }
 
-// (a0, a1) - (b0, b1) as one packed fp32x2 subtraction.
-__device__ __forceinline__ void sub_f32x2(float& o0, float& o1, float a0, float a1, float b0, float b1) {
-  asm("{\n\t.reg .b64 x, y, z;\n\t"
-      "mov.b64 x, {%2, %3};\n\tmov.b64 y, {%4, %5};\n\t"
-      "sub.rn.f32x2 z, x, y;\n\tmov.b64 {%0, %1}, z;\n\t}"
-      : "=f"(o0), "=f"(o1)
-      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
-}
-
 __device__ __forceinline__ float min3f(float a, float b, float c) {
   float r;
   asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -124,18 +119,12 @@ __device__ __forceinline__ float min16(const float* v) {
   return fminf(min3f(a0, a1, a2), min3f(a3, a4, v[15]));
 }
 
-// One 64-column block of one token row's accumulator: e = |r_j|^2 / 2 -
-// <x_t, r_j> for slots jb .. jb + 63, folded into the row's running list.
+// One 64-column block of one token row's accumulator, which holds
+// e = |r_j|^2 / 2 - <x_t, r_j> for slots jb .. jb + 63: fold it into the
+// row's running list.
 template <int KC>
-__device__ __forceinline__ void cand_block(float (&v)[64], const float* hn, int jb, int cnt, int cnt_lo,
-                                           bool first, float (&bd)[KC], int (&bi)[KC], float* sp, int sw) {
-  const float4* h4 = reinterpret_cast<const float4*>(hn + jb);
-#pragma unroll
-  for (int x4 = 0; x4 < 16; ++x4) {
-    const float4 t4 = __ldg(h4 + x4);
-    sub_f32x2(v[4 * x4], v[4 * x4 + 1], t4.x, t4.y, v[4 * x4], v[4 * x4 + 1]);
-    sub_f32x2(v[4 * x4 + 2], v[4 * x4 + 3], t4.z, t4.w, v[4 * x4 + 2], v[4 * x4 + 3]);
-  }
+__device__ __forceinline__ void cand_block(float (&v)[64], int jb, int cnt, int cnt_lo, bool first,
+                                           float (&bd)[KC], int (&bi)[KC], float* sp, int sw) {
   if (jb + 64 > cnt_lo) {
 #pragma unroll
     for (int x = 0; x < 64; ++x)
@@ -183,13 +172,16 @@ __device__ __forceinline__ void cand_block(float (&v)[64], const float* hn, int 
 template <int NKC, int KC>
 __global__ void __launch_bounds__(tcc::THREADS, 1)
     cand_tc_kernel(const __grid_constant__ CUtensorMap mapRK, const __grid_constant__ CUtensorMap mapRV,
-                   const TcParams P) {
+                   const __grid_constant__ CUtensorMap mapH, const TcParams P) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   constexpr int D = NKC * 64;
-  constexpr int SLOT = NKC * tcc::BATOM;                        // bytes of one reference tile
-  unsigned char* sB = smem;                                     // [NSLOT][NKC] atoms
-  float* spill = (float*)(sB + tcc::NSLOT * SLOT);              // [EPI_WARPS][32][CHUNK]
+  // one ring slot: NKC reference atoms, then the tile's split half-norm
+  // rows (128 x 32 bytes, 32-byte swizzle)
+  constexpr int SLOT = NKC * tcc::BATOM + tcc::HATOM;
+  unsigned char* sB = smem;                                     // [NSLOT] slots
+  unsigned char* sOnes = sB + tcc::NSLOT * SLOT;                // 128 rows of (1, 1, 1, 0, ...)
+  float* spill = (float*)(sOnes + tcc::HATOM);                  // [EPI_WARPS][32][CHUNK]
   uint64_t* b_full = (uint64_t*)((unsigned char*)spill + tcc::spill_bytes(KC));  // [NSLOT]
   uint64_t* b_empty = b_full + tcc::NSLOT;                      // [NSLOT]
   uint64_t* a_full = b_empty + tcc::NSLOT;                      // [1]
@@ -217,7 +209,20 @@ __global__ void __launch_bounds__(tcc::THREADS, 1)
   if (warp == tcc::PRODUCER_WARP && lane == 0) {
     prefetch_tensormap(&mapRK);
     prefetch_tensormap(&mapRV);
+    prefetch_tensormap(&mapH);
   }
+  // the ones operand of the norm MMA: row m = (1, 1, 1, 0 x 13), 32-byte
+  // swizzle (16-byte chunk c of row m sits at chunk c ^ ((m >> 2) & 1))
+  for (int i = threadIdx.x; i < tcc::TM * 2; i += blockDim.x) {
+    const int m = i >> 1, c = i & 1;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (c == 0) {
+      v.x = 0x3F803F80u;  // bf16 1.0, 1.0
+      v.y = 0x00003F80u;  // 1.0, 0
+    }
+    *reinterpret_cast<uint4*>(sOnes + m * 32 + ((c ^ ((m >> 2) & 1)) << 4)) = v;
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   if (warp == tcc::MMA_WARP) {
     tmem_alloc(tmem_slot, tcc::TMEM_COLS);
     tmem_relinquish();
@@ -246,6 +251,7 @@ __global__ void __launch_bounds__(tcc::THREADS, 1)
             else
               tma_load_3d(&mapRV, &b_full[sl], dst + kc * tcc::BATOM, (kc - HALF) * 64, r * tcc::RN, u.bh);
           }
+          tma_load_3d(&mapH, &b_full[sl], dst + NKC * tcc::BATOM, 0, r * tcc::RN, u.bh);
         }
       }
       if (!ok) {
@@ -285,6 +291,9 @@ __global__ void __launch_bounds__(tcc::THREADS, 1)
               umma_f16_ts(d, a + k16 * 8,
                            desc_kmajor_sw128(b_base + sl * SLOT + (k16 >> 2) * tcc::BATOM + (k16 & 3) * 32), idesc,
                            k16 != 0);
+            // + h_j: ones (A, shared memory) times the split half-norm rows
+            umma_f16(d, desc_kmajor_sw32(smem_u32(sOnes)), desc_kmajor_sw32(b_base + sl * SLOT + NKC * tcc::BATOM),
+                     idesc, 1u);
             umma_commit(&d_full[i]);
           }
           if (!ok) break;
@@ -324,10 +333,11 @@ __global__ void __launch_bounds__(tcc::THREADS, 1)
 #pragma unroll
           for (int v4 = 0; v4 < 8; ++v4) {
             const uint4 x = t < P.T ? __ldg(reinterpret_cast<const uint4*>(src) + v4) : make_uint4(0, 0, 0, 0);
-            w[4 * v4] = x.x;
-            w[4 * v4 + 1] = x.y;
-            w[4 * v4 + 2] = x.z;
-            w[4 * v4 + 3] = x.w;
+            // -x_t: flip the sign bits of both bf16 halves
+            w[4 * v4] = x.x ^ 0x80008000u;
+            w[4 * v4 + 1] = x.y ^ 0x80008000u;
+            w[4 * v4 + 2] = x.z ^ 0x80008000u;
+            w[4 * v4 + 3] = x.w ^ 0x80008000u;
           }
           tmem_st32(ta + c0, w);
         }
@@ -339,7 +349,6 @@ __global__ void __launch_bounds__(tcc::THREADS, 1)
       const int first = u.t0 + ti * tcc::TM;
       const int cnt = t < P.T ? min((t + P.s - 1) / P.s, P.n_ref) : 0;  // valid slots j < cnt
       const int cnt_lo = min((first + P.s - 1) / P.s, P.n_ref);         // smallest cnt in the tile
-      const float* hn = P.hnorm + (int64_t)u.bh * P.n_ref_cap;
       float bd[KC];
       int bi[KC];
 #pragma unroll
@@ -361,7 +370,7 @@ __global__ void __launch_bounds__(tcc::THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&d_empty[ti]);
           }
-          cand_block<KC>(v, hn, r * tcc::RN + hf * 64, cnt, cnt_lo, r == 0 && hf == 0, bd, bi, sp, sw);
+          cand_block<KC>(v, r * tcc::RN + hf * 64, cnt, cnt_lo, r == 0 && hf == 0, bd, bi, sp, sw);
         }
       }
       if (!ok) break;
@@ -418,6 +427,18 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims
   return r == CUDA_SUCCESS;
 }
 
+// The split half-norm plane: box 16 x RN rows, 32-byte swizzle.
+bool make_map_h(CUtensorMap* m, const void* base, const cuuint64_t* dims, const cuuint64_t* strides) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint32_t box[3] = {16, tcc::RN, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 int sm_count() {
   int dev = 0, n = kNumSMs;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
@@ -426,17 +447,17 @@ int sm_count() {
 
 template <int NKC, int KC>
 size_t smem_bytes() {
-  return 1024 + (size_t)tcc::NSLOT * NKC * tcc::BATOM + (size_t)tcc::spill_bytes(KC) + 256;
+  return 1024 + (size_t)tcc::NSLOT * (NKC * tcc::BATOM + tcc::HATOM) + tcc::HATOM + (size_t)tcc::spill_bytes(KC) + 256;
 }
 
 template <int NKC, int KC>
-cudaError_t launch_tc(const CUtensorMap& mRK, const CUtensorMap& mRV, const TcParams& P, int grid,
-                      cudaStream_t st) {
+cudaError_t launch_tc(const CUtensorMap& mRK, const CUtensorMap& mRV, const CUtensorMap& mH, const TcParams& P,
+                      int grid, cudaStream_t st) {
   auto kern = cand_tc_kernel<NKC, KC>;
   const size_t smem = smem_bytes<NKC, KC>();
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, tcc::THREADS, smem, st>>>(mRK, mRV, P);
+  kern<<<grid, tcc::THREADS, smem, st>>>(mRK, mRV, mH, P);
   return cudaGetLastError();
 }
 
@@ -453,7 +474,7 @@ cudaError_t launch_candidates_tc(const Plan& p, int T, const KVView& kv, const v
   if (n_code == 0) return cudaSuccess;
   const int n_ref = (int)n_ref_of(T, c.stride_s);
   const int d_h = c.d_h;
-  CUtensorMap mRK, mRV;
+  CUtensorMap mRK, mRV, mH;
   {
     const char* cb = (const char*)cache;
     cuuint64_t dims[3] = {(cuuint64_t)d_h, (cuuint64_t)n_ref, (cuuint64_t)c.batch * c.kv_heads};
@@ -461,6 +482,10 @@ cudaError_t launch_candidates_tc(const Plan& p, int T, const KVView& kv, const v
     if (!make_map(&mRK, cb + p.off_refk, 3, dims, str, tcc::RN) ||
         !make_map(&mRV, cb + p.off_refv, 3, dims, str, tcc::RN))
       return cudaErrorNotSupported;
+    // split half-norm rows: 16 bf16 (32 bytes) per reference, 32-byte swizzle
+    cuuint64_t hdims[3] = {16, (cuuint64_t)n_ref, (cuuint64_t)c.batch * c.kv_heads};
+    cuuint64_t hstr[2] = {32, (cuuint64_t)p.n_ref_cap * 32};
+    if (!make_map_h(&mH, (const char*)ws + p.ws_hsplit, hdims, hstr)) return cudaErrorNotSupported;
   }
   TcParams P;
   P.T = T;
@@ -484,8 +509,8 @@ cudaError_t launch_candidates_tc(const Plan& p, int T, const KVView& kv, const v
   const int grid = std::min(P.n_units, sm_count());
   ProfScope ps(p, st, KID_CAND_TC);
   if (d_h == 128)
-    return p.KC == 8 ? launch_tc<4, 8>(mRK, mRV, P, grid, st) : launch_tc<4, 12>(mRK, mRV, P, grid, st);
-  return p.KC == 8 ? launch_tc<2, 8>(mRK, mRV, P, grid, st) : launch_tc<2, 12>(mRK, mRV, P, grid, st);
+    return p.KC == 8 ? launch_tc<4, 8>(mRK, mRV, mH, P, grid, st) : launch_tc<4, 12>(mRK, mRV, mH, P, grid, st);
+  return p.KC == 8 ? launch_tc<2, 8>(mRK, mRV, mH, P, grid, st) : launch_tc<2, 12>(mRK, mRV, mH, P, grid, st);
 }
 
 }  // namespace dkv

@@ -24,7 +24,8 @@ template <typename T>
 __global__ void refpack_kernel(int s, int d_h, int H, int64_t n_ref, int64_t n_ref_cap,
                                const T* __restrict__ K, const T* __restrict__ V, int64_t sb,
                                int64_t sh, int64_t st, T* __restrict__ refk,
-                               T* __restrict__ refv, float* __restrict__ hnorm) {
+                               T* __restrict__ refv, float* __restrict__ hnorm,
+                               __nv_bfloat16* __restrict__ hsplit) {
   const int b = blockIdx.z, h = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t j = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
@@ -46,6 +47,23 @@ __global__ void refpack_kernel(int s, int d_h, int H, int64_t n_ref, int64_t n_r
   }
   acc = warp_sum(acc);
   if (lane == 0) hnorm[bh * n_ref_cap + j] = 0.5f * acc;
+  if (hsplit != nullptr && lane < 2) {
+    // h = 0.5 |x_j|^2 = hi + mid + lo in bf16 (24 significant bits), then
+    // zeros: the K = 16 row that the distance kernel's last MMA adds
+    const float hv = 0.5f * acc;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(hv);
+    const float r1 = hv - __bfloat162float(hi);
+    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+    __align__(16) __nv_bfloat16 row[8];
+    for (int i = 0; i < 8; ++i) row[i] = __float2bfloat16_rn(0.f);
+    if (lane == 0) {
+      row[0] = hi;
+      row[1] = mid;
+      row[2] = lo;
+    }
+    reinterpret_cast<uint4*>(hsplit + (bh * n_ref_cap + j) * 16)[lane] = *reinterpret_cast<const uint4*>(row);
+  }
 }
 
 cudaError_t launch_refpack(const Plan& p, int T, const KVView& kv, void* cache, void* ws,
@@ -62,13 +80,14 @@ cudaError_t launch_refpack(const Plan& p, int T, const KVView& kv, void* cache, 
     refpack_kernel<T_><<<grid, 256, 0, st>>>(c.stride_s, c.d_h, c.kv_heads, n_ref, p.n_ref_cap,
                                              (const T_*)kv.K, (const T_*)kv.V, kv.sb, kv.sh,
                                              kv.st, (T_*)(cb + p.off_refk),
-                                             (T_*)(cb + p.off_refv), hn);
+                                             (T_*)(cb + p.off_refv), hn,
+                                             (__nv_bfloat16*)((char*)ws + p.ws_hsplit));
   } else {
     refpack_kernel<float><<<grid, 256, 0, st>>>(c.stride_s, c.d_h, c.kv_heads, n_ref,
                                                  p.n_ref_cap, (const float*)kv.K,
                                                  (const float*)kv.V, kv.sb, kv.sh, kv.st,
                                                  (float*)(cb + p.off_refk),
-                                                 (float*)(cb + p.off_refv), hn);
+                                                 (float*)(cb + p.off_refv), hn, nullptr);
   }
   return cudaGetLastError();
 }

@@ -43,7 +43,7 @@ struct Plan {
   // cache layout (bytes from base)
   size_t off_refk, off_refv, off_code, off_idx, cache_bytes;
   // compress workspace
-  size_t ws_hnorm, ws_cand;
+  size_t ws_hnorm, ws_hsplit, ws_cand;
   // decode workspace
   int nslot_cap;         // decode partial slots per (b, head)
   int n_chunk_cap;       // combine blocks per (b, head)

@@ -122,6 +122,18 @@ __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t saddr) {
   return d;
 }
 
+// The same for a K-major operand with 32-byte rows (16 bf16) in the 32-byte
+// swizzle layout: 8-row groups 256 bytes apart.
+__device__ __forceinline__ uint64_t desc_kmajor_sw32(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+  d |= (uint64_t)1 << 16;
+  d |= (uint64_t)(256 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)6 << 61;                         // 32-byte swizzle
+  return d;
+}
+
 // Instruction descriptor of tcgen05.mma kind::f16 with bf16 A and B,
 // fp32 accumulator, both operands K-major, shape M x N.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
