@@ -102,6 +102,12 @@ def kernel_rooflines(sh, prof, peaks, peak_kind):
     tensor_peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     hbm_peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     out = {}
+    # DRAM bytes per launch from an ncu capture of this build on the 32k
+    # case, scaled by the units processed to the 128k workload (traffic
+    # grows with T and with the decode batch); null for other workloads
+    default = (sh.T, sh.Bc, sh.Bd, sh.H, sh.d_h, sh.s, sh.k, sh.d_c, sh.hidden) == \
+        (131072, 1, 8, 8, 128, 16, 4, 32, 256)
+    traffic = {"candidates_tc": 599e6, "encode_tc": 617e6, "decode_stream_tc": 649e6} if default else {}
 
     def add(name, bound, work, unit, peak, src):
         if name not in prof:
@@ -111,7 +117,7 @@ def kernel_rooflines(sh, prof, peaks, peak_kind):
         scale = 1e12 if unit == "TFLOP/s" else 1e9
         ach = work / sec / scale
         out[name] = {"kernel": name, "bound": bound, "achieved": ach, "peak": peak, "unit": unit,
-                     "frac": ach / peak, "traffic": None, "algorithmic_per_launch": work,
+                     "frac": ach / peak, "traffic": traffic.get(name), "algorithmic_per_launch": work,
                      "peak_source": src, "ms_per_launch": ms / n}
 
     src_t = f"{peak_kind} bf16 sustained (MEASURED_PEAKS bf16_tflops_sustained)" if peak_kind == "measured" \
@@ -306,7 +312,12 @@ def workload_config(sh):
             "T": sh.T, "layers": sh.L, "compress_batch": sh.Bc, "decode_batch": sh.Bd, "kv_heads": sh.H,
             "q_heads": sh.Hq, "d_h": sh.d_h, "stride_s": sh.s, "k": sh.k, "d_c": sh.d_c, "hidden": sh.hidden,
             "global_batch": sh.Bd, "seq_len": sh.T, "parallelism": "replicas",
-            "l2": "inputs larger than L2 (per step: 17 GB raw K/V compressed, 28.7 GB cache read)"}
+            "l2": f"inputs larger than L2 (per step: {raw_kv_bytes(sh) / 1e9:.2f} GB raw K/V compressed, "
+                  f"{sh.L * sh.decode_bytes_per_layer() / 1e9:.2f} GB cache read)"}
+
+
+def raw_kv_bytes(sh):
+    return sh.L * sh.Bc * sh.H * sh.T * 2 * sh.d_h * 2
 
 
 # ------------------------------------------------------------------- main
