@@ -189,6 +189,34 @@ def decode_phase(sh, w):
                              w["W"][l]["W4"], None, w["out"][l], w["ws_d"])
 
 
+def append_timing(sh, w, steps):
+    """Streaming append: one new token (the sequence's last, t = T - 1, a
+    non-reference token that searches all T/s references) per layer, for the
+    compress sequence; outside the timed step."""
+    from decode_attention_strided_b200 import deltakv as dkv
+    t = sh.T - 1
+    if t < 1 or t % sh.s == 0:
+        return None
+
+    def one():
+        for l in range(sh.L):
+            K, V = w["comp_in"][l]
+            dkv.append(w["pc"], t, sh.T, K, V, w["W"][l]["W1"], None, w["W"][l]["W2"], None,
+                       w["comp_cache"][l], w["ws_c"])
+
+    one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        one()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    return {"us_per_layer": ms / sh.L * 1e3, "ms_per_token_all_layers": ms, "sequences": sh.Bc,
+            "kv_heads": sh.H, "references_searched": (t + sh.s - 1) // sh.s}
+
+
 # ------------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -380,6 +408,7 @@ def main():
     prof_d = dkv.profile_collect(w["pd"])
     for p in (w["pc"], w["pd"]):
         dkv.set_profiling(p, False)
+    append = append_timing(sh, w, a.steps)
     status = max(dkv.device_status(w["pc"], w["ws_c"]), dkv.device_status(w["pd"], w["ws_d"]))
     step_ms = [e[0].elapsed_time(e[2]) for e in ev]
     comp_ms = [e[0].elapsed_time(e[1]) for e in ev]
@@ -433,7 +462,7 @@ def main():
         "metric": METRIC, "value": value, "unit": "Mtok/s", "n_gpus": world, "steps": a.steps,
         "warmup": a.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(sh),
-        "compress": compress, "decode_attn": decode_attn, "roofline": roof, "rooflines": rooflines,
+        "compress": compress, "decode_attn": decode_attn, "append": append, "roofline": roof, "rooflines": rooflines,
         "cpu_baseline": cpu,
         "e2e": e2e, "gpu_launches": launches, "kernels": {k_: {"launches": n, "ms": ms} for k_, (n, ms) in prof.items()},
         "clocks": clk, "device_status": status, "setup_s": setup_s, "wall_s": wall,

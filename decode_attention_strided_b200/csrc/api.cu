@@ -72,8 +72,8 @@ void build_plan(const deltakv_config& c, Plan& p) {
   w = align256(w + (size_t)(BH * p.n_ref_cap) * 4);
   p.ws_hsplit = w;  // 0.5 |x_j|^2 as three bf16 terms in a 16-element row (bf16 caches)
   w = align256(w + (size_t)(BH * p.n_ref_cap) * 32);
-  p.ws_cand = w;
-  w = align256(w + (size_t)(BH * p.n_code_cap * p.KC) * 4);
+  p.ws_cand = w;  // candidate plane; the append path's per-slice lists reuse it (at least 4 KB a head)
+  w = align256(w + std::max<size_t>((size_t)(BH * p.n_code_cap * p.KC) * 4, (size_t)BH * 4096));
   const size_t compress_end = w;
   w = kErrBytes;
   p.nslot_cap = (int)std::max<int64_t>(kMaxSplit, ceil_div64(kNumSMs, BH) + 1);
@@ -185,6 +185,26 @@ deltakv_status deltakv_compress(deltakv_plan_t plan, int32_t T, const void* K, c
     e = encode_tc_supported(p) ? launch_encode_tc(p, T, kv, W1, b1, W2, b2, cache, workspace, st)
                                : launch_encode(p, T, kv, W1, b1, W2, b2, cache, workspace, st);
   return from_cuda(e);
+}
+
+deltakv_status deltakv_append(deltakv_plan_t plan, int32_t T0, int32_t T1, const void* K, const void* V,
+                              const int64_t kv_strides[3], const void* W1, const float* b1, const void* W2,
+                              const float* b2, void* cache, void* workspace, size_t workspace_bytes,
+                              deltakv_stream_t stream) {
+  if (!plan) return DELTAKV_ERR_INVALID_ARG;
+  const Plan& p = plan->p;
+  if (T0 < 0 || T1 < T0 || T1 > p.cfg.max_T) return DELTAKV_ERR_INVALID_ARG;
+  if (T1 == T0) return DELTAKV_OK;
+  if (!K || !V || !kv_strides || !W1 || !W2 || !cache || !workspace) return DELTAKV_ERR_INVALID_ARG;
+  if (workspace_bytes < p.ws_bytes) return DELTAKV_ERR_WORKSPACE;
+  for (int i = 0; i < 3; ++i)
+    if (kv_strides[i] < 0 || (kv_strides[i] * p.esize) % 16 != 0) return DELTAKV_ERR_ALIGNMENT;
+  if (kv_strides[2] < p.cfg.d_h) return DELTAKV_ERR_INVALID_ARG;
+  if (!aligned16(K) || !aligned16(V) || !aligned16(W1) || !aligned16(W2) || !aligned16(cache) ||
+      !aligned16(workspace) || !aligned16(b1) || !aligned16(b2))
+    return DELTAKV_ERR_ALIGNMENT;
+  KVView kv{K, V, kv_strides[0], kv_strides[1], kv_strides[2]};
+  return from_cuda(launch_append(p, T0, T1, kv, W1, b1, W2, b2, cache, workspace, (cudaStream_t)stream));
 }
 
 deltakv_status deltakv_decode_attention(deltakv_plan_t plan, int32_t T, const void* q,

@@ -25,7 +25,8 @@ constexpr size_t kErrBytes = 256;
 // Kernels the library launches (profiling ids).
 enum KernelId {
   KID_REFPACK = 0, KID_CAND_SIMT, KID_CAND_TC, KID_ENCODE_SIMT, KID_ENCODE_TC, KID_RECONSTRUCT, KID_DEC_REF,
-  KID_DEC_PREP, KID_DEC_STREAM_SIMT, KID_DEC_STREAM_TC, KID_DEC_COMBINE, KID_DEC_FINAL, KID_COUNT
+  KID_DEC_PREP, KID_DEC_STREAM_SIMT, KID_DEC_STREAM_TC, KID_DEC_COMBINE, KID_DEC_FINAL,
+  KID_APPEND_REFS, KID_APPEND_ROWS, KID_COUNT
 };
 const char* kernel_name(int id);
 
@@ -83,6 +84,8 @@ cudaError_t launch_candidates_simt(const Plan& p, int T, const KVView& kv, const
 bool candidates_tc_supported(const Plan& p);
 cudaError_t launch_candidates_tc(const Plan& p, int T, const KVView& kv, const void* cache,
                                  void* ws, cudaStream_t st);
+cudaError_t launch_append(const Plan& p, int T0, int T1, const KVView& kv, const void* W1, const float* b1,
+                          const void* W2, const float* b2, void* cache, void* ws, cudaStream_t st);
 cudaError_t launch_encode(const Plan& p, int T, const KVView& kv, const void* W1, const float* b1,
                           const void* W2, const float* b2, void* cache, void* ws,
                           cudaStream_t st);

@@ -26,7 +26,7 @@ STATUS = {
 }
 
 SYMBOLS = ("deltakv_plan", "deltakv_plan_destroy", "deltakv_get_cache_layout", "deltakv_compress",
-           "deltakv_decode_attention", "deltakv_reconstruct", "deltakv_device_status",
+           "deltakv_append", "deltakv_decode_attention", "deltakv_reconstruct", "deltakv_device_status",
            "deltakv_decode_attention_noalloc", "deltakv_set_profiling", "deltakv_profile_collect",
            "deltakv_status_string", "deltakv_version")
 
@@ -74,6 +74,8 @@ def load_library(path: str = LIB_PATH):
     lib.deltakv_get_cache_layout.restype = ctypes.c_int
     lib.deltakv_compress.argtypes = [vp, i32, vp, vp, i64p, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.deltakv_compress.restype = ctypes.c_int
+    lib.deltakv_append.argtypes = [vp, i32, i32, vp, vp, i64p, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.deltakv_append.restype = ctypes.c_int
     lib.deltakv_decode_attention.argtypes = [vp, i32, vp, i64p, vp, vp, vp, vp, vp, vp, i64p, vp, sz, vp]
     lib.deltakv_decode_attention.restype = ctypes.c_int
     lib.deltakv_decode_attention_noalloc.argtypes = [vp, i32, vp, i64p, vp, vp, vp, vp, vp, vp, i64p, vp]
@@ -200,6 +202,18 @@ def compress(p: Plan, T: int, K, V, W1, b1, W2, b2, cache, workspace, stream=Non
         raise ValueError("K and V must share strides")
     _check("deltakv_compress", lib.deltakv_compress(
         p.handle, int(T), _ptr(K), _ptr(V), strides, _ptr(W1), _ptr(b1), _ptr(W2), _ptr(b2),
+        _ptr(cache), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def append(p: Plan, T0: int, T1: int, K, V, W1, b1, W2, b2, cache, workspace, stream=None):
+    """deltakv_append: extend a cache holding tokens [0, T0) to [0, T1);
+    K, V as for compress (only tokens [T0, T1) are read)."""
+    lib = load_library()
+    strides = (ctypes.c_int64 * 3)(K.stride(0), K.stride(1), K.stride(2))
+    if tuple(V.stride()[:3]) != tuple(K.stride()[:3]):
+        raise ValueError("K and V must share strides")
+    _check("deltakv_append", lib.deltakv_append(
+        p.handle, int(T0), int(T1), _ptr(K), _ptr(V), strides, _ptr(W1), _ptr(b1), _ptr(W2), _ptr(b2),
         _ptr(cache), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
 
 

@@ -133,6 +133,30 @@ deltakv_status deltakv_compress(deltakv_plan_t plan, int32_t T,
                                 void* cache, void* workspace, size_t workspace_bytes,
                                 deltakv_stream_t stream);
 
+/* Streaming compression ("Processo di Compressione" steps 1-4, applied as
+ * tokens arrive during decoding): extend a layer's packed cache that holds
+ * the compressed tokens [0, T0) to the tokens [0, T1).  New tokens with
+ * t mod s == 0 become references; every other new token t searches all
+ * references with slot j, j s < t (those appended by this call included)
+ * with exact float32 squared distances, keeps the k nearest (ties to the
+ * lower slot), and stores its code and slots.  The result equals
+ * deltakv_compress over [0, T1).
+ *   0 <= T0 <= T1 <= max_T; T0 == T1 returns DELTAKV_OK without launching.
+ *   cache      : device, as written by deltakv_compress(T0) or by earlier
+ *                appends up to T0 (the caller guarantees it); rows of the
+ *                tokens [T0, T1) are written, nothing else changes.
+ *   K, V       : device, as for deltakv_compress; only tokens [T0, T1) are
+ *                read.
+ *   W1, b1, W2, b2, workspace, stream: as for deltakv_compress.
+ * Runs on CUDA cores (a few tokens per call): one CTA per new token and
+ * kv-head.  Errors: as for deltakv_compress. */
+deltakv_status deltakv_append(deltakv_plan_t plan, int32_t T0, int32_t T1,
+                              const void* K, const void* V, const int64_t kv_strides[3],
+                              const void* W1, const float* b1,
+                              const void* W2, const float* b2,
+                              void* cache, void* workspace, size_t workspace_bytes,
+                              deltakv_stream_t stream);
+
 /* Decode attention over one layer's compressed cache ("Ricostruzione" and
  * section 4): for query head hq (kv-head hq / G),
  *   out = sum_t softmax_t(q . K_hat_t / sqrt(d_h)) V_hat_t over the T cached

@@ -105,4 +105,9 @@ def test_calls_reject_bad_arguments_before_any_launch(lib):
     assert lib.deltakv_decode_attention(p.handle, 0, fake, qs, fake, fake, None, fake, None, fake, qs, fake, ws, None) == 1
     assert lib.deltakv_decode_attention(p.handle, 100, fake, qs, fake, fake, None, fake, None, vp((1 << 20) + 4), qs, fake, ws, None) == 3
     assert lib.deltakv_reconstruct(p.handle, -1, fake, fake, None, fake, None, fake, fake, fake, ws, None) == 1
+    # append: T0 > T1, T1 beyond max_T, an empty range is a no-op, bad stride
+    assert lib.deltakv_append(p.handle, 600, 500, fake, fake, strides, fake, None, fake, None, fake, fake, ws, None) == 1
+    assert lib.deltakv_append(p.handle, 500, 2048, fake, fake, strides, fake, None, fake, None, fake, fake, ws, None) == 1
+    assert lib.deltakv_append(p.handle, 700, 700, None, None, None, None, None, None, None, None, None, 0, None) == 0
+    assert lib.deltakv_append(p.handle, 500, 600, fake, fake, bad, fake, None, fake, None, fake, fake, ws, None) == 3
     assert lib.deltakv_plan_destroy(None) == 0
