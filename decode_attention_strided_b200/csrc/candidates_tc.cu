@@ -146,11 +146,15 @@ __device__ __forceinline__ void cand_block(float (&v)[64], int jb, int cnt, int 
   for (int c = 0; c < 64 / tcc::CHUNK; ++c) {
     const float thr = bd[KC - 1];
     if (!__any_sync(0xffffffffu, cm[c] < thr)) continue;
-    // four independent partial masks keep the dependency chains short
-    uint32_t mp[4] = {0u, 0u, 0u, 0u};
+    // bit x = (v_x < thr): the sign of v_x - thr shifted in from the top
+    // (one funnel shift per value), in two independent 8-bit chains
+    uint32_t ma = 0u, mb = 0u;
 #pragma unroll
-    for (int x = 0; x < tcc::CHUNK; ++x) mp[x & 3] |= (v[c * tcc::CHUNK + x] < thr ? 1u : 0u) << x;
-    uint32_t m = (mp[0] | mp[1]) | (mp[2] | mp[3]);
+    for (int x = tcc::CHUNK / 2 - 1; x >= 0; --x) {
+      ma = __funnelshift_l(__float_as_uint(v[c * tcc::CHUNK + x] - thr), ma, 1);
+      mb = __funnelshift_l(__float_as_uint(v[c * tcc::CHUNK + tcc::CHUNK / 2 + x] - thr), mb, 1);
+    }
+    uint32_t m = ma | (mb << (tcc::CHUNK / 2));
     if (m) {
 #pragma unroll
       for (int i4 = 0; i4 < tcc::CHUNK / 4; ++i4)
@@ -162,7 +166,7 @@ __device__ __forceinline__ void cand_block(float (&v)[64], int jb, int cnt, int 
     while (m) {
       const int x = __ffs(m) - 1;
       m &= m - 1;
-      const float vx = sp[(((x >> 2) ^ sw) << 2) | (x & 3)];
+      const float vx = sp[x ^ (sw << 2)];  // float4 slot (x / 4) ^ sw, element x % 4
       topk_insert_inorder<KC>(bd, bi, vx, jb + c * tcc::CHUNK + x);
     }
     __syncwarp();
