@@ -155,6 +155,11 @@ __device__ __forceinline__ void cand_block(float (&v)[64], int jb, int cnt, int 
       mb = __funnelshift_l(__float_as_uint(v[c * tcc::CHUNK + tcc::CHUNK / 2 + x] - thr), mb, 1);
     }
     uint32_t m = ma | (mb << (tcc::CHUNK / 2));
+    if (!__any_sync(0xffffffffu, __popc(m) > 1)) {
+      // at most one candidate per lane: it is the chunk's minimum
+      if (m) topk_insert_inorder<KC>(bd, bi, cm[c], jb + c * tcc::CHUNK + __ffs(m) - 1);
+      continue;
+    }
     if (m) {
 #pragma unroll
       for (int i4 = 0; i4 < tcc::CHUNK / 4; ++i4)
