@@ -212,7 +212,7 @@ def append_timing(sh, w, steps):
         one()
     e1.record()
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / steps
+    ms = max_over_ranks([e0.elapsed_time(e1) / steps], dev, world)[0]
     return {"us_per_layer": ms / sh.L * 1e3, "ms_per_token_all_layers": ms, "sequences": sh.Bc,
             "kv_heads": sh.H, "references_searched": (t + sh.s - 1) // sh.s}
 
@@ -413,13 +413,7 @@ def main():
     step_ms = [e[0].elapsed_time(e[2]) for e in ev]
     comp_ms = [e[0].elapsed_time(e[1]) for e in ev]
     dec_ms = [e[1].elapsed_time(e[2]) for e in ev]
-    tot_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([tot_ms, sum(comp_ms), sum(dec_ms)], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        tot_ms, sc, sd = t.tolist()
-    else:
-        sc, sd = sum(comp_ms), sum(dec_ms)
+    tot_ms, sc, sd = max_over_ranks([sum(step_ms), sum(comp_ms), sum(dec_ms)], dev, world)
     ms_step = tot_ms / a.steps
     value = world * sh.T * sh.Bc * a.steps / (tot_ms / 1e3) / 1e6
 
@@ -452,7 +446,7 @@ def main():
 
     e2e = None
     if not a.no_e2e:
-        e2e = run_e2e(sh, w, dev, a)
+        e2e = run_e2e(sh, w, dev, a, world)
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         step_s, desc, nthreads = oracle_sample(sh, budget_s=12.0)
@@ -473,7 +467,18 @@ def main():
         torch.distributed.destroy_process_group()
 
 
-def run_e2e(sh, w, dev, a):
+def max_over_ranks(vals, dev, world):
+    """Element-wise maximum of per-rank timings over all ranks (every rank
+    calls it, in the same order); the identity on one rank."""
+    vals = [float(v) for v in vals]
+    if world <= 1:
+        return vals
+    t = torch.tensor(vals, dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
+
+
+def run_e2e(sh, w, dev, a, world=1):
     """Same step through the public API with host buffers: every layer's K/V
     is copied from pinned host memory before its compress call, and every
     decode copies its queries in and its output back."""
@@ -505,10 +510,10 @@ def run_e2e(sh, w, dev, a):
             ho[l].copy_(w["out"][l], non_blocking=True)
     e1.record()
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / steps
+    ms = max_over_ranks([e0.elapsed_time(e1) / steps], dev, world)[0]
     h2d = sh.L * (hK.numel() * 2 + hV.numel() * 2 + hq[0].numel() * 2)
     d2h = sh.L * ho[0].numel() * 4
-    return {"value": sh.T * sh.Bc / (ms / 1e3) / 1e6, "unit": "Mtok/s", "h2d_bytes_per_step": h2d,
+    return {"value": world * sh.T * sh.Bc / (ms / 1e3) / 1e6, "unit": "Mtok/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps}
 
 
