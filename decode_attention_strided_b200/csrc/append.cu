@@ -54,6 +54,23 @@ __device__ __forceinline__ void loadv(const float* p, float (&v)[N]) {
 }
 }  // namespace
 
+// Insert (d, j) into a list sorted by (distance, slot), branch-free: every
+// position is computed from the old list directly.  No-op when (d, j) does
+// not precede the last entry.
+template <int KC>
+__device__ __forceinline__ void topk_insert_any(float (&bd)[KC], int (&bi)[KC], float d, int j) {
+  bool lt[KC];
+#pragma unroll
+  for (int i = 0; i < KC; ++i) lt[i] = d < bd[i] || (d == bd[i] && j < bi[i]);
+#pragma unroll
+  for (int i = KC - 1; i > 0; --i) {
+    bd[i] = lt[i - 1] ? bd[i - 1] : (lt[i] ? d : bd[i]);
+    bi[i] = lt[i - 1] ? bi[i - 1] : (lt[i] ? j : bi[i]);
+  }
+  bd[0] = lt[0] ? d : bd[0];
+  bi[0] = lt[0] ? j : bi[0];
+}
+
 // New reference rows j in [j0, j1): copy K and V of token j s into the
 // reference planes.
 template <typename E>
@@ -167,7 +184,9 @@ __global__ void __launch_bounds__(kAppendThreads)
   const int d_h = P.d_h, D = 2 * d_h;
   const int64_t row = P.row0 + blockIdx.y;
   const int64_t t = token_of_code_row(row, P.s);
-  if (tid == 0) {
+  if (warp == 0) {
+    // merge the slices' lists: lane l folds slices l, l + 32, ..., then the
+    // lanes' lists meet in a shuffle tree
     float bd[kAppendKMax];
     int bi[kAppendKMax];
 #pragma unroll
@@ -176,15 +195,31 @@ __global__ void __launch_bounds__(kAppendThreads)
       bi[i] = INT_MAX;
     }
     const float* l = lists + ((int64_t)bh * gridDim.y + blockIdx.y) * nsplit * (2 * kAppendKMax);
-    for (int sp = 0; sp < nsplit; ++sp)
+    for (int sp = lane; sp < nsplit; sp += 32)
+#pragma unroll
       for (int i = 0; i < kAppendKMax; ++i) {
         const int j = __float_as_int(l[sp * 2 * kAppendKMax + kAppendKMax + i]);
-        if (j != INT_MAX) topk_insert<kAppendKMax>(bd, bi, l[sp * 2 * kAppendKMax + i], j);
+        topk_insert_any<kAppendKMax>(bd, bi, l[sp * 2 * kAppendKMax + i], j);
       }
-    int n = 0;
-    for (int i = 0; i < P.k; ++i)
-      if (bi[i] != INT_MAX) sel[n++] = bi[i];
-    sel_n = n;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      float od[kAppendKMax];
+      int oj[kAppendKMax];
+#pragma unroll
+      for (int i = 0; i < kAppendKMax; ++i) {
+        od[i] = __shfl_xor_sync(0xffffffffu, bd[i], o);
+        oj[i] = __shfl_xor_sync(0xffffffffu, bi[i], o);
+      }
+#pragma unroll
+      for (int i = 0; i < kAppendKMax; ++i)
+        topk_insert_any<kAppendKMax>(bd, bi, od[i], oj[i]);
+    }
+    if (lane == 0) {
+      int n = 0;
+      for (int i = 0; i < P.k; ++i)
+        if (bi[i] != INT_MAX) sel[n++] = bi[i];
+      sel_n = n;
+    }
   }
   __syncthreads();
   const int k_eff = sel_n;
@@ -208,30 +243,35 @@ __global__ void __launch_bounds__(kAppendThreads)
     for (int i = 0; i < NV; ++i) r[e0 + i] = x[i] - m[i] * inv;
   }
   __syncthreads();
-  // code = W2 act(W1 r + b1) + b2 (weight rows read 4 at a time; hidden is
-  // a multiple of 32, D of 128)
-  for (int u = tid; u < P.hidden; u += blockDim.x) {
-    float acc = b1 ? b1[u] : 0.f;
-    const E* w = W1 + (int64_t)u * D;
-    for (int e = 0; e < D; e += 4) {
-      float wv[4];
-      loadv<4>(w + e, wv);
+  // code = W2 act(W1 r + b1) + b2: a warp per weight row at a time, lane l
+  // multiplying elements [NV l, NV l + NV) of the row (D = 32 NV; hidden is
+  // a multiple of 32, so a W2 row is hidden / 32 elements a lane)
+  {
+    float rr[NV];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) acc = fmaf(wv[i], r[e + i], acc);
+    for (int i = 0; i < NV; ++i) rr[i] = r[lane * NV + i];
+    for (int u = warp; u < P.hidden; u += kAppendWarps) {
+      float wv[NV];
+      loadv<NV>(W1 + (int64_t)u * D + lane * NV, wv);
+      float acc = 0.f;
+#pragma unroll
+      for (int i = 0; i < NV; ++i) acc = fmaf(wv[i], rr[i], acc);
+      acc = warp_sum(acc);
+      if (lane == 0) hbuf[u] = act_eval(P.act, acc + (b1 ? b1[u] : 0.f));
     }
-    hbuf[u] = act_eval(P.act, acc);
   }
   __syncthreads();
-  for (int o = tid; o < P.d_c; o += blockDim.x) {
-    float acc = b2 ? b2[o] : 0.f;
+  for (int o = warp; o < P.d_c; o += kAppendWarps) {
+    float acc = 0.f;
     const E* w = W2 + (int64_t)o * P.hidden;
-    for (int u = 0; u < P.hidden; u += 4) {
+    for (int u = lane * 4; u < P.hidden; u += 128) {
       float wv[4];
       loadv<4>(w + u, wv);
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc = fmaf(wv[i], hbuf[u + i], acc);
     }
-    code[((int64_t)bh * P.n_code_cap + row) * P.d_c + o] = from_f<E>(acc);
+    acc = warp_sum(acc);
+    if (lane == 0) code[((int64_t)bh * P.n_code_cap + row) * P.d_c + o] = from_f<E>(acc + (b2 ? b2[o] : 0.f));
   }
   if (tid < P.k) idx[((int64_t)bh * P.n_code_cap + row) * P.k + tid] = tid < k_eff ? sel[tid] : -1;
 }
