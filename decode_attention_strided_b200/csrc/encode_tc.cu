@@ -9,19 +9,22 @@
 //   2. KV_R = their mean;  3. r = x_t - KV_R;
 //   4. code = W2 act(W1 r + b1) + b2  (code plane, rounded to bf16).
 //
-// One persistent CTA per SM, 8 warps.  W1 [hidden x D] and W2 [d_c x hidden]
-// stay in shared memory as fp16 for the whole launch (bf16 values are exact
-// in fp16); per 64-row tile:
-//   phase 1  8 lanes per token, 32 tokens in flight: gather the k + 4
-//            candidate rows, exact distances, choose k, reload them for the
-//            mean, residual r -> R tile (64 tokens x D, K-major)
-//   phase 2  tcgen05.mma  D1^T = W1 . R^T  (M = 128 hidden units per half,
-//            N = 64 tokens; fp32 in TMEM): TMEM lanes are hidden units
-//   phase 3  all 8 warps: thread = hidden unit, act(D1 + b1) over its 64
-//            tokens -> H tile stored as hidden rows of 64 tokens, which is
-//            the MN-major A operand of
-//   phase 4  tcgen05.mma  codes = H . W2^T  (M = 128 with 64 tokens, N = d_c)
-//   phase 5  TMEM -> + b2 -> bf16 codes
+// One persistent CTA per SM, 16 warps with fixed roles, per 64-row tile:
+//   gather warps (11)  16 lanes per token row; the row's x and candidate
+//            slots are loaded one row pass ahead, the k + 4 candidate rows
+//            together (kept in registers for the mean); exact fp32
+//            distances, each candidate ranked by one lane, the chosen set by
+//            ballot; r = x - mean -> R tile (64 tokens x D, K-major, hi and
+//            lo), double-buffered so the next tile's gather overlaps
+//   MMA warp  tcgen05.mma  D1^T = W1 . R^T  (A = W1 held in tensor memory
+//            for the whole launch, M = 128 hidden units per half, N = 64
+//            tokens); then codes = H . W2^T (A = the H tile through an
+//            MN-major descriptor, M = 128 with 64 tokens, N = d_c)
+//   activation warps (4)  thread = hidden unit: act(D1 + b1) over the tile's
+//            64 tokens -> H tile (hidden rows of 64 tokens, hi and lo), then
+//            TMEM -> + b2 -> bf16 codes
+// W1 and W2 are converted to fp16 once per launch (bf16 values of normal
+// range are exact in fp16).
 // Precision: every MMA operand that is not a weight is split into two fp16
 // terms, hi = fp16(v) and lo = fp16(v - hi), and multiplied twice, so r and
 // act(.) enter with about 22 significant bits.  With a single fp16 (or bf16)
