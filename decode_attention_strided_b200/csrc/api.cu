@@ -97,6 +97,8 @@ void build_plan(const deltakv_config& c, Plan& p) {
   w = align256(w + (size_t)(BH * p.nslot_cap * p.G * c.hidden) * 4);
   p.ws_ochunk = w;
   w = align256(w + (size_t)(BH * p.n_chunk_cap * p.G * (c.d_h + 1)) * 4);
+  p.ws_sparse = w;  // sparse decode: (m, l, output) of every share
+  w = align256(w + (size_t)(BH * kSparseSplits * p.G * (c.d_h + 2)) * 4);
   p.ws_bytes = std::max(compress_end, w);
 }
 
@@ -229,6 +231,30 @@ deltakv_status deltakv_decode_attention(deltakv_plan_t plan, int32_t T, const vo
     return DELTAKV_ERR_ALIGNMENT;
   return from_cuda(launch_decode(p, T, q, q_strides[0], q_strides[1], cache, W3, b3, W4, b4, out,
                                  out_strides[0], out_strides[1], workspace, (cudaStream_t)stream));
+}
+
+deltakv_status deltakv_decode_attention_sparse(deltakv_plan_t plan, int32_t T, const void* q,
+                                               const int64_t q_strides[2], const void* cache, const void* W3,
+                                               const float* b3, const void* W4, const float* b4,
+                                               const int32_t* tokens, int32_t n_sel, float* out,
+                                               const int64_t out_strides[2], void* workspace,
+                                               size_t workspace_bytes, deltakv_stream_t stream) {
+  if (!plan) return DELTAKV_ERR_INVALID_ARG;
+  const Plan& p = plan->p;
+  if (T < 1 || T > p.cfg.max_T || n_sel < 1) return DELTAKV_ERR_INVALID_ARG;
+  if (!q || !q_strides || !cache || !W3 || !W4 || !tokens || !out || !out_strides || !workspace)
+    return DELTAKV_ERR_INVALID_ARG;
+  if (workspace_bytes < p.ws_bytes) return DELTAKV_ERR_WORKSPACE;
+  if (q_strides[0] < 0 || q_strides[1] < 0 || out_strides[0] < 0 || out_strides[1] < 0)
+    return DELTAKV_ERR_INVALID_ARG;
+  if ((q_strides[0] * p.esize) % 16 || (q_strides[1] * p.esize) % 16 || (out_strides[0] * 4) % 16 ||
+      (out_strides[1] * 4) % 16)
+    return DELTAKV_ERR_ALIGNMENT;
+  if (!aligned16(q) || !aligned16(cache) || !aligned16(W3) || !aligned16(W4) || !aligned16(out) ||
+      !aligned16(workspace) || !aligned16(b3) || !aligned16(b4) || !aligned16(tokens))
+    return DELTAKV_ERR_ALIGNMENT;
+  return from_cuda(launch_decode_sparse(p, T, q, q_strides[0], q_strides[1], cache, W3, b3, W4, b4, tokens, n_sel,
+                                        out, out_strides[0], out_strides[1], workspace, (cudaStream_t)stream));
 }
 
 deltakv_status deltakv_reconstruct(deltakv_plan_t plan, int32_t T, const void* cache,

@@ -16,6 +16,7 @@ constexpr int kMaxCand = kMaxK + kExtraCand;
 constexpr int kMaxG = 8;          // query heads per kv-head
 constexpr int kMaxHidden = 256;
 constexpr int kMaxSplit = 32;     // decode splits per (sequence, kv-head)
+constexpr int kSparseSplits = 64;   // shares of one (sequence, kv-head)'s selection in sparse decode
 constexpr int kCombineSlots = 256;// reference slots per combine block
 constexpr int kNumSMs = 148;      // B200; used only to size launch grids
 
@@ -26,7 +27,7 @@ constexpr size_t kErrBytes = 256;
 enum KernelId {
   KID_REFPACK = 0, KID_CAND_SIMT, KID_CAND_TC, KID_ENCODE_SIMT, KID_ENCODE_TC, KID_RECONSTRUCT, KID_DEC_REF,
   KID_DEC_PREP, KID_DEC_STREAM_SIMT, KID_DEC_STREAM_TC, KID_DEC_COMBINE, KID_DEC_FINAL,
-  KID_APPEND_REFS, KID_APPEND_ROWS, KID_COUNT
+  KID_APPEND_REFS, KID_APPEND_ROWS, KID_SPARSE_ATTEND, KID_SPARSE_MERGE, KID_COUNT
 };
 const char* kernel_name(int id);
 
@@ -48,7 +49,7 @@ struct Plan {
   // decode workspace
   int nslot_cap;         // decode partial slots per (b, head)
   int n_chunk_cap;       // combine blocks per (b, head)
-  size_t ws_S, ws_Smax, ws_mref, ws_a, ws_cterm, ws_wtab, ws_part, ws_U, ws_ochunk;
+  size_t ws_S, ws_Smax, ws_mref, ws_a, ws_cterm, ws_wtab, ws_part, ws_U, ws_ochunk, ws_sparse;
   size_t ws_bytes;
 };
 
@@ -84,6 +85,10 @@ cudaError_t launch_candidates_simt(const Plan& p, int T, const KVView& kv, const
 bool candidates_tc_supported(const Plan& p);
 cudaError_t launch_candidates_tc(const Plan& p, int T, const KVView& kv, const void* cache,
                                  void* ws, cudaStream_t st);
+cudaError_t launch_decode_sparse(const Plan& p, int T, const void* q, int64_t qsb, int64_t qsh, const void* cache,
+                                 const void* W3, const float* b3, const void* W4, const float* b4,
+                                 const int32_t* tokens, int n_sel, float* out, int64_t osb, int64_t osh, void* ws,
+                                 cudaStream_t st);
 cudaError_t launch_append(const Plan& p, int T0, int T1, const KVView& kv, const void* W1, const float* b1,
                           const void* W2, const float* b2, void* cache, void* ws, cudaStream_t st);
 cudaError_t launch_encode(const Plan& p, int T, const KVView& kv, const void* W1, const float* b1,

@@ -26,7 +26,7 @@ STATUS = {
 }
 
 SYMBOLS = ("deltakv_plan", "deltakv_plan_destroy", "deltakv_get_cache_layout", "deltakv_compress",
-           "deltakv_append", "deltakv_decode_attention", "deltakv_reconstruct", "deltakv_device_status",
+           "deltakv_append", "deltakv_decode_attention", "deltakv_decode_attention_sparse", "deltakv_reconstruct", "deltakv_device_status",
            "deltakv_decode_attention_noalloc", "deltakv_set_profiling", "deltakv_profile_collect",
            "deltakv_status_string", "deltakv_version")
 
@@ -78,6 +78,9 @@ def load_library(path: str = LIB_PATH):
     lib.deltakv_append.restype = ctypes.c_int
     lib.deltakv_decode_attention.argtypes = [vp, i32, vp, i64p, vp, vp, vp, vp, vp, vp, i64p, vp, sz, vp]
     lib.deltakv_decode_attention.restype = ctypes.c_int
+    lib.deltakv_decode_attention_sparse.argtypes = [vp, i32, vp, i64p, vp, vp, vp, vp, vp, vp, i32, vp, i64p, vp,
+                                                    sz, vp]
+    lib.deltakv_decode_attention_sparse.restype = ctypes.c_int
     lib.deltakv_decode_attention_noalloc.argtypes = [vp, i32, vp, i64p, vp, vp, vp, vp, vp, vp, i64p, vp]
     lib.deltakv_decode_attention_noalloc.restype = ctypes.c_int
     lib.deltakv_reconstruct.argtypes = [vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
@@ -225,6 +228,20 @@ def decode_attention(p: Plan, T: int, q, cache, W3, b3, W4, b4, out, workspace, 
     _check("deltakv_decode_attention", lib.deltakv_decode_attention(
         p.handle, int(T), _ptr(q), qs, _ptr(cache), _ptr(W3), _ptr(b3), _ptr(W4), _ptr(b4), _ptr(out), os_,
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def decode_attention_sparse(p: Plan, T: int, q, cache, W3, b3, W4, b4, tokens, out, workspace, stream=None):
+    """deltakv_decode_attention_sparse: attention over the selected tokens
+    tokens [B, H, n_sel] (int32, contiguous) -> out [B, Hq, d_h] float32."""
+    lib = load_library()
+    if tokens.dtype != torch.int32 or not tokens.is_contiguous():
+        raise ValueError("tokens must be a contiguous int32 tensor [B, H, n_sel]")
+    qs = (ctypes.c_int64 * 2)(q.stride(0), q.stride(1))
+    os_ = (ctypes.c_int64 * 2)(out.stride(0), out.stride(1))
+    _check("deltakv_decode_attention_sparse", lib.deltakv_decode_attention_sparse(
+        p.handle, int(T), _ptr(q), qs, _ptr(cache), _ptr(W3), _ptr(b3), _ptr(W4), _ptr(b4), _ptr(tokens),
+        int(tokens.shape[-1]), _ptr(out), os_, _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
 
 
 def decode_attention_noalloc(p: Plan, T: int, q, cache, W3, b3, W4, b4, out, stream=None):

@@ -176,6 +176,29 @@ deltakv_status deltakv_decode_attention(deltakv_plan_t plan, int32_t T,
                                         void* workspace, size_t workspace_bytes,
                                         deltakv_stream_t stream);
 
+/* Sparse decode attention (section 4, reconstruction of only the tokens a
+ * sparse-attention selector such as OmniKV picks): for query head hq of
+ * kv-head h,
+ *   out = sum_{t in sel(b, h)} softmax_t(q . K_hat_t / sqrt(d_h)) V_hat_t,
+ * rebuilding only the selected tokens (reference rows as stored, the others
+ * as KV_R + W4 act(W3 code + b3) + b4) and never writing them out.
+ *   tokens : device int32 [B][H][n_sel], token indices in [0, T) chosen by
+ *            the caller (any order; an index outside [0, T) is skipped and
+ *            reported as DELTAKV_ERR_DEVICE_BOUNDS); n_sel >= 1.
+ *   every other argument as for deltakv_decode_attention.
+ * Runs on CUDA cores in float32: each CTA rebuilds 32 selected tokens at a
+ * time into shared memory and folds them into a running softmax; a second
+ * kernel merges the CTAs' shares. */
+deltakv_status deltakv_decode_attention_sparse(deltakv_plan_t plan, int32_t T,
+                                               const void* q, const int64_t q_strides[2],
+                                               const void* cache,
+                                               const void* W3, const float* b3,
+                                               const void* W4, const float* b4,
+                                               const int32_t* tokens, int32_t n_sel,
+                                               float* out, const int64_t out_strides[2],
+                                               void* workspace, size_t workspace_bytes,
+                                               deltakv_stream_t stream);
+
 /* Rebuild every token of one layer ("Ricostruzione") into dense float32
  * K_out, V_out [B][H][T][d_h] (contiguous).  For tests and debugging; the
  * decode path never materialises these. */

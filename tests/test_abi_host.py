@@ -110,4 +110,11 @@ def test_calls_reject_bad_arguments_before_any_launch(lib):
     assert lib.deltakv_append(p.handle, 500, 2048, fake, fake, strides, fake, None, fake, None, fake, fake, ws, None) == 1
     assert lib.deltakv_append(p.handle, 700, 700, None, None, None, None, None, None, None, None, None, 0, None) == 0
     assert lib.deltakv_append(p.handle, 500, 600, fake, fake, bad, fake, None, fake, None, fake, fake, ws, None) == 3
+    # sparse decode: no selection, NULL selection, misaligned selection
+    assert lib.deltakv_decode_attention_sparse(p.handle, 100, fake, qs, fake, fake, None, fake, None, fake, 0, fake, qs,
+                                               fake, ws, None) == 1
+    assert lib.deltakv_decode_attention_sparse(p.handle, 100, fake, qs, fake, fake, None, fake, None, None, 8, fake, qs,
+                                               fake, ws, None) == 1
+    assert lib.deltakv_decode_attention_sparse(p.handle, 100, fake, qs, fake, fake, None, fake, None,
+                                               vp((1 << 20) + 4), 8, fake, qs, fake, ws, None) == 3
     assert lib.deltakv_plan_destroy(None) == 0
