@@ -217,6 +217,34 @@ def append_timing(sh, w, steps):
             "kv_heads": sh.H, "references_searched": (t + sh.s - 1) // sh.s}
 
 
+def sparse_timing(sh, w, steps, n_sel=4096):
+    """Sparse decode over n_sel compressed tokens per (sequence, kv-head)
+    (t = 32 i + 7: none of them a reference, so every one is rebuilt), for
+    the decode batch, all layers; outside the timed step."""
+    from decode_attention_strided_b200 import deltakv as dkv
+    if 32 * (n_sel - 1) + 7 >= sh.T:
+        return None
+    dev = w["q"][0].device
+    sel = (torch.arange(n_sel, device=dev, dtype=torch.int32) * 32 + 7).expand(sh.Bd, sh.H, n_sel).contiguous()
+
+    def one():
+        for l in range(sh.L):
+            dkv.decode_attention_sparse(w["pd"], sh.T, w["q"][l], w["dec_cache"][l], w["W"][l]["W3"], None,
+                                        w["W"][l]["W4"], None, sel, w["out"][l], w["ws_d"])
+
+    one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        one()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    return {"ms_per_layer": ms / sh.L, "selected_tokens": n_sel, "batch": sh.Bd, "kv_heads": sh.H,
+            "rebuilt_tokens_per_s": sh.Bd * sh.H * n_sel * sh.L / (ms / 1e3)}
+
+
 # ------------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -409,6 +437,7 @@ def main():
     for p in (w["pc"], w["pd"]):
         dkv.set_profiling(p, False)
     append = append_timing(sh, w, a.steps)
+    sparse = sparse_timing(sh, w, a.steps)
     status = max(dkv.device_status(w["pc"], w["ws_c"]), dkv.device_status(w["pd"], w["ws_d"]))
     step_ms = [e[0].elapsed_time(e[2]) for e in ev]
     comp_ms = [e[0].elapsed_time(e[1]) for e in ev]
@@ -456,7 +485,7 @@ def main():
         "metric": METRIC, "value": value, "unit": "Mtok/s", "n_gpus": world, "steps": a.steps,
         "warmup": a.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(sh),
-        "compress": compress, "decode_attn": decode_attn, "append": append, "roofline": roof, "rooflines": rooflines,
+        "compress": compress, "decode_attn": decode_attn, "append": append, "sparse_decode": sparse, "roofline": roof, "rooflines": rooflines,
         "cpu_baseline": cpu,
         "e2e": e2e, "gpu_launches": launches, "kernels": {k_: {"launches": n, "ms": ms} for k_, (n, ms) in prof.items()},
         "clocks": clk, "device_status": status, "setup_s": setup_s, "wall_s": wall,

@@ -24,9 +24,12 @@ def _setup(c: Case):
     return inp, p, W, bias, cache, ws
 
 
-def _selection(c: Case, n_sel: int, seed: int):
+def _selection(c: Case, n_sel: int, seed: int, repeats: bool = False):
+    """Unsorted token indices per (sequence, kv-head); with `repeats` the
+    same token may appear more than once (it then counts once per
+    occurrence, as a gather followed by dense attention would)."""
     rng = np.random.default_rng(seed)
-    sel = np.stack([np.stack([rng.choice(c.T, n_sel, replace=False) for _ in range(c.H)]) for _ in range(c.B)])
+    sel = np.stack([np.stack([rng.choice(c.T, n_sel, replace=repeats) for _ in range(c.H)]) for _ in range(c.B)])
     return sel.astype(np.int32)
 
 
@@ -42,16 +45,21 @@ def _sparse(c, inp, p, W, bias, cache, ws, sel):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("name,case,n_sel", [
-    ("bf16_d128", Case(B=2, H=2, Hq=8, d_h=128, T=3000, s=16, k=4, d_c=32, hidden=256, dtype=dkv.BF16, n_lat=8), 700),
+@pytest.mark.parametrize("name,case,n_sel,repeats", [
+    ("bf16_d128", Case(B=2, H=2, Hq=8, d_h=128, T=3000, s=16, k=4, d_c=32, hidden=256, dtype=dkv.BF16, n_lat=8), 700,
+     False),
     ("bf16_d64_tanh_bias", Case(B=1, H=2, Hq=4, d_h=64, T=1500, s=8, k=2, d_c=16, hidden=128, dtype=dkv.BF16,
-                                act=dkv.ACT_GELU_TANH, biases=True), 37),
-    ("f32_G8", Case(B=1, H=1, Hq=8, d_h=64, T=900, s=4, k=3, d_c=32, hidden=64, dtype=dkv.F32, biases=True), 250),
+                                act=dkv.ACT_GELU_TANH, biases=True), 37, False),
+    ("f32_G8", Case(B=1, H=1, Hq=8, d_h=64, T=900, s=4, k=3, d_c=32, hidden=64, dtype=dkv.F32, biases=True), 250,
+     False),
+    ("bf16_G1_repeats", Case(B=2, H=2, Hq=2, d_h=128, T=700, s=16, k=4, d_c=32, hidden=256, dtype=dkv.BF16), 1500,
+     True),
+    ("bf16_one_token", Case(B=1, H=2, Hq=4, d_h=64, T=300, s=8, k=2, d_c=16, hidden=64, dtype=dkv.BF16), 1, False),
 ])
-def test_sparse_matches_oracle(name, case, n_sel):
+def test_sparse_matches_oracle(name, case, n_sel, repeats):
     c = case
     inp, p, W, bias, cache, ws = _setup(c)
-    sel = _selection(c, n_sel, 7)
+    sel = _selection(c, n_sel, 7, repeats)
     out, status = _sparse(c, inp, p, W, bias, cache, ws, sel)
     assert status == 0
     G = c.Hq // c.H
