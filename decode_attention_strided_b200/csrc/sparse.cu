@@ -79,6 +79,39 @@ template <> __device__ __forceinline__ float2 load2<__nv_bfloat16>(const __nv_bf
   return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
 }
 
+// Eight consecutive elements of a reference row, loaded in one go (16 bytes
+// of bf16, 32 of float) so that all of a token's slots are in flight together.
+template <typename E> struct Row8;
+template <> struct Row8<__nv_bfloat16> {
+  uint4 v;
+  __device__ __forceinline__ void load(const __nv_bfloat16* p) { v = __ldg(reinterpret_cast<const uint4*>(p)); }
+  __device__ __forceinline__ void add_to(float (&a)[8]) const {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      a[2 * i] += __uint_as_float(w[i] << 16);  // bf16 -> fp32 is exact
+      a[2 * i + 1] += __uint_as_float(w[i] & 0xffff0000u);
+    }
+  }
+};
+template <> struct Row8<float> {
+  float4 x, y;
+  __device__ __forceinline__ void load(const float* p) {
+    x = __ldg(reinterpret_cast<const float4*>(p));
+    y = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  }
+  __device__ __forceinline__ void add_to(float (&a)[8]) const {
+    a[0] += x.x;
+    a[1] += x.y;
+    a[2] += x.z;
+    a[3] += x.w;
+    a[4] += y.x;
+    a[5] += y.y;
+    a[6] += y.z;
+    a[7] += y.w;
+  }
+};
+
 // Sum each of N (a power of two <= 32) values over the warp.  Returns the
 // total of value g(lane) = the lane's position among the N groups of 32 / N
 // lanes; lanes with (lane % (32 / N)) == 0 hold distinct g.  log2(N) halving
@@ -105,7 +138,7 @@ __device__ __forceinline__ float warp_sum_scatter(float (&v)[N], int lane, int& 
 }
 
 template <typename E, int GM>
-__global__ void __launch_bounds__(kSpThreads)
+__global__ void __launch_bounds__(kSpThreads, GM <= 4 ? 2 : 1)
     sparse_attend_kernel(const SparseParams P, const E* __restrict__ q, const int32_t* __restrict__ tokens,
                          const E* __restrict__ refk, const E* __restrict__ refv, const E* __restrict__ code,
                          const int32_t* __restrict__ idx, const E* __restrict__ W3, const float* __restrict__ b3,
@@ -224,53 +257,64 @@ __global__ void __launch_bounds__(kSpThreads)
       t_next = (i0 + kSpR + tid < i_hi) ? tokens[bh * P.n_sel + i0 + kSpR + tid] : -1;
     }
     __syncthreads();
-    // codes (transposed) and slot lists of the coded tokens
-    for (int i = tid; i < kSpR * d_c; i += kSpThreads) {
-      const int r = i / d_c, e = i - r * d_c;
-      CsT[e * kSpRP + r] = kind[r] == 1 ? to_f(cd[code_row_of(tok[r], P.s) * d_c + e]) : 0.f;
-    }
-    for (int i = tid; i < kSpR * K; i += kSpThreads) {
-      const int r = i / K, j = i - r * K;
-      int v = -1;
-      if (kind[r] == 1) {
-        v = ix[code_row_of(tok[r], P.s) * K + j];
-        if (v >= n_ref) {
-          latch_error(err, DELTAKV_ERR_DEVICE_BOUNDS, (uint32_t)v);
-          v = -1;
+    // codes (transposed) and slot lists of the coded tokens: every load of
+    // the step is issued before the first store
+    {
+      float2 cv[4];
+      int cr[4], ce[4];
+      const int hc = d_c >> 1;
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int i = tid + m * kSpThreads;
+        cr[m] = -1;
+        cv[m] = make_float2(0.f, 0.f);
+        if (i < kSpR * hc) {
+          const int r = i / hc;
+          cr[m] = r;
+          ce[m] = 2 * (i - r * hc);
+          if (kind[r] == 1) cv[m] = load2(cd + code_row_of(tok[r], P.s) * d_c + ce[m]);
         }
       }
-      slots[i] = v < 0 ? -1 : v;
+      int sv = -1;
+      if (tid < kSpR * K) {
+        const int r = tid / K, j = tid - r * K;
+        if (kind[r] == 1) {
+          sv = ix[code_row_of(tok[r], P.s) * K + j];
+          if (sv >= n_ref) {
+            latch_error(err, DELTAKV_ERR_DEVICE_BOUNDS, (uint32_t)sv);
+            sv = -1;
+          }
+        }
+        slots[tid] = sv < 0 ? -1 : sv;
+      }
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+        if (cr[m] >= 0) {
+          CsT[ce[m] * kSpRP + cr[m]] = cv[m].x;
+          CsT[(ce[m] + 1) * kSpRP + cr[m]] = cv[m].y;
+        }
     }
     __syncthreads();
-    // reference part: the reference row itself, or the mean of the slots' rows
-    const int hd = d_h >> 1;
-    for (int i = tid; i < kSpR * hd; i += kSpThreads) {
-      const int r = i / hd, e = 2 * (i - r * hd), ty = kind[r];
-      float2 mk = make_float2(0.f, 0.f), mv = make_float2(0.f, 0.f);
-      if (ty == 0) {
-        const int64_t j = tok[r] / P.s;
-        mk = load2(rk + j * d_h + e);
-        mv = load2(rv + j * d_h + e);
-      } else if (ty == 1) {
-        int ke = 0;
-        for (int j2 = 0; j2 < K; ++j2) {
-          const int j = slots[r * K + j2];
-          if (j < 0) continue;
-          const float2 a = load2(rk + (int64_t)j * d_h + e), c = load2(rv + (int64_t)j * d_h + e);
-          mk.x += a.x;
-          mk.y += a.y;
-          mv.x += c.x;
-          mv.y += c.y;
-          ++ke;
-        }
-        const float kf = (float)max(ke, 1);
-        mk.x /= kf;
-        mk.y /= kf;
-        mv.x /= kf;
-        mv.y /= kf;
+    // reference part, issued now and consumed after the first decompressor
+    // layer: thread (ir, e8) sums elements e8 .. e8 + 7 of the rows of token
+    // ir's references (the reference row itself for a reference token)
+    const int per_row = d_h >> 3;
+    const bool has_item = tid < kSpR * per_row;
+    const int ir = has_item ? tid / per_row : 0;
+    const int e8 = has_item ? 8 * (tid - ir * per_row) : 0;
+    const int ity = has_item ? kind[ir] : -1;
+    Row8<E> rka[4], rva[4];
+    int js[4];
+#pragma unroll
+    for (int j2 = 0; j2 < 4; ++j2) {
+      int j = -1;
+      if (ity == 0 && j2 == 0) j = tok[ir] / P.s;
+      if (ity == 1 && j2 < K) j = slots[ir * K + j2];
+      js[j2] = j;
+      if (j >= 0) {
+        rka[j2].load(rk + (int64_t)j * d_h + e8);
+        rva[j2].load(rv + (int64_t)j * d_h + e8);
       }
-      *reinterpret_cast<float2*>(MK + r * d_h + e) = mk;
-      *reinterpret_cast<float2*>(MV + r * d_h + e) = mv;
     }
     // first decompressor layer: thread (n0, half) owns columns n0 and n0 + hidden/2
     // for the round's tokens 8 half .. 8 half + 7
@@ -302,6 +346,49 @@ __global__ void __launch_bounds__(kSpThreads)
         U[rr * hidden + n0] = on ? act_fast(P.act, a0[r]) : 0.f;
         U[rr * hidden + n1] = on ? act_fast(P.act, a1[r]) : 0.f;
       }
+    }
+    if (has_item) {
+      float mk[8], mv[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mk[i] = mv[i] = 0.f;
+      int ke = 0;
+#pragma unroll
+      for (int j2 = 0; j2 < 4; ++j2)
+        if (js[j2] >= 0) {
+          rka[j2].add_to(mk);
+          rva[j2].add_to(mv);
+          ++ke;
+        }
+      if (ity == 1 && K > 4) {  // slots 4 .. 7
+#pragma unroll
+        for (int j2 = 0; j2 < 4; ++j2) {
+          const int j = (4 + j2 < K) ? slots[ir * K + 4 + j2] : -1;
+          js[j2] = j;
+          if (j >= 0) {
+            rka[j2].load(rk + (int64_t)j * d_h + e8);
+            rva[j2].load(rv + (int64_t)j * d_h + e8);
+          }
+        }
+#pragma unroll
+        for (int j2 = 0; j2 < 4; ++j2)
+          if (js[j2] >= 0) {
+            rka[j2].add_to(mk);
+            rva[j2].add_to(mv);
+            ++ke;
+          }
+      }
+      const float kf = (float)max(ke, 1);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        mk[i] /= kf;
+        mv[i] /= kf;
+      }
+      float4* dk = reinterpret_cast<float4*>(MK + ir * d_h + e8);
+      float4* dv = reinterpret_cast<float4*>(MV + ir * d_h + e8);
+      dk[0] = make_float4(mk[0], mk[1], mk[2], mk[3]);
+      dk[1] = make_float4(mk[4], mk[5], mk[6], mk[7]);
+      dv[0] = make_float4(mv[0], mv[1], mv[2], mv[3]);
+      dv[1] = make_float4(mv[4], mv[5], mv[6], mv[7]);
     }
     __syncthreads();
     // logits: warp w takes tokens w and w + 8
