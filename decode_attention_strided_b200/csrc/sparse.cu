@@ -10,7 +10,7 @@
 // The selection is an input (the selector itself is not part of this path).
 //
 // Kernels: each CTA takes a contiguous share of one (sequence, kv-head)'s
-// selection, 16 tokens per round, and never forms K_hat or V_hat rows.  The
+// selection, 16 tokens per pass, and never forms K_hat or V_hat rows.  The
 // decompressor's output layer is linear, so for a non-reference token with
 // code c, u = act(W3 c + b3) and reference mean (mk, mv):
 //   q . k_hat = q . mk + (W4_K^T q) . u + q . b4_K
@@ -27,7 +27,7 @@
 namespace dkv {
 
 namespace {
-constexpr int kSpR = 16;           // tokens per round
+constexpr int kSpR = 16;           // tokens per pass
 constexpr int kSpRP = kSpR + 4;    // row stride of the transposed code tile (keeps float4 rows aligned)
 constexpr int kSpThreads = 256;
 constexpr int kSpWarps = kSpThreads / 32;
@@ -60,7 +60,7 @@ __host__ __device__ inline SpLayout sp_layout(int d_c, int hidden, int G, int d_
   L.qs = sp_take(o, G * d_h);             // q / sqrt(d_h), [G][d_h]
   L.qw = sp_take(o, G * hidden);          // W4_K^T q, [G][hidden]
   L.qb = sp_take(o, G);                   // q . b4_K
-  L.cst = sp_take(o, d_c * kSpRP);        // codes of the round, [d_c][kSpRP]
+  L.cst = sp_take(o, d_c * kSpRP);        // codes of the pass, [d_c][kSpRP]
   L.u = sp_take(o, kSpR * hidden);        // act(W3 c + b3), [kSpR][hidden]
   L.mk = sp_take(o, kSpR * d_h);          // K part of the reference mean (or the reference row)
   L.mv = sp_take(o, kSpR * d_h);          // V part
@@ -238,8 +238,8 @@ __global__ void __launch_bounds__(kSpThreads, GM <= 4 ? 2 : 1)
   if (tid < kSpR && i_lo + tid < i_hi) t_next = tokens[bh * P.n_sel + i_lo + tid];
 
   for (int i0 = i_lo; i0 < i_hi; i0 += kSpR) {
-    __syncthreads();  // the previous round's readers are done
-    // tokens of this round (loaded one round ahead)
+    __syncthreads();  // the previous pass's readers are done
+    // tokens of this pass (loaded one pass ahead)
     if (tid < kSpR) {
       int t = t_next, ty = -1;
       if (i0 + tid < i_hi) {
@@ -317,7 +317,7 @@ __global__ void __launch_bounds__(kSpThreads, GM <= 4 ? 2 : 1)
       }
     }
     // first decompressor layer: thread (n0, half) owns columns n0 and n0 + hidden/2
-    // for the round's tokens 8 half .. 8 half + 7
+    // for the pass's tokens 8 half .. 8 half + 7
     if (tid < hidden) {
       const int hh = hidden >> 1, n0 = tid % hh, half = tid / hh, n1 = n0 + hh;
       float a0[8], a1[8];
@@ -578,7 +578,7 @@ static cudaError_t sparse_launch(const Plan& p, int T, const void* q, int64_t qs
   P.qsh = qsh;
   P.scale = 1.0f / sqrtf((float)c.d_h);
   const int64_t BH = (int64_t)c.batch * c.kv_heads;
-  // shares of at least one round each, about two CTAs per SM in total
+  // shares of at least one pass each, about two CTAs per SM in total
   int nsplit = (int)std::min<int64_t>((n_sel + kSpR - 1) / kSpR, std::max<int64_t>(1, 2 * kNumSMs / BH));
   nsplit = std::max(1, std::min(nsplit, kSparseSplits));
   P.nsplit = nsplit;
