@@ -278,3 +278,47 @@ def test_attention_closed_forms(oracle_mod):
     Q = rng.normal(size=(3, 3))
     o = oracle_mod.attention(Q, K, V)
     assert np.array_equal(oracle_mod.attention(Q[::-1].copy(), K, V), o[::-1])
+
+
+# ------------------------------------------------- streaming and sparse use
+
+def test_compression_of_a_token_depends_only_on_its_prefix(oracle_mod):
+    """Compression looks only at earlier references (the "historical" tokens
+    of step 1), so a cache built over a prefix [0, T0) and extended later
+    holds exactly what one pass over [0, T) writes for those tokens; later
+    tokens, even references that nearly copy an earlier token, change nothing
+    before them.  A search over every reference would change the slots of 69
+    of the prefix's tokens here."""
+    from decode_attention_strided_b200 import synth
+    T, T0, d_h, s, k = 160, 97, 8, 4, 3
+    K, V = _tokens(T, d_h, 4, seed=21)
+    w = {n: t.double().numpy() for n, t in synth.codec_weights(0, d_h, 8, 32, dtype=torch.float32).items()}
+    full = oracle_mod.compress(K, V, w["W1"], None, w["W2"], None, s, k)
+    # make the later references near-copies of early tokens: a non-causal
+    # search would now pick them
+    first = -(-T0 // s) * s
+    for t in range(first, T, s):
+        K[t], V[t] = K[t - first + 1] + 1e-3, V[t - first + 1] - 1e-3
+    pre = oracle_mod.compress(K[:T0].copy(), V[:T0].copy(), w["W1"], None, w["W2"], None, s, k)
+    full2 = oracle_mod.compress(K, V, w["W1"], None, w["W2"], None, s, k)
+    for a, b, c in zip(pre, full, full2):
+        assert np.array_equal(a, b[:T0], equal_nan=True) and np.array_equal(a, c[:T0], equal_nan=True)
+    # and every selected slot of every token is strictly earlier than it
+    t_all = np.arange(T)[:, None]
+    sel = full2[0]
+    assert ((sel < 0) | (sel * s < t_all)).all()
+
+
+def test_attention_over_a_list_with_repeats(oracle_mod):
+    """Sparse decode attends over the caller's token list as given: a token
+    listed twice carries twice the weight.  Closed form for keys whose scaled
+    logits differ by delta: list [0, 0, 1] gives weights 2 : e^delta."""
+    rng = _rng(6)
+    V = rng.normal(size=(2, 4))
+    K = np.array([[0.0, 0, 0, 0], [2.0, 0, 0, 0]])
+    q = np.array([[1.0, 0, 0, 0]])
+    delta = 2.0 / math.sqrt(4.0)
+    want = (2 * V[0] + math.exp(delta) * V[1]) / (2 + math.exp(delta))
+    t = np.array([0, 0, 1])
+    got = oracle_mod.attention(q, K[t], V[t])[0]
+    assert np.allclose(got, want, rtol=1e-14, atol=1e-15)
