@@ -236,6 +236,11 @@ def decode_attention_sparse(p: Plan, T: int, q, cache, W3, b3, W4, b4, tokens, o
     lib = load_library()
     if tokens.dtype != torch.int32 or not tokens.is_contiguous():
         raise ValueError("tokens must be a contiguous int32 tensor [B, H, n_sel]")
+    # the library reads B * H * n_sel indices: a tensor of another shape
+    # would be read past its end
+    if tokens.dim() != 3 or tuple(tokens.shape[:2]) != (p.cfg.batch, p.cfg.kv_heads) or tokens.shape[2] < 1:
+        raise ValueError(f"tokens must have shape [{p.cfg.batch}, {p.cfg.kv_heads}, n_sel >= 1], "
+                         f"got {list(tokens.shape)}")
     qs = (ctypes.c_int64 * 2)(q.stride(0), q.stride(1))
     os_ = (ctypes.c_int64 * 2)(out.stride(0), out.stride(1))
     _check("deltakv_decode_attention_sparse", lib.deltakv_decode_attention_sparse(

@@ -118,3 +118,18 @@ def test_calls_reject_bad_arguments_before_any_launch(lib):
     assert lib.deltakv_decode_attention_sparse(p.handle, 100, fake, qs, fake, fake, None, fake, None,
                                                vp((1 << 20) + 4), 8, fake, qs, fake, ws, None) == 3
     assert lib.deltakv_plan_destroy(None) == 0
+
+
+def test_sparse_binding_rejects_a_selection_of_the_wrong_shape(lib):
+    """The library reads B * H * n_sel indices; the binding refuses any other
+    shape before calling it (tensors here are host tensors that are never
+    read)."""
+    import torch
+    cfg = dkv.Config(batch=2, kv_heads=4, q_heads=8, d_h=64, max_T=1000, stride_s=8, k=2, d_c=16, hidden=64)
+    p = dkv.plan(cfg)
+    x = torch.zeros(16)
+    for shape in [(4, 10), (1, 4, 10), (2, 2, 10), (2, 4, 0), (2, 4, 10, 1)]:
+        with pytest.raises(ValueError):
+            dkv.decode_attention_sparse(p, 100, x, x, x, None, x, None, torch.zeros(shape, dtype=torch.int32), x, x)
+    with pytest.raises(ValueError):  # wrong dtype
+        dkv.decode_attention_sparse(p, 100, x, x, x, None, x, None, torch.zeros((2, 4, 10), dtype=torch.int64), x, x)
