@@ -485,9 +485,9 @@ def main():
         "metric": METRIC, "value": value, "unit": "Mtok/s", "n_gpus": world, "steps": a.steps,
         "warmup": a.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(sh),
-        "compress": compress, "decode_attn": decode_attn, "append": append, "sparse_decode": sparse, "roofline": roof, "rooflines": rooflines,
-        "cpu_baseline": cpu,
-        "e2e": e2e, "gpu_launches": launches, "kernels": {k_: {"launches": n, "ms": ms} for k_, (n, ms) in prof.items()},
+        "compress": compress, "decode_attn": decode_attn, "append": append, "sparse_decode": sparse,
+        "roofline": roof, "rooflines": rooflines, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
+        "kernels": {k_: {"launches": n, "ms": ms} for k_, (n, ms) in prof.items()},
         "clocks": clk, "device_status": status, "setup_s": setup_s, "wall_s": wall,
     }
     if rank == 0:

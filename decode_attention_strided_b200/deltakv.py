@@ -26,9 +26,9 @@ STATUS = {
 }
 
 SYMBOLS = ("deltakv_plan", "deltakv_plan_destroy", "deltakv_get_cache_layout", "deltakv_compress",
-           "deltakv_append", "deltakv_decode_attention", "deltakv_decode_attention_sparse", "deltakv_reconstruct", "deltakv_device_status",
-           "deltakv_decode_attention_noalloc", "deltakv_set_profiling", "deltakv_profile_collect",
-           "deltakv_status_string", "deltakv_version")
+           "deltakv_append", "deltakv_decode_attention", "deltakv_decode_attention_sparse",
+           "deltakv_decode_attention_noalloc", "deltakv_reconstruct", "deltakv_device_status",
+           "deltakv_set_profiling", "deltakv_profile_collect", "deltakv_status_string", "deltakv_version")
 
 
 class DeltaKVError(RuntimeError):
