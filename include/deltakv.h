@@ -183,12 +183,15 @@ deltakv_status deltakv_decode_attention(deltakv_plan_t plan, int32_t T,
  * rebuilding only the selected tokens (reference rows as stored, the others
  * as KV_R + W4 act(W3 code + b3) + b4) and never writing them out.
  *   tokens : device int32 [B][H][n_sel], token indices in [0, T) chosen by
- *            the caller (any order; an index outside [0, T) is skipped and
- *            reported as DELTAKV_ERR_DEVICE_BOUNDS); n_sel >= 1.
+ *            the caller (any order; a repeated index counts once per
+ *            occurrence; an index outside [0, T) is skipped and reported as
+ *            DELTAKV_ERR_DEVICE_BOUNDS); n_sel >= 1; caller-owned, read only.
  *   every other argument as for deltakv_decode_attention.
- * Runs on CUDA cores in float32: each CTA rebuilds 32 selected tokens at a
- * time into shared memory and folds them into a running softmax; a second
- * kernel merges the CTAs' shares. */
+ * Runs on CUDA cores in float32, 16 selected tokens per pass of a CTA: the
+ * first decompressor layer per token, and the (linear) second layer folded
+ * into the query and applied once per CTA to the softmax-weighted sum of its
+ * activations, so no K_hat/V_hat row is formed; a second kernel merges the
+ * CTAs' shares. */
 deltakv_status deltakv_decode_attention_sparse(deltakv_plan_t plan, int32_t T,
                                                const void* q, const int64_t q_strides[2],
                                                const void* cache,
