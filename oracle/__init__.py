@@ -28,6 +28,7 @@ from .oracle import (  # noqa: F401
     lib_path,
     mlp,
     reconstruct,
+    reconstruct_rows,
     round_to,
     select,
 )

@@ -280,6 +280,44 @@ int deltakv_oracle_compress(int T, int d_h, int s, int k, int d_c, int hidden,
 
 /* ------------------------------------------------------- reconstruction */
 
+/* Rebuild token t ("Ricostruzione") into kh, vh [d_h] from what the cache
+ * holds for it: a reference token (t mod s == 0) is its stored row of K, V;
+ * any other token is KV_R + W4 act(W3 code + b3) + b4, where KV_R is the mean
+ * of the reference rows of the slots it (k entries, -1 unused) lists and
+ * code [d_c] is its stored code.  y and mean are caller scratch of 2*d_h. */
+static void reconstruct_token(int t, int d_h, int s, int k, int d_c, int hidden, int act,
+                              const double* K, const double* V,
+                              const int32_t* it, const double* code,
+                              const double* W3, const double* b3,
+                              const double* W4, const double* b4,
+                              double* kh, double* vh, double* y, double* mean)
+{
+    int D = 2 * d_h;
+    if (t % s == 0) {
+        for (int e = 0; e < d_h; ++e) {
+            kh[e] = K[(size_t)t * d_h + e];
+            vh[e] = V[(size_t)t * d_h + e];
+        }
+        return;
+    }
+    int k_eff = 0;
+    for (int e = 0; e < D; ++e) mean[e] = 0.0;
+    for (int i = 0; i < k; ++i) {
+        if (it[i] < 0) continue;
+        int u = it[i] * s;
+        for (int e = 0; e < d_h; ++e) {
+            mean[e] += K[(size_t)u * d_h + e];
+            mean[d_h + e] += V[(size_t)u * d_h + e];
+        }
+        ++k_eff;
+    }
+    deltakv_oracle_mlp(d_c, hidden, D, act, W3, b3, W4, b4, code, y);
+    for (int e = 0; e < d_h; ++e) {
+        kh[e] = mean[e] / (double)k_eff + y[e];
+        vh[e] = mean[d_h + e] / (double)k_eff + y[d_h + e];
+    }
+}
+
 /* Rebuild K_hat, V_hat [T][d_h] from what the compressed cache holds: the
  * reference rows (read from K, V at tokens j*s only), the slots idx and the
  * codes.  x_hat = KV_R + W4 act(W3 code + b3) + b4 for non-reference tokens. */
@@ -303,33 +341,51 @@ int deltakv_oracle_reconstruct(int T, int d_h, int s, int k, int d_c, int hidden
         double* y = (double*)malloc(sizeof(double) * (size_t)D);
         double* mean = (double*)malloc(sizeof(double) * (size_t)D);
 #pragma omp for schedule(dynamic, 16)
-        for (int t = 0; t < T; ++t) {
-            if (t % s == 0) {
-                for (int e = 0; e < d_h; ++e) {
-                    K_hat[(size_t)t * d_h + e] = K[(size_t)t * d_h + e];
-                    V_hat[(size_t)t * d_h + e] = V[(size_t)t * d_h + e];
-                }
-                continue;
-            }
-            const int32_t* it = idx + (size_t)t * k;
-            int k_eff = 0;
-            for (int e = 0; e < D; ++e) mean[e] = 0.0;
-            for (int i = 0; i < k; ++i) {
-                if (it[i] < 0) continue;
-                int u = it[i] * s;
-                for (int e = 0; e < d_h; ++e) {
-                    mean[e] += K[(size_t)u * d_h + e];
-                    mean[d_h + e] += V[(size_t)u * d_h + e];
-                }
-                ++k_eff;
-            }
-            deltakv_oracle_mlp(d_c, hidden, D, act, W3, b3, W4, b4,
-                               code + (size_t)t * d_c, y);
-            for (int e = 0; e < d_h; ++e) {
-                K_hat[(size_t)t * d_h + e] = mean[e] / (double)k_eff + y[e];
-                V_hat[(size_t)t * d_h + e] = mean[d_h + e] / (double)k_eff + y[d_h + e];
-            }
-        }
+        for (int t = 0; t < T; ++t)
+            reconstruct_token(t, d_h, s, k, d_c, hidden, act, K, V, idx + (size_t)t * k,
+                              code + (size_t)t * d_c, W3, b3, W4, b4,
+                              K_hat + (size_t)t * d_h, V_hat + (size_t)t * d_h, y, mean);
+        free(y);
+        free(mean);
+    }
+    return 0;
+}
+
+/* Rebuild only the tokens rows[0..n_rows) of a (sequence, kv-head) whose raw
+ * K, V are [T][d_h] (only their reference rows are read).  Row i of idx_rows
+ * [n_rows][k] and code_rows [n_rows][d_c] holds what the cache stores for
+ * token rows[i]; K_hat, V_hat [n_rows][d_h] receive the rebuilt rows.  Same
+ * arithmetic as deltakv_oracle_reconstruct, token by token. */
+int deltakv_oracle_reconstruct_rows(int T, int d_h, int s, int k, int d_c, int hidden, int act,
+                                    const double* K, const double* V,
+                                    int n_rows, const int32_t* rows,
+                                    const int32_t* idx_rows, const double* code_rows,
+                                    const double* W3, const double* b3,
+                                    const double* W4, const double* b4,
+                                    double* K_hat, double* V_hat, int n_threads)
+{
+    int D = 2 * d_h;
+    if (T < 0 || d_h <= 0 || s <= 0 || k <= 0 || d_c <= 0 || hidden <= 0 || n_rows < 0)
+        return -1;
+    for (int i = 0; i < n_rows; ++i) {
+        if (rows[i] < 0 || rows[i] >= T) return -1;
+        for (int j = 0; j < k; ++j)
+            if (idx_rows[(size_t)i * k + j] >= 0 && idx_rows[(size_t)i * k + j] * s >= rows[i]) return -1;
+    }
+#ifdef _OPENMP
+    if (n_threads > 0) omp_set_num_threads(n_threads);
+#else
+    (void)n_threads;
+#endif
+#pragma omp parallel
+    {
+        double* y = (double*)malloc(sizeof(double) * (size_t)D);
+        double* mean = (double*)malloc(sizeof(double) * (size_t)D);
+#pragma omp for schedule(dynamic, 16)
+        for (int i = 0; i < n_rows; ++i)
+            reconstruct_token(rows[i], d_h, s, k, d_c, hidden, act, K, V, idx_rows + (size_t)i * k,
+                              code_rows + (size_t)i * d_c, W3, b3, W4, b4,
+                              K_hat + (size_t)i * d_h, V_hat + (size_t)i * d_h, y, mean);
         free(y);
         free(mean);
     }

@@ -63,6 +63,9 @@ def _load():
             lib.deltakv_oracle_compress.argtypes = [ctypes.c_int] * 8 + [_dp] * 6 + [_ip, _dp, _dp, _dp, ctypes.c_int]
             lib.deltakv_oracle_reconstruct.restype = ctypes.c_int
             lib.deltakv_oracle_reconstruct.argtypes = [ctypes.c_int] * 7 + [_dp, _dp, _ip, _dp] + [_dp] * 4 + [_dp, _dp, ctypes.c_int]
+            lib.deltakv_oracle_reconstruct_rows.restype = ctypes.c_int
+            lib.deltakv_oracle_reconstruct_rows.argtypes = ([ctypes.c_int] * 7 + [_dp, _dp, ctypes.c_int, _ip, _ip, _dp]
+                                                            + [_dp] * 4 + [_dp, _dp, ctypes.c_int])
             lib.deltakv_oracle_attention.restype = ctypes.c_int
             lib.deltakv_oracle_attention.argtypes = [ctypes.c_int] * 3 + [_dp] * 4
             _lib = lib
@@ -171,6 +174,28 @@ def reconstruct(K, V, idx, code, W3, b3, W4, b4, s: int, act_kind: int = ACT_GEL
                                             _ptr(Kh), _ptr(Vh), int(n_threads))
     if rc != 0:
         raise ValueError("oracle reconstruct: invalid arguments")
+    return Kh, Vh
+
+
+def reconstruct_rows(K, V, rows, idx_rows, code_rows, W3, b3, W4, b4, s: int, act_kind: int = ACT_GELU_ERF,
+                     n_threads: int = 0):
+    """Rebuild only the tokens `rows` of one (sequence, kv-head): idx_rows
+    [n, k] and code_rows [n, d_c] are what the cache holds for them.  Returns
+    (K_hat, V_hat) [n, d_h]."""
+    K, V, code_rows, W3, b3, W4, b4 = _f64(K), _f64(V), _f64(code_rows), _f64(W3), _f64(b3), _f64(W4), _f64(b4)
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int32))
+    idx_rows = np.ascontiguousarray(np.asarray(idx_rows, dtype=np.int32))
+    T, d_h = K.shape
+    n, k = idx_rows.shape
+    d_c = code_rows.shape[1]
+    hidden = W3.shape[0]
+    Kh = np.empty((n, d_h), dtype=np.float64)
+    Vh = np.empty((n, d_h), dtype=np.float64)
+    rc = _load().deltakv_oracle_reconstruct_rows(T, d_h, int(s), k, d_c, hidden, int(act_kind), _ptr(K), _ptr(V),
+                                                 n, _ptr(rows, _ip), _ptr(idx_rows, _ip), _ptr(code_rows), _ptr(W3),
+                                                 _ptr(b3), _ptr(W4), _ptr(b4), _ptr(Kh), _ptr(Vh), int(n_threads))
+    if rc != 0:
+        raise ValueError("oracle reconstruct_rows: invalid arguments")
     return Kh, Vh
 
 

@@ -109,9 +109,33 @@ def test_gelu_matches_printed_normal_cdf(oracle_mod):
     assert oracle_mod.act(oracle_mod.ACT_GELU_ERF, 40.0) == 40.0
     assert oracle_mod.act(oracle_mod.ACT_GELU_ERF, -40.0) == 0.0
     assert oracle_mod.act(oracle_mod.ACT_NONE, -1.25) == -1.25
-    # tanh form: close to exact GELU (max gap below 1e-3) but not equal
-    gt = oracle_mod.act(oracle_mod.ACT_GELU_TANH, 1.0)
-    assert abs(gt - 0.841344746068543) < 1e-3 and gt != oracle_mod.act(oracle_mod.ACT_GELU_ERF, 1.0)
+
+
+def test_gelu_tanh_matches_values_worked_from_its_definition(oracle_mod):
+    """The tanh form z/2 (1 + tanh(sqrt(2/pi) (z + 0.044715 z^3))) against its
+    definition worked step by step in 60-digit decimal arithmetic
+    (tests/golden/gelu_tanh.json, written by make_gelu_tanh.py).  At 1e-15 this
+    catches any wrong constant (0.0447 for 0.044715 moves the value at z = 2 by
+    about 2e-6), a dropped half, a wrong power or a sign error."""
+    g = json.load(open(os.path.join(GOLDEN, "gelu_tanh.json")))
+    assert len(g["rows"]) >= 7
+    for r in g["rows"]:
+        want = float(r["gelu_tanh"])
+        got = oracle_mod.act(oracle_mod.ACT_GELU_TANH, r["z"])
+        assert abs(got - want) <= 4e-16 * max(1.0, abs(want)), (r["z"], got, want)
+
+
+def test_gelu_tanh_identities_and_limits(oracle_mod):
+    """tanh is odd, so f(z) - f(-z) = z/2 (1 + th) + z/2 (1 - th) = z for every
+    z; large |z| gives z and 0; and the form stays within the known worst-case
+    distance of exact GELU (4.73e-4, reached near |z| = 2.70) without being it."""
+    f = lambda z: oracle_mod.act(oracle_mod.ACT_GELU_TANH, float(z))  # noqa: E731
+    for z in np.linspace(-6.0, 6.0, 241):
+        assert abs(f(z) - f(-z) - z) <= 1e-15 * (1.0 + abs(z))
+    assert f(40.0) == 40.0 and f(-40.0) == 0.0 and f(0.0) == 0.0
+    zs = np.linspace(-8.0, 8.0, 16001)
+    gap = max(abs(f(z) - oracle_mod.act(oracle_mod.ACT_GELU_ERF, float(z))) for z in zs)
+    assert 4.6e-4 <= gap <= 4.8e-4, gap
 
 
 # ---------------------------------------------------------------------- MLP
@@ -165,6 +189,22 @@ def test_hand_worked_example(oracle_mod):
     assert out[0, 0] == pytest.approx(want, rel=1e-15)
 
 
+def test_hand_worked_example_row_by_row(oracle_mod):
+    """reconstruct_rows rebuilds the listed tokens of the worked example from
+    their slots and codes alone, in any order, to the hand-computed values."""
+    g = json.load(open(os.path.join(GOLDEN, "hand_example.json")))
+    K = np.array(g["K"], dtype=np.float64)[:, None]
+    V = np.array(g["V"], dtype=np.float64)[:, None]
+    arr = lambda v: None if v is None else np.array(v, dtype=np.float64)  # noqa: E731
+    rows = np.array([3, 0, 1, 4, 2])
+    idx = np.array(g["expect_idx"], dtype=np.int32)[rows]
+    code = np.array(g["expect_code"], dtype=np.float64)[rows]
+    Kh, Vh = oracle_mod.reconstruct_rows(K, V, rows, idx, code, arr(g["W3"]), arr(g["b3"]), arr(g["W4"]),
+                                         arr(g["b4"]), g["s"], oracle_mod.ACT_NONE)
+    assert Kh[:, 0].tolist() == [g["expect_K_hat"][t] for t in rows]
+    assert Vh[:, 0].tolist() == [g["expect_V_hat"][t] for t in rows]
+
+
 # ---------------------------------------------------------- invariants
 
 def _tokens(T, d_h, n_lat, seed=0, dtype=torch.float32):
@@ -206,6 +246,28 @@ def test_identity_codec_reconstructs_every_token(oracle_mod, k):
     assert exact.sum() > 0.9 * T
 
 
+def test_identity_codec_rebuilds_sampled_rows(oracle_mod):
+    """reconstruct_rows with the identity codec gives back the listed tokens
+    themselves (same exactness argument as the whole-sequence case) and the
+    reference rows as stored; a slot that is not strictly earlier than its
+    token is refused."""
+    from decode_attention_strided_b200 import synth
+    T, d_h, s, k = 300, 8, 4, 2
+    K, V = _tokens(T, d_h, 4, seed=5)
+    w = {n: t.double().numpy() for n, t in synth.identity_codec(d_h).items()}
+    idx, code, _, _ = oracle_mod.compress(K, V, w["W1"], None, w["W2"], None, s, k,
+                                          oracle_mod.ACT_NONE, oracle_mod.ROUND_NONE)
+    rows = _rng(8).choice(T, 60, replace=False)
+    Kh, Vh = oracle_mod.reconstruct_rows(K, V, rows, idx[rows], code[rows], w["W3"], None, w["W4"], None, s,
+                                         oracle_mod.ACT_NONE)
+    assert np.array_equal(Kh, K[rows]) and np.array_equal(Vh, V[rows])
+    bad = idx[rows].copy()
+    r = int(np.nonzero(rows % s)[0][0])
+    bad[r, 0] = rows[r] // s + 1
+    with pytest.raises(ValueError):
+        oracle_mod.reconstruct_rows(K, V, rows, bad, code[rows], w["W3"], None, w["W4"], None, s, oracle_mod.ACT_NONE)
+
+
 def test_token_equal_to_its_references_has_zero_residual(oracle_mod):
     """If the k chosen references all equal x_t, the residual and (with no
     biases, GELU(0) = 0) the code are exactly zero and x_t comes back."""
@@ -223,6 +285,8 @@ def test_token_equal_to_its_references_has_zero_residual(oracle_mod):
     assert (code[t] == 0.0).all()
     Kh, Vh = oracle_mod.reconstruct(K, V, idx, code, w["W3"], None, w["W4"], None, s)
     assert np.array_equal(Kh[t], K[t]) and np.array_equal(Vh[t], V[t])
+    Kr, Vr = oracle_mod.reconstruct_rows(K, V, [t], idx[t:t + 1], code[t:t + 1], w["W3"], None, w["W4"], None, s)
+    assert np.array_equal(Kr[0], K[t]) and np.array_equal(Vr[0], V[t])
 
 
 # --------------------------------------------------------------- attention
