@@ -20,6 +20,7 @@ from .oracle import (  # noqa: F401
     ROUND_BF16,
     ROUND_F32,
     ROUND_NONE,
+    ROUND_Q4,
     act,
     attention,
     build,
@@ -27,6 +28,7 @@ from .oracle import (  # noqa: F401
     compress_rows,
     lib_path,
     mlp,
+    quantize_row4,
     reconstruct,
     reconstruct_rows,
     round_to,

@@ -45,7 +45,7 @@
 #endif
 
 enum { ORACLE_ACT_GELU_ERF = 0, ORACLE_ACT_GELU_TANH = 1, ORACLE_ACT_NONE = 2 };
-enum { ORACLE_ROUND_NONE = 0, ORACLE_ROUND_F32 = 1, ORACLE_ROUND_BF16 = 2 };
+enum { ORACLE_ROUND_NONE = 0, ORACLE_ROUND_F32 = 1, ORACLE_ROUND_BF16 = 2, ORACLE_ROUND_Q4 = 3 };
 
 /* ---------------------------------------------------------------- helpers */
 
@@ -88,6 +88,31 @@ double deltakv_oracle_round(int mode, double v)
     if (mode == ORACLE_ROUND_BF16)
         return round_sig_bits(v, 8);
     return v;
+}
+
+/* 4-bit codes (the summary's section 5, "Efficienza di Memoria": the
+ * memory saving is largest combined with 4-bit quantisation; which tensors
+ * and which grid the summary does not say).  Reading taken: one code row
+ * (the d_c values of one compressed token) is quantised symmetrically to
+ * signed 4-bit integers with one scale per row,
+ *     scale = bf16(max_i |c_i| / 7),   q_i = clamp(rne(c_i / scale), -7, 7),
+ * and the stored (dequantised) code is q_i * scale.  A zero row has scale 0
+ * and q = 0.  rne is round to nearest, ties to even; the scale is rounded to
+ * bfloat16 first so that the value stored with the codes is the one they were
+ * quantised against.  Writes q[0..d_c) and returns the scale. */
+double deltakv_oracle_quantize_row4(int d_c, const double* c, int8_t* q)
+{
+    double amax = 0.0;
+    for (int i = 0; i < d_c; ++i)
+        if (fabs(c[i]) > amax) amax = fabs(c[i]);
+    double scale = deltakv_oracle_round(ORACLE_ROUND_BF16, amax / 7.0);
+    for (int i = 0; i < d_c; ++i) {
+        double v = scale > 0.0 ? nearbyint(c[i] / scale) : 0.0;
+        if (v > 7.0) v = 7.0;
+        if (v < -7.0) v = -7.0;
+        q[i] = (int8_t)v;
+    }
+    return scale;
 }
 
 static int ceil_div(int a, int b) { return (a + b - 1) / b; }
@@ -216,13 +241,20 @@ static void compress_token(int t, int d_h, int s, int k, int d_c, int hidden, in
     if (dk1) *dk1 = b;
     residual(t, d_h, s, k, K, V, it, r);
     deltakv_oracle_mlp(2 * d_h, hidden, d_c, act, W1, b1, W2, b2, r, c);
+    if (round_mode == ORACLE_ROUND_Q4) {
+        int8_t q[256];
+        double scale = deltakv_oracle_quantize_row4(d_c, c, q);
+        for (int o = 0; o < d_c; ++o) ct[o] = (double)q[o] * scale;
+        return;
+    }
     for (int o = 0; o < d_c; ++o) ct[o] = deltakv_oracle_round(round_mode, c[o]);
 }
 
 /* Compress the tokens listed in rows[0..n_rows) of one (sequence, kv-head)
  * whose K, V are [T][d_h].  Output row i belongs to token rows[i]:
  *   idx  [n_rows][k]   chosen slots (-1 for reference tokens and padding),
- *   code [n_rows][d_c] the stored code, rounded per round_mode (0 for refs),
+ *   code [n_rows][d_c] the stored code, rounded per round_mode (0 for refs;
+ *                      with ORACLE_ROUND_Q4 the dequantised 4-bit code),
  *   d_k, d_k1 [n_rows] the k-th and (k+1)-th smallest distances (NAN for
  *   references).  Tokens are independent, so the loop may run on several
  *   threads (n_threads <= 0 keeps the library default). */
@@ -236,6 +268,8 @@ int deltakv_oracle_compress_rows(int T, int d_h, int s, int k, int d_c, int hidd
                                  int n_threads)
 {
     if (T < 0 || d_h <= 0 || s <= 0 || k <= 0 || d_c <= 0 || hidden <= 0 || n_rows < 0)
+        return -1;
+    if (round_mode == ORACLE_ROUND_Q4 && d_c > 256)
         return -1;
     for (int i = 0; i < n_rows; ++i)
         if (rows[i] < 0 || rows[i] >= T) return -1;

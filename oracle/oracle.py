@@ -14,7 +14,7 @@ import threading
 import numpy as np
 
 ACT_GELU_ERF, ACT_GELU_TANH, ACT_NONE = 0, 1, 2
-ROUND_NONE, ROUND_F32, ROUND_BF16 = 0, 1, 2
+ROUND_NONE, ROUND_F32, ROUND_BF16, ROUND_Q4 = 0, 1, 2, 3
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "deltakv_oracle.c")
@@ -54,6 +54,8 @@ def _load():
             lib.deltakv_oracle_select.restype = ctypes.c_int
             lib.deltakv_oracle_select.argtypes = [
                 ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _dp, _dp, _ip, _dp, _dp]
+            lib.deltakv_oracle_quantize_row4.restype = ctypes.c_double
+            lib.deltakv_oracle_quantize_row4.argtypes = [ctypes.c_int, _dp, ctypes.POINTER(ctypes.c_int8)]
             lib.deltakv_oracle_mlp.restype = None
             lib.deltakv_oracle_mlp.argtypes = [
                 ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _dp, _dp, _dp, _dp, _dp, _dp]
@@ -88,6 +90,15 @@ def act(kind: int, z: float) -> float:
 def round_to(mode: int, v: float) -> float:
     """Round a double to float (ROUND_F32) or bfloat16 (ROUND_BF16), ties to even."""
     return _load().deltakv_oracle_round(int(mode), float(v))
+
+
+def quantize_row4(c):
+    """4-bit code of one row: returns (q int8 [d_c] in [-7, 7], scale) with
+    scale = bf16(max |c| / 7) and q = clamp(rne(c / scale), -7, 7)."""
+    c = _f64(c)
+    q = np.empty(c.shape[0], dtype=np.int8)
+    scale = _load().deltakv_oracle_quantize_row4(c.shape[0], _ptr(c), q.ctypes.data_as(ctypes.POINTER(ctypes.c_int8)))
+    return q, scale
 
 
 def select(t: int, K, V, s: int, k: int):

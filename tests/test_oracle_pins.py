@@ -386,3 +386,64 @@ def test_attention_over_a_list_with_repeats(oracle_mod):
     t = np.array([0, 0, 1])
     got = oracle_mod.attention(q, K[t], V[t])[0]
     assert np.allclose(got, want, rtol=1e-14, atol=1e-15)
+
+
+# ------------------------------------------------------------- 4-bit codes
+
+def test_quantize_row4_hand_example(oracle_mod):
+    """Worked by hand: c = (0.7, -1.4, 0.35, 0) has max |c| = 1.4 and
+    1.4 / 7 = 0.2 = 1.1001100110011..._2 x 2^-3; its bfloat16 keeps 8
+    significant bits, 1.1001100|1100... rounds up to 1.1001101_2 x 2^-3 =
+    205/1024.  Then c / scale = 3.4966, -6.9932, 1.7483, 0, so q = 3, -7, 2, 0."""
+    q, sc = oracle_mod.quantize_row4([0.7, -1.4, 0.35, 0.0])
+    assert sc == 205.0 / 1024.0
+    assert q.tolist() == [3, -7, 2, 0]
+
+
+def test_quantize_row4_round_trip_on_representable_rows(oracle_mod):
+    """A row that is exactly q * s, with s a bfloat16 value and integers
+    |q_i| <= 7 of which one is +-7, comes back as the same q and s."""
+    rng = _rng(31)
+    for _ in range(200):
+        m = int(rng.integers(128, 256))                  # 8 significant bits
+        s = m * 2.0 ** int(rng.integers(-20, 5))
+        d_c = int(rng.choice([16, 32, 64]))
+        q = rng.integers(-7, 8, size=d_c)
+        q[int(rng.integers(d_c))] = 7 if rng.random() < 0.5 else -7
+        got_q, got_s = oracle_mod.quantize_row4(q * s)
+        assert got_s == s and got_q.tolist() == q.tolist()
+
+
+def test_quantize_row4_ties_zero_row_and_error_bound(oracle_mod):
+    # scale 1: halfway values go to the even integer
+    q, sc = oracle_mod.quantize_row4([7.0, 0.5, 1.5, 2.5, -0.5, -2.5, -3.5])
+    assert sc == 1.0 and q.tolist() == [7, 0, 2, 2, 0, -2, -4]
+    q, sc = oracle_mod.quantize_row4(np.zeros(32))
+    assert sc == 0.0 and not q.any()
+    # every element within half a step of its dequantised value
+    rng = _rng(32)
+    for _ in range(100):
+        c = rng.normal(size=32) * rng.uniform(0.01, 10)
+        q, sc = oracle_mod.quantize_row4(c)
+        assert np.all(np.abs(q) <= 7)
+        assert np.all(np.abs(c - q * sc) <= sc / 2 * (1 + 1e-12) + 1e-300)
+
+
+def test_compress_with_4bit_codes_stores_quantised_rows(oracle_mod):
+    """With 4-bit codes every stored code row is the dequantised quantisation
+    of the code the compressor computes (the same compression without
+    rounding), and slots and distances are unchanged."""
+    from decode_attention_strided_b200 import synth
+    T, d_h, s, k = 150, 8, 4, 2
+    K, V = _tokens(T, d_h, 4, seed=33)
+    w = {n: t.double().numpy() for n, t in synth.codec_weights(0, d_h, 16, 32, dtype=torch.float32).items()}
+    raw = oracle_mod.compress(K, V, w["W1"], None, w["W2"], None, s, k, oracle_mod.ACT_GELU_ERF,
+                              oracle_mod.ROUND_NONE)
+    q4 = oracle_mod.compress(K, V, w["W1"], None, w["W2"], None, s, k, oracle_mod.ACT_GELU_ERF, oracle_mod.ROUND_Q4)
+    assert np.array_equal(raw[0], q4[0])
+    for t in range(T):
+        if t % s == 0:
+            assert not q4[1][t].any()
+            continue
+        q, sc = oracle_mod.quantize_row4(raw[1][t])
+        assert np.array_equal(q4[1][t], q * sc)
