@@ -10,8 +10,15 @@
 // below instead of a caller-supplied workspace.
 //
 // The array is kNoAllocScratchBytes (16 MiB) and, once this module is loaded
-// on a GPU, that GPU holds it until the process exits.  Plans whose workspace
-// is larger are rejected with DELTAKV_ERR_WORKSPACE.  Every call shares the
+// on a GPU, that GPU holds it until the process exits.  Only the decode's own
+// part of a plan's workspace has to fit, not the compress region: the error
+// word, the reference-logit and slot-weight tables (8 G / s bytes per token
+// of capacity and kv-head), the per-split partials (about 33 KB per kv-head
+// at G = 4, hidden 256) and the combine partials.  One 128k-token sequence
+// with 8 kv-heads and 4 query heads per kv-head needs about 3.6 MiB; batch 8
+// at 128k needs about 25 MiB and is refused.  Plans whose decode part is
+// larger than the array are rejected with DELTAKV_ERR_WORKSPACE.
+// Every call shares the
 // one array: calls that overlap on the GPU (on different streams, or from
 // different host threads without ordering) race on it.
 #include <mutex>
@@ -63,7 +70,7 @@ extern "C" deltakv_status deltakv_decode_attention_noalloc(
   const Plan& p = plan->p;
   if (T < 1 || T > p.cfg.max_T) return DELTAKV_ERR_INVALID_ARG;
   if (!q || !q_strides || !cache || !W3 || !W4 || !out || !out_strides) return DELTAKV_ERR_INVALID_ARG;
-  if (p.ws_bytes > kNoAllocScratchBytes) return DELTAKV_ERR_WORKSPACE;
+  if (p.ws_decode_end > kNoAllocScratchBytes) return DELTAKV_ERR_WORKSPACE;
   if (q_strides[0] < 0 || q_strides[1] < 0 || out_strides[0] < 0 || out_strides[1] < 0)
     return DELTAKV_ERR_INVALID_ARG;
   if ((q_strides[0] * p.esize) % 16 || (q_strides[1] * p.esize) % 16 || (out_strides[0] * 4) % 16 ||
