@@ -52,6 +52,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of the phase with the given parity (test_wait never
+// suspends the thread, so a loop over several barriers polls each in turn).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete.  Returns false if
 // `abort` became non-zero or the time limit passed.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
@@ -63,6 +77,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
       if (*abort) return false;
       if (globaltimer() - t0 > kWaitLimitNs) return false;
     }
+  }
+}
+
+// Wait for the phase with the given parity regardless of any abort flag, for
+// at most kWaitLimitNs.  This is the wait on the way out of a kernel: the
+// copies and MMAs a thread issued must have landed before the block releases
+// its shared and tensor memory, even when a role gave up early.  Returns
+// false if the time limit passed.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 63) == 0 && globaltimer() - t0 > kWaitLimitNs) return false;
   }
 }
 
@@ -175,6 +203,15 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                    smem_u32(bar))
                : "memory");
+}
+
+// Wait (bounded, ignoring any abort flag) until every tcgen05 operation this
+// thread issued has completed: one more commit onto `bar`, a barrier of
+// count 1 that is used for nothing else, then its first phase.  Returns
+// false if the time limit passed.
+__device__ __forceinline__ bool umma_drain(uint64_t* bar) {
+  umma_commit(bar);
+  return mbar_wait_drain(bar, 0);
 }
 
 // 32 consecutive fp32 columns of this thread's TMEM lane.
