@@ -28,7 +28,8 @@ deltakv_status validate_config(const deltakv_config* c) {
       c->stride_s < 1 || c->k < 1 || c->d_c < 1 || c->hidden < 1 || c->d_h < 1)
     return DELTAKV_ERR_INVALID_ARG;
   if (c->q_heads % c->kv_heads != 0) return DELTAKV_ERR_INVALID_ARG;
-  if (c->dtype != DELTAKV_BF16 && c->dtype != DELTAKV_F32) return DELTAKV_ERR_INVALID_ARG;
+  if (c->dtype != DELTAKV_BF16 && c->dtype != DELTAKV_F32 && c->dtype != DELTAKV_BF16_CODE4)
+    return DELTAKV_ERR_INVALID_ARG;
   if (c->act != DELTAKV_ACT_GELU_ERF && c->act != DELTAKV_ACT_GELU_TANH &&
       c->act != DELTAKV_ACT_NONE)
     return DELTAKV_ERR_INVALID_ARG;
@@ -40,6 +41,9 @@ deltakv_status validate_config(const deltakv_config* c) {
   if (!(c->d_c == 16 || c->d_c == 32 || c->d_c == 64 || identity)) return DELTAKV_ERR_UNSUPPORTED;
   if (identity && c->d_c * c->hidden > 128 * 128) return DELTAKV_ERR_UNSUPPORTED;
   if (c->max_T > (1 << 26)) return DELTAKV_ERR_UNSUPPORTED;
+  if (c->dtype == DELTAKV_BF16_CODE4 &&
+      (identity || (c->hidden != 128 && c->hidden != 256) || c->act == DELTAKV_ACT_NONE))
+    return DELTAKV_ERR_UNSUPPORTED;
   return DELTAKV_OK;
 }
 
@@ -47,7 +51,9 @@ void build_plan(const deltakv_config& c, Plan& p) {
   p.cfg = c;
   p.G = c.q_heads / c.kv_heads;
   p.D = 2 * c.d_h;
-  p.esize = c.dtype == DELTAKV_BF16 ? 2 : 4;
+  p.bf16 = c.dtype != DELTAKV_F32;
+  p.code4 = c.dtype == DELTAKV_BF16_CODE4;
+  p.esize = p.bf16 ? 2 : 4;
   p.KC = c.k + kExtraCand <= 8 ? 8 : 12;
   const int64_t BH = (int64_t)c.batch * c.kv_heads;
   const int64_t n_ref_max = n_ref_of(c.max_T, c.stride_s);
@@ -61,9 +67,15 @@ void build_plan(const deltakv_config& c, Plan& p) {
   p.off_refv = off;
   off = align256(off + (size_t)(BH * p.n_ref_cap * c.d_h) * p.esize);
   p.off_code = off;
-  off = align256(off + (size_t)(BH * p.n_code_cap * c.d_c) * p.esize);
+  off = align256(off + (p.code4 ? (size_t)(BH * p.n_code_cap * c.d_c) / 2
+                                : (size_t)(BH * p.n_code_cap * c.d_c) * p.esize));
   p.off_idx = off;
   off = align256(off + (size_t)(BH * p.n_code_cap * c.k) * 4);
+  p.off_cscale = 0;
+  if (p.code4) {
+    p.off_cscale = off;
+    off = align256(off + (size_t)(BH * p.n_code_cap) * 2);
+  }
   p.cache_bytes = off;
   // workspace: error word, then the compress region and the decode region
   // side by side (a call uses one of them).
@@ -97,6 +109,7 @@ void build_plan(const deltakv_config& c, Plan& p) {
   w = align256(w + (size_t)(BH * p.nslot_cap * p.G * c.hidden) * 4);
   p.ws_ochunk = w;
   w = align256(w + (size_t)(BH * p.n_chunk_cap * p.G * (c.d_h + 1)) * 4);
+  p.ws_decode_end = w;
   p.ws_sparse = w;  // sparse decode: (m, l, output) of every share
   w = align256(w + (size_t)(BH * kSparseSplits * p.G * (c.d_h + 2)) * 4);
   p.ws_bytes = std::max(compress_end, w);
@@ -154,6 +167,7 @@ deltakv_status deltakv_get_cache_layout(deltakv_plan_t plan, deltakv_cache_layou
   out->total_bytes = p.cache_bytes;
   out->n_ref_cap = p.n_ref_cap;
   out->n_code_cap = p.n_code_cap;
+  out->code_scale_offset = p.off_cscale;
   return DELTAKV_OK;
 }
 

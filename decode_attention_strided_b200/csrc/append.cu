@@ -8,7 +8,11 @@
 // earlier references (slots j with j s < t, including references appended by
 // the same call), keeps the k nearest by squared L2 over [K ; V] (ties to the
 // lower slot), subtracts their mean and compresses the residual with the MLP.
-// The result is identical to compressing [0, T1) in one call.
+// The slots are the exact top-k of float32 distances, so they match the oracle
+// under the same near-tie rule as compression in one call; where two
+// references lie within float32 rounding of the same distance the two paths
+// may keep different ones.  Everything else is what one call over [0, T1)
+// writes.
 //
 // Few tokens arrive per call, so the kernels are plain CUDA-core code with
 // exact fp32 distances (no candidate search and re-rank): each new token's
@@ -89,6 +93,7 @@ __global__ void append_refs_kernel(int s, int d_h, int H, int64_t j0, int64_t n_
 
 struct AppendParams {
   int s, d_h, H, k, d_c, hidden, act;
+  __nv_bfloat16* cscale;  // per-row scales of 4-bit codes, else null
   int64_t row0;  // first code row of the call
   int64_t n_ref_cap, n_code_cap;
   int64_t sb, sh, st;
@@ -177,7 +182,7 @@ __global__ void __launch_bounds__(kAppendThreads)
                          const E* __restrict__ W1, const float* __restrict__ b1, const E* __restrict__ W2,
                          const float* __restrict__ b2, const E* __restrict__ refk, const E* __restrict__ refv,
                          const float* __restrict__ lists, E* __restrict__ code, int32_t* __restrict__ idx) {
-  __shared__ float r[2 * 128], hbuf[kMaxHidden];
+  __shared__ float r[2 * 128], hbuf[kMaxHidden], cbuf[64];
   __shared__ int sel[kAppendKMax], sel_n;
   const int bh = blockIdx.z, b = bh / P.H, h = bh % P.H;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -271,7 +276,31 @@ __global__ void __launch_bounds__(kAppendThreads)
       for (int i = 0; i < 4; ++i) acc = fmaf(wv[i], hbuf[u + i], acc);
     }
     acc = warp_sum(acc);
-    if (lane == 0) code[((int64_t)bh * P.n_code_cap + row) * P.d_c + o] = from_f<E>(acc + (b2 ? b2[o] : 0.f));
+    if (lane == 0) {
+      const float cv = acc + (b2 ? b2[o] : 0.f);
+      if (P.cscale) cbuf[o] = cv;
+      else code[((int64_t)bh * P.n_code_cap + row) * P.d_c + o] = from_f<E>(cv);
+    }
+  }
+  if (P.cscale) {
+    // 4-bit codes: the whole row's scale first, then the packed nibbles
+    __syncthreads();
+    if (tid == 0) {
+      float amax = 0.f;
+      for (int o = 0; o < P.d_c; ++o) amax = fmaxf(amax, fabsf(cbuf[o]));
+      const __nv_bfloat16 sb = __float2bfloat16_rn(amax / 7.0f);
+      const float sc = __bfloat162float(sb);
+      uint8_t* c8 = reinterpret_cast<uint8_t*>(code) + ((int64_t)bh * P.n_code_cap + row) * (P.d_c / 2);
+      for (int o = 0; o < P.d_c; o += 2) {
+        int q0 = 0, q1 = 0;
+        if (sc > 0.f) {
+          q0 = (int)fminf(fmaxf(rintf(__fdiv_rn(cbuf[o], sc)), -7.f), 7.f);
+          q1 = (int)fminf(fmaxf(rintf(__fdiv_rn(cbuf[o + 1], sc)), -7.f), 7.f);
+        }
+        c8[o / 2] = (uint8_t)((q0 & 0xF) | ((q1 & 0xF) << 4));
+      }
+      P.cscale[(int64_t)bh * P.n_code_cap + row] = sb;
+    }
   }
   if (tid < P.k) idx[((int64_t)bh * P.n_code_cap + row) * P.k + tid] = tid < k_eff ? sel[tid] : -1;
 }
@@ -303,6 +332,7 @@ static cudaError_t append_launch(const Plan& p, int T0, int T1, const KVView& kv
     P.row0 = r0;
     P.n_ref_cap = p.n_ref_cap;
     P.n_code_cap = p.n_code_cap;
+    P.cscale = p.code4 ? (__nv_bfloat16*)(cb + p.off_cscale) : nullptr;
     P.sb = kv.sb;
     P.sh = kv.sh;
     P.st = kv.st;
@@ -349,7 +379,7 @@ static cudaError_t append_launch(const Plan& p, int T0, int T1, const KVView& kv
 
 cudaError_t launch_append(const Plan& p, int T0, int T1, const KVView& kv, const void* W1, const float* b1,
                           const void* W2, const float* b2, void* cache, void* ws, cudaStream_t st) {
-  if (p.cfg.dtype == DELTAKV_BF16)
+  if (p.bf16)
     return append_launch<__nv_bfloat16>(p, T0, T1, kv, W1, b1, W2, b2, cache, ws, st);
   return append_launch<float>(p, T0, T1, kv, W1, b1, W2, b2, cache, ws, st);
 }

@@ -85,6 +85,46 @@ __device__ __forceinline__ float2 gelu_fast2(float x0, float x1) {
   return make_float2(fmaxf(x0, 0.0f) - p0, fmaxf(x1, 0.0f) - p1);
 }
 
+// Exact GELU for the decode token loop, where the activation count sets the
+// pace: x Phi(x) ~= x/2 (1 + tanh(y)) with y = xc (c1 + c3 xc^2 + c5 xc^4)
+// and xc = clamp(x, -8, 8) (one min.xorsign.abs).  (c1, c3, c5) is the
+// builder's own minimax fit of this form to exact GELU on [-8, 8] (the
+// argument rises monotonically there; beyond it tanh is saturated and the
+// form returns x or 0): |form - GELU| <= 2.6e-5 with an exact tanh.  tanh
+// itself comes from the special-function unit (tanh.approx.f32, whose
+// relative error the tests measure), the rest runs as packed fp32x2
+// arithmetic; so one activation costs one MUFU operation and about five
+// issue slots, against about fifteen for gelu_fast.
+__device__ __forceinline__ float2 gelu_tanhfit2(float x0, float x1) {
+  float a0, a1;
+  asm("min.xorsign.abs.f32 %0, %1, %2;" : "=f"(a0) : "f"(x0), "f"(8.0f));
+  asm("min.xorsign.abs.f32 %0, %1, %2;" : "=f"(a1) : "f"(x1), "f"(8.0f));
+  unsigned long long xc, xx, s, p, y, u;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(xc) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(xx) : "f"(x0), "f"(x1));
+  asm("mul.rn.f32x2 %0, %1, %1;" : "=l"(s) : "l"(xc));
+  asm("{\n\t.reg .b64 c5, c3, c1;\n\t"
+      "mov.b64 c5, {%2, %2};\n\tmov.b64 c3, {%3, %3};\n\tmov.b64 c1, {%4, %4};\n\t"
+      "fma.rn.f32x2 %0, c5, %1, c3;\n\t"
+      "fma.rn.f32x2 %0, %0, %1, c1;\n\t}"
+      : "=l"(p)
+      : "l"(s), "f"(-3.515167919e-04f), "f"(3.700564429e-02f), "f"(7.975078821e-01f));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(y) : "l"(p), "l"(xc));
+  float y0, y1, t0, t1;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(y0), "=f"(y1) : "l"(y));
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t0) : "f"(y0));
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t1) : "f"(y1));
+  asm("{\n\t.reg .b64 hf, t, h;\n\t"
+      "mov.b64 hf, {%2, %2};\n\tmov.b64 t, {%3, %4};\n\t"
+      "mul.rn.f32x2 h, %1, hf;\n\t"
+      "fma.rn.f32x2 %0, h, t, h;\n\t}"
+      : "=l"(u)
+      : "l"(xx), "f"(0.5f), "f"(t0), "f"(t1));
+  float u0, u1;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(u0), "=f"(u1) : "l"(u));
+  return make_float2(u0, u1);
+}
+
 // The activation inside the tensor-core kernels: exact GELU through
 // gelu_fast, the other forms as in act_eval.
 __device__ __forceinline__ float act_fast(int act, float z) {
@@ -139,6 +179,42 @@ __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
   return v;
+}
+
+// Element e of code row `row` (a row index of the whole plane).  With 4-bit
+// codes (cscale non-null) the plane holds d_c / 2 bytes per row, element 2i in
+// the low nibble of byte i and 2i + 1 in its high nibble, two's complement,
+// and the value is q * scale[row] (exact in fp32: |q| <= 7 times a bf16).
+template <typename E>
+__device__ __forceinline__ float code_at(const E* code, const __nv_bfloat16* cscale, int64_t row, int d_c, int e) {
+  if (cscale != nullptr) {
+    const int b = reinterpret_cast<const int8_t*>(code)[row * (d_c >> 1) + (e >> 1)];
+    const int qv = (e & 1) ? (b >> 4) : ((int)(int8_t)(b << 4) >> 4);
+    return (float)qv * __bfloat162float(cscale[row]);
+  }
+  return to_f(code[row * d_c + e]);
+}
+
+// Quantise one code row to 4 bits: scale = bf16(max |c| / 7), q =
+// clamp(rne(c / scale), -7, 7), packed two per byte (low nibble first) into
+// `out` (n / 2 bytes).  Returns the scale.
+template <int N>
+__device__ __forceinline__ __nv_bfloat16 quantize_row4(const float (&c)[N], uint8_t (&out)[N / 2]) {
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < N; ++i) amax = fmaxf(amax, fabsf(c[i]));
+  const __nv_bfloat16 sb = __float2bfloat16_rn(amax / 7.0f);
+  const float sc = __bfloat162float(sb);
+#pragma unroll
+  for (int i = 0; i < N; i += 2) {
+    int q0 = 0, q1 = 0;
+    if (sc > 0.f) {
+      q0 = (int)fminf(fmaxf(rintf(__fdiv_rn(c[i], sc)), -7.f), 7.f);
+      q1 = (int)fminf(fmaxf(rintf(__fdiv_rn(c[i + 1], sc)), -7.f), 7.f);
+    }
+    out[i / 2] = (uint8_t)((q0 & 0xF) | ((q1 & 0xF) << 4));
+  }
+  return sb;
 }
 
 // Code row of non-reference token t.

@@ -75,7 +75,7 @@ cudaError_t launch_refpack(const Plan& p, int T, const KVView& kv, void* cache, 
   char* cb = (char*)cache;
   float* hn = (float*)((char*)ws + p.ws_hnorm);
   ProfScope ps(p, st, KID_REFPACK);
-  if (c.dtype == DELTAKV_BF16) {
+  if (p.bf16) {
     using T_ = __nv_bfloat16;
     refpack_kernel<T_><<<grid, 256, 0, st>>>(c.stride_s, c.d_h, c.kv_heads, n_ref, p.n_ref_cap,
                                              (const T_*)kv.K, (const T_*)kv.V, kv.sb, kv.sh,
@@ -190,7 +190,7 @@ static cudaError_t cand_simt_launch(const Plan& p, int T, const KVView& kv, cons
 cudaError_t launch_candidates_simt(const Plan& p, int T, const KVView& kv, const void* cache,
                                    void* ws, cudaStream_t st) {
   if (n_code_of(T, p.cfg.stride_s) == 0) return cudaSuccess;
-  if (p.cfg.dtype == DELTAKV_BF16)
+  if (p.bf16)
     return p.KC == 8 ? cand_simt_launch<__nv_bfloat16, 8>(p, T, kv, cache, ws, st)
                      : cand_simt_launch<__nv_bfloat16, 12>(p, T, kv, cache, ws, st);
   return p.KC == 8 ? cand_simt_launch<float, 8>(p, T, kv, cache, ws, st)
@@ -254,6 +254,9 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
     for (int i = 0; i < KC; ++i) {
       int j = cr[i];
+      // the tensor-core search may mark the first slot with kExactFlag; this
+      // kernel re-ranks every row, so the mark is dropped
+      if (i == 0 && j >= 0) j &= ~kExactFlag;
       if (j >= 0 && (int64_t)j * s >= t) {  // not an earlier reference: drop it
         latch_error(err, DELTAKV_ERR_DEVICE_BOUNDS, (uint32_t)j);
         j = -1;
@@ -389,7 +392,8 @@ cudaError_t launch_encode(const Plan& p, int T, const KVView& kv, const void* W1
                           const void* W2, const float* b2, void* cache, void* ws,
                           cudaStream_t st) {
   if (n_code_of(T, p.cfg.stride_s) == 0) return cudaSuccess;
-  if (p.cfg.dtype == DELTAKV_BF16)
+  if (p.code4) return cudaErrorNotSupported;  // 4-bit codes are written by the tensor-core encoder
+  if (p.bf16)
     return p.KC == 8 ? encode_launch<__nv_bfloat16, 8>(p, T, kv, W1, b1, W2, b2, cache, ws, st)
                      : encode_launch<__nv_bfloat16, 12>(p, T, kv, W1, b1, W2, b2, cache, ws, st);
   return p.KC == 8 ? encode_launch<float, 8>(p, T, kv, W1, b1, W2, b2, cache, ws, st)
@@ -405,6 +409,7 @@ __global__ void __launch_bounds__(256)
     reconstruct_kernel(int T_, int s, int d_h, int H, int k, int d_c, int hidden, int act,
                        int64_t n_ref_cap, int64_t n_code_cap, const T* __restrict__ refk,
                        const T* __restrict__ refv, const T* __restrict__ code,
+                       const __nv_bfloat16* __restrict__ cscale,
                        const int32_t* __restrict__ idx, const T* __restrict__ W3,
                        const float* __restrict__ b3, const T* __restrict__ W4,
                        const float* __restrict__ b4, float* __restrict__ Kout,
@@ -423,7 +428,7 @@ __global__ void __launch_bounds__(256)
     int r = i / d_c, o = i - r * d_c;
     int64_t t = t0 + r;
     float v = 0.f;
-    if (t < T_ && t % s != 0) v = to_f(code[(bh * n_code_cap + code_row_of(t, s)) * d_c + o]);
+    if (t < T_ && t % s != 0) v = code_at(code, cscale, bh * n_code_cap + code_row_of(t, s), d_c, o);
     Cs[i] = v;
   }
   __syncthreads();
@@ -473,7 +478,7 @@ cudaError_t launch_reconstruct(const Plan& p, int T, const void* cache, const vo
   dim3 grid((unsigned)ceil_div64(T, 32), c.kv_heads, c.batch);
   const char* cb = (const char*)cache;
   ProfScope ps(p, st, KID_RECONSTRUCT);
-  if (c.dtype == DELTAKV_BF16) {
+  if (p.bf16) {
     using T_ = __nv_bfloat16;
     auto kern = reconstruct_kernel<T_>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -481,7 +486,9 @@ cudaError_t launch_reconstruct(const Plan& p, int T, const void* cache, const vo
     kern<<<grid, 256, smem, st>>>(T, c.stride_s, c.d_h, c.kv_heads, c.k, c.d_c, c.hidden,
                                   (int)c.act, p.n_ref_cap, p.n_code_cap,
                                   (const T_*)(cb + p.off_refk), (const T_*)(cb + p.off_refv),
-                                  (const T_*)(cb + p.off_code), (const int32_t*)(cb + p.off_idx),
+                                  (const T_*)(cb + p.off_code),
+                                  p.code4 ? (const __nv_bfloat16*)(cb + p.off_cscale) : nullptr,
+                                  (const int32_t*)(cb + p.off_idx),
                                   (const T_*)W3, b3, (const T_*)W4, b4, Kout, Vout, (uint32_t*)ws);
   } else {
     auto kern = reconstruct_kernel<float>;
@@ -490,7 +497,7 @@ cudaError_t launch_reconstruct(const Plan& p, int T, const void* cache, const vo
     kern<<<grid, 256, smem, st>>>(T, c.stride_s, c.d_h, c.kv_heads, c.k, c.d_c, c.hidden,
                                   (int)c.act, p.n_ref_cap, p.n_code_cap,
                                   (const float*)(cb + p.off_refk), (const float*)(cb + p.off_refv),
-                                  (const float*)(cb + p.off_code),
+                                  (const float*)(cb + p.off_code), nullptr,
                                   (const int32_t*)(cb + p.off_idx), (const float*)W3, b3,
                                   (const float*)W4, b4, Kout, Vout, (uint32_t*)ws);
   }

@@ -164,6 +164,7 @@ __global__ void __launch_bounds__(256)
     decode_stream_kernel(int T_, int s, int d_h, int H, int G, int k, int d_c, int hidden,
                          int act, int ns, int64_t n_ref_cap, int64_t n_code_cap,
                          int n_refblk, int n_refblk_cap, const T* __restrict__ code,
+                         const __nv_bfloat16* __restrict__ cscale,
                          const int32_t* __restrict__ idx, const T* __restrict__ W3,
                          const float* __restrict__ b3, const float* __restrict__ a,
                          const float* __restrict__ cterm, const float* __restrict__ S,
@@ -220,14 +221,14 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
     for (int i = 0; i < 8; ++i) Uw[g][i] = 0.f;
   }
-  const T* cb = code + bh * n_code_cap * d_c;
+  const int64_t crow0 = bh * n_code_cap;  // plane row of this (sequence, kv-head)'s first code
   const int32_t* ib = idx + bh * n_code_cap * k;
   const float* Sb = S + bh * n_ref_cap * G;
 
   for (int64_t row = c0 + warp; row < c1; row += 8) {
     // the code row, staged in this warp's slice of shared memory
     float* cr = cw + warp * d_c;
-    for (int e = lane; e < d_c; e += 32) cr[e] = to_f(cb[row * d_c + e]);
+    for (int e = lane; e < d_c; e += 32) cr[e] = code_at(code, cscale, crow0 + row, d_c, e);
     __syncwarp();
     float u[8];
 #pragma unroll
@@ -525,6 +526,7 @@ static cudaError_t decode_launch(const Plan& p, int T, const void* q, int64_t qs
   const E* refk = (const E*)(cb + p.off_refk);
   const E* refv = (const E*)(cb + p.off_refv);
   const E* code = (const E*)(cb + p.off_code);
+  const __nv_bfloat16* cscale = p.code4 ? (const __nv_bfloat16*)(cb + p.off_cscale) : nullptr;
   const int32_t* idx = (const int32_t*)(cb + p.off_idx);
   float* S = (float*)(w + p.ws_S);
   float* Smax = (float*)(w + p.ws_Smax);
@@ -575,7 +577,7 @@ static cudaError_t decode_launch(const Plan& p, int T, const void* q, int64_t qs
     if (e != cudaSuccess) return e;
     ProfScope ps(p, st, KID_DEC_STREAM_SIMT);
     ks<<<dim3(ns, H, B), 256, smem, st>>>(T, c.stride_s, c.d_h, H, G, c.k, c.d_c, c.hidden, (int)c.act, ns,
-                                          p.n_ref_cap, p.n_code_cap, n_refblk, n_refblk_cap, code, idx,
+                                          p.n_ref_cap, p.n_code_cap, n_refblk, n_refblk_cap, code, cscale, idx,
                                           (const E*)W3, b3, a, cterm, S, Smax, wtab, part, Upart,
                                           wt_in_smem, p.nslot_cap, (uint32_t*)ws);
     e = cudaGetLastError();
@@ -601,7 +603,7 @@ cudaError_t launch_decode(const Plan& p, int T, const void* q, int64_t qsb, int6
                           const void* cache, const void* W3, const float* b3, const void* W4,
                           const float* b4, float* out, int64_t osb, int64_t osh, void* ws,
                           cudaStream_t st) {
-  if (p.cfg.dtype == DELTAKV_BF16)
+  if (p.bf16)
     return decode_launch<__nv_bfloat16>(p, T, q, qsb, qsh, cache, W3, b3, W4, b4, out, osb, osh,
                                         ws, st);
   return decode_launch<float>(p, T, q, qsb, qsh, cache, W3, b3, W4, b4, out, osb, osh, ws, st);

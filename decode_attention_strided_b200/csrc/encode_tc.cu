@@ -4,18 +4,23 @@
 // DeltaKV summary, section 3, "Processo di Compressione" steps 1-4 (the
 // selection is finished here from the k + 4 candidates the tensor-core search
 // kept):
-//   1. exact fp32 distances |x_t - r_j|^2 to the candidates; the k smallest
-//      by (distance, slot) are the token's references (idx plane);
+//   1. a row whose approximate ranking the search marked exact (every gap
+//      among its first k + 1 candidates above the fp32 error bound of the
+//      ranking key) takes its first k candidates as they are; any other row
+//      gets exact fp32 distances |x_t - r_j|^2 to all candidates and the k
+//      smallest by (distance, slot) are its references (idx plane);
 //   2. KV_R = their mean;  3. r = x_t - KV_R;
 //   4. code = W2 act(W1 r + b1) + b2  (code plane, rounded to bf16).
 //
 // One persistent CTA per SM, 16 warps with fixed roles, per 64-row tile:
 //   gather warps (11)  16 lanes per token row; the row's x and candidate
-//            slots are loaded one row pass ahead, the k + 4 candidate rows
-//            together (kept in registers for the mean); exact fp32
-//            distances, each candidate ranked by one lane, the chosen set by
-//            ballot; r = x - mean -> R tile (64 tokens x D, K-major, hi and
-//            lo), double-buffered so the next tile's gather overlaps
+//            slots are loaded one row pass ahead; an exact row loads only its
+//            k references; a re-ranked row loads its k + 4 candidate rows four
+//            at a time, gets exact fp32 distances, each candidate ranked by
+//            one lane, the chosen set by ballot over the row's 16 lanes (the
+//            two rows of a warp may take different paths); r = x - mean ->
+//            R tile (64 tokens x D, K-major, hi and lo), double-buffered so
+//            the next tile's gather overlaps
 //   MMA warp  tcgen05.mma  D1^T = W1 . R^T  (A = W1 held in tensor memory
 //            for the whole launch, M = 128 hidden units per half, N = 64
 //            tokens); then codes = H . W2^T (A = the H tile through an
@@ -109,6 +114,34 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// One code row of 4-bit codes from the GEMM2 accumulator (TMEM lane = row,
+// DC fp32 columns from taddr): + b2, quantised by quantize_row4 and stored as
+// DC / 2 bytes plus its bf16 scale when `live`.  Warp-collective (every lane
+// runs the TMEM loads).
+template <int DC>
+__device__ __forceinline__ void store_code4_row(uint32_t taddr, const float* b2, uint8_t* dst, __nv_bfloat16* sdst,
+                                                bool live) {
+  float cv[DC];
+#pragma unroll
+  for (int c0 = 0; c0 < DC; c0 += 16) {
+    float v[16];
+    tmem_ld16(taddr + c0, v);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) cv[c0 + i] = v[i] + (b2 ? b2[c0 + i] : 0.f);
+  }
+  uint8_t pk[DC / 2];
+  const __nv_bfloat16 sb = quantize_row4<DC>(cv, pk);
+  if (live) {
+    if constexpr (DC == 16) {
+      *reinterpret_cast<uint2*>(dst) = *reinterpret_cast<const uint2*>(pk);
+    } else {
+#pragma unroll
+      for (int i = 0; i < DC / 32; ++i) reinterpret_cast<uint4*>(dst)[i] = reinterpret_cast<const uint4*>(pk)[i];
+    }
+    *sdst = sb;
+  }
+}
+
 struct EncParams {
   int T, s, d_h, H, k, d_c, hidden, act, BH;
   int64_t n_code, n_ref, n_ref_cap, n_code_cap;
@@ -122,6 +155,7 @@ struct EncParams {
   const __nv_bfloat16* refk;
   const __nv_bfloat16* refv;
   __nv_bfloat16* code;
+  __nv_bfloat16* cscale;  // 4-bit codes: per-row scales (the code plane then holds d_c / 2 bytes a row)
   int32_t* idx;
   const int32_t* cand;
   uint32_t* err;
@@ -153,16 +187,18 @@ __device__ __forceinline__ void unpack_row(const uint4 (&r)[RowPack<EPL>::V4], f
   }
 }
 
-__device__ __forceinline__ float group16_sum(float v) {
-  v += __shfl_xor_sync(0xffffffffu, v, 8, 16);
-  v += __shfl_xor_sync(0xffffffffu, v, 4, 16);
-  v += __shfl_xor_sync(0xffffffffu, v, 2, 16);
-  v += __shfl_xor_sync(0xffffffffu, v, 1, 16);
+// Sum over the 16 lanes of one row group (`mask` names exactly those lanes).
+__device__ __forceinline__ float group16_sum(float v, unsigned mask) {
+  v += __shfl_xor_sync(mask, v, 8, 16);
+  v += __shfl_xor_sync(mask, v, 4, 16);
+  v += __shfl_xor_sync(mask, v, 2, 16);
+  v += __shfl_xor_sync(mask, v, 1, 16);
   return v;
 }
 
-// Candidate rows loaded together: all of them when there are 8, else 4.
-template <int KC> struct CandBatch { static constexpr int N = KC == 8 ? 8 : 4; };
+// Candidate rows of a re-ranked row are loaded four at a time; the chosen
+// ones are loaded again (from L2) for the mean.
+template <int KC> struct CandBatch { static constexpr int N = 4; };
 
 template <int ACT>
 __device__ __forceinline__ float enc_act(float v) {
@@ -207,6 +243,7 @@ __device__ __forceinline__ void gather_prefetch(const EncParams& P, const Gather
 
 struct EncBars {
   uint64_t r_full[2], r_empty[2], d1_full, d1_empty, h_full, h_empty, d2_full, d2_empty;
+  uint64_t drain;  // the MMA warp's last commit
 };
 
 template <int EPL, int KC, int ACT>
@@ -252,6 +289,7 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
     mbar_init(&bars->h_empty, 1);
     mbar_init(&bars->d2_full, 1);
     mbar_init(&bars->d2_empty, enc::ACT_WARPS);
+    mbar_init(&bars->drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -330,15 +368,62 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
         }
         int cj[KC];
         float cd[KC];
+        // a row whose approximate ranking already fixes the exact choice
+        // (flag in its first slot, set by the distance kernel) takes its
+        // first k slots as they are; the others are re-ranked exactly
+        const int c0raw = __shfl_sync(0xffffffffu, myc, 0, 16);
+        const bool exact = c0raw >= 0 && (c0raw & kExactFlag) != 0;
 #pragma unroll
         for (int c = 0; c < KC; ++c) {
           int j = __shfl_sync(0xffffffffu, myc, c, 16);
+          if (c == 0 && j >= 0) j &= ~kExactFlag;
           if (j >= 0 && (int64_t)j * P.s >= g.t) {  // not an earlier reference: drop it
             if (s16 == 0) latch_error(P.err, DELTAKV_ERR_DEVICE_BOUNDS, (uint32_t)j);
             j = -1;
           }
           cj[c] = j;
         }
+        const unsigned gmask = 0xFFFFu << (16 * grp);
+        if (exact) {
+          // the list is in ascending order with the valid slots first
+          int n_valid = 0;
+#pragma unroll
+          for (int c = 0; c < KC; ++c) n_valid += cj[c] >= 0 ? 1 : 0;
+          const int k_eff = min(P.k, n_valid);
+          if (g.live && s16 < P.k) {
+            int js = -1;
+#pragma unroll
+            for (int c = 0; c < KC; ++c)
+              if (c == s16) js = cj[c];
+            P.idx[((int64_t)bh * P.n_code_cap + g.row) * P.k + s16] = s16 < k_eff ? js : -1;
+          }
+          const float inv = 1.0f / (float)max(k_eff, 1);
+          // the chosen rows, four in flight at a time
+#pragma unroll
+          for (int b0 = 0; b0 < kMaxK; b0 += 4) {
+            if (b0 < k_eff) {
+              uint4 rr[4][RowPack<EPL>::V4];
+#pragma unroll
+              for (int u = 0; u < 4; ++u)
+                if (b0 + u < k_eff) load_row<EPL>(rs + (int64_t)cj[b0 + u] * P.d_h, rr[u]);
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                if (b0 + u < k_eff) {
+#pragma unroll
+                  for (int i = 0; i < RowPack<EPL>::V4; ++i) {
+                    const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&rr[u][i]);
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
+                      const float2 v = __bfloat1622float2(p2[x]);
+                      xr[8 * i + 2 * x] = fmaf(-inv, v.x, xr[8 * i + 2 * x]);
+                      xr[8 * i + 2 * x + 1] = fmaf(-inv, v.y, xr[8 * i + 2 * x + 1]);
+                    }
+                  }
+                }
+              }
+            }
+          }
+        } else {
         // exact distances, NB candidate rows in flight at a time; with
         // NB == KC the rows stay in registers for the mean
         uint4 rr[NB][RowPack<EPL>::V4];
@@ -373,7 +458,7 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
               asm("mov.b64 {%0, %1}, %2;" : "=f"(e0), "=f"(e1) : "l"(acc));
               part = e0 + e1;
             }
-            part = group16_sum(part);
+            part = group16_sum(part, gmask);
             cd[c0 + u] = cj[c0 + u] >= 0 ? part : FLT_MAX;
           }
         }
@@ -394,7 +479,7 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
         for (int c = 0; c < KC; ++c)
           rank += (cj[c] >= 0 && (cd[c] < my_d || (cd[c] == my_d && cj[c] < my_j))) ? 1 : 0;
         const bool pick = s16 < KC && my_j >= 0 && rank < P.k;
-        const uint32_t chosen = (__ballot_sync(0xffffffffu, pick) >> (16 * grp)) & 0xFFFFu;
+        const uint32_t chosen = (__ballot_sync(gmask, pick) >> (16 * grp)) & 0xFFFFu;
         const int k_eff = min(P.k, n_valid);
         if (g.live) {
           int32_t* idx_row = P.idx + ((int64_t)bh * P.n_code_cap + g.row) * P.k;
@@ -425,6 +510,7 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
             }
           }
         }
+        }  // re-rank
         // r = hi + lo (fp16) into the R tile: row n, columns e0 .. e0 + EPL
 #pragma unroll
         for (int v = 0; v < EPL / 8; ++v) {
@@ -500,6 +586,8 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
         latch_error(P.err, DELTAKV_ERR_DEVICE_TIMEOUT, 11);
         *abort_flag = 1;
       }
+      // every MMA issued has completed before tensor memory is released
+      if (!umma_drain(&bars->drain)) latch_error(P.err, DELTAKV_ERR_DEVICE_TIMEOUT, 13);
     }
   } else if (warp >= enc::ACT0 && warp < enc::ACT0 + enc::ACT_WARPS) {
     // ------------------- activation H = act(D1 + b1), then the code store
@@ -555,7 +643,17 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
       // codes = D2 + b2 (TMEM lanes 0-63: the first two activation warps)
       if (!mbar_wait(&bars->d2_full, it & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      if (q < 2) {
+      if (q < 2 && P.cscale) {
+        const int bh = tile / P.tiles_per_bh;
+        const int64_t row = (int64_t)(tile % P.tiles_per_bh) * enc::ROWS + q * 32 + lane;
+        const int64_t prow = (int64_t)bh * P.n_code_cap + row;
+        const uint32_t ta = tmem + ((uint32_t)(q * 32) << 16) + enc::D2_COL;
+        uint8_t* dst = reinterpret_cast<uint8_t*>(P.code) + prow * (P.d_c / 2);
+        const bool live = row < P.n_code;
+        if (P.d_c == 16) store_code4_row<16>(ta, P.b2, dst, P.cscale + prow, live);
+        else if (P.d_c == 32) store_code4_row<32>(ta, P.b2, dst, P.cscale + prow, live);
+        else store_code4_row<64>(ta, P.b2, dst, P.cscale + prow, live);
+      } else if (q < 2) {
         const int bh = tile / P.tiles_per_bh;
         const int64_t row = (int64_t)(tile % P.tiles_per_bh) * enc::ROWS + q * 32 + lane;
         for (int c0 = 0; c0 < P.d_c; c0 += 16) {
@@ -601,7 +699,7 @@ size_t encode_tc_smem(const Plan& p) {
 
 bool encode_tc_supported(const Plan& p) {
   const auto& c = p.cfg;
-  return c.dtype == DELTAKV_BF16 && (c.d_h == 64 || c.d_h == 128) && (c.hidden == 128 || c.hidden == 256) &&
+  return p.bf16 && (c.d_h == 64 || c.d_h == 128) && (c.hidden == 128 || c.hidden == 256) &&
          c.d_c % 16 == 0 && c.d_c <= 64 && encode_tc_smem(p) <= 227 * 1024;
 }
 
@@ -654,6 +752,7 @@ cudaError_t launch_encode_tc(const Plan& p, int T, const KVView& kv, const void*
   P.refk = (const __nv_bfloat16*)(cb + p.off_refk);
   P.refv = (const __nv_bfloat16*)(cb + p.off_refv);
   P.code = (__nv_bfloat16*)(cb + p.off_code);
+  P.cscale = p.code4 ? (__nv_bfloat16*)(cb + p.off_cscale) : nullptr;
   P.idx = (int32_t*)(cb + p.off_idx);
   P.cand = (const int32_t*)((char*)ws + p.ws_cand);
   P.err = (uint32_t*)ws;

@@ -13,6 +13,9 @@ namespace dkv {
 constexpr int kMaxK = 8;          // references per token
 constexpr int kExtraCand = 4;     // extra candidates the distance kernel keeps
 constexpr int kMaxCand = kMaxK + kExtraCand;
+// Set in the first candidate slot of a row whose approximate ranking already
+// fixes the exact k nearest and their order (slot numbers stay below 2^26).
+constexpr int32_t kExactFlag = 1 << 30;
 constexpr int kMaxG = 8;          // query heads per kv-head
 constexpr int kMaxHidden = 256;
 constexpr int kMaxSplit = 32;     // decode splits per (sequence, kv-head)
@@ -38,18 +41,21 @@ struct Plan {
   deltakv_config cfg;
   int G;                 // q_heads / kv_heads
   int D;                 // 2 d_h
-  int esize;             // bytes per element of dtype
+  int esize;             // bytes per element of K, V, refs and weights
+  bool bf16;             // element type bf16 (BF16 or BF16_CODE4)
+  bool code4;            // codes stored as 4-bit pairs with a bf16 scale per row
   int KC;                // candidates per token kept by the distance kernel
   int64_t n_ref_cap;     // reference rows per (b, head)
   int64_t n_code_cap;    // code rows per (b, head)
   // cache layout (bytes from base)
-  size_t off_refk, off_refv, off_code, off_idx, cache_bytes;
+  size_t off_refk, off_refv, off_code, off_idx, off_cscale, cache_bytes;
   // compress workspace
   size_t ws_hnorm, ws_hsplit, ws_cand;
   // decode workspace
   int nslot_cap;         // decode partial slots per (b, head)
   int n_chunk_cap;       // combine blocks per (b, head)
   size_t ws_S, ws_Smax, ws_mref, ws_a, ws_cterm, ws_wtab, ws_part, ws_U, ws_ochunk, ws_sparse;
+  size_t ws_decode_end;  // error word + the dense decode's regions (S .. ochunk)
   size_t ws_bytes;
 };
 

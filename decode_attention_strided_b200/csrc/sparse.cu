@@ -39,6 +39,7 @@ struct SparseParams {
   int T, s, d_h, H, G, k, d_c, hidden, act, n_sel, per, nsplit;
   int64_t n_ref_cap, n_code_cap, qsb, qsh;
   float scale;  // 1 / sqrt(d_h)
+  const __nv_bfloat16* cscale;  // per-row scales of 4-bit codes, else null
 };
 
 // Shared-memory carve-up (in floats; every region starts on 16 bytes).
@@ -272,7 +273,15 @@ __global__ void __launch_bounds__(kSpThreads, GM <= 4 ? 2 : 1)
           const int r = i / hc;
           cr[m] = r;
           ce[m] = 2 * (i - r * hc);
-          if (kind[r] == 1) cv[m] = load2(cd + code_row_of(tok[r], P.s) * d_c + ce[m]);
+          if (kind[r] == 1) {
+            if (P.cscale) {
+              const int64_t crow = bh * P.n_code_cap + code_row_of(tok[r], P.s);
+              cv[m] = make_float2(code_at(code, P.cscale, crow, d_c, ce[m]),
+                                  code_at(code, P.cscale, crow, d_c, ce[m] + 1));
+            } else {
+              cv[m] = load2(cd + code_row_of(tok[r], P.s) * d_c + ce[m]);
+            }
+          }
         }
       }
       int sv = -1;
@@ -577,6 +586,7 @@ static cudaError_t sparse_launch(const Plan& p, int T, const void* q, int64_t qs
   P.qsb = qsb;
   P.qsh = qsh;
   P.scale = 1.0f / sqrtf((float)c.d_h);
+  P.cscale = p.code4 ? (const __nv_bfloat16*)((const char*)cache + p.off_cscale) : nullptr;
   const int64_t BH = (int64_t)c.batch * c.kv_heads;
   // shares of at least one pass each, about two CTAs per SM in total
   int nsplit = (int)std::min<int64_t>((n_sel + kSpR - 1) / kSpR, std::max<int64_t>(1, 2 * kNumSMs / BH));
@@ -598,7 +608,7 @@ cudaError_t launch_decode_sparse(const Plan& p, int T, const void* q, int64_t qs
                                  const void* W3, const float* b3, const void* W4, const float* b4,
                                  const int32_t* tokens, int n_sel, float* out, int64_t osb, int64_t osh, void* ws,
                                  cudaStream_t st) {
-  if (p.cfg.dtype == DELTAKV_BF16)
+  if (p.bf16)
     return sparse_launch<__nv_bfloat16>(p, T, q, qsb, qsh, cache, W3, b3, W4, b4, tokens, n_sel, out, osb, osh, ws,
                                         st);
   return sparse_launch<float>(p, T, q, qsb, qsh, cache, W3, b3, W4, b4, tokens, n_sel, out, osb, osh, ws, st);

@@ -17,7 +17,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "_lib", "libdeltakv.so")
 
-BF16, F32 = 0, 1
+BF16, F32, BF16_CODE4 = 0, 1, 2
 ACT_GELU_ERF, ACT_GELU_TANH, ACT_NONE = 0, 1, 2
 
 STATUS = {
@@ -28,7 +28,11 @@ STATUS = {
 SYMBOLS = ("deltakv_plan", "deltakv_plan_destroy", "deltakv_get_cache_layout", "deltakv_compress",
            "deltakv_append", "deltakv_decode_attention", "deltakv_decode_attention_sparse",
            "deltakv_decode_attention_noalloc", "deltakv_reconstruct", "deltakv_device_status",
-           "deltakv_set_profiling", "deltakv_profile_collect", "deltakv_status_string", "deltakv_version")
+           "deltakv_set_profiling", "deltakv_profile_collect", "deltakv_status_string", "deltakv_version",
+           "deltakv_test_activation")
+
+# forms of deltakv_test_activation (include/deltakv_testing.h)
+TEST_ACT_GELU_ERFF, TEST_ACT_GELU_FAST, TEST_ACT_GELU_FAST2, TEST_ACT_GELU_TANH, TEST_ACT_GELU_TANHFIT2 = 0, 1, 2, 3, 4
 
 
 class DeltaKVError(RuntimeError):
@@ -47,7 +51,7 @@ class _Layout(ctypes.Structure):
     _fields_ = [("ref_k_offset", ctypes.c_size_t), ("ref_v_offset", ctypes.c_size_t),
                 ("code_offset", ctypes.c_size_t), ("idx_offset", ctypes.c_size_t),
                 ("total_bytes", ctypes.c_size_t), ("n_ref_cap", ctypes.c_int64),
-                ("n_code_cap", ctypes.c_int64)]
+                ("n_code_cap", ctypes.c_int64), ("code_scale_offset", ctypes.c_size_t)]
 
 
 class _KernelTime(ctypes.Structure):
@@ -95,6 +99,8 @@ def load_library(path: str = LIB_PATH):
     lib.deltakv_status_string.restype = ctypes.c_char_p
     lib.deltakv_version.argtypes = []
     lib.deltakv_version.restype = ctypes.c_int32
+    lib.deltakv_test_activation.argtypes = [i32, vp, vp, ctypes.c_int64, vp]
+    lib.deltakv_test_activation.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -115,7 +121,7 @@ class Config:
     layers: int = 1
 
     def torch_dtype(self):
-        return torch.bfloat16 if self.dtype == BF16 else torch.float32
+        return torch.float32 if self.dtype == F32 else torch.bfloat16
 
 
 def _check(fn, code):
@@ -172,24 +178,43 @@ class Plan:
         return torch.zeros(self.workspace_bytes, dtype=torch.uint8, device=device)
 
     def cache_planes(self, cache: torch.Tensor):
-        """Views of the four planes of a cache buffer: ref_k, ref_v
+        """Views of the planes of a cache buffer: ref_k, ref_v
         [B,H,n_ref_cap,d_h], code [B,H,n_code_cap,d_c] and idx
-        [B,H,n_code_cap,k] (int32)."""
+        [B,H,n_code_cap,k] (int32); with 4-bit codes, code is the packed
+        uint8 plane [B,H,n_code_cap,d_c/2] and code_scale [B,H,n_code_cap]
+        (bf16) holds the per-row scales."""
         c, L = self.cfg, self.layout
         dt = c.torch_dtype()
-        es = 2 if c.dtype == BF16 else 4
+        es = 4 if c.dtype == F32 else 2
         B, H = c.batch, c.kv_heads
 
         def view(off, rows, cols, dtype, esize):
             n = B * H * rows * cols
             return cache[off:off + n * esize].view(dtype).view(B, H, rows, cols)
 
-        return {
+        planes = {
             "ref_k": view(L["ref_k_offset"], L["n_ref_cap"], c.d_h, dt, es),
             "ref_v": view(L["ref_v_offset"], L["n_ref_cap"], c.d_h, dt, es),
-            "code": view(L["code_offset"], L["n_code_cap"], c.d_c, dt, es),
             "idx": view(L["idx_offset"], L["n_code_cap"], c.k, torch.int32, 4),
         }
+        if c.dtype == BF16_CODE4:
+            planes["code"] = view(L["code_offset"], L["n_code_cap"], c.d_c // 2, torch.uint8, 1)
+            planes["code_scale"] = view(L["code_scale_offset"], L["n_code_cap"], 1, torch.bfloat16, 2)[..., 0]
+        else:
+            planes["code"] = view(L["code_offset"], L["n_code_cap"], c.d_c, dt, es)
+        return planes
+
+    def dequantized_codes(self, cache: torch.Tensor):
+        """Code rows as float32 [B,H,n_code_cap,d_c]: the stored values, or for
+        4-bit codes q * scale unpacked (low nibble first, two's complement)."""
+        pl = self.cache_planes(cache)
+        if self.cfg.dtype != BF16_CODE4:
+            return pl["code"].float()
+        b = pl["code"].to(torch.int16)
+        lo = ((b & 0xF) ^ 8) - 8
+        hi = ((b >> 4) ^ 8) - 8
+        q = torch.stack([lo, hi], dim=-1).flatten(-2).float()
+        return q * pl["code_scale"].float()[..., None]
 
 
 def plan(cfg: Config) -> Plan:
@@ -285,6 +310,17 @@ def profile_collect(p: Plan) -> dict:
     n = ctypes.c_int32()
     _check("deltakv_profile_collect", load_library().deltakv_profile_collect(p.handle, buf, 16, ctypes.byref(n)))
     return {buf[i].name.decode(): (int(buf[i].launches), float(buf[i].total_ms)) for i in range(n.value)}
+
+
+def test_activation(form: int, x, y, stream=None):
+    """deltakv_test_activation: y = form(x) on the device (float32 tensors of
+    the same length; test support, include/deltakv_testing.h)."""
+    if x.dtype != torch.float32 or y.dtype != torch.float32 or not x.is_contiguous() or not y.is_contiguous():
+        raise ValueError("x and y must be contiguous float32 tensors")
+    if x.numel() != y.numel():
+        raise ValueError("x and y must have the same length")
+    _check("deltakv_test_activation", load_library().deltakv_test_activation(
+        int(form), _ptr(x), _ptr(y), int(x.numel()), _stream(stream)))
 
 
 def version() -> int:

@@ -51,7 +51,14 @@ typedef enum {
     DELTAKV_ERR_DEVICE_BOUNDS = 7   /* a kernel met an out-of-range index */
 } deltakv_status;
 
-typedef enum { DELTAKV_BF16 = 0, DELTAKV_F32 = 1 } deltakv_dtype;
+/* Element types.  DELTAKV_BF16_CODE4: K, V, queries, weights and reference
+ * rows in bfloat16, and every code row quantised to 4 bits ("Efficienza di
+ * Memoria", section 5 of the summary: the saving is largest combined with
+ * 4-bit quantisation): per compressed token one scale = bf16(max |c| / 7)
+ * and signed 4-bit q = clamp(rne(c / scale), -7, 7), the stored code being
+ * q * scale.  Needs d_c in {16, 32, 64}, hidden in {128, 256} and a
+ * nonlinear act (it runs on the tensor-core compressor and decoder). */
+typedef enum { DELTAKV_BF16 = 0, DELTAKV_F32 = 1, DELTAKV_BF16_CODE4 = 2 } deltakv_dtype;
 
 /* Nonlinearity between the two linear layers of the compressor and of the
  * decompressor.  GELU_ERF is x * Phi(x). */
@@ -90,10 +97,15 @@ typedef struct CUstream_st* deltakv_stream_t;  /* same type as cudaStream_t */
  *                  whole (slot j = token j s);
  *   code         : [B][H][n_code_cap][d_c] dtype  -- one row per non-reference
  *                  token, in token order: token t (t mod s != 0) is row
- *                  t - floor(t / s) - 1;
+ *                  t - floor(t / s) - 1; with DELTAKV_BF16_CODE4 a row is
+ *                  d_c / 2 bytes, element 2i in the low nibble of byte i and
+ *                  2i + 1 in its high nibble (two's complement);
  *   idx          : [B][H][n_code_cap][k]   int32  -- its reference slots in
  *                  ascending (distance, slot) order, -1 where fewer than k
- *                  earlier references exist.
+ *                  earlier references exist;
+ *   code_scale   : [B][H][n_code_cap]      bf16   -- with DELTAKV_BF16_CODE4
+ *                  only, each code row's scale (code_scale_offset is 0 and
+ *                  the plane absent otherwise).
  * For a cache holding T tokens the first ceil(T/s) reference rows and the
  * first T - ceil(T/s) code/idx rows of each (b, head) are used. */
 typedef struct {
@@ -101,6 +113,7 @@ typedef struct {
     size_t total_bytes;
     int64_t n_ref_cap;
     int64_t n_code_cap;
+    size_t code_scale_offset;
 } deltakv_cache_layout;
 
 /* Validate `cfg`, build a host-side plan, and report the bytes of one layer's
@@ -139,8 +152,11 @@ deltakv_status deltakv_compress(deltakv_plan_t plan, int32_t T,
  * t mod s == 0 become references; every other new token t searches all
  * references with slot j, j s < t (those appended by this call included)
  * with exact float32 squared distances, keeps the k nearest (ties to the
- * lower slot), and stores its code and slots.  The result equals
- * deltakv_compress over [0, T1).
+ * lower slot), and stores its code and slots.  The slots match the exact
+ * selection under the same near-tie rule as deltakv_compress's (where two
+ * references lie within float32 rounding of the same distance, append and
+ * compress may keep different ones); everything else equals compressing
+ * [0, T1) in one call.
  *   0 <= T0 <= T1 <= max_T; T0 == T1 returns DELTAKV_OK without launching.
  *   cache      : device, as written by deltakv_compress(T0) or by earlier
  *                appends up to T0 (the caller guarantees it); rows of the
@@ -219,8 +235,12 @@ deltakv_status deltakv_reconstruct(deltakv_plan_t plan, int32_t T, const void* c
  * the workspace: scratch comes from a 16 MiB array that the library holds in
  * device memory (every GPU that loads this part of the library keeps it until
  * the process exits).  The paper has no counterpart to this entry point.
- *  - Plans whose workspace_bytes exceeds 16 MiB: DELTAKV_ERR_WORKSPACE,
- *    nothing launched.
+ *  - Only the decode part of the plan's workspace must fit in 16 MiB (the
+ *    compress part is not used): the reference-logit and slot-weight tables,
+ *    8 G / s bytes per token of capacity and kv-head, plus about 33 KB per
+ *    kv-head of partials at G = 4, hidden 256.  One 128k-token sequence with
+ *    8 kv-heads fits (about 3.6 MiB); batch 8 at 128k does not.  A plan whose
+ *    decode part is larger: DELTAKV_ERR_WORKSPACE, nothing launched.
  *  - Nothing is allocated: no cudaMalloc, no cudaFree, no allocating library
  *    call.  The first call on a device looks up the array's device address
  *    (once per device); make that first call before any stream capture.

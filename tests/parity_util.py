@@ -31,7 +31,12 @@ ATTN_MAX_ABS = 5e-3
 
 
 def recon_tol(dtype):
-    return 1e-2 if dtype == dkv.BF16 else 1e-5
+    return 1e-5 if dtype == dkv.F32 else 1e-2
+
+
+def round_mode(dtype):
+    """The oracle's rounding of stored codes for a cache element type."""
+    return {dkv.F32: oracle.ROUND_F32, dkv.BF16: oracle.ROUND_BF16, dkv.BF16_CODE4: oracle.ROUND_Q4}[dtype]
 
 
 @dataclasses.dataclass
@@ -65,7 +70,7 @@ class Inputs:
 
 
 def make_inputs(c: Case) -> Inputs:
-    tdt = torch.bfloat16 if c.dtype == dkv.BF16 else torch.float32
+    tdt = torch.float32 if c.dtype == dkv.F32 else torch.bfloat16
     K, V = synth.kv(c.layer, c.layer, c.B, c.H, c.T, c.d_h, c.n_lat, dtype=tdt)
     if c.identity:
         W = synth.identity_codec(c.d_h, dtype=tdt)
@@ -127,7 +132,7 @@ def run_gpu(c: Case, inp: Inputs, decode=True) -> GpuResult:
     n_code = c.T - math.ceil(c.T / c.s)
     return GpuResult(
         idx=planes["idx"][:, :, :n_code].cpu().numpy(),
-        code=planes["code"][:, :, :n_code].float().cpu().double().numpy(),
+        code=p.dequantized_codes(cache)[:, :, :n_code].cpu().double().numpy(),
         K_hat=Kh.cpu().double().numpy(), V_hat=Vh.cpu().double().numpy(),
         out=out.cpu().double().numpy(), status=status, kernels=kernels)
 
@@ -148,7 +153,7 @@ def run_oracle_head(c: Case, inp: Inputs, b: int, h: int) -> OracleHead:
     V = inp.V[b, h].double().numpy()
     W = {n: t.double().numpy() for n, t in inp.W.items()}
     bias = {n: (None if t is None else t.double().numpy()) for n, t in inp.bias.items()}
-    rmode = oracle.ROUND_BF16 if c.dtype == dkv.BF16 else oracle.ROUND_F32
+    rmode = round_mode(c.dtype)
     idx, code, dk, dk1 = oracle.compress(K, V, W["W1"], bias["b1"], W["W2"], bias["b2"], c.s, c.k, c.act, rmode)
     Kh, Vh = oracle.reconstruct(K, V, idx, code, W["W3"], bias["b3"], W["W4"], bias["b4"], c.s, c.act)
     G = c.Hq // c.H
@@ -190,6 +195,42 @@ def check_indices(gpu_idx, o_idx, o_dk, o_dk1, K, V, tokens, s):
         for a, b in zip(d, d[1:]):
             assert a <= b * (1 + NEAR_TIE_REL), "order not ascending beyond the margin: " + ctx
     return len(tokens), n_flagged
+
+
+def q4_code_delta(W2):
+    """Per code element, a bound on the GPU's own error in the unrounded code
+    c: its GELU is within 1.2e-5 of the exact one, which W2 carries into
+    element e with gain sum_h |W2[e, h]|; every other step is fp32 or finer."""
+    return 1.2e-5 * np.abs(np.asarray(W2, dtype=np.float64)).sum(axis=1) + 1e-6
+
+
+def q4_other_rounding(c_raw, delta):
+    """Another 4-bit code the GPU may legitimately store for each row of
+    c_raw (the oracle's unrounded codes): every element whose rounding
+    changes within +-delta is pushed across its boundary, the largest
+    element too when the scale changes within it, and the pushed row goes
+    through the oracle's own quantiser.  Returns (dequantised rows, mask of
+    rows that differ from the oracle's code)."""
+    c_raw = np.asarray(c_raw, dtype=np.float64)
+    alt = np.empty_like(c_raw)
+    changed = np.zeros(c_raw.shape[0], dtype=bool)
+    for r, c in enumerate(c_raw):
+        q, sc = oracle.quantize_row4(c)
+        push = np.zeros_like(c)
+        if sc > 0:
+            lo = np.clip(np.rint((c - delta) / sc), -7, 7)
+            hi = np.clip(np.rint((c + delta) / sc), -7, 7)
+            push = np.where(lo != q, -delta, np.where(hi != q, delta, 0.0))
+        e = int(np.argmax(np.abs(c)))
+        amax = abs(c[e])
+        if oracle.round_to(oracle.ROUND_BF16, (amax + delta[e]) / 7.0) != sc:
+            push[e] = np.sign(c[e]) * delta[e]
+        elif oracle.round_to(oracle.ROUND_BF16, max(amax - delta[e], 0.0) / 7.0) != sc:
+            push[e] = -np.sign(c[e]) * delta[e]
+        q2, sc2 = oracle.quantize_row4(c + push)
+        alt[r] = q2.astype(np.float64) * sc2
+        changed[r] = not np.array_equal(alt[r], q.astype(np.float64) * sc)
+    return alt, changed
 
 
 def rel_l2(a, b):

@@ -20,9 +20,14 @@ def lib():
 
 
 def _declared_symbols():
-    text = open(os.path.join(ROOT, "include", "deltakv.h")).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(deltakv_[a-z_]+)\s*\(", text)))
+    names = set()
+    for hdr in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if not hdr.endswith(".h"):
+            continue
+        text = open(os.path.join(ROOT, "include", hdr)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names |= set(re.findall(r"\b(deltakv_[a-z_]+)\s*\(", text))
+    return sorted(names)
 
 
 def test_every_declared_symbol_is_exported(lib):
@@ -32,6 +37,16 @@ def test_every_declared_symbol_is_exported(lib):
     for name in declared:
         assert hasattr(lib, name), name
     assert set(declared) == set(dkv.SYMBOLS)
+
+
+def test_test_activation_rejects_bad_arguments(lib):
+    """The test-support entry point validates before launching: an unknown
+    form, a negative length or a NULL pointer are refused; n = 0 is a no-op."""
+    assert lib.deltakv_test_activation(9, None, None, 4, None) == 1
+    assert lib.deltakv_test_activation(5, None, None, 4, None) == 1
+    assert lib.deltakv_test_activation(0, None, None, -1, None) == 1
+    assert lib.deltakv_test_activation(0, None, None, 4, None) == 1
+    assert lib.deltakv_test_activation(0, None, None, 0, None) == 0
 
 
 def test_version_and_status_strings(lib):
@@ -133,3 +148,19 @@ def test_sparse_binding_rejects_a_selection_of_the_wrong_shape(lib):
             dkv.decode_attention_sparse(p, 100, x, x, x, None, x, None, torch.zeros(shape, dtype=torch.int32), x, x)
     with pytest.raises(ValueError):  # wrong dtype
         dkv.decode_attention_sparse(p, 100, x, x, x, None, x, None, torch.zeros((2, 4, 10), dtype=torch.int64), x, x)
+
+
+def test_layout_of_4bit_codes(lib):
+    """DELTAKV_BF16_CODE4: the code plane holds d_c / 2 bytes a row and a
+    bf16 scale plane follows the slot plane; unsupported shapes are refused."""
+    p = dkv.plan(_cfg(dtype=dkv.BF16_CODE4))
+    L = p.layout
+    B, H, n_code = 8, 8, 131072 - 8192
+    assert L["idx_offset"] - L["code_offset"] == B * H * n_code * 16
+    assert L["code_scale_offset"] >= L["idx_offset"] + B * H * n_code * 4 * 4
+    assert L["total_bytes"] >= L["code_scale_offset"] + B * H * n_code * 2
+    assert dkv.plan(_cfg()).layout["code_scale_offset"] == 0
+    for bad in (dict(act=dkv.ACT_NONE), dict(hidden=64)):
+        with pytest.raises(dkv.DeltaKVError) as ei:
+            dkv.plan(_cfg(dtype=dkv.BF16_CODE4, **bad))
+        assert ei.value.code == 2
