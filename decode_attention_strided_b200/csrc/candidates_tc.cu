@@ -29,16 +29,6 @@
 // The ranking key e is formed inside the accumulator: A holds -x_t, and one
 // more K = 16 MMA per tile adds a ones row times the bf16 split of h_j (three
 // terms, 24 significant bits), so the epilogue reads e directly.
-// Exactness flag: at the end of its sweep each token row checks whether its
-// approximate list already fixes the exact choice.  The key e = h_j - x . r_j
-// is a sum of D products and three h terms, each added in fp32 (in any order,
-// rounding or truncating), and h_j itself is an fp32 sum of D squares, so
-// |e - e_exact| <= GAMMA (|x| |r_j| + h_j) with GAMMA = (2 D + 8) 2^-23
-// (Cauchy-Schwarz bounds the sum of |x_i r_ji| by |x| |r_j|).  When every gap
-// between neighbours among the first k + 1 entries exceeds the sum of their
-// bounds, the first k entries are the exact k nearest, in the exact order;
-// the row's first slot then carries kExactFlag and the encode kernel skips
-// its re-rank.
 // Shape choices: an M = 128 MMA occupies the tensor pipe for at least about
 // 58 cycles whatever its N, so N = 128 (64 cycles of math) keeps it math-bound;
 // with A in tensor memory each MMA reads only its 4 KB of B from shared
@@ -74,7 +64,7 @@ __host__ __device__ constexpr int spill_bytes(int) { return EPI_WARPS * SPILL; }
 }  // namespace tcc
 
 struct TcParams {
-  int T, s, H, BH, n_units, n_pairs, d_h, k;
+  int T, s, H, BH, n_units, n_pairs, d_h;
   int n_ref;
   int64_t n_ref_cap, n_code_cap;
   const __nv_bfloat16* K;
@@ -343,13 +333,11 @@ __global__ void __launch_bounds__(tcc::THREADS, 1)
       // A of token tile ti: this thread's token row, [K ; V] as bf16 pairs.
       // Every MMA that read it in the previous unit is complete: this warp
       // consumed that unit's last accumulator of tile ti.
-      float x2 = 0.f;  // |x_t|^2, for the exactness flag
       {
         const int b = u.bh / P.H, h = u.bh % P.H;
         const __nv_bfloat16* kr = P.K + b * P.sb + h * P.sh + (int64_t)t * P.st;
         const __nv_bfloat16* vr = P.V + b * P.sb + h * P.sh + (int64_t)t * P.st;
         const uint32_t ta = tmem + ((uint32_t)(q * 32) << 16) + tcc::A_COL + ti * 128;
-        unsigned long long sq = 0ull;  // packed fp32x2 partial sums of squares
 #pragma unroll 1
         for (int c0 = 0; c0 < D / 2; c0 += 32) {
           // columns c0 .. c0 + 31 hold elements 2 c0 .. 2 c0 + 63 of [K ; V]
@@ -364,20 +352,9 @@ __global__ void __launch_bounds__(tcc::THREADS, 1)
             w[4 * v4 + 1] = x.y ^ 0x80008000u;
             w[4 * v4 + 2] = x.z ^ 0x80008000u;
             w[4 * v4 + 3] = x.w ^ 0x80008000u;
-            const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              // a bf16 pair widened to fp32 is a shift and a mask
-              const float lo = __uint_as_float(xw[i] << 16), hi = __uint_as_float(xw[i] & 0xFFFF0000u);
-              asm("{\n\t.reg .b64 v;\n\tmov.b64 v, {%1, %2};\n\tfma.rn.f32x2 %0, v, v, %0;\n\t}"
-                  : "+l"(sq) : "f"(lo), "f"(hi));
-            }
           }
           tmem_st32(ta + c0, w);
         }
-        float s0, s1;
-        asm("mov.b64 {%0, %1}, %2;" : "=f"(s0), "=f"(s1) : "l"(sq));
-        x2 = s0 + s1;
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -412,27 +389,9 @@ __global__ void __launch_bounds__(tcc::THREADS, 1)
       }
       if (!ok) break;
       if (t < P.T && (t % P.s) != 0) {
-        // exactness: every gap between neighbours among the first k + 1
-        // entries (the first k and their boundary to the next) must exceed
-        // the sum of the two entries' error bounds
-        const float gamma = (float)(2 * D + 8) * 1.1920928955078125e-07f;  // (2 D + 8) 2^-23
-        const float xn = sqrtf(x2);
-        const float* hn = P.hnorm + (int64_t)u.bh * P.n_ref_cap;
-        bool exact = true;
-        float bprev = 0.f;
-#pragma unroll
-        for (int x = 0; x < KC; ++x) {
-          if (x <= P.k && bi[x] != INT_MAX) {
-            const float h = __ldg(hn + bi[x]);
-            const float b = gamma * fmaf(xn, sqrtf(2.f * h), h);
-            if (x > 0 && !(bd[x] - bd[x - 1] > b + bprev)) exact = false;
-            bprev = b;
-          }
-        }
         int32_t* o = P.cand + ((int64_t)u.bh * P.n_code_cap + (t - t / P.s - 1)) * KC;
 #pragma unroll
         for (int x = 0; x < KC; ++x) o[x] = bi[x] == INT_MAX ? -1 : bi[x];
-        if (exact && bi[0] != INT_MAX) o[0] = bi[0] | kExactFlag;
       }
     }
     if (!ok) {
@@ -548,7 +507,6 @@ cudaError_t launch_candidates_tc(const Plan& p, int T, const KVView& kv, const v
   P.H = c.kv_heads;
   P.BH = c.batch * c.kv_heads;
   P.d_h = d_h;
-  P.k = c.k;
   P.K = (const __nv_bfloat16*)kv.K;
   P.V = (const __nv_bfloat16*)kv.V;
   P.sb = kv.sb;

@@ -254,9 +254,6 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
     for (int i = 0; i < KC; ++i) {
       int j = cr[i];
-      // the tensor-core search may mark the first slot with kExactFlag; this
-      // kernel re-ranks every row, so the mark is dropped
-      if (i == 0 && j >= 0) j &= ~kExactFlag;
       if (j >= 0 && (int64_t)j * s >= t) {  // not an earlier reference: drop it
         latch_error(err, DELTAKV_ERR_DEVICE_BOUNDS, (uint32_t)j);
         j = -1;

@@ -4,30 +4,27 @@
 // DeltaKV summary, section 3, "Processo di Compressione" steps 1-4 (the
 // selection is finished here from the k + 4 candidates the tensor-core search
 // kept):
-//   1. a row whose approximate ranking the search marked exact (every gap
-//      among its first k + 1 candidates above the fp32 error bound of the
-//      ranking key) takes its first k candidates as they are; any other row
-//      gets exact fp32 distances |x_t - r_j|^2 to all candidates and the k
-//      smallest by (distance, slot) are its references (idx plane);
+//   1. exact fp32 distances |x_t - r_j|^2 to the candidates; the k smallest
+//      by (distance, slot) are the token's references (idx plane);
 //   2. KV_R = their mean;  3. r = x_t - KV_R;
-//   4. code = W2 act(W1 r + b1) + b2  (code plane, rounded to bf16).
+//   4. code = W2 act(W1 r + b1) + b2  (code plane: bf16, or 4-bit values with
+//      one bf16 scale per row).
 //
 // One persistent CTA per SM, 16 warps with fixed roles, per 64-row tile:
 //   gather warps (11)  16 lanes per token row; the row's x and candidate
-//            slots are loaded one row pass ahead; an exact row loads only its
-//            k references; a re-ranked row loads its k + 4 candidate rows four
-//            at a time, gets exact fp32 distances, each candidate ranked by
-//            one lane, the chosen set by ballot over the row's 16 lanes (the
-//            two rows of a warp may take different paths); r = x - mean ->
-//            R tile (64 tokens x D, K-major, hi and lo), double-buffered so
-//            the next tile's gather overlaps
+//            slots are loaded one row pass ahead, the k + 4 candidate rows
+//            together when k + 4 = 8 (kept in registers for the mean), four at
+//            a time otherwise; exact fp32 distances, each candidate ranked by
+//            one lane, the chosen set by ballot; r = x - mean -> R tile (64
+//            tokens x D, K-major, hi and lo), double-buffered so the next
+//            tile's gather overlaps
 //   MMA warp  tcgen05.mma  D1^T = W1 . R^T  (A = W1 held in tensor memory
 //            for the whole launch, M = 128 hidden units per half, N = 64
 //            tokens); then codes = H . W2^T (A = the H tile through an
 //            MN-major descriptor, M = 128 with 64 tokens, N = d_c)
 //   activation warps (4)  thread = hidden unit: act(D1 + b1) over the tile's
 //            64 tokens -> H tile (hidden rows of 64 tokens, hi and lo), then
-//            TMEM -> + b2 -> bf16 codes
+//            TMEM -> + b2 -> bf16 codes (or 4-bit codes and their scale)
 // W1 and W2 are converted to fp16 once per launch (bf16 values of normal
 // range are exact in fp16).
 // Precision: every MMA operand that is not a weight is split into two fp16
@@ -196,9 +193,10 @@ __device__ __forceinline__ float group16_sum(float v, unsigned mask) {
   return v;
 }
 
-// Candidate rows of a re-ranked row are loaded four at a time; the chosen
-// ones are loaded again (from L2) for the mean.
-template <int KC> struct CandBatch { static constexpr int N = 4; };
+// Candidate rows in flight at a time: all of them when there are 8 (they
+// stay in registers for the mean), else four (the chosen ones are loaded
+// again, from L2, for the mean).
+template <int KC> struct CandBatch { static constexpr int N = KC == 8 ? 8 : 4; };
 
 template <int ACT>
 __device__ __forceinline__ float enc_act(float v) {
@@ -368,15 +366,9 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
         }
         int cj[KC];
         float cd[KC];
-        // a row whose approximate ranking already fixes the exact choice
-        // (flag in its first slot, set by the distance kernel) takes its
-        // first k slots as they are; the others are re-ranked exactly
-        const int c0raw = __shfl_sync(0xffffffffu, myc, 0, 16);
-        const bool exact = c0raw >= 0 && (c0raw & kExactFlag) != 0;
 #pragma unroll
         for (int c = 0; c < KC; ++c) {
           int j = __shfl_sync(0xffffffffu, myc, c, 16);
-          if (c == 0 && j >= 0) j &= ~kExactFlag;
           if (j >= 0 && (int64_t)j * P.s >= g.t) {  // not an earlier reference: drop it
             if (s16 == 0) latch_error(P.err, DELTAKV_ERR_DEVICE_BOUNDS, (uint32_t)j);
             j = -1;
@@ -384,46 +376,6 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
           cj[c] = j;
         }
         const unsigned gmask = 0xFFFFu << (16 * grp);
-        if (exact) {
-          // the list is in ascending order with the valid slots first
-          int n_valid = 0;
-#pragma unroll
-          for (int c = 0; c < KC; ++c) n_valid += cj[c] >= 0 ? 1 : 0;
-          const int k_eff = min(P.k, n_valid);
-          if (g.live && s16 < P.k) {
-            int js = -1;
-#pragma unroll
-            for (int c = 0; c < KC; ++c)
-              if (c == s16) js = cj[c];
-            P.idx[((int64_t)bh * P.n_code_cap + g.row) * P.k + s16] = s16 < k_eff ? js : -1;
-          }
-          const float inv = 1.0f / (float)max(k_eff, 1);
-          // the chosen rows, four in flight at a time
-#pragma unroll
-          for (int b0 = 0; b0 < kMaxK; b0 += 4) {
-            if (b0 < k_eff) {
-              uint4 rr[4][RowPack<EPL>::V4];
-#pragma unroll
-              for (int u = 0; u < 4; ++u)
-                if (b0 + u < k_eff) load_row<EPL>(rs + (int64_t)cj[b0 + u] * P.d_h, rr[u]);
-#pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                if (b0 + u < k_eff) {
-#pragma unroll
-                  for (int i = 0; i < RowPack<EPL>::V4; ++i) {
-                    const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&rr[u][i]);
-#pragma unroll
-                    for (int x = 0; x < 4; ++x) {
-                      const float2 v = __bfloat1622float2(p2[x]);
-                      xr[8 * i + 2 * x] = fmaf(-inv, v.x, xr[8 * i + 2 * x]);
-                      xr[8 * i + 2 * x + 1] = fmaf(-inv, v.y, xr[8 * i + 2 * x + 1]);
-                    }
-                  }
-                }
-              }
-            }
-          }
-        } else {
         // exact distances, NB candidate rows in flight at a time; with
         // NB == KC the rows stay in registers for the mean
         uint4 rr[NB][RowPack<EPL>::V4];
@@ -510,7 +462,6 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
             }
           }
         }
-        }  // re-rank
         // r = hi + lo (fp16) into the R tile: row n, columns e0 .. e0 + EPL
 #pragma unroll
         for (int v = 0; v < EPL / 8; ++v) {

@@ -13,9 +13,6 @@ namespace dkv {
 constexpr int kMaxK = 8;          // references per token
 constexpr int kExtraCand = 4;     // extra candidates the distance kernel keeps
 constexpr int kMaxCand = kMaxK + kExtraCand;
-// Set in the first candidate slot of a row whose approximate ranking already
-// fixes the exact k nearest and their order (slot numbers stay below 2^26).
-constexpr int32_t kExactFlag = 1 << 30;
 constexpr int kMaxG = 8;          // query heads per kv-head
 constexpr int kMaxHidden = 256;
 constexpr int kMaxSplit = 32;     // decode splits per (sequence, kv-head)
