@@ -9,7 +9,8 @@ One step = the whole path over one batch of synthetic input:
   * decode: one query per sequence for a batch of 8 sequences of 131072
     cached tokens, 32 layers, 32 query heads / 8 kv-heads, over caches
     compressed (untimed) before the run.
-`value` is compressed tokens per second over the whole step (Mtok/s);
+`value` is the metric's compress Mtok/s: tokens compressed per second of the
+compress phase of the timed steps (`step_Mtok_s` divides by the whole step);
 `decode_attn` reports the decode phase in GB/s of algorithmic bytes.
 
 Prints one JSON line (rank 0).  `--impl reference` times the fp64 CPU oracle
@@ -48,6 +49,10 @@ def parse():
     ap.add_argument("--decode-batch", type=int, default=8)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="single-layer sweep over s, k, d_c, T: one JSON line per point instead of the step")
+    ap.add_argument("--sweep-T", default="4096,16384,65536,131072")
+    ap.add_argument("--sweep-reps", type=int, default=5)
     return ap.parse_args()
 
 
@@ -64,11 +69,11 @@ def load_peaks():
 # ------------------------------------------------------------------ workload
 
 class Shape:
-    def __init__(self, a):
+    def __init__(self, a, s=16, k=4, d_c=32, T=None):
         self.L = a.layers
-        self.T = a.T
+        self.T = a.T if T is None else T
         self.H, self.Hq, self.d_h = 8, 32, 128
-        self.s, self.k, self.d_c, self.hidden = 16, 4, 32, 256
+        self.s, self.k, self.d_c, self.hidden = s, k, d_c, 256
         self.Bc, self.Bd = 1, a.decode_batch
         self.n_lat = 8
         self.n_ref = math.ceil(self.T / self.s)
@@ -134,6 +139,34 @@ def kernel_rooflines(sh, prof, peaks, peak_kind):
     add("decode_stream_tc", "hbm", stream_bytes, "GB/s", hbm_peak, src_h)
     add("decode_stream_simt", "hbm", stream_bytes, "GB/s", hbm_peak, src_h)
     return out
+
+
+MUFU_PER_CLK_PER_SM = 16       # special-function unit results per clock per SM (fp32 tanh.approx)
+MMA_MIN_CYCLES = 56            # an M = 128, N <= 64 tcgen05.mma occupies the tensor pipe this long (measured)
+
+
+def decode_bounds(sh, peaks, sm_mhz):
+    """Floors of the decode token loop for one layer, in ms, and the binding
+    one.  hbm: the algorithmic bytes at the copy peak; tensor: the folded
+    decode's MMA FLOPs per compressed token (decompressor layer 1, logits
+    against [a_hi, a_lo], U against [P_hi, P_lo]) at the bf16 peak; mma_issue:
+    the same MMAs counted as instructions at the measured minimum occupancy
+    of a small-N tcgen05.mma; sfu: one special-function (tanh) result per
+    activation."""
+    clk = (sm_mhz or SM_MAX_MHZ) * 1e6
+    tok_heads = sh.Bd * sh.H * sh.n_code
+    G = sh.Hq // sh.H
+    flops = 2 * tok_heads * (sh.d_c * sh.hidden + 2 * sh.hidden * 2 * G + 2 * sh.hidden * 2 * G)
+    hbm_ms = sh.decode_bytes_per_layer() / (peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]) * 1e9) * 1e3
+    tensor_ms = flops / (peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]) * 1e12) * 1e3
+    chunks_per_sm = math.ceil(tok_heads / 128) / NUM_SMS
+    g1_cycles = max(MMA_MIN_CYCLES, sh.hidden // 2) * math.ceil(sh.d_c / 16)
+    mma_cycles = g1_cycles + MMA_MIN_CYCLES * (sh.hidden // 16) + MMA_MIN_CYCLES * (sh.hidden // 128) * 8
+    mma_ms = chunks_per_sm * mma_cycles / clk * 1e3
+    sfu_ms = tok_heads * sh.hidden / (NUM_SMS * MUFU_PER_CLK_PER_SM * clk) * 1e3
+    b = {"hbm_ms": hbm_ms, "tensor_ms": tensor_ms, "mma_issue_ms": mma_ms, "sfu_ms": sfu_ms, "clock_mhz": clk / 1e6}
+    b["binding"] = max(("hbm_ms", "tensor_ms", "mma_issue_ms", "sfu_ms"), key=lambda k: b[k])
+    return b
 
 
 def build_workload(sh, dev):
@@ -245,6 +278,86 @@ def sparse_timing(sh, w, steps, n_sel=4096):
             "rebuilt_tokens_per_s": sh.Bd * sh.H * n_sel * sh.L / (ms / 1e3)}
 
 
+# -------------------------------------------------------------------- sweep
+
+def run_sweep(a, dev):
+    """The single-layer sweep: 8 kv-heads, d_h 128, bf16, hidden 256, the
+    same generator; s in {4, 8, 16, 32} x k in {1, 2, 4, 8} x d_c in {16, 32,
+    64} x T in --sweep-T.  Per point: compress of one sequence (Mtok/s and
+    the fraction of the sustained bf16 peak its search and MLP FLOPs reach)
+    and decode at batch 8 with 32 query heads over caches compressed
+    beforehand (GB/s of algorithmic bytes and the fraction of HBM copy
+    bandwidth).  K/V are generated once per T and reused by every point."""
+    from decode_attention_strided_b200 import deltakv as dkv
+    from decode_attention_strided_b200 import synth
+    peaks, peak_kind = load_peaks()
+    tpk = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    Bd, reps = 8, max(1, a.sweep_reps)
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    n_pts = 0
+    t_all = time.perf_counter()
+    for T in [int(x) for x in a.sweep_T.split(",")]:
+        base = Shape(a, T=T)
+        K = torch.empty((Bd, base.H, T, base.d_h), dtype=torch.bfloat16, device=dev)
+        V = torch.empty_like(K)
+        for b in range(Bd):
+            for h in range(base.H):
+                x = synth.head_tokens(0, 0, b, h, T, base.d_h, base.n_lat, torch.bfloat16, dev)
+                K[b, h].copy_(x[:, :base.d_h])
+                V[b, h].copy_(x[:, base.d_h:])
+        q = synth.queries(0, Bd, base.Hq, base.d_h, device=dev)
+        out = torch.empty((Bd, base.Hq, base.d_h), dtype=torch.float32, device=dev)
+        for s_ in (4, 8, 16, 32):
+            for k_ in (1, 2, 4, 8):
+                for dc in (16, 32, 64):
+                    sh = Shape(a, s=s_, k=k_, d_c=dc, T=T)
+                    sh.Bd = Bd
+                    W = {n: t.to(dev) for n, t in synth.codec_weights(0, sh.d_h, dc, sh.hidden).items()}
+                    mk = lambda B: dkv.plan(dkv.Config(batch=B, kv_heads=sh.H, q_heads=sh.Hq, d_h=sh.d_h,  # noqa
+                                                       max_T=T, stride_s=s_, k=k_, d_c=dc, hidden=sh.hidden))
+                    pc, pd = mk(1), mk(Bd)
+                    cc, cd = pc.alloc_cache(dev), pd.alloc_cache(dev)
+                    wc, wd = pc.alloc_workspace(dev), pd.alloc_workspace(dev)
+                    Kc, Vc = K[:1], V[:1]
+                    dkv.compress(pd, T, K, V, W["W1"], None, W["W2"], None, cd, wd)
+                    for _ in range(2):
+                        dkv.compress(pc, T, Kc, Vc, W["W1"], None, W["W2"], None, cc, wc)
+                        dkv.decode_attention(pd, T, q, cd, W["W3"], None, W["W4"], None, out, wd)
+                    torch.cuda.synchronize()
+                    e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+                    e[0].record()
+                    for _ in range(reps):
+                        dkv.compress(pc, T, Kc, Vc, W["W1"], None, W["W2"], None, cc, wc)
+                    e[1].record()
+                    for _ in range(reps):
+                        dkv.decode_attention(pd, T, q, cd, W["W3"], None, W["W4"], None, out, wd)
+                    e[2].record()
+                    torch.cuda.synchronize()
+                    ms_c = e[0].elapsed_time(e[1]) / reps
+                    ms_d = e[1].elapsed_time(e[2]) / reps
+                    fl = sh.cand_flops_per_layer(1) + sh.mlp_flops_per_layer(1)
+                    db = sh.decode_bytes_per_layer()
+                    st = max(dkv.device_status(pc, wc), dkv.device_status(pd, wd))
+                    per_tok = (sh.n_ref * 2 * sh.d_h * 2 + sh.n_code * (dc * 2 + k_ * 4)) / T
+                    pt = {"point": {"s": s_, "k": k_, "d_c": dc, "T": T}, "compress_ms": ms_c,
+                          "compress_Mtok_s": T / (ms_c / 1e3) / 1e6,
+                          "compress_tensor_frac": fl / (ms_c / 1e3) / 1e12 / tpk,
+                          "decode_ms": ms_d, "decode_GB_s": db / (ms_d / 1e3) / 1e9,
+                          "decode_hbm_frac": db / (ms_d / 1e3) / 1e9 / hbm,
+                          "cache_bytes_per_token_head": per_tok, "cache_frac_of_bf16": per_tok / (4 * sh.d_h),
+                          "decode_batch": Bd, "q_heads": sh.Hq, "kv_heads": sh.H, "device_status": st}
+                    print(json.dumps(pt), flush=True)
+                    n_pts += 1
+                    del cc, cd, wc, wd, pc, pd
+        del K, V
+        torch.cuda.empty_cache()
+    clk = clocks.stop()
+    print(json.dumps({"sweep_points": n_pts, "wall_s": time.perf_counter() - t_all, "clocks": clk,
+                      "peaks": {"bf16_tflops_sustained": tpk, "hbm_gbs": hbm, "source": peak_kind}}), flush=True)
+
+
 # ------------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -324,6 +437,12 @@ def oracle_sample(sh, budget_s=12.0, threads=0):
             break
         n_rows *= 4
     per_row_c = t_c / n_rows
+    # one thread on a small bounded sample of the same rows: the per-unit cost
+    # of the oracle without threading
+    n1 = max(16, min(n_rows, 256))
+    t0 = time.perf_counter()
+    oracle.compress_rows(K, V, W["W1"], None, W["W2"], None, sh.s, sh.k, rows[:n1], n_threads=1)
+    per_row_c_1t = (time.perf_counter() - t0) / n1
     # decode: reconstruct a prefix of the cache and attend over it
     Tp = min(sh.T, 16384)
     idx, code, _, _ = oracle.compress(K[:Tp], V[:Tp], W["W1"], None, W["W2"], None, sh.s, sh.k, n_threads=nthreads)
@@ -331,12 +450,17 @@ def oracle_sample(sh, budget_s=12.0, threads=0):
     Kh, Vh = oracle.reconstruct(K[:Tp], V[:Tp], idx, code, W["W3"], None, W["W4"], None, sh.s, n_threads=nthreads)
     q = np.random.default_rng(1).normal(size=(sh.Hq // sh.H, sh.d_h))
     oracle.attention(q, Kh, Vh)
-    per_row_d = (time.perf_counter() - t0) / Tp
+    t_d = time.perf_counter() - t0
+    per_row_d = t_d / Tp
     step_s = sh.L * (per_row_c * sh.T * sh.H * sh.Bc + per_row_d * sh.T * sh.H * sh.Bd)
     desc = (f"oracle compress_rows on {n_rows} uniformly drawn rows of one (layer, kv-head) at T={sh.T} "
-            f"({t_c:.2f}s) + reconstruct/attend over a {Tp}-token prefix; extrapolated to the full step "
-            f"({sh.L} layers x {sh.H} heads compress, {sh.Bd} x {sh.H} heads decode)")
-    return step_s, desc, nthreads
+            f"({t_c:.2f}s) + reconstruct/attend over a {Tp}-token prefix ({t_d:.2f}s); extrapolated to the full "
+            f"step ({sh.L} layers x {sh.H} heads compress, {sh.Bd} x {sh.H} heads decode)")
+    info = {"extrapolated": True, "measured_s": t_c + t_d, "sampled_compress_rows": int(n_rows),
+            "sampled_decode_prefix": int(Tp), "threads": int(nthreads),
+            "single_thread_s_per_compressed_row": per_row_c_1t,
+            "threaded_s_per_compressed_row": per_row_c}
+    return step_s, desc, nthreads, info
 
 
 def run_reference(a, rank):
@@ -344,19 +468,25 @@ def run_reference(a, rank):
     if rank != 0:
         return
     per_step = []
-    desc, nthreads = "", 0
+    desc, nthreads, info, measured = "", 0, {}, 0.0
     for i in range(a.warmup + a.steps):
-        step_s, desc, nthreads = oracle_sample(sh, budget_s=8.0)
+        step_s, desc, nthreads, info = oracle_sample(sh, budget_s=8.0)
         if i >= a.warmup:
             per_step.append(step_s)
+            measured += info["measured_s"]
     step_s = statistics.median(per_step)
-    value = sh.T * sh.Bc / step_s / 1e6
+    # the metric's compress Mtok/s: the compress share of the extrapolated step
+    comp_s = sh.L * info["threaded_s_per_compressed_row"] * sh.T * sh.H * sh.Bc
+    value = sh.T * sh.Bc / comp_s / 1e6
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "Mtok/s", "n_gpus": a.gpus,
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(sh),
-        "cpu_baseline": {"value": value, "unit": "Mtok/s", "cores": nthreads, "kind": "oracle", "sample": desc},
+        "extrapolated": True, "measured_sample_s": measured,
+        "step_Mtok_s": sh.T * sh.Bc / step_s / 1e6,
+        "cpu_baseline": {"value": value, "unit": "Mtok/s", "cores": nthreads, "kind": "oracle", "sample": desc,
+                         **info},
         "e2e": {"value": value, "unit": "Mtok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -397,6 +527,12 @@ def main():
     dev = f"cuda:{local}"
     from decode_attention_strided_b200 import deltakv as dkv
     dkv.load_library()  # fails loudly if the CUDA library is not built
+    if a.sweep:
+        if rank == 0:
+            run_sweep(a, dev)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
 
     sh = Shape(a)
     t_setup = time.perf_counter()
@@ -444,7 +580,11 @@ def main():
     dec_ms = [e[1].elapsed_time(e[2]) for e in ev]
     tot_ms, sc, sd = max_over_ranks([sum(step_ms), sum(comp_ms), sum(dec_ms)], dev, world)
     ms_step = tot_ms / a.steps
-    value = world * sh.T * sh.Bc * a.steps / (tot_ms / 1e3) / 1e6
+    # value: the metric's compress Mtok/s, tokens compressed by all ranks per
+    # second of the compress phase (the timed region also runs the decode,
+    # reported in decode_attn; step_Mtok_s divides by the whole step)
+    value = world * sh.T * sh.Bc * a.steps / (sc / 1e3) / 1e6
+    step_rate = world * sh.T * sh.Bc * a.steps / (tot_ms / 1e3) / 1e6
 
     peaks, peak_kind = load_peaks()
     # dominant kernel of the step
@@ -467,6 +607,7 @@ def main():
         if k_ in prof:
             n, ms = prof[k_]
             decode_attn["stream_kernel_ms_per_launch"] = ms / n
+    decode_attn["bounds"] = decode_bounds(sh, peaks, clk.get("sm_mhz"))
     comp_fl = sh.cand_flops_per_layer(sh.Bc) + sh.mlp_flops_per_layer(sh.Bc)
     compress = {"value": sh.T * sh.Bc / (sc / a.steps / 1e3) / 1e6, "unit": "Mtok/s",
                 "ms": sc / a.steps,
@@ -478,14 +619,15 @@ def main():
         e2e = run_e2e(sh, w, dev, a, world)
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
-        step_s, desc, nthreads = oracle_sample(sh, budget_s=12.0)
-        cpu = {"value": sh.T * sh.Bc / step_s / 1e6, "unit": "Mtok/s", "cores": nthreads, "kind": "oracle",
-               "sample": desc}
+        step_s, desc, nthreads, info = oracle_sample(sh, budget_s=12.0)
+        comp_s = sh.L * info["threaded_s_per_compressed_row"] * sh.T * sh.H * sh.Bc
+        cpu = {"value": sh.T * sh.Bc / comp_s / 1e6, "unit": "Mtok/s", "cores": nthreads, "kind": "oracle",
+               "sample": desc, "step_Mtok_s": sh.T * sh.Bc / step_s / 1e6, **info}
     line = {
         "metric": METRIC, "value": value, "unit": "Mtok/s", "n_gpus": world, "steps": a.steps,
         "warmup": a.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(sh),
-        "compress": compress, "decode_attn": decode_attn, "append": append, "sparse_decode": sparse,
+        "step_Mtok_s": step_rate, "compress": compress, "decode_attn": decode_attn, "append": append, "sparse_decode": sparse,
         "roofline": roof, "rooflines": rooflines, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
         "kernels": {k_: {"launches": n, "ms": ms} for k_, (n, ms) in prof.items()},
         "clocks": clk, "device_status": status, "setup_s": setup_s, "wall_s": wall,
@@ -524,26 +666,31 @@ def run_e2e(sh, w, dev, a, world=1):
     h2d = d2h = 0
     steps = max(1, min(a.steps, 3))
     torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(steps):
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for i in range(steps):
+        ev[i][0].record()
         for l in range(sh.L):
             dK.copy_(hK, non_blocking=True)
             dV.copy_(hV, non_blocking=True)
             dkv.compress(w["pc"], sh.T, dK, dV, w["W"][l]["W1"], None, w["W"][l]["W2"], None,
                          w["comp_cache"][l], w["ws_c"])
+        ev[i][1].record()
         for l in range(sh.L):
             dq.copy_(hq[l], non_blocking=True)
             dkv.decode_attention(w["pd"], sh.T, dq, w["dec_cache"][l], w["W"][l]["W3"], None, w["W"][l]["W4"],
                                  None, w["out"][l], w["ws_d"])
             ho[l].copy_(w["out"][l], non_blocking=True)
-    e1.record()
+        ev[i][2].record()
     torch.cuda.synchronize()
-    ms = max_over_ranks([e0.elapsed_time(e1) / steps], dev, world)[0]
+    ms, ms_c = max_over_ranks([sum(e[0].elapsed_time(e[2]) for e in ev) / steps,
+                               sum(e[0].elapsed_time(e[1]) for e in ev) / steps], dev, world)
     h2d = sh.L * (hK.numel() * 2 + hV.numel() * 2 + hq[0].numel() * 2)
     d2h = sh.L * ho[0].numel() * 4
-    return {"value": world * sh.T * sh.Bc / (ms / 1e3) / 1e6, "unit": "Mtok/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps}
+    # value: compress Mtok/s with every layer's K/V copied in (the metric);
+    # step_Mtok_s and ms_per_step cover the whole step with the decode copies
+    return {"value": world * sh.T * sh.Bc / (ms_c / 1e3) / 1e6, "unit": "Mtok/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "compress_ms_per_step": ms_c,
+            "step_Mtok_s": world * sh.T * sh.Bc / (ms / 1e3) / 1e6, "steps": steps}
 
 
 if __name__ == "__main__":

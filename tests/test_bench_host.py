@@ -57,3 +57,20 @@ def test_roofline_fields():
     # traffic is only quoted for the workload it was measured on
     r2 = bench.kernel_rooflines(_shape(T=65536), prof, peaks, "measured")
     assert r2["candidates_tc"]["traffic"] is None
+
+
+def test_decode_bounds_of_the_128k_batch8_layer():
+    """The decode token loop's floors, recomputed: 8 x 8 x 122880 compressed
+    token-heads; 256 activations each at 16 special-function results per clock
+    on 148 SMs; 960 chunks per sequence-head of 2 GEMM1 MMAs (128 cycles at
+    N = 256) plus 16 z and 16 U MMAs at the 56-cycle minimum."""
+    sh = _shape()
+    b = bench.decode_bounds(sh, {"hbm_gbs": 5000.0, "bf16_tflops_sustained": 1000.0}, 2000.0)
+    th = 8 * 8 * (131072 - 8192)
+    assert math.isclose(b["sfu_ms"], th * 256 / (148 * 16 * 2e9) * 1e3)
+    assert math.isclose(b["hbm_ms"], sh.decode_bytes_per_layer() / 5e12 * 1e3)
+    chunks = 8 * 8 * 960
+    assert math.isclose(b["mma_issue_ms"], chunks / 148 * (2 * 128 + 16 * 56 + 16 * 56) / 2e9 * 1e3)
+    flops = 2 * th * (32 * 256 + 2 * 256 * 8 + 2 * 256 * 8)
+    assert math.isclose(b["tensor_ms"], flops / 1e15 * 1e3)
+    assert b["binding"] in ("sfu_ms", "mma_issue_ms")
