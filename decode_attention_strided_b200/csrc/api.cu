@@ -88,7 +88,10 @@ void build_plan(const deltakv_config& c, Plan& p) {
   w = align256(w + std::max<size_t>((size_t)(BH * p.n_code_cap * p.KC) * 4, (size_t)BH * 4096));
   const size_t compress_end = w;
   w = kErrBytes;
-  p.nslot_cap = (int)std::max<int64_t>(kMaxSplit, ceil_div64(kNumSMs, BH) + 1);
+  // partial slots of one (sequence, kv-head): the CTAs its chunks span; with
+  // sequences of different lengths one sequence's kv-heads may hold nearly
+  // all chunks, so the bound is taken per kv-head count
+  p.nslot_cap = (int)std::max<int64_t>(kMaxSplit, ceil_div64(kNumSMs, c.kv_heads) + 2);
   const int64_t n_refblk_cap = ceil_div64(p.n_ref_cap, 64);
   p.n_chunk_cap = (int)ceil_div64(p.n_ref_cap, kCombineSlots);
   p.ws_S = w;
@@ -109,6 +112,8 @@ void build_plan(const deltakv_config& c, Plan& p) {
   w = align256(w + (size_t)(BH * p.nslot_cap * p.G * c.hidden) * 4);
   p.ws_ochunk = w;
   w = align256(w + (size_t)(BH * p.n_chunk_cap * p.G * (c.d_h + 1)) * 4);
+  p.ws_cho = w;  // then the checked lengths [batch]
+  w = align256(w + (size_t)(BH + 1 + c.batch) * 4);
   p.ws_decode_end = w;
   p.ws_sparse = w;  // sparse decode: (m, l, output) of every share
   w = align256(w + (size_t)(BH * kSparseSplits * p.G * (c.d_h + 2)) * 4);
@@ -243,8 +248,73 @@ deltakv_status deltakv_decode_attention(deltakv_plan_t plan, int32_t T, const vo
   if (!aligned16(q) || !aligned16(cache) || !aligned16(W3) || !aligned16(W4) || !aligned16(out) ||
       !aligned16(workspace) || !aligned16(b3) || !aligned16(b4))
     return DELTAKV_ERR_ALIGNMENT;
-  return from_cuda(launch_decode(p, T, q, q_strides[0], q_strides[1], cache, W3, b3, W4, b4, out,
-                                 out_strides[0], out_strides[1], workspace, (cudaStream_t)stream));
+  const SeqLens sl{nullptr, T, T};
+  return from_cuda(launch_decode(p, contiguous_view(p, cache), sl, q, q_strides[0], q_strides[1], W3, b3, W4, b4,
+                                 out, out_strides[0], out_strides[1], workspace, (cudaStream_t)stream));
+}
+
+deltakv_status deltakv_page_pool_layout(deltakv_plan_t plan, int32_t n_pages, deltakv_page_layout* out) {
+  if (!plan || !out || n_pages < 1) return DELTAKV_ERR_INVALID_ARG;
+  const Plan& p = plan->p;
+  const PoolLayout L = pool_layout(p, n_pages);
+  out->refs_per_page = (int32_t)L.rp;
+  out->codes_per_page = (int32_t)L.cp;
+  out->tokens_per_page = (int32_t)(L.rp * p.cfg.stride_s);
+  out->n_pages = n_pages;
+  out->ref_k_offset = L.off_refk;
+  out->ref_v_offset = L.off_refv;
+  out->code_offset = L.off_code;
+  out->idx_offset = L.off_idx;
+  out->code_scale_offset = L.off_cscale;
+  out->pool_bytes = L.bytes;
+  return DELTAKV_OK;
+}
+
+deltakv_status deltakv_pages_from_cache(deltakv_plan_t plan, int32_t T, const void* cache,
+                                        const int32_t* page_table, int32_t max_pages, void* pool, int32_t n_pages,
+                                        void* workspace, size_t workspace_bytes, deltakv_stream_t stream) {
+  if (!plan) return DELTAKV_ERR_INVALID_ARG;
+  const Plan& p = plan->p;
+  if (T < 1 || T > p.cfg.max_T || n_pages < 1 || !cache || !page_table || !pool || !workspace)
+    return DELTAKV_ERR_INVALID_ARG;
+  const int64_t tpp = (int64_t)kPageRefs * p.cfg.stride_s;
+  if (max_pages < ceil_div64(T, tpp)) return DELTAKV_ERR_INVALID_ARG;
+  if (workspace_bytes < p.ws_bytes) return DELTAKV_ERR_WORKSPACE;
+  if (!aligned16(cache) || !aligned16(pool) || !aligned16(workspace) || ((uintptr_t)page_table & 3))
+    return DELTAKV_ERR_ALIGNMENT;
+  const PoolLayout L = pool_layout(p, n_pages);
+  return from_cuda(launch_pages_from_cache(p, T, cache, L, pool, n_pages, page_table, max_pages, workspace,
+                                           (cudaStream_t)stream));
+}
+
+deltakv_status deltakv_decode_attention_paged(deltakv_plan_t plan, const int32_t* seq_lens, int32_t max_len,
+                                              const void* q, const int64_t q_strides[2], const void* pool,
+                                              int32_t n_pages, const int32_t* page_table, int32_t max_pages,
+                                              const void* W3, const float* b3, const void* W4, const float* b4,
+                                              float* out, const int64_t out_strides[2], void* workspace,
+                                              size_t workspace_bytes, deltakv_stream_t stream) {
+  if (!plan) return DELTAKV_ERR_INVALID_ARG;
+  const Plan& p = plan->p;
+  if (max_len < 1 || max_len > p.cfg.max_T || n_pages < 1) return DELTAKV_ERR_INVALID_ARG;
+  if (!seq_lens || !q || !q_strides || !pool || !page_table || !W3 || !W4 || !out || !out_strides || !workspace)
+    return DELTAKV_ERR_INVALID_ARG;
+  const int64_t tpp = (int64_t)kPageRefs * p.cfg.stride_s;
+  if (max_pages < ceil_div64(max_len, tpp)) return DELTAKV_ERR_INVALID_ARG;
+  if (workspace_bytes < p.ws_bytes) return DELTAKV_ERR_WORKSPACE;
+  if (q_strides[0] < 0 || q_strides[1] < 0 || out_strides[0] < 0 || out_strides[1] < 0)
+    return DELTAKV_ERR_INVALID_ARG;
+  if ((q_strides[0] * p.esize) % 16 || (q_strides[1] * p.esize) % 16 || (out_strides[0] * 4) % 16 ||
+      (out_strides[1] * 4) % 16)
+    return DELTAKV_ERR_ALIGNMENT;
+  if (!aligned16(q) || !aligned16(pool) || !aligned16(W3) || !aligned16(W4) || !aligned16(out) ||
+      !aligned16(workspace) || !aligned16(b3) || !aligned16(b4) || ((uintptr_t)seq_lens & 3) ||
+      ((uintptr_t)page_table & 3))
+    return DELTAKV_ERR_ALIGNMENT;
+  const PoolLayout L = pool_layout(p, n_pages);
+  const CacheView cv = pool_view(p, L, pool, n_pages, page_table, max_pages, workspace);
+  const SeqLens sl{seq_lens, max_len, max_len};
+  return from_cuda(launch_decode(p, cv, sl, q, q_strides[0], q_strides[1], W3, b3, W4, b4, out, out_strides[0],
+                                 out_strides[1], workspace, (cudaStream_t)stream));
 }
 
 deltakv_status deltakv_decode_attention_sparse(deltakv_plan_t plan, int32_t T, const void* q,

@@ -34,15 +34,17 @@ constexpr int kRefBlockSlots = 64;
 // ------------------------------------------------------------ decode_ref
 template <typename T>
 __global__ void __launch_bounds__(256)
-    decode_ref_kernel(int64_t n_ref, int64_t n_ref_cap, int d_h, int H, int G, float c,
-                      const T* __restrict__ q, int64_t qsb, int64_t qsh,
-                      const T* __restrict__ refk, float* __restrict__ S,
-                      float* __restrict__ Smax, int n_refblk_cap, float* __restrict__ wtab) {
+    decode_ref_kernel(SeqLens sl, int s_, int64_t n_ref_cap, int d_h, int H, int G, float c,
+                      const T* __restrict__ q, int64_t qsb, int64_t qsh, CacheView cv,
+                      float* __restrict__ S, float* __restrict__ Smax, int n_refblk_cap,
+                      float* __restrict__ wtab) {
   __shared__ float qs[kMaxG][128];
   __shared__ float wmax[8][kMaxG];
   const int b = blockIdx.z, h = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t bh = (int64_t)b * H + h;
+  const int64_t n_ref = n_ref_of(sl.T(b), s_);
+  const T* refk = reinterpret_cast<const T*>(cv.base + cv.off_refk);
   for (int i = threadIdx.x; i < G * d_h; i += blockDim.x) {
     int g = i / d_h, e = i - g * d_h;
     qs[g][e] = c * to_f(q[b * qsb + (int64_t)(h * G + g) * qsh + e]);
@@ -54,7 +56,7 @@ __global__ void __launch_bounds__(256)
   for (int i = 0; i < kRefBlockSlots / 8; ++i) {
     int64_t j = (int64_t)blockIdx.x * kRefBlockSlots + warp * (kRefBlockSlots / 8) + i;
     if (j >= n_ref) break;
-    const T* kr = refk + (bh * n_ref_cap + j) * d_h;
+    const T* kr = refk + cv.ref_row(bh, j) * d_h;
     float kv[4];
 #pragma unroll
     for (int q4 = 0; q4 < 4; ++q4) {
@@ -161,11 +163,9 @@ __global__ void __launch_bounds__(256)
 // U and l use a per-warp running maximum.
 template <typename T>
 __global__ void __launch_bounds__(256)
-    decode_stream_kernel(int T_, int s, int d_h, int H, int G, int k, int d_c, int hidden,
-                         int act, int ns, int64_t n_ref_cap, int64_t n_code_cap,
-                         int n_refblk, int n_refblk_cap, const T* __restrict__ code,
-                         const __nv_bfloat16* __restrict__ cscale,
-                         const int32_t* __restrict__ idx, const T* __restrict__ W3,
+    decode_stream_kernel(SeqLens sl, int s, int d_h, int H, int G, int k, int d_c, int hidden,
+                         int act, int ns, int64_t n_ref_cap, int n_refblk, int n_refblk_cap, CacheView cv,
+                         const T* __restrict__ W3,
                          const float* __restrict__ b3, const float* __restrict__ a,
                          const float* __restrict__ cterm, const float* __restrict__ S,
                          const float* __restrict__ Smax, float* __restrict__ wtab_g,
@@ -181,9 +181,14 @@ __global__ void __launch_bounds__(256)
   const int b = blockIdx.z, h = blockIdx.y, split = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
   const int64_t bh = (int64_t)b * H + h;
-  const int64_t n_ref = (T_ + s - 1) / s;
-  const int64_t n_code = T_ - n_ref;
+  const int64_t n_ref = n_ref_of(sl.T(b), s);
+  const int64_t n_code = sl.T(b) - n_ref;
   const int64_t c0 = n_code * split / ns, c1 = n_code * (split + 1) / ns;
+  const T* code = reinterpret_cast<const T*>(cv.base + cv.off_code);
+  // the scale plane exists with 4-bit codes only (its offset is 0 otherwise)
+  const __nv_bfloat16* cscale =
+      cv.off_cscale ? reinterpret_cast<const __nv_bfloat16*>(cv.base + cv.off_cscale) : nullptr;
+  const int32_t* idx = reinterpret_cast<const int32_t*>(cv.base + cv.off_idx);
   // the kv-head's slot-weight table (zeroed by decode_ref), relative to
   // m_ref; with room in shared memory the block sums into a private copy first
   float* wtab = wt_in_smem ? wt : wtab_g + bh * n_ref_cap * G;
@@ -221,14 +226,13 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
     for (int i = 0; i < 8; ++i) Uw[g][i] = 0.f;
   }
-  const int64_t crow0 = bh * n_code_cap;  // plane row of this (sequence, kv-head)'s first code
-  const int32_t* ib = idx + bh * n_code_cap * k;
   const float* Sb = S + bh * n_ref_cap * G;
 
   for (int64_t row = c0 + warp; row < c1; row += 8) {
     // the code row, staged in this warp's slice of shared memory
     float* cr = cw + warp * d_c;
-    for (int e = lane; e < d_c; e += 32) cr[e] = code_at(code, cscale, crow0 + row, d_c, e);
+    const int64_t prow = cv.code_row(bh, row);  // plane row of the code and of its slots
+    for (int e = lane; e < d_c; e += 32) cr[e] = code_at(code, cscale, prow, d_c, e);
     __syncwarp();
     float u[8];
 #pragma unroll
@@ -243,7 +247,7 @@ __global__ void __launch_bounds__(256)
     }
     __syncwarp();
     // reference part of the logits
-    int j = lane < k ? ib[row * k + lane] : -1;
+    int j = lane < k ? idx[prow * k + lane] : -1;
     if (j >= n_ref) { latch_error(err, DELTAKV_ERR_DEVICE_BOUNDS, (uint32_t)j); j = -1; }
     const unsigned valid = __ballot_sync(0xffffffffu, j >= 0);
     const int k_eff = __popc(valid);
@@ -320,15 +324,22 @@ __global__ void __launch_bounds__(256)
 // Partial (m, l, U) slots per kv-head: a fixed count for the CUDA-core
 // stream kernel, the CTAs of the even chunk split for the tensor-core one.
 struct SlotInfo {
-  int tc, ns, n_ch, grid, nslot_cap;
-  int64_t N;
+  int tc, ns, grid, nslot_cap, BH;
+  int n_ch;            // chunks per (sequence, kv-head) when every sequence has the same length
+  const int32_t* cho;  // else the chunk offsets [BH + 1] (decode_sched_kernel)
 };
+
+__device__ __forceinline__ int64_t chunk_off(const SlotInfo& si, int64_t bh) {
+  return si.cho ? (int64_t)si.cho[bh] : bh * si.n_ch;
+}
 
 __device__ __forceinline__ int slots_of(const SlotInfo& si, int64_t bh) {
   if (!si.tc) return si.ns;
-  if (si.n_ch == 0) return 0;
-  const int64_t first = (bh * si.n_ch * si.grid) / si.N;
-  const int64_t last = (((bh + 1) * si.n_ch - 1) * si.grid) / si.N;
+  const int64_t x0 = chunk_off(si, bh), x1 = chunk_off(si, bh + 1), N = chunk_off(si, si.BH);
+  if (x1 == x0) return 0;
+  const int64_t g = N < si.grid ? N : si.grid;  // the CTAs that got chunks (as in the token loop)
+  const int64_t first = (x0 * g) / N;
+  const int64_t last = ((x1 - 1) * g) / N;
   return (int)(last - first + 1);
 }
 
@@ -354,8 +365,8 @@ __device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
 // w_j = 2^(S_j - M) + 2^(m_ref - M) sum_splits wtab, then sum_j w_j V_ref_j.
 template <typename T>
 __global__ void __launch_bounds__(256)
-    decode_combine_kernel(int T_, int s, int d_h, int H, int G, SlotInfo si, int64_t n_ref_cap,
-                          int n_chunk_cap, const T* __restrict__ refv, const float* __restrict__ S,
+    decode_combine_kernel(SeqLens sl, int s, int d_h, int H, int G, SlotInfo si, int64_t n_ref_cap,
+                          int n_chunk_cap, CacheView cv, const float* __restrict__ S,
                           const float* __restrict__ mref, const float* __restrict__ wtab_g,
                           const float* __restrict__ part, float* __restrict__ ochunk) {
   __shared__ float wts[kCombineSlots][kMaxG];
@@ -364,8 +375,9 @@ __global__ void __launch_bounds__(256)
   const int b = blockIdx.z, h = blockIdx.y, ch = blockIdx.x, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int64_t bh = (int64_t)b * H + h;
-  const int64_t n_ref = (T_ + s - 1) / s;
+  const int64_t n_ref = n_ref_of(sl.T(b), s);
   const int64_t j0 = (int64_t)ch * kCombineSlots;
+  if (j0 >= n_ref) return;  // past this sequence's references (its final reads n_chunk of its own)
   if (tid < G) {
     const float m = mref[bh * G + tid];
     mrefg[tid] = m;
@@ -401,7 +413,7 @@ __global__ void __launch_bounds__(256)
   __syncthreads();
   // sum_j w_j V_ref_j: thread = (slot group, 8 consecutive elements); every
   // V row segment is loaded once (16 bytes of bf16) for all heads of the group
-  const T* vb = refv + bh * n_ref_cap * d_h;
+  const T* refv = reinterpret_cast<const T*>(cv.base + cv.off_refv);
   const int eg = d_h / 8, e8 = tid % eg, js = tid / eg, njs = blockDim.x / eg;
   float acc[kMaxG][8];
 #pragma unroll
@@ -412,7 +424,7 @@ __global__ void __launch_bounds__(256)
     const int64_t j = j0 + jj;
     if (j >= n_ref) break;
     float v[8];
-    load8(vb + j * d_h + e8 * 8, v);
+    load8(refv + cv.ref_row(bh, j) * d_h + e8 * 8, v);
 #pragma unroll
     for (int g = 0; g < kMaxG; ++g) {
       if (g < G) {
@@ -452,7 +464,7 @@ __global__ void __launch_bounds__(256)
 // ---------------------------------------------------------- decode_final
 template <typename T>
 __global__ void __launch_bounds__(256)
-    decode_final_kernel(int T_, int s, int d_h, int H, int G, int hidden, SlotInfo si, int n_chunk,
+    decode_final_kernel(SeqLens sl, int s, int d_h, int H, int G, int hidden, SlotInfo si,
                         int n_chunk_cap, const T* __restrict__ W4, const float* __restrict__ b4,
                         const float* __restrict__ mref, const float* __restrict__ part,
                         const float* __restrict__ Upart, const float* __restrict__ ochunk,
@@ -463,6 +475,7 @@ __global__ void __launch_bounds__(256)
   const int64_t bh = (int64_t)b * H + h;
   const int ns = slots_of(si, bh);
   const int64_t pb0 = bh * si.nslot_cap;
+  const int n_chunk = (int)((n_ref_of(sl.T(b), s) + kCombineSlots - 1) / kCombineSlots);
   {
     // warp g: the maximum, the token-loop denominator and the reference
     // denominator of head g (the chunks' sums split over the lanes)
@@ -510,24 +523,67 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// ---------------------------------------------------------- decode_sched
+// Sequences of different lengths: their lengths checked against [1, T_max]
+// (an out-of-range length is reported and read as 1) into `lens`, which the
+// other kernels read, and the chunk offsets of the tensor-core token loop:
+// cho[bh] = sum over earlier (sequence, kv-head) pairs of their 128-row
+// chunk counts, cho[BH] the total.  One block.
+__global__ void __launch_bounds__(1024)
+    decode_sched_kernel(const int32_t* __restrict__ Tin, int B, int H, int s, int T_max,
+                        int32_t* __restrict__ lens, int32_t* __restrict__ cho, uint32_t* __restrict__ err) {
+  __shared__ int32_t part[1024];
+  __shared__ int32_t Ts[1024];
+  const int BH = B * H, tid = threadIdx.x;
+  for (int b = tid; b < B; b += blockDim.x) {
+    int32_t t = Tin[b];
+    if (t < 1 || t > T_max) {
+      if (atomicCAS(err, 0u, (uint32_t)DELTAKV_ERR_DEVICE_BOUNDS) == 0u) err[1] = (uint32_t)t;
+      t = 1;
+    }
+    lens[b] = t;
+    if (b < 1024) Ts[b] = t;
+  }
+  __syncthreads();
+  const int32_t* Tb = B <= 1024 ? Ts : lens;
+  const int per = (BH + blockDim.x - 1) / blockDim.x;  // (sequence, kv-head) pairs per thread
+  int32_t sum = 0;
+  for (int i = 0; i < per; ++i) {
+    const int bh = tid * per + i;
+    if (bh < BH) sum += (int32_t)((n_code_of(Tb[bh / H], s) + 127) / 128);
+  }
+  part[tid] = sum;
+  __syncthreads();
+  if (tid == 0) {
+    int32_t run = 0;
+    for (int t = 0; t < (int)blockDim.x; ++t) {
+      const int32_t v = part[t];
+      part[t] = run;
+      run += v;
+    }
+    cho[BH] = run;
+  }
+  __syncthreads();
+  int32_t run = part[tid];
+  for (int i = 0; i < per; ++i) {
+    const int bh = tid * per + i;
+    if (bh < BH) {
+      cho[bh] = run;
+      run += (int32_t)((n_code_of(Tb[bh / H], s) + 127) / 128);
+    }
+  }
+}
+
 // ------------------------------------------------------------- launcher
 template <typename E>
-static cudaError_t decode_launch(const Plan& p, int T, const void* q, int64_t qsb, int64_t qsh,
-                                 const void* cache, const void* W3, const float* b3,
-                                 const void* W4, const float* b4, float* out, int64_t osb,
-                                 int64_t osh, void* ws, cudaStream_t st) {
+static cudaError_t decode_launch(const Plan& p, const CacheView& cv, const SeqLens& sl_in, const void* q, int64_t qsb,
+                                 int64_t qsh, const void* W3, const float* b3, const void* W4, const float* b4,
+                                 float* out, int64_t osb, int64_t osh, void* ws, cudaStream_t st) {
   const auto& c = p.cfg;
   const int H = c.kv_heads, B = c.batch, G = p.G;
-  const int64_t n_ref = n_ref_of(T, c.stride_s);
-  const int64_t n_code = n_code_of(T, c.stride_s);
+  const int64_t n_ref = n_ref_of(sl_in.T_max, c.stride_s);  // the longest sequence's; shorter ones stop early
   const float cs = kLog2e / sqrtf((float)c.d_h);
-  const char* cb = (const char*)cache;
   char* w = (char*)ws;
-  const E* refk = (const E*)(cb + p.off_refk);
-  const E* refv = (const E*)(cb + p.off_refv);
-  const E* code = (const E*)(cb + p.off_code);
-  const __nv_bfloat16* cscale = p.code4 ? (const __nv_bfloat16*)(cb + p.off_cscale) : nullptr;
-  const int32_t* idx = (const int32_t*)(cb + p.off_idx);
   float* S = (float*)(w + p.ws_S);
   float* Smax = (float*)(w + p.ws_Smax);
   float* a = (float*)(w + p.ws_a);
@@ -537,14 +593,25 @@ static cudaError_t decode_launch(const Plan& p, int T, const void* q, int64_t qs
   float* part = (float*)(w + p.ws_part);
   float* Upart = (float*)(w + p.ws_U);
   float* ochunk = (float*)(w + p.ws_ochunk);
+  int32_t* cho = (int32_t*)(w + p.ws_cho);
+  int32_t* lens = cho + (int64_t)B * H + 1;
+  SeqLens sl = sl_in;
+  if (sl.Tb) {
+    // checked lengths and chunk offsets first: every later kernel reads them
+    decode_sched_kernel<<<1, 1024, 0, st>>>(sl_in.Tb, B, H, c.stride_s, sl.T_max, lens, cho, (uint32_t*)ws);
+    cudaError_t e0 = cudaGetLastError();
+    if (e0 != cudaSuccess) return e0;
+    sl.Tb = lens;
+  }
   const int n_refblk = (int)ceil_div64(n_ref, kRefBlockSlots);
   const int n_refblk_cap = (int)ceil_div64(p.n_ref_cap, kRefBlockSlots);
   const int n_chunk = (int)ceil_div64(n_ref, kCombineSlots);
 
   {
     ProfScope ps(p, st, KID_DEC_REF);
-    decode_ref_kernel<E><<<dim3(n_refblk, H, B), 256, 0, st>>>(
-        n_ref, p.n_ref_cap, c.d_h, H, G, cs, (const E*)q, qsb, qsh, refk, S, Smax, n_refblk_cap, wtab);
+    decode_ref_kernel<E><<<dim3(n_refblk, H, B), 256, 0, st>>>(sl, c.stride_s, p.n_ref_cap, c.d_h, H, G, cs,
+                                                               (const E*)q, qsb, qsh, cv, S, Smax, n_refblk_cap,
+                                                               wtab);
   }
   {
     ProfScope ps(p, st, KID_DEC_PREP);
@@ -554,18 +621,22 @@ static cudaError_t decode_launch(const Plan& p, int T, const void* q, int64_t qs
   }
   SlotInfo si{};
   si.nslot_cap = p.nslot_cap;
+  si.BH = B * H;
   cudaError_t e = cudaErrorNotSupported;
   if (decode_tc_supported(p)) {
-    e = launch_decode_tc(p, T, cache, W3, b3, ws, st);
+    const int32_t* chop = sl.Tb ? cho : nullptr;
+    int grid = 0;
+    e = launch_decode_tc(p, cv, sl, chop, W3, b3, ws, st, &grid);
     if (e == cudaSuccess) {
       si.tc = 1;
-      si.n_ch = (int)ceil_div64(n_code, 128);
-      si.N = (int64_t)si.n_ch * B * H;
-      si.grid = decode_tc_grid(p, si.N);
+      si.n_ch = (int)ceil_div64(n_code_of(sl.T_all, c.stride_s), 128);
+      si.cho = chop;
+      si.grid = grid;
     }
   }
   if (e == cudaErrorNotSupported) {
     // splits: enough blocks for about two waves, never more rows than splits
+    const int64_t n_code = n_code_of(sl.T_max, c.stride_s);
     int ns = (int)ceil_div64(2 * kNumSMs, (int64_t)B * H);
     ns = (int)std::min<int64_t>(std::min<int64_t>(ns, p.nslot_cap), std::max<int64_t>(1, n_code / 64));
     size_t base = sizeof(float) * (size_t)(c.d_c * c.hidden + 2 * G * c.hidden + 4 * kMaxG + 8 * c.d_c);
@@ -576,10 +647,9 @@ static cudaError_t decode_launch(const Plan& p, int T, const void* q, int64_t qs
     e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     ProfScope ps(p, st, KID_DEC_STREAM_SIMT);
-    ks<<<dim3(ns, H, B), 256, smem, st>>>(T, c.stride_s, c.d_h, H, G, c.k, c.d_c, c.hidden, (int)c.act, ns,
-                                          p.n_ref_cap, p.n_code_cap, n_refblk, n_refblk_cap, code, cscale, idx,
-                                          (const E*)W3, b3, a, cterm, S, Smax, wtab, part, Upart,
-                                          wt_in_smem, p.nslot_cap, (uint32_t*)ws);
+    ks<<<dim3(ns, H, B), 256, smem, st>>>(sl, c.stride_s, c.d_h, H, G, c.k, c.d_c, c.hidden, (int)c.act, ns,
+                                          p.n_ref_cap, n_refblk, n_refblk_cap, cv, (const E*)W3, b3, a, cterm,
+                                          S, Smax, wtab, part, Upart, wt_in_smem, p.nslot_cap, (uint32_t*)ws);
     e = cudaGetLastError();
     si.tc = 0;
     si.ns = ns;
@@ -588,25 +658,40 @@ static cudaError_t decode_launch(const Plan& p, int T, const void* q, int64_t qs
   {
     ProfScope ps(p, st, KID_DEC_COMBINE);
     decode_combine_kernel<E><<<dim3(n_chunk, H, B), 256, 0, st>>>(
-        T, c.stride_s, c.d_h, H, G, si, p.n_ref_cap, p.n_chunk_cap, refv, S, mref, wtab, part, ochunk);
+        sl, c.stride_s, c.d_h, H, G, si, p.n_ref_cap, p.n_chunk_cap, cv, S, mref, wtab, part, ochunk);
   }
   {
     ProfScope ps(p, st, KID_DEC_FINAL);
     decode_final_kernel<E><<<dim3(1, H, B), 256, 0, st>>>(
-        T, c.stride_s, c.d_h, H, G, c.hidden, si, n_chunk, p.n_chunk_cap, (const E*)W4, b4, mref, part, Upart,
-        ochunk, out, osb, osh);
+        sl, c.stride_s, c.d_h, H, G, c.hidden, si, p.n_chunk_cap, (const E*)W4, b4, mref, part, Upart, ochunk,
+        out, osb, osh);
   }
   return cudaGetLastError();
 }
 
-cudaError_t launch_decode(const Plan& p, int T, const void* q, int64_t qsb, int64_t qsh,
-                          const void* cache, const void* W3, const float* b3, const void* W4,
-                          const float* b4, float* out, int64_t osb, int64_t osh, void* ws,
-                          cudaStream_t st) {
+CacheView contiguous_view(const Plan& p, const void* cache) {
+  CacheView v{};
+  v.base = (const char*)cache;
+  v.off_refk = p.off_refk;
+  v.off_refv = p.off_refv;
+  v.off_code = p.off_code;
+  v.off_idx = p.off_idx;
+  v.off_cscale = p.off_cscale;
+  v.rp = p.n_ref_cap;
+  v.cp = p.n_code_cap;
+  v.n_pages = (int64_t)p.cfg.batch * p.cfg.kv_heads;
+  v.ptab = nullptr;
+  v.max_pages = 1;
+  v.err = nullptr;
+  return v;
+}
+
+cudaError_t launch_decode(const Plan& p, const CacheView& cv, const SeqLens& sl, const void* q, int64_t qsb,
+                          int64_t qsh, const void* W3, const float* b3, const void* W4, const float* b4, float* out,
+                          int64_t osb, int64_t osh, void* ws, cudaStream_t st) {
   if (p.bf16)
-    return decode_launch<__nv_bfloat16>(p, T, q, qsb, qsh, cache, W3, b3, W4, b4, out, osb, osh,
-                                        ws, st);
-  return decode_launch<float>(p, T, q, qsb, qsh, cache, W3, b3, W4, b4, out, osb, osh, ws, st);
+    return decode_launch<__nv_bfloat16>(p, cv, sl, q, qsb, qsh, W3, b3, W4, b4, out, osb, osh, ws, st);
+  return decode_launch<float>(p, cv, sl, q, qsb, qsh, W3, b3, W4, b4, out, osb, osh, ws, st);
 }
 
 }  // namespace dkv

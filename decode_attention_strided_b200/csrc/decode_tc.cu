@@ -43,6 +43,7 @@
 #include <climits>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 
 #include <cuda_fp16.h>
 
@@ -84,9 +85,11 @@ __host__ __device__ inline int64_t dtc_owner(int64_t x, int64_t N, int grid) { r
 
 struct DecTcParams {
   int s, d_h, G, k, d_c, hidden, act, H, BH;
-  int64_t n_code, n_ref, n_ref_cap, n_code_cap;
-  int n_ch;
-  int64_t N;
+  int64_t n_ref_cap;
+  CacheView cv;         // where the codes and slots are (contiguous cache or page pool)
+  SeqLens sl;           // tokens of every sequence
+  int n_ch_all;         // chunks per (sequence, kv-head) when every sequence has T_all tokens
+  const int32_t* cho;   // else chunk offsets per (sequence, kv-head), [BH + 1]
   int grid, nslot_cap, n_refblk, n_refblk_cap;
   int code_swz;        // 32, 64 or 128: bytes per swizzled row of the code tile
   int code_atoms;      // 64-column atoms of the code tile (2 when d_c = 128)
@@ -231,7 +234,7 @@ struct DecLayout {
     zb = o;   o = dtc_align(o + 2 * zb_b);
     u = o;    o = dtc_align(o + 2 * u_b);
     p = o;    o = dtc_align(o + p_b);
-    fl = o;   o += 256 * sizeof(float);
+    fl = o;   o += 128 * sizeof(float);  // 112 used (below)
     bar = o;  o += 32 * 8;
     total = o;
   }
@@ -281,8 +284,38 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
   const int G = P.G, hidden = P.hidden, part_w = hidden / dtc::PARTS;
-  const int64_t x_begin = dtc_begin(blockIdx.x, P.N, P.grid), x_end = dtc_begin(blockIdx.x + 1, P.N, P.grid);
+  // the flattened (sequence, kv-head, chunk) list: chunk x belongs to the
+  // last bh with coff(bh) <= x; every role visits its chunks in order and
+  // walks bh forward from the previous one
+  auto coff = [&](int bh) -> int64_t { return P.cho ? (int64_t)P.cho[bh] : (int64_t)bh * P.n_ch_all; };
+  const int64_t N = coff(P.BH);
+  // the chunks go to the first min(grid, N) CTAs (every one of them gets at
+  // least one, so the CTAs that share a (sequence, kv-head) are consecutive);
+  // the rest have nothing to do
+  const int gridp = (int)(N < P.grid ? N : P.grid);
+  const bool has = (int)blockIdx.x < gridp;
+  const int64_t x_begin = has ? dtc_begin(blockIdx.x, N, gridp) : 0;
+  const int64_t x_end = has ? dtc_begin(blockIdx.x + 1, N, gridp) : 0;
   const int n_local = (int)(x_end - x_begin);
+  int bh_start = 0;
+  if (n_local > 0) {
+    if (!P.cho) {
+      bh_start = (int)(x_begin / P.n_ch_all);
+    } else {
+      int lo = 0, hi = P.BH - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) / 2;
+        if (coff(mid) <= x_begin) lo = mid; else hi = mid - 1;
+      }
+      bh_start = lo;
+    }
+  }
+  auto bh_of = [&](int64_t x, int hint) {
+    int bh = hint;
+    while (bh + 1 < P.BH && coff(bh + 1) <= x) ++bh;
+    return bh;
+  };
+  auto n_code_bh = [&](int bh) -> int64_t { return n_code_of(P.sl.T(bh / P.H), P.s); };
 
   // ---- one-time set-up: W3 (K-major, swizzled like the code tile; bf16, or
   // fp16 next to 4-bit codes, whose expanded values q * scale fp16 holds
@@ -351,16 +384,17 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
       const int swz = P.code_swz, hb = P.d_c / 2;
       bool ok = true;
       int issued = 0;
+      int pbh = bh_start, ebh = bh_start;  // issuing and expanding cursors
       for (int it = 0; it <= n_local && ok; ++it) {
         if (it < n_local) {
           const int64_t x = x_begin + it;
-          const int bh = (int)(x / P.n_ch);
-          const int64_t row0 = (x % P.n_ch) * dtc::CH;
+          pbh = bh_of(x, pbh);
+          const int64_t row0 = (x - coff(pbh)) * dtc::CH;
           const int st = it % NST;
           ok = mbar_wait(&in_empty[st], ((it / NST) & 1) ^ 1, abort_flag);
           if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
           if (lane == 0) {
-            const int64_t prow = (int64_t)bh * P.n_code_cap + row0;
+            const int64_t prow = P.cv.code_row(pbh, row0);
             mbar_arrive_expect_tx(&in_full[st], c4_bytes + s_bytes + idx_bytes);
             bulk_load(sStg(st), P.code4p + prow * hb, c4_bytes, &in_full[st]);
             bulk_load(sStg(st) + c4_bytes, P.cscale + prow, s_bytes, &in_full[st]);
@@ -372,13 +406,15 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
           const int j = it - 1, sj = j % NST;
           ok = mbar_wait(&in_full[sj], (j / NST) & 1, abort_flag);
           if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-          const int64_t row0 = ((x_begin + j) % P.n_ch) * dtc::CH;
+          ebh = bh_of(x_begin + j, ebh);
+          const int64_t row0 = (x_begin + j - coff(ebh)) * dtc::CH;
+          const int64_t n_code = n_code_bh(ebh);
           const uint8_t* c8 = sStg(sj);
           const __nv_bfloat16* sc = reinterpret_cast<const __nv_bfloat16*>(sStg(sj) + c4_bytes);
           unsigned char* tile = sCode(sj);
 #pragma unroll 1
           for (int r = lane; r < dtc::CH; r += 32) {
-            const bool valid = row0 + r < P.n_code;
+            const bool valid = row0 + r < n_code;
             const float scale = valid ? __bfloat162float(sc[r]) : 0.f;
             for (int e8 = 0; e8 < P.d_c; e8 += 8) {
               const uint32_t w = *reinterpret_cast<const uint32_t*>(c8 + r * hb + e8 / 2);  // 8 codes
@@ -416,18 +452,22 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
       const uint32_t code_bytes = (uint32_t)(dtc::CH * P.d_c * 2), idx_bytes = (uint32_t)(dtc::CH * P.k * 4);
       bool ok = true;
       int issued = 0;
+      int bh = bh_start;
       for (int it = 0; it < n_local && ok; ++it) {
         const int64_t x = x_begin + it;
-        const int bh = (int)(x / P.n_ch);
-        const int64_t row0 = (x % P.n_ch) * dtc::CH;
+        bh = bh_of(x, bh);
+        const int64_t row0 = (x - coff(bh)) * dtc::CH;
+        // a chunk never straddles a page: a page holds a multiple of 128 code rows
+        const int64_t prow = P.cv.code_row(bh, row0);
         const int st = it % NST;
         ok = mbar_wait(&in_empty[st], ((it / NST) & 1) ^ 1, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         if (lane == 0) {
           mbar_arrive_expect_tx(&in_full[st], code_bytes + idx_bytes);
           for (int a = 0; a < P.code_atoms; ++a)
-            tma_load_3d(&mapC, &in_full[st], sCode(st) + (size_t)a * dtc::CH * 128, a * 64, (int)row0, bh);
-          bulk_load(sIdx(st), P.idx + ((int64_t)bh * P.n_code_cap + row0) * P.k, idx_bytes, &in_full[st]);
+            tma_load_3d(&mapC, &in_full[st], sCode(st) + (size_t)a * dtc::CH * 128, a * 64, (int)(prow % P.cv.cp),
+                        (int)(prow / P.cv.cp));
+          bulk_load(sIdx(st), P.idx + prow * P.k, idx_bytes, &in_full[st]);
         }
         __syncwarp();
         issued = it + 1;
@@ -486,7 +526,7 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
       } else {
         ok = false;
       }
-      int useg = -1, uprev = -1;
+      int useg = -1, uprev = -1, ubh = bh_start;
       for (int i = 0; i < n_local && ok; ++i) {
         if (i + 1 < n_local) {
           ok = mbar_wait(d1_free, i & 1, abort_flag) && code_wait(i + 1);
@@ -495,7 +535,7 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
           gemm1(i + 1);
         }
         const int jb = i & 1;
-        const int ubh = (int)((x_begin + i) / P.n_ch);
+        ubh = bh_of(x_begin + i, ubh);
         const bool first = ubh != uprev;
         ok = mbar_wait(&p_full[jb], (i >> 1) & 1, abort_flag) &&
              (!first || useg < 0 || mbar_wait(ua_free, useg & 1, abort_flag));
@@ -536,12 +576,20 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
     const int q = warp & 3, n = q * 32 + lane;
     const int hh = aw >> 2;                 // hidden range
     bool ok = true;
-    int prev_bh = -1, seg_count = 0;
+    int prev_bh = -1, seg_count = 0, bh = bh_start;
+    int64_t seg_x0 = 0, seg_ncode = 0;  // the segment's first chunk and row count
     const float* av = sAv(0);
     for (int it = 0; it < n_local && ok; ++it) {
       const int64_t x = x_begin + it;
-      const int bh = (int)(x / P.n_ch);
+      bh = bh_of(x, bh);
       const int ub = it & 1;
+      if (bh != prev_bh) {
+        seg_x0 = coff(bh);
+        seg_ncode = n_code_bh(bh);
+      }
+      // rows past the sequence's last compressed token (the chunk's padding)
+      // hold whatever the buffer holds: their u is zero
+      const bool rvalid = (x - seg_x0) * dtc::CH + n < seg_ncode;
       if (bh != prev_bh) {
         // a_g of this kv-head into the buffer of this segment's parity, as
         // pairs of adjacent hidden units per head (heads >= G zero).  Its
@@ -574,7 +622,10 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
       // is computed (a wait covers every earlier load, so each wait comes
       // right before its sub-block is used)
       uint32_t ra[16], rc[16];
-      auto block = [&](const uint32_t (&r)[16], int c0) {
+      // masked: the chunk holds rows past the sequence's last compressed
+      // token (only the last chunk of a (sequence, kv-head) can); their u is
+      // set to zero (the rows hold whatever the buffer holds)
+      auto block = [&](const uint32_t (&r)[16], int c0, auto masked) {
 #pragma unroll
         for (int v8 = 0; v8 < 2; ++v8) {
           uint4 pk;
@@ -593,6 +644,9 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
               u2 = gelu_tanhfit2(z0, z1);
             } else {
               u2 = make_float2(act_eval(ACT, z0), act_eval(ACT, z1));
+            }
+            if constexpr (decltype(masked)::value) {
+              if (!rvalid) u2 = make_float2(0.f, 0.f);
             }
             h2[x2] = __floats2half2_rn(u2.x, u2.y);
             const float* ap = av + ((c0 + e) >> 1) * GP * 2;
@@ -613,27 +667,34 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
       const int nsb = part_w / 16;  // even: part_w is 32, 64 or 128
-      tmem_ld_issue(trow, ra);
+      auto run = [&](auto masked) {
+        tmem_ld_issue(trow, ra);
 #pragma unroll 1
-      for (int sb = 0; sb < nsb; sb += 2) {
-        const int c0 = hh * part_w + 16 * sb;
-        const bool last = sb + 2 >= nsb;
-        tmem_ld_wait(ra);
-        tmem_ld_issue(trow + 16 * (sb + 1), rc);
-        if (last) {
-          // both last sub-blocks in registers: D1 goes to the next GEMM1 two
-          // sub-blocks before the end of this chunk's work
-          tmem_ld_wait(rc);
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(d1_free);
+        for (int sb = 0; sb < nsb; sb += 2) {
+          const int c0 = hh * part_w + 16 * sb;
+          const bool last = sb + 2 >= nsb;
+          tmem_ld_wait(ra);
+          tmem_ld_issue(trow + 16 * (sb + 1), rc);
+          if (last) {
+            // both last sub-blocks in registers: D1 goes to the next GEMM1
+            // two sub-blocks before the end of this chunk's work
+            tmem_ld_wait(rc);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(d1_free);
+          }
+          block(ra, c0, masked);
+          if (!last) {
+            tmem_ld_wait(rc);
+            tmem_ld_issue(trow + 16 * (sb + 2), ra);
+          }
+          block(rc, c0 + 16, masked);
         }
-        block(ra, c0);
-        if (!last) {
-          tmem_ld_wait(rc);
-          tmem_ld_issue(trow + 16 * (sb + 2), ra);
-        }
-        block(rc, c0 + 16);
+      };
+      if ((x - seg_x0 + 1) * dtc::CH <= seg_ncode) {
+        run(std::false_type{});
+      } else {
+        run(std::true_type{});
       }
       if (!ok) break;
       {
@@ -664,15 +725,18 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
       wsc[g] = 1.f;
     }
     bool ok = true;
-    int prev_bh = -1, seg_first = 0;
+    int prev_bh = -1, seg_first = 0, bh = bh_start;
+    int64_t n_code = 0, n_ref = 0;
     for (int it = 0; it < n_local && ok; ++it) {
       const int64_t x = x_begin + it;
-      const int bh = (int)(x / P.n_ch);
-      const int64_t row0 = (x % P.n_ch) * dtc::CH;
+      bh = bh_of(x, bh);
+      const int64_t row0 = (x - coff(bh)) * dtc::CH;
       const int st = it % NST, zb = it & 1;
       if (bh != prev_bh) {
         prev_bh = bh;
         seg_first = it;
+        n_code = n_code_bh(bh);
+        n_ref = n_ref_of(P.sl.T(bh / P.H), P.s);
         named_bar(3, dtc::SMX * 32);
         if (sw == 0 && lane < G) {
           const int g = lane;
@@ -690,7 +754,7 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
       // the chunk's slots into registers and the reference logits S[idx]
       // requested; the ring stage is then free for the producer
       const int64_t row = row0 + n;
-      const bool valid = row < P.n_code;
+      const bool valid = row < n_code;
       if (!mbar_wait(&in_full[st], (it / NST) & 1, abort_flag)) { ok = false; break; }
       int js[kMaxK];
       {
@@ -707,10 +771,10 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
       for (int i = 0; i < kMaxK; ++i) {
         sv[i] = make_float4(0.f, 0.f, 0.f, 0.f);
         const int j = js[i];
-        if (j >= 0 && j < P.n_ref) {
+        if (j >= 0 && j < n_ref) {
           ++k_eff;
           if (G == 4) sv[i] = __ldg(reinterpret_cast<const float4*>(Sb + (int64_t)j * 4));
-        } else if (j >= P.n_ref) {
+        } else if (j >= n_ref) {
           latch_error(P.err, DELTAKV_ERR_DEVICE_BOUNDS, (uint32_t)j);
           js[i] = -1;
         }
@@ -862,13 +926,13 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
           }
         }
       }
-      const bool seg_end = (it == n_local - 1) || ((x + 1) / P.n_ch != bh);
+      const bool seg_end = (it == n_local - 1) || (x + 1 >= coff(bh + 1));
       if (seg_end) {
         // the segment's U once its last MMA is complete, then its denominator
         ok = mbar_wait(&ua_done[it & 1], (it >> 1) & 1, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         tc_fence_after();
-        const int64_t pb = (int64_t)bh * P.nslot_cap + (int64_t)blockIdx.x - dtc_owner((int64_t)bh * P.n_ch, P.N, P.grid);
+        const int64_t pb = (int64_t)bh * P.nslot_cap + (int64_t)blockIdx.x - dtc_owner(coff(bh), N, gridp);
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
           if (h2 < hidden / 128) {
@@ -963,30 +1027,32 @@ int decode_tc_grid(const Plan& p, int64_t N) {
   return (int)std::min<int64_t>(N, kNumSMs);
 }
 
-cudaError_t launch_decode_tc(const Plan& p, int T, const void* cache, const void* W3, const float* b3,
-                             void* ws, cudaStream_t st) {
+cudaError_t launch_decode_tc(const Plan& p, const CacheView& cv, const SeqLens& sl, const int32_t* cho,
+                             const void* W3, const float* b3, void* ws, cudaStream_t st, int* grid_out) {
   const auto& c = p.cfg;
-  const int64_t n_code = n_code_of(T, c.stride_s);
-  const int n_ch = (int)ceil_div64(n_code, dtc::CH);
   const int BH = c.batch * c.kv_heads;
-  const int64_t N = (int64_t)n_ch * BH;
-  if (N == 0) return cudaSuccess;
-  const char* cb = (const char*)cache;
+  const int n_ch_all = (int)ceil_div64(n_code_of(sl.T_all, c.stride_s), dtc::CH);
+  // with one length for all, the grid covers the chunks; else one CTA per SM
+  // (CTAs past the end of the list have nothing to do)
+  const int grid = cho ? kNumSMs : decode_tc_grid(p, (int64_t)n_ch_all * BH);
+  *grid_out = grid;
+  if (grid == 0) return cudaSuccess;
   char* w = (char*)ws;
   DecTcParams P;
   P.s = c.stride_s; P.d_h = c.d_h; P.G = p.G; P.k = c.k; P.d_c = c.d_c; P.hidden = c.hidden;
   P.act = (int)c.act; P.H = c.kv_heads; P.BH = BH;
-  P.n_code = n_code; P.n_ref = n_ref_of(T, c.stride_s); P.n_ref_cap = p.n_ref_cap; P.n_code_cap = p.n_code_cap;
-  P.n_ch = n_ch; P.N = N; P.grid = decode_tc_grid(p, N); P.nslot_cap = p.nslot_cap;
-  P.n_refblk = (int)ceil_div64(P.n_ref, 64);
+  P.n_ref_cap = p.n_ref_cap;
+  P.cv = cv; P.sl = sl; P.n_ch_all = n_ch_all; P.cho = cho;
+  P.grid = grid; P.nslot_cap = p.nslot_cap;
+  P.n_refblk = (int)ceil_div64(n_ref_of(sl.T_max, c.stride_s), 64);
   P.n_refblk_cap = (int)ceil_div64(p.n_ref_cap, 64);
   P.code_swz = c.d_c >= 64 ? 128 : c.d_c * 2;
   P.code_atoms = c.d_c > 64 ? c.d_c / 64 : 1;
   P.nst = decode_tc_stages(p);
   P.code4 = p.code4 ? 1 : 0;
-  P.code4p = (const uint8_t*)(cb + p.off_code);
-  P.cscale = p.code4 ? (const __nv_bfloat16*)(cb + p.off_cscale) : nullptr;
-  P.idx = (const int32_t*)(cb + p.off_idx);
+  P.code4p = (const uint8_t*)(cv.base + cv.off_code);
+  P.cscale = p.code4 ? (const __nv_bfloat16*)(cv.base + cv.off_cscale) : nullptr;
+  P.idx = (const int32_t*)(cv.base + cv.off_idx);
   P.W3 = (const __nv_bfloat16*)W3; P.b3 = b3;
   P.a = (const float*)(w + p.ws_a); P.cterm = (const float*)(w + p.ws_cterm);
   P.S = (const float*)(w + p.ws_S); P.Smax = (const float*)(w + p.ws_Smax);
@@ -996,14 +1062,16 @@ cudaError_t launch_decode_tc(const Plan& p, int T, const void* cache, const void
   CUtensorMap mapC;
   memset(&mapC, 0, sizeof(mapC));  // unused with 4-bit codes (the producer copies them untiled)
   if (!p.code4) {
-    cuuint64_t dims[3] = {(cuuint64_t)c.d_c, (cuuint64_t)n_code, (cuuint64_t)BH};
-    cuuint64_t str[2] = {(cuuint64_t)c.d_c * 2, (cuuint64_t)p.n_code_cap * c.d_c * 2};
+    // pages of cp code rows; rows past a sequence's last token are loaded
+    // as they are and masked by the activation and softmax warps
+    cuuint64_t dims[3] = {(cuuint64_t)c.d_c, (cuuint64_t)cv.cp, (cuuint64_t)cv.n_pages};
+    cuuint64_t str[2] = {(cuuint64_t)c.d_c * 2, (cuuint64_t)cv.cp * c.d_c * 2};
     cuuint32_t box[3] = {(cuuint32_t)std::min(c.d_c, 64), (cuuint32_t)dtc::CH, 1};
     cuuint32_t es[3] = {1, 1, 1};
     const CUtensorMapSwizzle sw = P.code_swz == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
                                   : P.code_swz == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
                                                      : CU_TENSOR_MAP_SWIZZLE_32B;
-    if (encode_fn_dec()(&mapC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<char*>(cb + p.off_code), dims,
+    if (encode_fn_dec()(&mapC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<char*>(cv.base + cv.off_code), dims,
                         str, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorNotSupported;

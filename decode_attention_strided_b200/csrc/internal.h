@@ -52,7 +52,9 @@ struct Plan {
   int nslot_cap;         // decode partial slots per (b, head)
   int n_chunk_cap;       // combine blocks per (b, head)
   size_t ws_S, ws_Smax, ws_mref, ws_a, ws_cterm, ws_wtab, ws_part, ws_U, ws_ochunk, ws_sparse;
-  size_t ws_decode_end;  // error word + the dense decode's regions (S .. ochunk)
+  size_t ws_cho;         // sequences of different lengths: int32 chunk offsets [batch * kv_heads + 1], then the
+                         // checked lengths [batch]
+  size_t ws_decode_end;  // error word + the dense decode's regions (S .. cho)
   size_t ws_bytes;
 };
 
@@ -67,18 +69,82 @@ struct ProfScope {
   int slot;
 };
 
-inline int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
+__host__ __device__ inline int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Number of references and of compressed rows for a cache of T tokens.
-inline int64_t n_ref_of(int64_t T, int s) { return T <= 0 ? 0 : ceil_div64(T, s); }
-inline int64_t n_code_of(int64_t T, int s) { return T - n_ref_of(T, s); }
+__host__ __device__ inline int64_t n_ref_of(int64_t T, int s) { return T <= 0 ? 0 : ceil_div64(T, s); }
+__host__ __device__ inline int64_t n_code_of(int64_t T, int s) { return T - n_ref_of(T, s); }
 
 struct KVView {
   const void* K;
   const void* V;
   int64_t sb, sh, st;    // element strides: batch, head, token
 };
+
+// Where a decode reads the compressed cache.  Each plane (reference K and V
+// rows, code rows, slot rows, 4-bit scales) is an array of pages; page p
+// holds rp reference rows and cp code rows of one (sequence, kv-head).  The
+// contiguous cache of a plan is the case of one page per (sequence,
+// kv-head): rp = n_ref_cap, cp = n_code_cap, page of (bh, 0) = bh.  A page
+// pool instead maps logical page l of (sequence, kv-head) bh to
+// ptab[bh * max_pages + l].
+struct CacheView {
+  const char* base;
+  size_t off_refk, off_refv, off_code, off_idx, off_cscale;
+  int64_t rp, cp;        // reference rows and code rows per page
+  int64_t n_pages;       // pages in each plane
+  const int32_t* ptab;   // device [batch * kv_heads][max_pages], or null
+  int max_pages;
+  uint32_t* err;         // the workspace error word: a page index outside [0, n_pages) is reported there
+#ifdef __CUDACC__
+  __device__ int64_t page(int64_t bh, int64_t l) const {
+    if (!ptab) return bh;
+    const int64_t pg = ptab[bh * max_pages + l];
+    if (pg < 0 || pg >= n_pages) {  // read page 0 instead (in bounds) and report
+      if (atomicCAS(err, 0u, (uint32_t)DELTAKV_ERR_DEVICE_BOUNDS) == 0u) err[1] = (uint32_t)pg;
+      return 0;
+    }
+    return pg;
+  }
+  // physical row of reference slot j / compressed row r of (sequence, kv-head)
+  // bh; a pool page holds 128 reference rows (rp == 128) and fewer than 2^31
+  // rows of any plane
+  __device__ int64_t ref_row(int64_t bh, int64_t j) const {
+    if (!ptab) return bh * rp + j;
+    return page(bh, j >> 7) * 128 + (j & 127);
+  }
+  __device__ int64_t code_row(int64_t bh, int64_t r) const {
+    if (!ptab) return bh * cp + r;
+    const uint32_t l = (uint32_t)r / (uint32_t)cp;
+    return page(bh, l) * cp + (r - (int64_t)l * cp);
+  }
+#endif
+};
+
+// Token counts of one decode: sequence b holds Tb[b] tokens (a device array)
+// or, when Tb is null, T_all; T_max bounds them all.
+struct SeqLens {
+  const int32_t* Tb;
+  int T_all, T_max;
+  __device__ int T(int b) const { return Tb ? Tb[b] : T_all; }
+};
+
+// The contiguous cache of a plan as a CacheView.
+CacheView contiguous_view(const Plan& p, const void* cache);
+
+// Page pools: 128 blocks of s tokens per page.
+constexpr int kPageRefs = 128;
+struct PoolLayout {
+  int64_t rp, cp;  // reference rows and code rows per page
+  size_t off_refk, off_refv, off_code, off_idx, off_cscale, bytes;
+};
+PoolLayout pool_layout(const Plan& p, int64_t n_pages);
+CacheView pool_view(const Plan& p, const PoolLayout& L, const void* pool, int64_t n_pages, const int32_t* ptab,
+                    int max_pages, void* ws);
+// Copy the contiguous cache of every (sequence, kv-head) (T tokens) into its pages.
+cudaError_t launch_pages_from_cache(const Plan& p, int T, const void* cache, const PoolLayout& L, void* pool,
+                                    int64_t n_pages, const int32_t* ptab, int max_pages, void* ws, cudaStream_t st);
 
 // ---- compress ----
 cudaError_t launch_refpack(const Plan& p, int T, const KVView& kv, void* cache, void* ws,
@@ -108,12 +174,13 @@ cudaError_t launch_reconstruct(const Plan& p, int T, const void* cache, const vo
 // ---- decode ----
 bool decode_tc_supported(const Plan& p);
 int decode_tc_grid(const Plan& p, int64_t N);
-cudaError_t launch_decode_tc(const Plan& p, int T, const void* cache, const void* W3, const float* b3,
-                             void* ws, cudaStream_t st);
-cudaError_t launch_decode(const Plan& p, int T, const void* q, int64_t qsb, int64_t qsh,
-                          const void* cache, const void* W3, const float* b3, const void* W4,
-                          const float* b4, float* out, int64_t osb, int64_t osh, void* ws,
-                          cudaStream_t st);
+// The token loop on the tensor cores; cho: chunk offsets per (sequence,
+// kv-head) when the lengths differ (else null); the grid used goes to *grid.
+cudaError_t launch_decode_tc(const Plan& p, const CacheView& cv, const SeqLens& sl, const int32_t* cho,
+                             const void* W3, const float* b3, void* ws, cudaStream_t st, int* grid);
+cudaError_t launch_decode(const Plan& p, const CacheView& cv, const SeqLens& sl, const void* q, int64_t qsb,
+                          int64_t qsh, const void* W3, const float* b3, const void* W4, const float* b4, float* out,
+                          int64_t osb, int64_t osh, void* ws, cudaStream_t st);
 
 }  // namespace dkv
 

@@ -85,7 +85,8 @@ extern "C" deltakv_status deltakv_decode_attention_noalloc(
   // The array keeps the previous call's contents; only the error word must
   // start at zero (every other region is written before it is read).
   if (cudaMemsetAsync(scratch, 0, kErrBytes, st) != cudaSuccess) return DELTAKV_ERR_CUDA;
-  cudaError_t e = launch_decode(p, T, q, q_strides[0], q_strides[1], cache, W3, b3, W4, b4, out,
-                                out_strides[0], out_strides[1], scratch, st);
+  const SeqLens sl{nullptr, T, T};
+  cudaError_t e = launch_decode(p, contiguous_view(p, cache), sl, q, q_strides[0], q_strides[1], W3, b3, W4, b4,
+                                out, out_strides[0], out_strides[1], scratch, st);
   return e == cudaSuccess ? DELTAKV_OK : DELTAKV_ERR_CUDA;
 }

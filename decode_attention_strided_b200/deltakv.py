@@ -29,7 +29,8 @@ SYMBOLS = ("deltakv_plan", "deltakv_plan_destroy", "deltakv_get_cache_layout", "
            "deltakv_append", "deltakv_decode_attention", "deltakv_decode_attention_sparse",
            "deltakv_decode_attention_noalloc", "deltakv_reconstruct", "deltakv_device_status",
            "deltakv_set_profiling", "deltakv_profile_collect", "deltakv_status_string", "deltakv_version",
-           "deltakv_test_activation")
+           "deltakv_test_activation", "deltakv_page_pool_layout", "deltakv_pages_from_cache",
+           "deltakv_decode_attention_paged")
 
 # forms of deltakv_test_activation (include/deltakv_testing.h)
 TEST_ACT_GELU_ERFF, TEST_ACT_GELU_FAST, TEST_ACT_GELU_FAST2, TEST_ACT_GELU_TANH, TEST_ACT_GELU_TANHFIT2 = 0, 1, 2, 3, 4
@@ -52,6 +53,14 @@ class _Layout(ctypes.Structure):
                 ("code_offset", ctypes.c_size_t), ("idx_offset", ctypes.c_size_t),
                 ("total_bytes", ctypes.c_size_t), ("n_ref_cap", ctypes.c_int64),
                 ("n_code_cap", ctypes.c_int64), ("code_scale_offset", ctypes.c_size_t)]
+
+
+class _PageLayout(ctypes.Structure):
+    _fields_ = [("refs_per_page", ctypes.c_int32), ("codes_per_page", ctypes.c_int32),
+                ("tokens_per_page", ctypes.c_int32), ("n_pages", ctypes.c_int32),
+                ("ref_k_offset", ctypes.c_size_t), ("ref_v_offset", ctypes.c_size_t),
+                ("code_offset", ctypes.c_size_t), ("idx_offset", ctypes.c_size_t),
+                ("code_scale_offset", ctypes.c_size_t), ("pool_bytes", ctypes.c_size_t)]
 
 
 class _KernelTime(ctypes.Structure):
@@ -101,6 +110,13 @@ def load_library(path: str = LIB_PATH):
     lib.deltakv_version.restype = ctypes.c_int32
     lib.deltakv_test_activation.argtypes = [i32, vp, vp, ctypes.c_int64, vp]
     lib.deltakv_test_activation.restype = ctypes.c_int
+    lib.deltakv_page_pool_layout.argtypes = [vp, i32, ctypes.POINTER(_PageLayout)]
+    lib.deltakv_page_pool_layout.restype = ctypes.c_int
+    lib.deltakv_pages_from_cache.argtypes = [vp, i32, vp, vp, i32, vp, i32, vp, sz, vp]
+    lib.deltakv_pages_from_cache.restype = ctypes.c_int
+    lib.deltakv_decode_attention_paged.argtypes = [vp, vp, i32, vp, i64p, vp, i32, vp, i32, vp, vp, vp, vp, vp,
+                                                   i64p, vp, sz, vp]
+    lib.deltakv_decode_attention_paged.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -284,6 +300,54 @@ def decode_attention_noalloc(p: Plan, T: int, q, cache, W3, b3, W4, b4, out, str
     _check("deltakv_decode_attention_noalloc", lib.deltakv_decode_attention_noalloc(
         p.handle, int(T), _ptr(q), qs, _ptr(cache), _ptr(W3), _ptr(b3), _ptr(W4), _ptr(b4), _ptr(out), os_,
         _stream(stream)))
+
+
+def page_pool_layout(p: Plan, n_pages: int) -> dict:
+    """deltakv_page_pool_layout: geometry and plane offsets of a pool of
+    n_pages pages (128 blocks of s tokens each)."""
+    lib = load_library()
+    lay = _PageLayout()
+    _check("deltakv_page_pool_layout", lib.deltakv_page_pool_layout(p.handle, int(n_pages), ctypes.byref(lay)))
+    return {f: getattr(lay, f) for f, _ in _PageLayout._fields_}
+
+
+def alloc_pool(p: Plan, n_pages: int, device="cuda"):
+    """A zeroed page pool of n_pages pages (uint8, pool_bytes)."""
+    return torch.zeros(page_pool_layout(p, n_pages)["pool_bytes"], dtype=torch.uint8, device=device)
+
+
+def _page_table(p: Plan, page_table):
+    if page_table.dtype != torch.int32 or not page_table.is_contiguous() or page_table.dim() != 3 or \
+            tuple(page_table.shape[:2]) != (p.cfg.batch, p.cfg.kv_heads):
+        raise ValueError(f"page_table must be a contiguous int32 tensor [{p.cfg.batch}, {p.cfg.kv_heads}, "
+                         f"max_pages], got {page_table.dtype} {list(page_table.shape)}")
+    return int(page_table.shape[2])
+
+
+def pages_from_cache(p: Plan, T: int, cache, page_table, pool, n_pages: int, workspace, stream=None):
+    """deltakv_pages_from_cache: copy the contiguous cache (T tokens per
+    sequence) into the pool pages page_table [B, H, max_pages] names."""
+    lib = load_library()
+    max_pages = _page_table(p, page_table)
+    _check("deltakv_pages_from_cache", lib.deltakv_pages_from_cache(
+        p.handle, int(T), _ptr(cache), _ptr(page_table), max_pages, _ptr(pool), int(n_pages), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def decode_attention_paged(p: Plan, seq_lens, max_len: int, q, pool, n_pages: int, page_table, W3, b3, W4, b4,
+                           out, workspace, stream=None):
+    """deltakv_decode_attention_paged: decode over a paged cache whose
+    sequences hold seq_lens [B] (int32, device) tokens each."""
+    lib = load_library()
+    if seq_lens.dtype != torch.int32 or not seq_lens.is_contiguous() or seq_lens.numel() != p.cfg.batch:
+        raise ValueError(f"seq_lens must be a contiguous int32 tensor of {p.cfg.batch} lengths")
+    max_pages = _page_table(p, page_table)
+    qs = (ctypes.c_int64 * 2)(q.stride(0), q.stride(1))
+    os_ = (ctypes.c_int64 * 2)(out.stride(0), out.stride(1))
+    _check("deltakv_decode_attention_paged", lib.deltakv_decode_attention_paged(
+        p.handle, _ptr(seq_lens), int(max_len), _ptr(q), qs, _ptr(pool), int(n_pages), _ptr(page_table), max_pages,
+        _ptr(W3), _ptr(b3), _ptr(W4), _ptr(b4), _ptr(out), os_, _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
 def reconstruct(p: Plan, T: int, cache, W3, b3, W4, b4, K_out, V_out, workspace, stream=None):

@@ -257,6 +257,81 @@ deltakv_status deltakv_decode_attention_noalloc(deltakv_plan_t plan, int32_t T,
                                                 float* out, const int64_t out_strides[2],
                                                 deltakv_stream_t stream);
 
+/* ---- Paged compressed cache (section 4, "Implementazione: Sparse-vLLM":
+ * the memory manager that holds the irregular compressed layout, decoupled
+ * from the attention kernels).  The cache of one (sequence, kv-head) is a
+ * list of pages, each 128 consecutive blocks of s tokens: 128 reference
+ * rows, 128 (s - 1) code rows, their slot rows and (4-bit codes) their
+ * scales.  Pages come from a pool shared by the batch; a page table maps
+ * logical page l of (sequence b, kv-head h) to a physical page, so sequences
+ * of different lengths share one pool and grow a page at a time.
+ *
+ * Pool layout: five planes (ref_k, ref_v, code, idx, code_scale), each an
+ * array of n_pages pages; page p of a plane holds its rows p rows_per_page ..
+ * (p + 1) rows_per_page - 1, laid out like the contiguous cache's rows.
+ * Token t of a sequence is in logical page t / tokens_per_page; reference
+ * slot j in page j / refs_per_page, row j mod refs_per_page; compressed row
+ * r (as in the contiguous layout) in page r / codes_per_page, row r mod
+ * codes_per_page. */
+typedef struct {
+    int32_t refs_per_page;    /* 128 */
+    int32_t codes_per_page;   /* 128 (s - 1) */
+    int32_t tokens_per_page;  /* 128 s */
+    int32_t n_pages;
+    size_t ref_k_offset, ref_v_offset, code_offset, idx_offset, code_scale_offset;
+    size_t pool_bytes;        /* 256-byte aligned */
+} deltakv_page_layout;
+
+/* Layout of a pool of n_pages (>= 1) pages for `plan`'s configuration.  No
+ * device work.  Errors: INVALID_ARG. */
+deltakv_status deltakv_page_pool_layout(deltakv_plan_t plan, int32_t n_pages, deltakv_page_layout* out);
+
+/* Copy the compressed cache of every (sequence, kv-head) of `cache` (the
+ * plan's contiguous layout, T tokens per sequence, as deltakv_compress and
+ * deltakv_append write it) into its pages of `pool`:
+ *   page_table : device int32 [B][H][max_pages]; entries of the logical pages
+ *                l < ceil(T / tokens_per_page) name physical pages in
+ *                [0, n_pages) (distinct pages are the caller's business; an
+ *                entry outside the range is skipped and reported as
+ *                DELTAKV_ERR_DEVICE_BOUNDS by deltakv_device_status);
+ *   pool       : device, deltakv_page_pool_layout(n_pages).pool_bytes, 16-byte
+ *                aligned; the rows of the used pages are written, nothing else.
+ *   workspace  : the plan's workspace (its error word only).
+ * Errors: INVALID_ARG (T outside [1, max_T], max_pages too small, NULL),
+ * ALIGNMENT, WORKSPACE, CUDA. */
+deltakv_status deltakv_pages_from_cache(deltakv_plan_t plan, int32_t T, const void* cache,
+                                        const int32_t* page_table, int32_t max_pages,
+                                        void* pool, int32_t n_pages,
+                                        void* workspace, size_t workspace_bytes,
+                                        deltakv_stream_t stream);
+
+/* Decode attention over a paged cache whose sequences may differ in length:
+ * the same result as deltakv_decode_attention on each sequence b alone with
+ * T = seq_lens[b] (up to float32 summation order).
+ *   seq_lens  : device int32 [B], 1 <= seq_lens[b] <= max_len (a length out
+ *               of range is read as 1 and reported as DEVICE_BOUNDS);
+ *   max_len   : host, 1 <= max_len <= max_T, the longest of them;
+ *   pool, n_pages, page_table, max_pages: as for deltakv_pages_from_cache,
+ *               every logical page l < ceil(seq_lens[b] / tokens_per_page)
+ *               of (b, h) mapped (max_pages >= ceil(max_len /
+ *               tokens_per_page)); a page index out of range is read as page
+ *               0 and reported as DEVICE_BOUNDS;
+ *   everything else as for deltakv_decode_attention.
+ * The tensor-core token loop splits the flattened (sequence, kv-head, 128-row
+ * chunk) list evenly over one CTA per SM, so a long sequence among short ones
+ * is shared out like any other work.  Errors: as for
+ * deltakv_decode_attention, plus INVALID_ARG for max_len, n_pages or
+ * max_pages out of range. */
+deltakv_status deltakv_decode_attention_paged(deltakv_plan_t plan, const int32_t* seq_lens, int32_t max_len,
+                                              const void* q, const int64_t q_strides[2],
+                                              const void* pool, int32_t n_pages,
+                                              const int32_t* page_table, int32_t max_pages,
+                                              const void* W3, const float* b3,
+                                              const void* W4, const float* b4,
+                                              float* out, const int64_t out_strides[2],
+                                              void* workspace, size_t workspace_bytes,
+                                              deltakv_stream_t stream);
+
 /* Synchronise `stream`, read and clear the error word that the kernels latch
  * in `workspace`, and return DELTAKV_OK, DEVICE_TIMEOUT or DEVICE_BOUNDS. */
 deltakv_status deltakv_device_status(deltakv_plan_t plan, void* workspace,

@@ -164,3 +164,51 @@ def test_layout_of_4bit_codes(lib):
         with pytest.raises(dkv.DeltaKVError) as ei:
             dkv.plan(_cfg(dtype=dkv.BF16_CODE4, **bad))
         assert ei.value.code == 2
+
+
+def test_page_pool_layout(lib):
+    """A page holds 128 blocks of s tokens: 128 reference rows and 128 (s - 1)
+    code rows; each plane is an array of n_pages pages, 256-byte aligned."""
+    for dtype, code_row in ((dkv.BF16, 64), (dkv.BF16_CODE4, 16)):
+        p = dkv.plan(_cfg(dtype=dtype))
+        L = dkv.page_pool_layout(p, 10)
+        assert (L["refs_per_page"], L["codes_per_page"], L["tokens_per_page"]) == (128, 1920, 2048)
+        assert L["ref_v_offset"] - L["ref_k_offset"] == 10 * 128 * 128 * 2
+        assert L["code_offset"] - L["ref_v_offset"] == 10 * 128 * 128 * 2
+        assert L["idx_offset"] - L["code_offset"] == 10 * 1920 * code_row
+        if dtype == dkv.BF16_CODE4:
+            assert L["code_scale_offset"] == L["idx_offset"] + 10 * 1920 * 4 * 4
+            assert L["pool_bytes"] == L["code_scale_offset"] + 10 * 1920 * 2
+        else:
+            assert L["code_scale_offset"] == 0 and L["pool_bytes"] == L["idx_offset"] + 10 * 1920 * 4 * 4
+        assert all(L[k] % 256 == 0 for k in ("ref_v_offset", "code_offset", "idx_offset", "pool_bytes"))
+    p = dkv.plan(_cfg(stride_s=4))
+    assert dkv.page_pool_layout(p, 1)["codes_per_page"] == 384
+    with pytest.raises(dkv.DeltaKVError):
+        dkv.page_pool_layout(p, 0)
+
+
+def test_paged_calls_reject_bad_arguments_before_any_launch(lib):
+    p = dkv.plan(_cfg(batch=2, kv_heads=1, q_heads=4, max_T=5000))
+    vp = ctypes.c_void_p
+    fake = vp(1 << 20)
+    ws = p.workspace_bytes
+    qs = (ctypes.c_int64 * 2)(4 * 128, 128)
+    dec = lib.deltakv_decode_attention_paged
+    # max_len out of range, no pages, too few pages per sequence for max_len (2048 tokens a page)
+    assert dec(p.handle, fake, 0, fake, qs, fake, 4, fake, 3, fake, None, fake, None, fake, qs, fake, ws, None) == 1
+    assert dec(p.handle, fake, 5001, fake, qs, fake, 4, fake, 3, fake, None, fake, None, fake, qs, fake, ws, None) == 1
+    assert dec(p.handle, fake, 5000, fake, qs, fake, 0, fake, 3, fake, None, fake, None, fake, qs, fake, ws, None) == 1
+    assert dec(p.handle, fake, 5000, fake, qs, fake, 4, fake, 2, fake, None, fake, None, fake, qs, fake, ws, None) == 1
+    # NULL lengths or page table, small workspace, misaligned pool
+    assert dec(p.handle, None, 5000, fake, qs, fake, 4, fake, 3, fake, None, fake, None, fake, qs, fake, ws, None) == 1
+    assert dec(p.handle, fake, 5000, fake, qs, fake, 4, None, 3, fake, None, fake, None, fake, qs, fake, ws, None) == 1
+    assert dec(p.handle, fake, 5000, fake, qs, fake, 4, fake, 3, fake, None, fake, None, fake, qs, fake, ws - 1,
+               None) == 4
+    assert dec(p.handle, fake, 5000, fake, qs, vp((1 << 20) + 8), 4, fake, 3, fake, None, fake, None, fake, qs, fake,
+               ws, None) == 3
+    cp = lib.deltakv_pages_from_cache
+    assert cp(p.handle, 0, fake, fake, 3, fake, 4, fake, ws, None) == 1
+    assert cp(p.handle, 5000, fake, fake, 2, fake, 4, fake, ws, None) == 1
+    assert cp(p.handle, 5000, fake, fake, 3, fake, 4, fake, ws - 1, None) == 4
+    assert cp(p.handle, 5000, fake, vp((1 << 20) + 2), 3, fake, 4, fake, ws, None) == 3
