@@ -184,12 +184,13 @@ __device__ __forceinline__ void unpack_row(const uint4 (&r)[RowPack<EPL>::V4], f
   }
 }
 
-// Sum over the 16 lanes of one row group (`mask` names exactly those lanes).
-__device__ __forceinline__ float group16_sum(float v, unsigned mask) {
-  v += __shfl_xor_sync(mask, v, 8, 16);
-  v += __shfl_xor_sync(mask, v, 4, 16);
-  v += __shfl_xor_sync(mask, v, 2, 16);
-  v += __shfl_xor_sync(mask, v, 1, 16);
+// Sum over the 16 lanes of each row group; the whole warp takes part (a
+// constant full mask: both groups run every shuffle together).
+__device__ __forceinline__ float group16_sum(float v) {
+  v += __shfl_xor_sync(0xffffffffu, v, 8, 16);
+  v += __shfl_xor_sync(0xffffffffu, v, 4, 16);
+  v += __shfl_xor_sync(0xffffffffu, v, 2, 16);
+  v += __shfl_xor_sync(0xffffffffu, v, 1, 16);
   return v;
 }
 
@@ -375,7 +376,6 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
           }
           cj[c] = j;
         }
-        const unsigned gmask = 0xFFFFu << (16 * grp);
         // exact distances, NB candidate rows in flight at a time; with
         // NB == KC the rows stay in registers for the mean
         uint4 rr[NB][RowPack<EPL>::V4];
@@ -410,7 +410,7 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
               asm("mov.b64 {%0, %1}, %2;" : "=f"(e0), "=f"(e1) : "l"(acc));
               part = e0 + e1;
             }
-            part = group16_sum(part, gmask);
+            part = group16_sum(part);
             cd[c0 + u] = cj[c0 + u] >= 0 ? part : FLT_MAX;
           }
         }
@@ -431,7 +431,7 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
         for (int c = 0; c < KC; ++c)
           rank += (cj[c] >= 0 && (cd[c] < my_d || (cd[c] == my_d && cj[c] < my_j))) ? 1 : 0;
         const bool pick = s16 < KC && my_j >= 0 && rank < P.k;
-        const uint32_t chosen = (__ballot_sync(gmask, pick) >> (16 * grp)) & 0xFFFFu;
+        const uint32_t chosen = (__ballot_sync(0xffffffffu, pick) >> (16 * grp)) & 0xFFFFu;
         const int k_eff = min(P.k, n_valid);
         if (g.live) {
           int32_t* idx_row = P.idx + ((int64_t)bh * P.n_code_cap + g.row) * P.k;
