@@ -180,6 +180,7 @@ deltakv_status deltakv_compress(deltakv_plan_t plan, int32_t T, const void* K, c
                                 const int64_t kv_strides[3], const void* W1, const float* b1,
                                 const void* W2, const float* b2, void* cache, void* workspace,
                                 size_t workspace_bytes, deltakv_stream_t stream) {
+  NvtxRange nvtx("deltakv_compress");
   if (!plan) return DELTAKV_ERR_INVALID_ARG;
   const Plan& p = plan->p;
   if (T < 0 || T > p.cfg.max_T) return DELTAKV_ERR_INVALID_ARG;
@@ -212,6 +213,7 @@ deltakv_status deltakv_append(deltakv_plan_t plan, int32_t T0, int32_t T1, const
                               const int64_t kv_strides[3], const void* W1, const float* b1, const void* W2,
                               const float* b2, void* cache, void* workspace, size_t workspace_bytes,
                               deltakv_stream_t stream) {
+  NvtxRange nvtx("deltakv_append");
   if (!plan) return DELTAKV_ERR_INVALID_ARG;
   const Plan& p = plan->p;
   if (T0 < 0 || T1 < T0 || T1 > p.cfg.max_T) return DELTAKV_ERR_INVALID_ARG;
@@ -234,6 +236,7 @@ deltakv_status deltakv_decode_attention(deltakv_plan_t plan, int32_t T, const vo
                                         const float* b4, float* out,
                                         const int64_t out_strides[2], void* workspace,
                                         size_t workspace_bytes, deltakv_stream_t stream) {
+  NvtxRange nvtx("deltakv_decode_attention");
   if (!plan) return DELTAKV_ERR_INVALID_ARG;
   const Plan& p = plan->p;
   if (T < 1 || T > p.cfg.max_T) return DELTAKV_ERR_INVALID_ARG;
@@ -273,6 +276,7 @@ deltakv_status deltakv_page_pool_layout(deltakv_plan_t plan, int32_t n_pages, de
 deltakv_status deltakv_pages_from_cache(deltakv_plan_t plan, int32_t T, const void* cache,
                                         const int32_t* page_table, int32_t max_pages, void* pool, int32_t n_pages,
                                         void* workspace, size_t workspace_bytes, deltakv_stream_t stream) {
+  NvtxRange nvtx("deltakv_pages_from_cache");
   if (!plan) return DELTAKV_ERR_INVALID_ARG;
   const Plan& p = plan->p;
   if (T < 1 || T > p.cfg.max_T || n_pages < 1 || !cache || !page_table || !pool || !workspace)
@@ -293,6 +297,7 @@ deltakv_status deltakv_decode_attention_paged(deltakv_plan_t plan, const int32_t
                                               const void* W3, const float* b3, const void* W4, const float* b4,
                                               float* out, const int64_t out_strides[2], void* workspace,
                                               size_t workspace_bytes, deltakv_stream_t stream) {
+  NvtxRange nvtx("deltakv_decode_attention_paged");
   if (!plan) return DELTAKV_ERR_INVALID_ARG;
   const Plan& p = plan->p;
   if (max_len < 1 || max_len > p.cfg.max_T || n_pages < 1) return DELTAKV_ERR_INVALID_ARG;
@@ -323,6 +328,7 @@ deltakv_status deltakv_decode_attention_sparse(deltakv_plan_t plan, int32_t T, c
                                                const int32_t* tokens, int32_t n_sel, float* out,
                                                const int64_t out_strides[2], void* workspace,
                                                size_t workspace_bytes, deltakv_stream_t stream) {
+  NvtxRange nvtx("deltakv_decode_attention_sparse");
   if (!plan) return DELTAKV_ERR_INVALID_ARG;
   const Plan& p = plan->p;
   if (T < 1 || T > p.cfg.max_T || n_sel < 1) return DELTAKV_ERR_INVALID_ARG;
@@ -345,6 +351,7 @@ deltakv_status deltakv_reconstruct(deltakv_plan_t plan, int32_t T, const void* c
                                    const void* W3, const float* b3, const void* W4,
                                    const float* b4, float* K_out, float* V_out, void* workspace,
                                    size_t workspace_bytes, deltakv_stream_t stream) {
+  NvtxRange nvtx("deltakv_reconstruct");
   if (!plan) return DELTAKV_ERR_INVALID_ARG;
   const Plan& p = plan->p;
   if (T < 0 || T > p.cfg.max_T) return DELTAKV_ERR_INVALID_ARG;

@@ -8,7 +8,19 @@
 
 #include "deltakv.h"
 
+#include <nvtx3/nvToolsExt.h>
+
 namespace dkv {
+
+// An NVTX range over one C-ABI call, named after the call: a tool that
+// records NVTX ranges (nsys, ncu --nvtx) files the call's kernels under that
+// name.  With no tool attached a push or pop costs a test of a null pointer.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 constexpr int kMaxK = 8;          // references per token
 constexpr int kExtraCand = 4;     // extra candidates the distance kernel keeps

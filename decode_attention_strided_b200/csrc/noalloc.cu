@@ -66,6 +66,7 @@ extern "C" deltakv_status deltakv_decode_attention_noalloc(
     deltakv_plan_t plan, int32_t T, const void* q, const int64_t q_strides[2], const void* cache,
     const void* W3, const float* b3, const void* W4, const float* b4, float* out,
     const int64_t out_strides[2], deltakv_stream_t stream) {
+  NvtxRange nvtx("deltakv_decode_attention_noalloc");
   if (!plan) return DELTAKV_ERR_INVALID_ARG;
   const Plan& p = plan->p;
   if (T < 1 || T > p.cfg.max_T) return DELTAKV_ERR_INVALID_ARG;

@@ -337,7 +337,13 @@ deltakv_status deltakv_decode_attention_paged(deltakv_plan_t plan, const int32_t
 deltakv_status deltakv_device_status(deltakv_plan_t plan, void* workspace,
                                      deltakv_stream_t stream);
 
-/* Benchmark support: per-kernel device time.  While profiling is on for a
+/* Tracing: every call that launches kernels (compress, append, the decode
+ * calls, pages_from_cache, reconstruct) opens an NVTX range named after the
+ * call for its duration, so a tool that records NVTX ranges shows each
+ * call's kernels under its name.  Without such a tool the ranges cost a
+ * pointer test each.
+ *
+ * Benchmark support: per-kernel device time.  While profiling is on for a
  * plan, every kernel its calls launch is bracketed by two CUDA events
  * recorded on the call's own stream (host-side bookkeeping only; the kernels
  * are unchanged).  deltakv_profile_collect waits for the recorded events,
