@@ -139,6 +139,23 @@ __device__ __forceinline__ void store_code4_row(uint32_t taddr, const float* b2,
   }
 }
 
+// n / d for 0 <= n < 2^31 by one multiply-high, one add and one shift
+// (division by an invariant integer, Granlund and Montgomery 1994, Thm 4.2:
+// l = ceil(log2 d), m = floor(2^32 (2^l - d) / d) + 1; the add cannot wrap
+// because n < 2^31).
+struct FastDiv {
+  uint32_t m, l;
+  __device__ __forceinline__ uint32_t div(uint32_t n) const { return (__umulhi(n, m) + n) >> l; }
+};
+inline FastDiv make_fastdiv(uint32_t d) {
+  uint32_t l = 0;
+  while (((uint64_t)1 << l) < d) ++l;
+  FastDiv f;
+  f.m = (uint32_t)((((uint64_t)1 << 32) * (((uint64_t)1 << l) - d)) / d + 1);
+  f.l = l;
+  return f;
+}
+
 struct EncParams {
   int T, s, d_h, H, k, d_c, hidden, act, BH;
   int64_t n_code, n_ref, n_ref_cap, n_code_cap;
@@ -157,6 +174,8 @@ struct EncParams {
   const int32_t* cand;
   uint32_t* err;
   int n_tiles, tiles_per_bh;
+  FastDiv div_tiles, div_sm1, div_H;  // by tiles_per_bh, s - 1 and H
+  float inv_k;                          // 1 / k, rounded as the device rounds 1.0f / k
 };
 
 // EPL: elements of [K ; V] per lane with 16 lanes per row (D / 16).
@@ -208,6 +227,7 @@ __device__ __forceinline__ float enc_act(float v) {
 // Row n of a 64-row tile: its code row, token and this lane's x slice.
 struct GatherRow {
   int64_t row, t;
+  int64_t last_ref;        // the latest reference before token t (slot q of row = q (s - 1) + r)
   bool inrow;              // n < ROWS (the last pass of a tile may run past it)
   const __nv_bfloat16* x;  // this lane's slice of x_t (valid when live)
   const int32_t* cand;     // the row's candidate slots
@@ -217,13 +237,20 @@ struct GatherRow {
 template <int KC>
 __device__ __forceinline__ GatherRow gather_row(const EncParams& P, int tile, int n, bool inK, int e0) {
   GatherRow g;
-  const int bh = tile / P.tiles_per_bh;
-  g.row = (int64_t)(tile % P.tiles_per_bh) * enc::ROWS + n;
+  // unsigned 32-bit index arithmetic: tiles, rows and tokens of one
+  // (sequence, kv-head) are below 2^31
+  const uint32_t bh = P.div_tiles.div((uint32_t)tile);
+  const uint32_t row = ((uint32_t)tile - bh * (uint32_t)P.tiles_per_bh) * enc::ROWS + (uint32_t)n;
+  g.row = row;
   g.inrow = n < enc::ROWS;
   g.live = g.inrow && g.row < P.n_code;
-  g.t = g.live ? (g.row / (P.s - 1)) * P.s + (g.row % (P.s - 1)) + 1 : 0;
-  const int b = bh / P.H, h = bh % P.H;
-  g.x = (inK ? P.K + e0 : P.V + (e0 - P.d_h)) + b * P.sb + h * P.sh + g.t * P.st;
+  // row = q (s - 1) + r with r < s - 1 is token t = q s + r + 1 = row + q + 1;
+  // the references before it are slots 0 .. q
+  const uint32_t q = P.div_sm1.div(row);
+  g.t = g.live ? (int64_t)(row + q + 1u) : 0;
+  g.last_ref = q;
+  const uint32_t b = P.div_H.div(bh), h = bh - b * (uint32_t)P.H;
+  g.x = (inK ? P.K + e0 : P.V + (e0 - P.d_h)) + (int64_t)b * P.sb + (int64_t)h * P.sh + g.t * P.st;
   g.cand = P.cand + ((int64_t)bh * P.n_code_cap + g.row) * KC;
   return g;
 }
@@ -370,7 +397,7 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
 #pragma unroll
         for (int c = 0; c < KC; ++c) {
           int j = __shfl_sync(0xffffffffu, myc, c, 16);
-          if (j >= 0 && (int64_t)j * P.s >= g.t) {  // not an earlier reference: drop it
+          if (j >= 0 && j > g.last_ref) {  // not an earlier reference: drop it
             if (s16 == 0) latch_error(P.err, DELTAKV_ERR_DEVICE_BOUNDS, (uint32_t)j);
             j = -1;
           }
@@ -439,7 +466,8 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
           if (s16 >= k_eff && s16 < P.k) idx_row[s16] = -1;
         }
         // r = x - mean of the chosen rows, formed in place as x - sum_c inv r_c
-        const float inv = 1.0f / (float)max(k_eff, 1);
+        // (k_eff < k only for the earliest tokens, which see fewer than k references)
+        const float inv = k_eff == P.k ? P.inv_k : 1.0f / (float)max(k_eff, 1);
 #pragma unroll
         for (int c = 0; c < KC; ++c) {
           if (chosen & (1u << c)) {
@@ -709,6 +737,10 @@ cudaError_t launch_encode_tc(const Plan& p, int T, const KVView& kv, const void*
   P.err = (uint32_t*)ws;
   P.tiles_per_bh = (int)ceil_div64(n_code, enc::ROWS);
   P.n_tiles = P.tiles_per_bh * P.BH;
+  P.div_tiles = make_fastdiv((uint32_t)P.tiles_per_bh);
+  P.div_sm1 = make_fastdiv((uint32_t)(P.s - 1));
+  P.div_H = make_fastdiv((uint32_t)P.H);
+  P.inv_k = 1.0f / (float)c.k;  // IEEE division, correctly rounded on host and device alike
   int dev = 0, sms = kNumSMs;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = std::min(P.n_tiles, sms);
