@@ -107,12 +107,14 @@ def kernel_rooflines(sh, prof, peaks, peak_kind):
     tensor_peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     hbm_peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     out = {}
-    # DRAM bytes per launch from an ncu capture of this build on the 32k
-    # case, scaled by the units processed to the 128k workload (traffic
-    # grows with T and with the decode batch); null for other workloads
+    # DRAM bytes per launch from ncu captures of this build: the distance
+    # and encode kernels on one 128k launch each; the token loop on the 32k
+    # case, scaled by the units processed to the 128k workload (its traffic
+    # grows with T and the decode batch); null for other workloads and for
+    # kernels changed since their capture
     default = (sh.T, sh.Bc, sh.Bd, sh.H, sh.d_h, sh.s, sh.k, sh.d_c, sh.hidden) == \
         (131072, 1, 8, 8, 128, 16, 4, 32, 256)
-    traffic = {"candidates_tc": 598e6, "encode_tc": 614.6e6, "decode_stream_tc": 668.9e6} if default else {}
+    traffic = {"candidates_tc": 624.0e6, "encode_tc": 641.1e6, "decode_stream_tc": 668.9e6} if default else {}
 
     def add(name, bound, work, unit, peak, src):
         if name not in prof:
