@@ -11,8 +11,9 @@
 //      one bf16 scale per row).
 //
 // One persistent CTA per SM, 16 warps with fixed roles, per 64-row tile:
-//   gather warps (11)  16 lanes per token row; the row's x and candidate
-//            slots are loaded one row pass ahead, the k + 4 candidate rows
+//   gather warps (11)  16 lanes per token row, a pair of rows at a time,
+//            pairs claimed from a shared counter in tile order; the next
+//            pair's x and candidate slots are loaded ahead, the k + 4 candidate rows
 //            together when k + 4 = 8 (kept in registers for the mean), four at
 //            a time otherwise; exact fp32 distances, each candidate ranked by
 //            one lane, the chosen set by ballot; r = x - mean -> R tile (64
@@ -290,6 +291,7 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
   EncBars* bars = (EncBars*)(sW2 + (((size_t)hid_atoms * P.d_c * 128 + 1023) & ~size_t(1023)));
   uint32_t* tmem_slot = (uint32_t*)(bars + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+  uint32_t* q_claim = tmem_slot + 2;  // the row-pair counter of the gather
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
 
@@ -305,8 +307,9 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
     *reinterpret_cast<uint4*>(sW2 + sw128_offset(o, c8, P.d_c)) = out;
   }
   if (tid == 0) {
-    mbar_init(&bars->r_full[0], enc::GATHER_WARPS);
-    mbar_init(&bars->r_full[1], enc::GATHER_WARPS);
+    mbar_init(&bars->r_full[0], enc::ROWS / 2);  // one arrival per row pair
+    mbar_init(&bars->r_full[1], enc::ROWS / 2);
+    *q_claim = 0;
     mbar_init(&bars->r_empty[0], 1);
     mbar_init(&bars->r_empty[1], 1);
     mbar_init(&bars->d1_full, 1);
@@ -360,155 +363,176 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
   __syncthreads();
   tc_fence_after();
 
-  if (warp < enc::GATHER_WARPS) {
-    // ------------------------------------ gather: re-rank, mean, residual
-    const int grp = lane >> 4, s16 = lane & 15;  // row within the warp's 2, lane within the row
-    const int e0 = s16 * EPL;                      // this lane's first element of [K ; V]
-    const bool inK = e0 < P.d_h;
-    constexpr int NB = CandBatch<KC>::N;
-    constexpr int PASSES = (enc::ROWS + 2 * enc::GATHER_WARPS - 1) / (2 * enc::GATHER_WARPS);
-    bool ok = true;
-    // The x slice and candidate slot of the next row pass are loaded one pass
-    // ahead, so only the candidate rows' latency sits on a pass's path.
-    uint4 pf_x[RowPack<EPL>::V4];
-    int pf_c = -1;
-    if (n_local > 0) gather_prefetch<EPL, KC>(P, gather_row<KC>(P, blockIdx.x, warp * 2 + grp, inK, e0), s16, pf_x, pf_c);
-    for (int it = 0; it < n_local && ok; ++it) {
-      const int tile = blockIdx.x + it * gridDim.x, rb = it & 1;
-      const int bh = tile / P.tiles_per_bh;
-      // this lane's slice of reference row j: rs + j d_h
-      const __nv_bfloat16* rs = (inK ? P.refk + e0 : P.refv + (e0 - P.d_h)) + (int64_t)bh * P.n_ref_cap * P.d_h;
-      unsigned char* sRb = sR + rb * 2 * r_part;
-      if (it >= 2 && !mbar_wait(&bars->r_empty[rb], ((it >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
-#pragma unroll 1
-      for (int pass = 0; pass < PASSES; ++pass) {
-        const int n = pass * 2 * enc::GATHER_WARPS + warp * 2 + grp;
-        const GatherRow g = gather_row<KC>(P, tile, n, inK, e0);
-        float xr[EPL];
-        unpack_row<EPL>(pf_x, xr);
-        const int myc = pf_c;
-        {
-          const int ntile = pass + 1 < PASSES ? tile : tile + gridDim.x;
-          const int nn = pass + 1 < PASSES ? n + 2 * enc::GATHER_WARPS : warp * 2 + grp;  // may pass ROWS: not live
-          if (ntile < P.n_tiles) gather_prefetch<EPL, KC>(P, gather_row<KC>(P, ntile, nn, inK, e0), s16, pf_x, pf_c);
+  // ---- the gather: exact re-rank, mean, residual, one row pair at a time
+  // A tile's 64 rows are 32 pairs; a warp takes one pair (16 lanes a row).
+  // Pairs are claimed from one counter in shared memory in tile order (claim
+  // c is pair c % 32 of this CTA's tile c / 32), so a warp that finishes
+  // early takes the next pair instead of idling behind a fixed share of the
+  // rows.  Each pair arrives once on its tile's r_full.
+  constexpr int PAIRS = enc::ROWS / 2;
+  const int grp = lane >> 4, s16 = lane & 15;  // row within the pair, lane within the row
+  const int e0 = s16 * EPL;                    // this lane's first element of [K ; V]
+  const bool inK = e0 < P.d_h;
+  constexpr int NB = CandBatch<KC>::N;
+  // The x slice and candidate slot of the next pair are loaded before the
+  // current pair's work, so only the candidate rows' latency sits on its path.
+  uint4 pf_x[RowPack<EPL>::V4];
+  int pf_c = -1;
+  auto claim = [&]() -> uint32_t {
+    uint32_t c = 0;
+    if (lane == 0) c = atomicAdd(q_claim, 1u);
+    return __shfl_sync(0xffffffffu, c, 0);
+  };
+  auto valid = [&](uint32_t c) { return c / PAIRS < (uint32_t)n_local; };
+  auto prefetch = [&](uint32_t c) {
+    const int tile = blockIdx.x + (int)(c / PAIRS) * gridDim.x;
+    gather_prefetch<EPL, KC>(P, gather_row<KC>(P, tile, (int)(c % PAIRS) * 2 + grp, inK, e0), s16, pf_x, pf_c);
+  };
+  // pair c, whose x slices and slots are in pf_x / pf_c; the loads of pair
+  // cn (when valid) are issued before the work
+  auto process = [&](uint32_t c, uint32_t cn) -> bool {
+    const int it = (int)(c / PAIRS), rb = it & 1;
+    const int tile = blockIdx.x + it * gridDim.x;
+    // the R buffer is free once GEMM1 of the tile two back is complete
+    if (it >= 2 && !mbar_wait(&bars->r_empty[rb], ((it >> 1) - 1) & 1, abort_flag)) return false;
+    const int bh = (int)P.div_tiles.div((uint32_t)tile);
+    // this lane's slice of reference row j: rs + j d_h
+    const __nv_bfloat16* rs = (inK ? P.refk + e0 : P.refv + (e0 - P.d_h)) + (int64_t)bh * P.n_ref_cap * P.d_h;
+    unsigned char* sRb = sR + rb * 2 * r_part;
+    const int n = (int)(c % PAIRS) * 2 + grp;
+    const GatherRow g = gather_row<KC>(P, tile, n, inK, e0);
+    float xr[EPL];
+    unpack_row<EPL>(pf_x, xr);
+    const int myc = pf_c;
+    if (valid(cn)) prefetch(cn);
+      int cj[KC];
+      float cd[KC];
+#pragma unroll
+      for (int c = 0; c < KC; ++c) {
+        int j = __shfl_sync(0xffffffffu, myc, c, 16);
+        if (j >= 0 && j > g.last_ref) {  // not an earlier reference: drop it
+          if (s16 == 0) latch_error(P.err, DELTAKV_ERR_DEVICE_BOUNDS, (uint32_t)j);
+          j = -1;
         }
-        int cj[KC];
-        float cd[KC];
+        cj[c] = j;
+      }
+      // exact distances, NB candidate rows in flight at a time; with
+      // NB == KC the rows stay in registers for the mean
+      uint4 rr[NB][RowPack<EPL>::V4];
 #pragma unroll
-        for (int c = 0; c < KC; ++c) {
-          int j = __shfl_sync(0xffffffffu, myc, c, 16);
-          if (j >= 0 && j > g.last_ref) {  // not an earlier reference: drop it
-            if (s16 == 0) latch_error(P.err, DELTAKV_ERR_DEVICE_BOUNDS, (uint32_t)j);
-            j = -1;
-          }
-          cj[c] = j;
+      for (int c0 = 0; c0 < KC; c0 += NB) {
+#pragma unroll
+        for (int u = 0; u < NB; ++u) {
+          const int j = cj[c0 + u];
+          if (j >= 0) load_row<EPL>(rs + (int64_t)j * P.d_h, rr[u]);
         }
-        // exact distances, NB candidate rows in flight at a time; with
-        // NB == KC the rows stay in registers for the mean
-        uint4 rr[NB][RowPack<EPL>::V4];
 #pragma unroll
-        for (int c0 = 0; c0 < KC; c0 += NB) {
-#pragma unroll
-          for (int u = 0; u < NB; ++u) {
-            const int j = cj[c0 + u];
-            if (j >= 0) load_row<EPL>(rs + (int64_t)j * P.d_h, rr[u]);
-          }
-#pragma unroll
-          for (int u = 0; u < NB; ++u) {
-            float part = 0.f;
-            if (cj[c0 + u] >= 0) {
-              // even and odd elements accumulate in the two lanes of a packed
-              // fp32x2 register
-              unsigned long long acc = 0ull;
-#pragma unroll
-              for (int i = 0; i < RowPack<EPL>::V4; ++i) {
-                const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&rr[u][i]);
-#pragma unroll
-                for (int x = 0; x < 4; ++x) {
-                  const float2 v = __bfloat1622float2(p2[x]);
-                  asm("{\n\t.reg .b64 a, b, d;\n\t"
-                      "mov.b64 a, {%1, %2};\n\tmov.b64 b, {%3, %4};\n\t"
-                      "sub.rn.f32x2 d, a, b;\n\tfma.rn.f32x2 %0, d, d, %0;\n\t}"
-                      : "+l"(acc)
-                      : "f"(xr[8 * i + 2 * x]), "f"(xr[8 * i + 2 * x + 1]), "f"(v.x), "f"(v.y));
-                }
-              }
-              float e0, e1;
-              asm("mov.b64 {%0, %1}, %2;" : "=f"(e0), "=f"(e1) : "l"(acc));
-              part = e0 + e1;
-            }
-            part = group16_sum(part);
-            cd[c0 + u] = cj[c0 + u] >= 0 ? part : FLT_MAX;
-          }
-        }
-        // the k smallest (distance, slot), ascending: lane c of the row ranks
-        // candidate c against the others; ranks below k are the references
-        float my_d = FLT_MAX;
-        int my_j = -1, n_valid = 0;
-#pragma unroll
-        for (int c = 0; c < KC; ++c) {
-          if (s16 == c) {
-            my_d = cd[c];
-            my_j = cj[c];
-          }
-          n_valid += cj[c] >= 0 ? 1 : 0;
-        }
-        int rank = 0;
-#pragma unroll
-        for (int c = 0; c < KC; ++c)
-          rank += (cj[c] >= 0 && (cd[c] < my_d || (cd[c] == my_d && cj[c] < my_j))) ? 1 : 0;
-        const bool pick = s16 < KC && my_j >= 0 && rank < P.k;
-        const uint32_t chosen = (__ballot_sync(0xffffffffu, pick) >> (16 * grp)) & 0xFFFFu;
-        const int k_eff = min(P.k, n_valid);
-        if (g.live) {
-          int32_t* idx_row = P.idx + ((int64_t)bh * P.n_code_cap + g.row) * P.k;
-          if (pick) idx_row[rank] = my_j;
-          if (s16 >= k_eff && s16 < P.k) idx_row[s16] = -1;
-        }
-        // r = x - mean of the chosen rows, formed in place as x - sum_c inv r_c
-        // (k_eff < k only for the earliest tokens, which see fewer than k references)
-        const float inv = k_eff == P.k ? P.inv_k : 1.0f / (float)max(k_eff, 1);
-#pragma unroll
-        for (int c = 0; c < KC; ++c) {
-          if (chosen & (1u << c)) {
-            uint4 rc[RowPack<EPL>::V4];
-            if constexpr (NB == KC) {
-#pragma unroll
-              for (int i = 0; i < RowPack<EPL>::V4; ++i) rc[i] = rr[c][i];
-            } else {
-              load_row<EPL>(rs + (int64_t)cj[c] * P.d_h, rc);  // reloaded: it is in L2
-            }
+        for (int u = 0; u < NB; ++u) {
+          float part = 0.f;
+          if (cj[c0 + u] >= 0) {
+            // even and odd elements accumulate in the two lanes of a packed
+            // fp32x2 register
+            unsigned long long acc = 0ull;
 #pragma unroll
             for (int i = 0; i < RowPack<EPL>::V4; ++i) {
-              const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&rc[i]);
+              const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&rr[u][i]);
 #pragma unroll
               for (int x = 0; x < 4; ++x) {
                 const float2 v = __bfloat1622float2(p2[x]);
-                xr[8 * i + 2 * x] = fmaf(-inv, v.x, xr[8 * i + 2 * x]);
-                xr[8 * i + 2 * x + 1] = fmaf(-inv, v.y, xr[8 * i + 2 * x + 1]);
+                asm("{\n\t.reg .b64 a, b, d;\n\t"
+                    "mov.b64 a, {%1, %2};\n\tmov.b64 b, {%3, %4};\n\t"
+                    "sub.rn.f32x2 d, a, b;\n\tfma.rn.f32x2 %0, d, d, %0;\n\t}"
+                    : "+l"(acc)
+                    : "f"(xr[8 * i + 2 * x]), "f"(xr[8 * i + 2 * x + 1]), "f"(v.x), "f"(v.y));
               }
+            }
+            float e0, e1;
+            asm("mov.b64 {%0, %1}, %2;" : "=f"(e0), "=f"(e1) : "l"(acc));
+            part = e0 + e1;
+          }
+          part = group16_sum(part);
+          cd[c0 + u] = cj[c0 + u] >= 0 ? part : FLT_MAX;
+        }
+      }
+      // the k smallest (distance, slot), ascending: lane c of the row ranks
+      // candidate c against the others; ranks below k are the references
+      float my_d = FLT_MAX;
+      int my_j = -1, n_valid = 0;
+#pragma unroll
+      for (int c = 0; c < KC; ++c) {
+        if (s16 == c) {
+          my_d = cd[c];
+          my_j = cj[c];
+        }
+        n_valid += cj[c] >= 0 ? 1 : 0;
+      }
+      int rank = 0;
+#pragma unroll
+      for (int c = 0; c < KC; ++c)
+        rank += (cj[c] >= 0 && (cd[c] < my_d || (cd[c] == my_d && cj[c] < my_j))) ? 1 : 0;
+      const bool pick = s16 < KC && my_j >= 0 && rank < P.k;
+      const uint32_t chosen = (__ballot_sync(0xffffffffu, pick) >> (16 * grp)) & 0xFFFFu;
+      const int k_eff = min(P.k, n_valid);
+      if (g.live) {
+        int32_t* idx_row = P.idx + ((int64_t)bh * P.n_code_cap + g.row) * P.k;
+        if (pick) idx_row[rank] = my_j;
+        if (s16 >= k_eff && s16 < P.k) idx_row[s16] = -1;
+      }
+      // r = x - mean of the chosen rows, formed in place as x - sum_c inv r_c
+      // (k_eff < k only for the earliest tokens, which see fewer than k references)
+      const float inv = k_eff == P.k ? P.inv_k : 1.0f / (float)max(k_eff, 1);
+#pragma unroll
+      for (int c = 0; c < KC; ++c) {
+        if (chosen & (1u << c)) {
+          uint4 rc[RowPack<EPL>::V4];
+          if constexpr (NB == KC) {
+#pragma unroll
+            for (int i = 0; i < RowPack<EPL>::V4; ++i) rc[i] = rr[c][i];
+          } else {
+            load_row<EPL>(rs + (int64_t)cj[c] * P.d_h, rc);  // reloaded: it is in L2
+          }
+#pragma unroll
+          for (int i = 0; i < RowPack<EPL>::V4; ++i) {
+            const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&rc[i]);
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+              const float2 v = __bfloat1622float2(p2[x]);
+              xr[8 * i + 2 * x] = fmaf(-inv, v.x, xr[8 * i + 2 * x]);
+              xr[8 * i + 2 * x + 1] = fmaf(-inv, v.y, xr[8 * i + 2 * x + 1]);
             }
           }
         }
-        // r = hi + lo (fp16) into the R tile: row n, columns e0 .. e0 + EPL
+      }
+      // r = hi + lo (fp16) into the R tile: row n, columns e0 .. e0 + EPL
 #pragma unroll
-        for (int v = 0; v < EPL / 8; ++v) {
-          __half2 hi2[4], lo2[4];
+      for (int v = 0; v < EPL / 8; ++v) {
+        __half2 hi2[4], lo2[4];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int i = 8 * v + 2 * q;
-            split_half2(g.live ? xr[i] : 0.f, g.live ? xr[i + 1] : 0.f, hi2[q], lo2[q]);
-          }
-          if (g.inrow) {
-            const uint32_t off = sw128_offset(n, e0 + 8 * v, enc::ROWS);
-            *reinterpret_cast<uint4*>(sRb + off) = *reinterpret_cast<const uint4*>(hi2);
-            *reinterpret_cast<uint4*>(sRb + r_part + off) = *reinterpret_cast<const uint4*>(lo2);
-          }
+        for (int q = 0; q < 4; ++q) {
+          const int i = 8 * v + 2 * q;
+          split_half2(g.live ? xr[i] : 0.f, g.live ? xr[i + 1] : 0.f, hi2[q], lo2[q]);
+        }
+        if (g.inrow) {
+          const uint32_t off = sw128_offset(n, e0 + 8 * v, enc::ROWS);
+          *reinterpret_cast<uint4*>(sRb + off) = *reinterpret_cast<const uint4*>(hi2);
+          *reinterpret_cast<uint4*>(sRb + r_part + off) = *reinterpret_cast<const uint4*>(lo2);
         }
       }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->r_full[rb]);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars->r_full[rb]);
+    return true;
+  };
+
+  if (warp < enc::GATHER_WARPS) {
+    // ------------------------------------ gather warps: pairs until none is left
+    bool ok = true;
+    uint32_t c = claim();
+    if (valid(c)) prefetch(c);
+    while (ok && valid(c)) {
+      const uint32_t cn = claim();
+      ok = process(c, cn);
+      c = cn;
     }
     if (!ok) {
       if (lane == 0) latch_error(P.err, DELTAKV_ERR_DEVICE_TIMEOUT, 10);
@@ -619,6 +643,11 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->h_full);
+      // this tile's codes wait for GEMM2, which the MMA warp issues after
+      // GEMM1 of the next tile: meanwhile take row pairs of the next tile
+      // (a pair claimed from the tile after it is worked too: its R buffer
+      // is free, GEMM1 of this tile being complete)
+      if (!ok) break;
       // codes = D2 + b2 (TMEM lanes 0-63: the first two activation warps)
       if (!mbar_wait(&bars->d2_full, it & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
