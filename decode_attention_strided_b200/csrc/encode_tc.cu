@@ -13,10 +13,11 @@
 // One persistent CTA per SM, 16 warps with fixed roles, per 64-row tile:
 //   gather warps (11)  16 lanes per token row, a pair of rows at a time,
 //            pairs claimed from a shared counter in tile order; the next
-//            pair's x and candidate slots are loaded ahead, the k + 4 candidate rows
-//            together when k + 4 = 8 (kept in registers for the mean), four at
-//            a time otherwise; exact fp32 distances, each candidate ranked by
-//            one lane, the chosen set by ballot; r = x - mean -> R tile (64
+//            pair's x and candidate slots are loaded ahead, and with k + 4 = 8
+//            its candidate rows too, at the end of the current pair's work
+//            (kept in registers for the mean), else four at a time; exact
+//            fp32 distances, each candidate ranked by one lane, the chosen
+//            set by ballot; r = x - mean -> R tile (64
 //            tokens x D, K-major, hi and lo), double-buffered so the next
 //            tile's gather overlaps
 //   MMA warp  tcgen05.mma  D1^T = W1 . R^T  (A = W1 held in tensor memory
@@ -388,6 +389,30 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
     const int tile = blockIdx.x + (int)(c / PAIRS) * gridDim.x;
     gather_prefetch<EPL, KC>(P, gather_row<KC>(P, tile, (int)(c % PAIRS) * 2 + grp, inK, e0), s16, pf_x, pf_c);
   };
+  // the next pair's candidate slots (checked) and, with k + 4 = 8, its
+  // candidate rows: loaded at the end of the current pair's work
+  uint4 nrr[NB][RowPack<EPL>::V4];
+  int ncj[KC];
+  auto load_cands = [&](uint32_t c) {
+    const int tile = blockIdx.x + (int)(c / PAIRS) * gridDim.x;
+    const GatherRow g = gather_row<KC>(P, tile, (int)(c % PAIRS) * 2 + grp, inK, e0);
+    const int bh = (int)P.div_tiles.div((uint32_t)tile);
+    const __nv_bfloat16* rs = (inK ? P.refk + e0 : P.refv + (e0 - P.d_h)) + (int64_t)bh * P.n_ref_cap * P.d_h;
+#pragma unroll
+    for (int cc = 0; cc < KC; ++cc) {
+      int j = __shfl_sync(0xffffffffu, pf_c, cc, 16);
+      if (j >= 0 && j > g.last_ref) {  // not an earlier reference: drop it
+        if (s16 == 0) latch_error(P.err, DELTAKV_ERR_DEVICE_BOUNDS, (uint32_t)j);
+        j = -1;
+      }
+      ncj[cc] = j;
+    }
+    if constexpr (NB == KC) {
+#pragma unroll
+      for (int u = 0; u < NB; ++u)
+        if (ncj[u] >= 0) load_row<EPL>(rs + (int64_t)ncj[u] * P.d_h, nrr[u]);
+    }
+  };
   // pair c, whose x slices and slots are in pf_x / pf_c; the loads of pair
   // cn (when valid) are issued before the work
   auto process = [&](uint32_t c, uint32_t cn) -> bool {
@@ -403,121 +428,122 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
     const GatherRow g = gather_row<KC>(P, tile, n, inK, e0);
     float xr[EPL];
     unpack_row<EPL>(pf_x, xr);
-    const int myc = pf_c;
+    int cj[KC];
+    float cd[KC];
+#pragma unroll
+    for (int u = 0; u < KC; ++u) cj[u] = ncj[u];
+    uint4 rr[NB][RowPack<EPL>::V4];
+    if constexpr (NB == KC) {
+#pragma unroll
+      for (int u = 0; u < NB; ++u)
+#pragma unroll
+        for (int i = 0; i < RowPack<EPL>::V4; ++i) rr[u][i] = nrr[u][i];
+    }
     if (valid(cn)) prefetch(cn);
-      int cj[KC];
-      float cd[KC];
+    // exact distances; with NB == KC the rows were loaded at the end of the
+    // previous pair and stay in registers for the mean, else NB at a time
 #pragma unroll
-      for (int c = 0; c < KC; ++c) {
-        int j = __shfl_sync(0xffffffffu, myc, c, 16);
-        if (j >= 0 && j > g.last_ref) {  // not an earlier reference: drop it
-          if (s16 == 0) latch_error(P.err, DELTAKV_ERR_DEVICE_BOUNDS, (uint32_t)j);
-          j = -1;
-        }
-        cj[c] = j;
-      }
-      // exact distances, NB candidate rows in flight at a time; with
-      // NB == KC the rows stay in registers for the mean
-      uint4 rr[NB][RowPack<EPL>::V4];
-#pragma unroll
-      for (int c0 = 0; c0 < KC; c0 += NB) {
+    for (int c0 = 0; c0 < KC; c0 += NB) {
+      if constexpr (NB != KC) {
 #pragma unroll
         for (int u = 0; u < NB; ++u) {
           const int j = cj[c0 + u];
           if (j >= 0) load_row<EPL>(rs + (int64_t)j * P.d_h, rr[u]);
         }
-#pragma unroll
-        for (int u = 0; u < NB; ++u) {
-          float part = 0.f;
-          if (cj[c0 + u] >= 0) {
-            // even and odd elements accumulate in the two lanes of a packed
-            // fp32x2 register
-            unsigned long long acc = 0ull;
-#pragma unroll
-            for (int i = 0; i < RowPack<EPL>::V4; ++i) {
-              const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&rr[u][i]);
-#pragma unroll
-              for (int x = 0; x < 4; ++x) {
-                const float2 v = __bfloat1622float2(p2[x]);
-                asm("{\n\t.reg .b64 a, b, d;\n\t"
-                    "mov.b64 a, {%1, %2};\n\tmov.b64 b, {%3, %4};\n\t"
-                    "sub.rn.f32x2 d, a, b;\n\tfma.rn.f32x2 %0, d, d, %0;\n\t}"
-                    : "+l"(acc)
-                    : "f"(xr[8 * i + 2 * x]), "f"(xr[8 * i + 2 * x + 1]), "f"(v.x), "f"(v.y));
-              }
-            }
-            float e0, e1;
-            asm("mov.b64 {%0, %1}, %2;" : "=f"(e0), "=f"(e1) : "l"(acc));
-            part = e0 + e1;
-          }
-          part = group16_sum(part);
-          cd[c0 + u] = cj[c0 + u] >= 0 ? part : FLT_MAX;
-        }
       }
-      // the k smallest (distance, slot), ascending: lane c of the row ranks
-      // candidate c against the others; ranks below k are the references
-      float my_d = FLT_MAX;
-      int my_j = -1, n_valid = 0;
 #pragma unroll
-      for (int c = 0; c < KC; ++c) {
-        if (s16 == c) {
-          my_d = cd[c];
-          my_j = cj[c];
-        }
-        n_valid += cj[c] >= 0 ? 1 : 0;
-      }
-      int rank = 0;
-#pragma unroll
-      for (int c = 0; c < KC; ++c)
-        rank += (cj[c] >= 0 && (cd[c] < my_d || (cd[c] == my_d && cj[c] < my_j))) ? 1 : 0;
-      const bool pick = s16 < KC && my_j >= 0 && rank < P.k;
-      const uint32_t chosen = (__ballot_sync(0xffffffffu, pick) >> (16 * grp)) & 0xFFFFu;
-      const int k_eff = min(P.k, n_valid);
-      if (g.live) {
-        int32_t* idx_row = P.idx + ((int64_t)bh * P.n_code_cap + g.row) * P.k;
-        if (pick) idx_row[rank] = my_j;
-        if (s16 >= k_eff && s16 < P.k) idx_row[s16] = -1;
-      }
-      // r = x - mean of the chosen rows, formed in place as x - sum_c inv r_c
-      // (k_eff < k only for the earliest tokens, which see fewer than k references)
-      const float inv = k_eff == P.k ? P.inv_k : 1.0f / (float)max(k_eff, 1);
-#pragma unroll
-      for (int c = 0; c < KC; ++c) {
-        if (chosen & (1u << c)) {
-          uint4 rc[RowPack<EPL>::V4];
-          if constexpr (NB == KC) {
-#pragma unroll
-            for (int i = 0; i < RowPack<EPL>::V4; ++i) rc[i] = rr[c][i];
-          } else {
-            load_row<EPL>(rs + (int64_t)cj[c] * P.d_h, rc);  // reloaded: it is in L2
-          }
+      for (int u = 0; u < NB; ++u) {
+        float part = 0.f;
+        if (cj[c0 + u] >= 0) {
+          // even and odd elements accumulate in the two lanes of a packed
+          // fp32x2 register
+          unsigned long long acc = 0ull;
 #pragma unroll
           for (int i = 0; i < RowPack<EPL>::V4; ++i) {
-            const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&rc[i]);
+            const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&rr[u][i]);
 #pragma unroll
             for (int x = 0; x < 4; ++x) {
               const float2 v = __bfloat1622float2(p2[x]);
-              xr[8 * i + 2 * x] = fmaf(-inv, v.x, xr[8 * i + 2 * x]);
-              xr[8 * i + 2 * x + 1] = fmaf(-inv, v.y, xr[8 * i + 2 * x + 1]);
+              asm("{\n\t.reg .b64 a, b, d;\n\t"
+                  "mov.b64 a, {%1, %2};\n\tmov.b64 b, {%3, %4};\n\t"
+                  "sub.rn.f32x2 d, a, b;\n\tfma.rn.f32x2 %0, d, d, %0;\n\t}"
+                  : "+l"(acc)
+                  : "f"(xr[8 * i + 2 * x]), "f"(xr[8 * i + 2 * x + 1]), "f"(v.x), "f"(v.y));
             }
+          }
+          float e0, e1;
+          asm("mov.b64 {%0, %1}, %2;" : "=f"(e0), "=f"(e1) : "l"(acc));
+          part = e0 + e1;
+        }
+        part = group16_sum(part);
+        cd[c0 + u] = cj[c0 + u] >= 0 ? part : FLT_MAX;
+      }
+    }
+    // the k smallest (distance, slot), ascending: lane c of the row ranks
+    // candidate c against the others; ranks below k are the references
+    float my_d = FLT_MAX;
+    int my_j = -1, n_valid = 0;
+#pragma unroll
+    for (int c = 0; c < KC; ++c) {
+      if (s16 == c) {
+        my_d = cd[c];
+        my_j = cj[c];
+      }
+      n_valid += cj[c] >= 0 ? 1 : 0;
+    }
+    int rank = 0;
+#pragma unroll
+    for (int c = 0; c < KC; ++c)
+      rank += (cj[c] >= 0 && (cd[c] < my_d || (cd[c] == my_d && cj[c] < my_j))) ? 1 : 0;
+    const bool pick = s16 < KC && my_j >= 0 && rank < P.k;
+    const uint32_t chosen = (__ballot_sync(0xffffffffu, pick) >> (16 * grp)) & 0xFFFFu;
+    const int k_eff = min(P.k, n_valid);
+    if (g.live) {
+      int32_t* idx_row = P.idx + ((int64_t)bh * P.n_code_cap + g.row) * P.k;
+      if (pick) idx_row[rank] = my_j;
+      if (s16 >= k_eff && s16 < P.k) idx_row[s16] = -1;
+    }
+    // r = x - mean of the chosen rows, formed in place as x - sum_c inv r_c
+    // (k_eff < k only for the earliest tokens, which see fewer than k references)
+    const float inv = k_eff == P.k ? P.inv_k : 1.0f / (float)max(k_eff, 1);
+#pragma unroll
+    for (int c = 0; c < KC; ++c) {
+      if (chosen & (1u << c)) {
+        uint4 rc[RowPack<EPL>::V4];
+        if constexpr (NB == KC) {
+#pragma unroll
+          for (int i = 0; i < RowPack<EPL>::V4; ++i) rc[i] = rr[c][i];
+        } else {
+          load_row<EPL>(rs + (int64_t)cj[c] * P.d_h, rc);  // reloaded: it is in L2
+        }
+#pragma unroll
+        for (int i = 0; i < RowPack<EPL>::V4; ++i) {
+          const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&rc[i]);
+#pragma unroll
+          for (int x = 0; x < 4; ++x) {
+            const float2 v = __bfloat1622float2(p2[x]);
+            xr[8 * i + 2 * x] = fmaf(-inv, v.x, xr[8 * i + 2 * x]);
+            xr[8 * i + 2 * x + 1] = fmaf(-inv, v.y, xr[8 * i + 2 * x + 1]);
           }
         }
       }
-      // r = hi + lo (fp16) into the R tile: row n, columns e0 .. e0 + EPL
+    }
+    if (valid(cn)) load_cands(cn);
+    // r = hi + lo (fp16) into the R tile: row n, columns e0 .. e0 + EPL
 #pragma unroll
-      for (int v = 0; v < EPL / 8; ++v) {
-        __half2 hi2[4], lo2[4];
+    for (int v = 0; v < EPL / 8; ++v) {
+      __half2 hi2[4], lo2[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int i = 8 * v + 2 * q;
-          split_half2(g.live ? xr[i] : 0.f, g.live ? xr[i + 1] : 0.f, hi2[q], lo2[q]);
-        }
-        if (g.inrow) {
-          const uint32_t off = sw128_offset(n, e0 + 8 * v, enc::ROWS);
-          *reinterpret_cast<uint4*>(sRb + off) = *reinterpret_cast<const uint4*>(hi2);
-          *reinterpret_cast<uint4*>(sRb + r_part + off) = *reinterpret_cast<const uint4*>(lo2);
-        }
+      for (int q = 0; q < 4; ++q) {
+        const int i = 8 * v + 2 * q;
+        split_half2(g.live ? xr[i] : 0.f, g.live ? xr[i + 1] : 0.f, hi2[q], lo2[q]);
       }
+      if (g.inrow) {
+        const uint32_t off = sw128_offset(n, e0 + 8 * v, enc::ROWS);
+        *reinterpret_cast<uint4*>(sRb + off) = *reinterpret_cast<const uint4*>(hi2);
+        *reinterpret_cast<uint4*>(sRb + r_part + off) = *reinterpret_cast<const uint4*>(lo2);
+      }
+    }
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(&bars->r_full[rb]);
@@ -528,7 +554,10 @@ __global__ void __launch_bounds__(enc::THREADS, 1) encode_tc_kernel(const EncPar
     // ------------------------------------ gather warps: pairs until none is left
     bool ok = true;
     uint32_t c = claim();
-    if (valid(c)) prefetch(c);
+    if (valid(c)) {
+      prefetch(c);
+      load_cands(c);
+    }
     while (ok && valid(c)) {
       const uint32_t cn = claim();
       ok = process(c, cn);
