@@ -31,6 +31,23 @@ namespace dkv {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kRefBlockSlots = 64;
 
+// Eight consecutive elements as floats (16-byte aligned for bf16, 32 for fp32).
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
+  const uint4 r = __ldg(reinterpret_cast<const uint4*>(p));
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&r);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+__device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p)), b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
 // ------------------------------------------------------------ decode_ref
 template <typename T>
 __global__ void __launch_bounds__(256)
@@ -343,22 +360,6 @@ __device__ __forceinline__ int slots_of(const SlotInfo& si, int64_t bh) {
   return (int)(last - first + 1);
 }
 
-// Eight consecutive elements as floats (16-byte aligned for bf16, 32 for fp32).
-__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
-  const uint4 r = __ldg(reinterpret_cast<const uint4*>(p));
-  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&r);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 f = __bfloat1622float2(h[i]);
-    v[2 * i] = f.x;
-    v[2 * i + 1] = f.y;
-  }
-}
-__device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
-  const float4 a = __ldg(reinterpret_cast<const float4*>(p)), b = __ldg(reinterpret_cast<const float4*>(p) + 1);
-  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-}
 
 // -------------------------------------------------------- decode_combine
 // M_g = max(m_ref, split maxima).  For 256 slots: weights
@@ -420,17 +421,32 @@ __global__ void __launch_bounds__(256)
   for (int g = 0; g < kMaxG; ++g)
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[g][i] = 0.f;
-  for (int jj = js; jj < kCombineSlots; jj += njs) {
-    const int64_t j = j0 + jj;
-    if (j >= n_ref) break;
-    float v[8];
-    load8(refv + cv.ref_row(bh, j) * d_h + e8 * 8, v);
+  // four rows' loads in flight at a time
+  for (int jj0 = js; jj0 < kCombineSlots; jj0 += 4 * njs) {
+    float v[4][8];
 #pragma unroll
-    for (int g = 0; g < kMaxG; ++g) {
-      if (g < G) {
-        const float w = wts[jj][g];
+    for (int u = 0; u < 4; ++u) {
+      const int jj = jj0 + u * njs;
+      const int64_t j = j0 + jj;
+      if (jj < kCombineSlots && j < n_ref) {
+        load8(refv + cv.ref_row(bh, j) * d_h + e8 * 8, v[u]);
+      } else {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[g][i] = fmaf(w, v[i], acc[g][i]);
+        for (int i = 0; i < 8; ++i) v[u][i] = 0.f;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int jj = jj0 + u * njs;
+      if (jj < kCombineSlots) {
+#pragma unroll
+        for (int g = 0; g < kMaxG; ++g) {
+          if (g < G) {
+            const float w = wts[jj][g];  // 0 past the sequence's references
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[g][i] = fmaf(w, v[u][i], acc[g][i]);
+          }
+        }
       }
     }
   }
@@ -511,15 +527,44 @@ __global__ void __launch_bounds__(256)
     Ut[g][n] = acc;
   }
   __syncthreads();
+  // the reference chunks' sums: threads over (head, element), chunk loads
+  // independent of one another
+  __shared__ float Oc[kMaxG][128];
   for (int o = tid; o < G * d_h; o += blockDim.x) {
-    int g = o / d_h, e = o - g * d_h;
+    const int g = o / d_h, e = o - g * d_h;
     float acc = 0.f;
+#pragma unroll 8
     for (int c = 0; c < n_chunk; ++c) acc += ochunk[((bh * n_chunk_cap + c) * G + g) * (d_h + 1) + e];
+    Oc[g][e] = acc;
+  }
+  __syncthreads();
+  // W4_V . U: a warp per output element, its lanes over the hidden units
+  // (8 consecutive weights per 16-byte load), every head of the group at once
+  const int warp = tid >> 5, lane = tid & 31;
+  for (int e = warp; e < d_h; e += (int)(blockDim.x >> 5)) {
     const T* w4 = W4 + (int64_t)(d_h + e) * hidden;
-    float y = 0.f;
-    for (int n = 0; n < hidden; ++n) y = fmaf(to_f(w4[n]), Ut[g][n], y);
-    acc += y + (b4 ? b4[d_h + e] * Lnr[g] : 0.f);
-    out[b * osb + (int64_t)(h * G + g) * osh + e] = acc / Lall[g];
+    float y[kMaxG];
+#pragma unroll
+    for (int g = 0; g < kMaxG; ++g) y[g] = 0.f;
+    for (int n0 = lane * 8; n0 < hidden; n0 += 256) {
+      float w[8];
+      load8(w4 + n0, w);
+#pragma unroll
+      for (int g = 0; g < kMaxG; ++g)
+        if (g < G)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) y[g] = fmaf(w[i], Ut[g][n0 + i], y[g]);
+    }
+#pragma unroll
+    for (int g = 0; g < kMaxG; ++g) {
+      if (g < G) {
+        const float yg = warp_sum(y[g]);
+        if (lane == g) {
+          const float acc = Oc[g][e] + yg + (b4 ? b4[d_h + e] * Lnr[g] : 0.f);
+          out[b * osb + (int64_t)(h * G + g) * osh + e] = acc / Lall[g];
+        }
+      }
+    }
   }
 }
 
