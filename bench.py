@@ -114,7 +114,7 @@ def kernel_rooflines(sh, prof, peaks, peak_kind):
     # kernels changed since their capture
     default = (sh.T, sh.Bc, sh.Bd, sh.H, sh.d_h, sh.s, sh.k, sh.d_c, sh.hidden) == \
         (131072, 1, 8, 8, 128, 16, 4, 32, 256)
-    traffic = {"candidates_tc": 624.0e6, "decode_stream_tc": 668.9e6} if default else {}
+    traffic = {"candidates_tc": 624.0e6, "encode_tc": 640.0e6, "decode_stream_tc": 668.9e6} if default else {}
 
     def add(name, bound, work, unit, peak, src):
         if name not in prof:

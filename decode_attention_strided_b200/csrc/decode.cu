@@ -49,63 +49,81 @@ __device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
 }
 
 // ------------------------------------------------------------ decode_ref
+// One thread per reference row (64 rows per CTA): the row's d_h elements
+// with 16-byte loads, every head's dot product at once against the scaled
+// queries in shared memory (stored element-major, so one 16-byte shared load
+// gives four heads), S and the cleared slot weights written as one vector
+// per row.
 template <typename T>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(kRefBlockSlots)
     decode_ref_kernel(SeqLens sl, int s_, int64_t n_ref_cap, int d_h, int H, int G, float c,
                       const T* __restrict__ q, int64_t qsb, int64_t qsh, CacheView cv,
                       float* __restrict__ S, float* __restrict__ Smax, int n_refblk_cap,
                       float* __restrict__ wtab) {
-  __shared__ float qs[kMaxG][128];
-  __shared__ float wmax[8][kMaxG];
-  const int b = blockIdx.z, h = blockIdx.y;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __shared__ __align__(16) float qt[128][kMaxG];  // [element][head]
+  __shared__ float wmax[kRefBlockSlots / 32][kMaxG];
+  const int b = blockIdx.z, h = blockIdx.y, tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
   const int64_t bh = (int64_t)b * H + h;
   const int64_t n_ref = n_ref_of(sl.T(b), s_);
   const T* refk = reinterpret_cast<const T*>(cv.base + cv.off_refk);
-  for (int i = threadIdx.x; i < G * d_h; i += blockDim.x) {
-    int g = i / d_h, e = i - g * d_h;
-    qs[g][e] = c * to_f(q[b * qsb + (int64_t)(h * G + g) * qsh + e]);
+  for (int i = tid; i < kMaxG * d_h; i += blockDim.x) {
+    const int g = i % kMaxG, e = i / kMaxG;
+    qt[e][g] = g < G ? c * to_f(q[b * qsb + (int64_t)(h * G + g) * qsh + e]) : 0.f;
   }
   __syncthreads();
-  float mx[kMaxG];
+  const int64_t j = (int64_t)blockIdx.x * kRefBlockSlots + tid;
+  float acc[kMaxG];
 #pragma unroll
-  for (int g = 0; g < kMaxG; ++g) mx[g] = -INFINITY;
-  for (int i = 0; i < kRefBlockSlots / 8; ++i) {
-    int64_t j = (int64_t)blockIdx.x * kRefBlockSlots + warp * (kRefBlockSlots / 8) + i;
-    if (j >= n_ref) break;
+  for (int g = 0; g < kMaxG; ++g) acc[g] = 0.f;
+  if (j < n_ref) {
     const T* kr = refk + cv.ref_row(bh, j) * d_h;
-    float kv[4];
+#pragma unroll 4
+    for (int e0 = 0; e0 < d_h; e0 += 8) {
+      float v[8];
+      load8(kr + e0, v);
 #pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4) {
-      int e = lane + 32 * q4;
-      kv[q4] = e < d_h ? to_f(kr[e]) : 0.f;
-    }
-#pragma unroll
-    for (int g = 0; g < kMaxG; ++g) {
-      if (g < G) {
-        float acc = 0.f;
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          int e = lane + 32 * q4;
-          if (e < d_h) acc = fmaf(qs[g][e], kv[q4], acc);
-        }
-        acc = warp_sum(acc);
-        mx[g] = fmaxf(mx[g], acc);
-        if (lane == 0) {
-          S[(bh * n_ref_cap + j) * G + g] = acc;
-          wtab[(bh * n_ref_cap + j) * G + g] = 0.f;
+      for (int i = 0; i < 8; ++i) {
+        const float4 qa = *reinterpret_cast<const float4*>(&qt[e0 + i][0]);
+        acc[0] = fmaf(qa.x, v[i], acc[0]);
+        acc[1] = fmaf(qa.y, v[i], acc[1]);
+        acc[2] = fmaf(qa.z, v[i], acc[2]);
+        acc[3] = fmaf(qa.w, v[i], acc[3]);
+        if (G > 4) {
+          const float4 qb = *reinterpret_cast<const float4*>(&qt[e0 + i][4]);
+          acc[4] = fmaf(qb.x, v[i], acc[4]);
+          acc[5] = fmaf(qb.y, v[i], acc[5]);
+          acc[6] = fmaf(qb.z, v[i], acc[6]);
+          acc[7] = fmaf(qb.w, v[i], acc[7]);
         }
       }
     }
-  }
-  if (lane == 0)
+    float* so = S + (bh * n_ref_cap + j) * G;
+    float* wo = wtab + (bh * n_ref_cap + j) * G;
+    if (G == 4) {
+      *reinterpret_cast<float4*>(so) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      *reinterpret_cast<float4*>(wo) = make_float4(0.f, 0.f, 0.f, 0.f);
+    } else {
 #pragma unroll
-    for (int g = 0; g < kMaxG; ++g) wmax[warp][g] = mx[g];
+      for (int g = 0; g < kMaxG; ++g)
+        if (g < G) {
+          so[g] = acc[g];
+          wo[g] = 0.f;
+        }
+    }
+  }
+#pragma unroll
+  for (int g = 0; g < kMaxG; ++g) {
+    float m = j < n_ref ? acc[g] : -INFINITY;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) wmax[warp][g] = m;
+  }
   __syncthreads();
-  if (threadIdx.x < G) {
+  if (tid < G) {
     float m = -INFINITY;
-    for (int w = 0; w < 8; ++w) m = fmaxf(m, wmax[w][threadIdx.x]);
-    Smax[(bh * n_refblk_cap + blockIdx.x) * G + threadIdx.x] = m;
+    for (int w = 0; w < kRefBlockSlots / 32; ++w) m = fmaxf(m, wmax[w][tid]);
+    Smax[(bh * n_refblk_cap + blockIdx.x) * G + tid] = m;
   }
 }
 
@@ -654,7 +672,7 @@ static cudaError_t decode_launch(const Plan& p, const CacheView& cv, const SeqLe
 
   {
     ProfScope ps(p, st, KID_DEC_REF);
-    decode_ref_kernel<E><<<dim3(n_refblk, H, B), 256, 0, st>>>(sl, c.stride_s, p.n_ref_cap, c.d_h, H, G, cs,
+    decode_ref_kernel<E><<<dim3(n_refblk, H, B), kRefBlockSlots, 0, st>>>(sl, c.stride_s, p.n_ref_cap, c.d_h, H, G, cs,
                                                                (const E*)q, qsb, qsh, cv, S, Smax, n_refblk_cap,
                                                                wtab);
   }
