@@ -653,8 +653,9 @@ def max_over_ranks(vals, dev, world):
 
 def run_e2e(sh, w, dev, a, world=1):
     """Same step through the public API with host buffers: every layer's K/V
-    is copied from pinned host memory before its compress call, and every
-    decode copies its queries in and its output back."""
+    is copied from pinned host memory (on a copy stream, into one of two
+    device buffers, so layer l + 1's copy overlaps layer l's compress call),
+    and every decode copies its queries in and its output back."""
     from decode_attention_strided_b200 import deltakv as dkv
     K0, V0 = w["comp_in"][0]
     hK = torch.empty(K0.shape, dtype=K0.dtype, pin_memory=True)
@@ -663,20 +664,35 @@ def run_e2e(sh, w, dev, a, world=1):
     hV.copy_(V0)
     hq = [q.cpu().pin_memory() for q in w["q"]]
     ho = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in w["out"]]
-    dK, dV = torch.empty_like(K0), torch.empty_like(V0)
+    dK = [torch.empty_like(K0) for _ in range(2)]
+    dV = [torch.empty_like(V0) for _ in range(2)]
     dq = torch.empty_like(w["q"][0])
+    main = torch.cuda.current_stream()
+    cs = torch.cuda.Stream(device=main.device)
+    copied = [torch.cuda.Event() for _ in range(2)]
+    consumed = [torch.cuda.Event() for _ in range(2)]
+    used = [False, False]
     h2d = d2h = 0
     steps = max(1, min(a.steps, 3))
     torch.cuda.synchronize()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
     for i in range(steps):
-        ev[i][0].record()
+        ev[i][0].record(main)
+        cs.wait_event(ev[i][0])  # every copy of the step inside the timed region
         for l in range(sh.L):
-            dK.copy_(hK, non_blocking=True)
-            dV.copy_(hV, non_blocking=True)
-            dkv.compress(w["pc"], sh.T, dK, dV, w["W"][l]["W1"], None, w["W"][l]["W2"], None,
+            b = l & 1
+            with torch.cuda.stream(cs):
+                if used[b]:
+                    cs.wait_event(consumed[b])  # the compress call that read this buffer is done
+                dK[b].copy_(hK, non_blocking=True)
+                dV[b].copy_(hV, non_blocking=True)
+                copied[b].record(cs)
+            main.wait_event(copied[b])
+            dkv.compress(w["pc"], sh.T, dK[b], dV[b], w["W"][l]["W1"], None, w["W"][l]["W2"], None,
                          w["comp_cache"][l], w["ws_c"])
-        ev[i][1].record()
+            consumed[b].record(main)
+            used[b] = True
+        ev[i][1].record(main)
         for l in range(sh.L):
             dq.copy_(hq[l], non_blocking=True)
             dkv.decode_attention(w["pd"], sh.T, dq, w["dec_cache"][l], w["W"][l]["W3"], None, w["W"][l]["W4"],
