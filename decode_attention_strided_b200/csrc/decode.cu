@@ -382,7 +382,8 @@ __device__ __forceinline__ int slots_of(const SlotInfo& si, int64_t bh) {
 // -------------------------------------------------------- decode_combine
 // M_g = max(m_ref, split maxima).  For 256 slots: weights
 // w_j = 2^(S_j - M) + 2^(m_ref - M) sum_splits wtab, then sum_j w_j V_ref_j.
-template <typename T>
+// GP: heads per kv-head as laid out in registers (4 or 8, at least G).
+template <typename T, int GP>
 __global__ void __launch_bounds__(256)
     decode_combine_kernel(SeqLens sl, int s, int d_h, int H, int G, SlotInfo si, int64_t n_ref_cap,
                           int n_chunk_cap, CacheView cv, const float* __restrict__ S,
@@ -406,13 +407,13 @@ __global__ void __launch_bounds__(256)
     Mg[tid] = M;
   }
   __syncthreads();
-  float lsum[kMaxG];
+  float lsum[GP];
 #pragma unroll
-  for (int g = 0; g < kMaxG; ++g) lsum[g] = 0.f;
+  for (int g = 0; g < GP; ++g) lsum[g] = 0.f;
   for (int jj = tid; jj < kCombineSlots; jj += blockDim.x) {
     const int64_t j = j0 + jj;
 #pragma unroll
-    for (int g = 0; g < kMaxG; ++g) {
+    for (int g = 0; g < GP; ++g) {
       if (g < G) {
         float w = 0.f;
         if (j < n_ref) {
@@ -425,7 +426,7 @@ __global__ void __launch_bounds__(256)
     }
   }
 #pragma unroll
-  for (int g = 0; g < kMaxG; ++g) {
+  for (int g = 0; g < GP; ++g) {
     const float ls = warp_sum(lsum[g]);
     if (lane == 0 && g < G) lw[warp][g] = ls;
   }
@@ -434,9 +435,9 @@ __global__ void __launch_bounds__(256)
   // V row segment is loaded once (16 bytes of bf16) for all heads of the group
   const T* refv = reinterpret_cast<const T*>(cv.base + cv.off_refv);
   const int eg = d_h / 8, e8 = tid % eg, js = tid / eg, njs = blockDim.x / eg;
-  float acc[kMaxG][8];
+  float acc[GP][8];
 #pragma unroll
-  for (int g = 0; g < kMaxG; ++g)
+  for (int g = 0; g < GP; ++g)
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[g][i] = 0.f;
   // four rows' loads in flight at a time
@@ -458,7 +459,7 @@ __global__ void __launch_bounds__(256)
       const int jj = jj0 + u * njs;
       if (jj < kCombineSlots) {
 #pragma unroll
-        for (int g = 0; g < kMaxG; ++g) {
+        for (int g = 0; g < GP; ++g) {
           if (g < G) {
             const float w = wts[jj][g];  // 0 past the sequence's references
 #pragma unroll
@@ -471,12 +472,12 @@ __global__ void __launch_bounds__(256)
   // lanes that share e8 hold different slot groups: fold them, then the warps
   for (int o = eg; o < 32; o <<= 1)
 #pragma unroll
-    for (int g = 0; g < kMaxG; ++g)
+    for (int g = 0; g < GP; ++g)
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[g][i] += __shfl_xor_sync(0xffffffffu, acc[g][i], o);
   if (lane < eg) {
 #pragma unroll
-    for (int g = 0; g < kMaxG; ++g)
+    for (int g = 0; g < GP; ++g)
       if (g < G)
 #pragma unroll
         for (int i = 0; i < 8; ++i) red[warp][g][e8 * 8 + i] = acc[g][i];
@@ -720,8 +721,12 @@ static cudaError_t decode_launch(const Plan& p, const CacheView& cv, const SeqLe
   if (e != cudaSuccess) return e;
   {
     ProfScope ps(p, st, KID_DEC_COMBINE);
-    decode_combine_kernel<E><<<dim3(n_chunk, H, B), 256, 0, st>>>(
-        sl, c.stride_s, c.d_h, H, G, si, p.n_ref_cap, p.n_chunk_cap, cv, S, mref, wtab, part, ochunk);
+    if (G <= 4)
+      decode_combine_kernel<E, 4><<<dim3(n_chunk, H, B), 256, 0, st>>>(
+          sl, c.stride_s, c.d_h, H, G, si, p.n_ref_cap, p.n_chunk_cap, cv, S, mref, wtab, part, ochunk);
+    else
+      decode_combine_kernel<E, 8><<<dim3(n_chunk, H, B), 256, 0, st>>>(
+          sl, c.stride_s, c.d_h, H, G, si, p.n_ref_cap, p.n_chunk_cap, cv, S, mref, wtab, part, ochunk);
   }
   {
     ProfScope ps(p, st, KID_DEC_FINAL);
