@@ -49,7 +49,7 @@ def test_roofline_fields():
     work = sh.cand_flops_per_layer(1)
     assert c["bound"] == "tensor" and c["unit"] == "TFLOP/s" and c["peak"] == 1000.0
     assert math.isclose(c["achieved"], work / 2.5e-3 / 1e12) and math.isclose(c["frac"], c["achieved"] / 1000.0)
-    assert c["ms_per_launch"] == 2.5 and c["traffic"] == 598e6
+    assert c["ms_per_launch"] == 2.5 and c["traffic"] == 624e6
     d = r["decode_stream_tc"]
     stream = 8 * 8 * (131072 - 8192) * (32 * 2 + 4 * 4)
     assert d["bound"] == "hbm" and math.isclose(d["achieved"], stream / 2e-3 / 1e9)
