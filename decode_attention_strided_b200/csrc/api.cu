@@ -117,6 +117,12 @@ void build_plan(const deltakv_config& c, Plan& p) {
   p.ws_decode_end = w;
   p.ws_sparse = w;  // sparse decode: (m, l, output) of every share
   w = align256(w + (size_t)(BH * kSparseSplits * p.G * (c.d_h + 2)) * 4);
+  p.ws_mult = w;
+  w = align256(w + (size_t)(BH * p.n_ref_cap) * 4);
+  p.ws_rowlist = w;  // room for every selected token of a (sequence, kv-head)
+  w = align256(w + (size_t)(BH * (p.n_code_cap + p.n_ref_cap)) * 4);
+  p.ws_ncode = w;
+  w = align256(w + (size_t)BH * 4);
   p.ws_bytes = std::max(compress_end, w);
 }
 
@@ -343,8 +349,14 @@ deltakv_status deltakv_decode_attention_sparse(deltakv_plan_t plan, int32_t T, c
   if (!aligned16(q) || !aligned16(cache) || !aligned16(W3) || !aligned16(W4) || !aligned16(out) ||
       !aligned16(workspace) || !aligned16(b3) || !aligned16(b4) || !aligned16(tokens))
     return DELTAKV_ERR_ALIGNMENT;
-  return from_cuda(launch_decode_sparse(p, T, q, q_strides[0], q_strides[1], cache, W3, b3, W4, b4, tokens, n_sel,
-                                        out, out_strides[0], out_strides[1], workspace, (cudaStream_t)stream));
+  // the tensor-core token loop over the gathered rows where the plan and the
+  // selection fit it, else the CUDA-core sparse kernels
+  cudaError_t e = launch_decode_sparse_tc(p, T, q, q_strides[0], q_strides[1], cache, W3, b3, W4, b4, tokens, n_sel,
+                                          out, out_strides[0], out_strides[1], workspace, (cudaStream_t)stream);
+  if (e == cudaErrorNotSupported)
+    e = launch_decode_sparse(p, T, q, q_strides[0], q_strides[1], cache, W3, b3, W4, b4, tokens, n_sel, out,
+                             out_strides[0], out_strides[1], workspace, (cudaStream_t)stream);
+  return from_cuda(e);
 }
 
 deltakv_status deltakv_reconstruct(deltakv_plan_t plan, int32_t T, const void* cache,

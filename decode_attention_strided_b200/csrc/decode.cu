@@ -388,7 +388,8 @@ __global__ void __launch_bounds__(256)
     decode_combine_kernel(SeqLens sl, int s, int d_h, int H, int G, SlotInfo si, int64_t n_ref_cap,
                           int n_chunk_cap, CacheView cv, const float* __restrict__ S,
                           const float* __restrict__ mref, const float* __restrict__ wtab_g,
-                          const float* __restrict__ part, float* __restrict__ ochunk) {
+                          const float* __restrict__ part, float* __restrict__ ochunk,
+                          const int32_t* __restrict__ mult) {
   __shared__ float wts[kCombineSlots][kMaxG];
   __shared__ float Mg[kMaxG], mrefg[kMaxG], lw[8][kMaxG];
   __shared__ float red[8][kMaxG][128];
@@ -417,7 +418,10 @@ __global__ void __launch_bounds__(256)
       if (g < G) {
         float w = 0.f;
         if (j < n_ref) {
-          const float own = exp2f(S[(bh * n_ref_cap + j) * G + g] - Mg[g]);
+          // a reference's own term counts once per selection of it (sparse
+          // decode), once otherwise
+          float own = exp2f(S[(bh * n_ref_cap + j) * G + g] - Mg[g]);
+          if (mult) own *= (float)mult[bh * n_ref_cap + j];
           w = own + wtab_g[(bh * n_ref_cap + j) * G + g] * exp2f(mrefg[g] - Mg[g]);
           lsum[g] += own;
         }
@@ -639,10 +643,146 @@ __global__ void __launch_bounds__(1024)
 }
 
 // ------------------------------------------------------------- launcher
+// ------------------------------------------------- sparse selection
+// One block per (sequence, kv-head): the selected reference tokens are
+// counted per slot (a token selected twice counts twice), the selected other
+// tokens' compressed rows listed (in any order) for the token loop, and their
+// number kept; an index outside [0, T) is reported and skipped.
+__global__ void __launch_bounds__(256)
+    sparse_select_kernel(int T, int s, int64_t n_ref_cap, int64_t rl_cap, int n_sel,
+                         const int32_t* __restrict__ tokens, int32_t* __restrict__ mult,
+                         int32_t* __restrict__ rowlist, int32_t* __restrict__ ncode, uint32_t* __restrict__ err) {
+  __shared__ int cnt;
+  const int64_t bh = blockIdx.x;
+  const int64_t n_ref = n_ref_of(T, s);
+  int32_t* m = mult + bh * n_ref_cap;
+  for (int64_t j = threadIdx.x; j < n_ref; j += blockDim.x) m[j] = 0;
+  if (threadIdx.x == 0) cnt = 0;
+  __syncthreads();
+  for (int i = threadIdx.x; i < n_sel; i += blockDim.x) {
+    const int t = tokens[bh * n_sel + i];
+    if (t < 0 || t >= T) {
+      latch_error(err, DELTAKV_ERR_DEVICE_BOUNDS, (uint32_t)t);
+      continue;
+    }
+    if (t % s == 0) {
+      atomicAdd(&m[t / s], 1);
+    } else {
+      const int pos = atomicAdd(&cnt, 1);
+      rowlist[bh * rl_cap + pos] = t - t / s - 1;
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) ncode[bh] = cnt;
+}
+
+// Chunk offsets of the token loop over the listed rows: cho[bh] = sum over
+// earlier (sequence, kv-head) pairs of their 128-row chunk counts.  One block.
+__global__ void __launch_bounds__(1024)
+    sparse_cho_kernel(int BH, const int32_t* __restrict__ ncode, int32_t* __restrict__ cho) {
+  __shared__ int32_t part[1024];
+  const int tid = threadIdx.x;
+  const int per = (BH + blockDim.x - 1) / blockDim.x;
+  int32_t sum = 0;
+  for (int i = 0; i < per; ++i) {
+    const int bh = tid * per + i;
+    if (bh < BH) sum += (ncode[bh] + 127) / 128;
+  }
+  part[tid] = sum;
+  __syncthreads();
+  if (tid == 0) {
+    int32_t run = 0;
+    for (int t = 0; t < (int)blockDim.x; ++t) {
+      const int32_t v = part[t];
+      part[t] = run;
+      run += v;
+    }
+    cho[BH] = run;
+  }
+  __syncthreads();
+  int32_t run = part[tid];
+  for (int i = 0; i < per; ++i) {
+    const int bh = tid * per + i;
+    if (bh < BH) {
+      cho[bh] = run;
+      run += (ncode[bh] + 127) / 128;
+    }
+  }
+}
+
+// The stabilising maximum of a sparse decode, per (sequence, kv-head, head):
+// the largest logit estimate over the selection -- S_j of each selected
+// reference, the mean of S over the slots of each selected other token (its
+// logit less the a . u and constant terms, which the token loop's lazy
+// rescaling absorbs).  The dense decode's maximum over every reference can
+// lie far above all selected logits, and their softmax weights would then
+// underflow in the token loop's fp16 P tile.  One block per (sequence,
+// kv-head); 0 when nothing valid is selected.
+__global__ void __launch_bounds__(256)
+    sparse_mref_kernel(int T, int s, int G, int k, int64_t n_ref_cap, int64_t n_code_cap, int64_t rl_cap,
+                       const float* __restrict__ S, const int32_t* __restrict__ mult,
+                       const int32_t* __restrict__ rowlist, const int32_t* __restrict__ ncode,
+                       const int32_t* __restrict__ idx, float* __restrict__ mref) {
+  __shared__ float red[8][kMaxG];
+  const int64_t bh = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t n_ref = n_ref_of(T, s);
+  const float* Sb = S + bh * n_ref_cap * G;
+  float m[kMaxG];
+#pragma unroll
+  for (int g = 0; g < kMaxG; ++g) m[g] = -INFINITY;
+  for (int64_t j = tid; j < n_ref; j += blockDim.x) {
+    if (mult[bh * n_ref_cap + j] > 0)
+#pragma unroll
+      for (int g = 0; g < kMaxG; ++g)
+        if (g < G) m[g] = fmaxf(m[g], Sb[j * G + g]);
+  }
+  const int nc = ncode[bh];
+  for (int i = tid; i < nc; i += blockDim.x) {
+    const int64_t r = rowlist[bh * rl_cap + i];
+    const int32_t* ir = idx + (bh * n_code_cap + r) * k;
+    float sum[kMaxG];
+#pragma unroll
+    for (int g = 0; g < kMaxG; ++g) sum[g] = 0.f;
+    int ke = 0;
+    for (int q = 0; q < k; ++q) {
+      const int j = ir[q];
+      if (j < 0 || j >= n_ref) continue;
+      ++ke;
+#pragma unroll
+      for (int g = 0; g < kMaxG; ++g)
+        if (g < G) sum[g] += Sb[(int64_t)j * G + g];
+    }
+    if (ke > 0)
+#pragma unroll
+      for (int g = 0; g < kMaxG; ++g)
+        if (g < G) m[g] = fmaxf(m[g], sum[g] / (float)ke);
+  }
+#pragma unroll
+  for (int g = 0; g < kMaxG; ++g) {
+    float v = m[g];
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    if (lane == 0) red[warp][g] = v;
+  }
+  __syncthreads();
+  if (tid < G) {
+    float v = -INFINITY;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) v = fmaxf(v, red[w][tid]);
+    mref[bh * G + tid] = v == -INFINITY ? 0.f : v;
+  }
+}
+
+// Selected tokens of a sparse decode on the tensor-core token loop.
+struct SparseSel {
+  const int32_t* tokens;
+  int n_sel;
+};
+
 template <typename E>
 static cudaError_t decode_launch(const Plan& p, const CacheView& cv, const SeqLens& sl_in, const void* q, int64_t qsb,
                                  int64_t qsh, const void* W3, const float* b3, const void* W4, const float* b4,
-                                 float* out, int64_t osb, int64_t osh, void* ws, cudaStream_t st) {
+                                 float* out, int64_t osb, int64_t osh, void* ws, cudaStream_t st,
+                                 const SparseSel* sel = nullptr) {
   const auto& c = p.cfg;
   const int H = c.kv_heads, B = c.batch, G = p.G;
   const int64_t n_ref = n_ref_of(sl_in.T_max, c.stride_s);  // the longest sequence's; shorter ones stop early
@@ -660,6 +800,24 @@ static cudaError_t decode_launch(const Plan& p, const CacheView& cv, const SeqLe
   int32_t* cho = (int32_t*)(w + p.ws_cho);
   int32_t* lens = cho + (int64_t)B * H + 1;
   SeqLens sl = sl_in;
+  int32_t* mult = nullptr;
+  int32_t* rowlist = nullptr;
+  int32_t* ncode = nullptr;
+  if (sel) {
+    // the selection: reference multiplicities, the listed compressed rows and
+    // the token loop's chunk offsets over them
+    mult = (int32_t*)(w + p.ws_mult);
+    rowlist = (int32_t*)(w + p.ws_rowlist);
+    ncode = (int32_t*)(w + p.ws_ncode);
+    {
+      ProfScope ps(p, st, KID_SPARSE_SELECT);
+      sparse_select_kernel<<<B * H, 256, 0, st>>>(sl.T_all, c.stride_s, p.n_ref_cap, p.n_code_cap + p.n_ref_cap,
+                                                  sel->n_sel, sel->tokens, mult, rowlist, ncode, (uint32_t*)ws);
+      sparse_cho_kernel<<<1, 1024, 0, st>>>(B * H, ncode, cho);
+    }
+    cudaError_t e0 = cudaGetLastError();
+    if (e0 != cudaSuccess) return e0;
+  }
   if (sl.Tb) {
     // checked lengths and chunk offsets first: every later kernel reads them
     decode_sched_kernel<<<1, 1024, 0, st>>>(sl_in.Tb, B, H, c.stride_s, sl.T_max, lens, cho, (uint32_t*)ws);
@@ -683,14 +841,22 @@ static cudaError_t decode_launch(const Plan& p, const CacheView& cv, const SeqLe
                                                          qsh, (const E*)W4, b4, a, cterm, Smax, n_refblk,
                                                          n_refblk_cap, mref);
   }
+  if (sel) {
+    ProfScope ps(p, st, KID_SPARSE_SELECT);
+    sparse_mref_kernel<<<B * H, 256, 0, st>>>(sl.T_all, c.stride_s, G, c.k, p.n_ref_cap, p.n_code_cap,
+                                              p.n_code_cap + p.n_ref_cap, S, mult, rowlist, ncode,
+                                              (const int32_t*)(cv.base + cv.off_idx), mref);
+    cudaError_t e1 = cudaGetLastError();
+    if (e1 != cudaSuccess) return e1;
+  }
   SlotInfo si{};
   si.nslot_cap = p.nslot_cap;
   si.BH = B * H;
   cudaError_t e = cudaErrorNotSupported;
   if (decode_tc_supported(p)) {
-    const int32_t* chop = sl.Tb ? cho : nullptr;
+    const int32_t* chop = (sl.Tb || sel) ? cho : nullptr;
     int grid = 0;
-    e = launch_decode_tc(p, cv, sl, chop, W3, b3, ws, st, &grid);
+    e = launch_decode_tc(p, cv, sl, chop, W3, b3, ws, st, &grid, rowlist, ncode, p.n_code_cap + p.n_ref_cap);
     if (e == cudaSuccess) {
       si.tc = 1;
       si.n_ch = (int)ceil_div64(n_code_of(sl.T_all, c.stride_s), 128);
@@ -698,6 +864,7 @@ static cudaError_t decode_launch(const Plan& p, const CacheView& cv, const SeqLe
       si.grid = grid;
     }
   }
+  if (e == cudaErrorNotSupported && sel) return e;  // the caller takes the CUDA-core sparse kernels
   if (e == cudaErrorNotSupported) {
     // splits: enough blocks for about two waves, never more rows than splits
     const int64_t n_code = n_code_of(sl.T_max, c.stride_s);
@@ -723,10 +890,10 @@ static cudaError_t decode_launch(const Plan& p, const CacheView& cv, const SeqLe
     ProfScope ps(p, st, KID_DEC_COMBINE);
     if (G <= 4)
       decode_combine_kernel<E, 4><<<dim3(n_chunk, H, B), 256, 0, st>>>(
-          sl, c.stride_s, c.d_h, H, G, si, p.n_ref_cap, p.n_chunk_cap, cv, S, mref, wtab, part, ochunk);
+          sl, c.stride_s, c.d_h, H, G, si, p.n_ref_cap, p.n_chunk_cap, cv, S, mref, wtab, part, ochunk, mult);
     else
       decode_combine_kernel<E, 8><<<dim3(n_chunk, H, B), 256, 0, st>>>(
-          sl, c.stride_s, c.d_h, H, G, si, p.n_ref_cap, p.n_chunk_cap, cv, S, mref, wtab, part, ochunk);
+          sl, c.stride_s, c.d_h, H, G, si, p.n_ref_cap, p.n_chunk_cap, cv, S, mref, wtab, part, ochunk, mult);
   }
   {
     ProfScope ps(p, st, KID_DEC_FINAL);
@@ -752,6 +919,20 @@ CacheView contiguous_view(const Plan& p, const void* cache) {
   v.max_pages = 1;
   v.err = nullptr;
   return v;
+}
+
+cudaError_t launch_decode_sparse_tc(const Plan& p, int T, const void* q, int64_t qsb, int64_t qsh, const void* cache,
+                                    const void* W3, const float* b3, const void* W4, const float* b4,
+                                    const int32_t* tokens, int n_sel, float* out, int64_t osb, int64_t osh, void* ws,
+                                    cudaStream_t st) {
+  // the row list holds up to n_code_cap + n_ref_cap entries per (sequence, kv-head)
+  if (!decode_tc_supported(p) || p.code4 || (int64_t)n_sel > p.n_code_cap + p.n_ref_cap) return cudaErrorNotSupported;
+  const SparseSel sel{tokens, n_sel};
+  const CacheView cv = contiguous_view(p, cache);
+  const SeqLens sl{nullptr, T, T};
+  if (p.bf16)
+    return decode_launch<__nv_bfloat16>(p, cv, sl, q, qsb, qsh, W3, b3, W4, b4, out, osb, osh, ws, st, &sel);
+  return decode_launch<float>(p, cv, sl, q, qsb, qsh, W3, b3, W4, b4, out, osb, osh, ws, st, &sel);
 }
 
 cudaError_t launch_decode(const Plan& p, const CacheView& cv, const SeqLens& sl, const void* q, int64_t qsb,

@@ -90,6 +90,11 @@ struct DecTcParams {
   SeqLens sl;           // tokens of every sequence
   int n_ch_all;         // chunks per (sequence, kv-head) when every sequence has T_all tokens
   const int32_t* cho;   // else chunk offsets per (sequence, kv-head), [BH + 1]
+  // Gathered rows (sparse decode): the compressed rows of (sequence, kv-head)
+  // bh are rowlist[bh * rl_cap + i], i < ncode[bh], not rows 0 .. n_code - 1
+  const int32_t* rowlist;
+  const int32_t* ncode;
+  int64_t rl_cap;
   int grid, nslot_cap, n_refblk, n_refblk_cap;
   int code_swz;        // 32, 64 or 128: bytes per swizzled row of the code tile
   int code_atoms;      // 64-column atoms of the code tile (2 when d_c = 128)
@@ -315,7 +320,9 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
     while (bh + 1 < P.BH && coff(bh + 1) <= x) ++bh;
     return bh;
   };
-  auto n_code_bh = [&](int bh) -> int64_t { return n_code_of(P.sl.T(bh / P.H), P.s); };
+  auto n_code_bh = [&](int bh) -> int64_t {
+    return P.ncode ? (int64_t)P.ncode[bh] : n_code_of(P.sl.T(bh / P.H), P.s);
+  };
 
   // ---- one-time set-up: W3 (K-major, swizzled like the code tile; bf16, or
   // fp16 next to 4-bit codes, whose expanded values q * scale fp16 holds
@@ -372,7 +379,50 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == dtc::PRODUCER && P.code4) {
+  if (warp == dtc::PRODUCER && P.rowlist) {
+    // ------------------------------------------ producer, gathered rows
+    // the chunk's rows are entries of the (sequence, kv-head)'s row list: the
+    // warp copies each row's codes into the swizzled code tile and its slots
+    // into the slot tile with plain loads and stores (rows past the list's
+    // end: zero codes, no slots), then marks the stage full
+    if (n_local > 0) {
+      bool ok = true;
+      int bh = bh_start;
+      const int swz = P.code_swz, row_elems = swz / 2;
+      const char* cbase = P.cv.base + P.cv.off_code;
+      for (int it = 0; it < n_local && ok; ++it) {
+        const int64_t x = x_begin + it;
+        bh = bh_of(x, bh);
+        const int64_t row0 = (x - coff(bh)) * dtc::CH;
+        const int64_t n_code = n_code_bh(bh);
+        const int st = it % NST;
+        ok = mbar_wait(&in_empty[st], ((it / NST) & 1) ^ 1, abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        unsigned char* tile = sCode(st);
+        int32_t* sidx = sIdx(st);
+#pragma unroll 1
+        for (int r = lane; r < dtc::CH; r += 32) {
+          const bool valid = row0 + r < n_code;
+          const int64_t cr = valid ? (int64_t)P.rowlist[(int64_t)bh * P.rl_cap + row0 + r] : 0;
+          const int64_t prow = P.cv.code_row(bh, cr);
+          const uint4* src = reinterpret_cast<const uint4*>(cbase + prow * P.d_c * 2);
+          for (int e = 0; e < P.d_c; e += 8) {  // 16 bytes: 8 bf16 codes
+            const uint4 v = valid ? __ldg(src + e / 8) : make_uint4(0u, 0u, 0u, 0u);
+            const int atom = e / row_elems, col = e % row_elems;
+            *reinterpret_cast<uint4*>(tile + (size_t)atom * dtc::CH * swz + swz_off(r, col * 2, swz)) = v;
+          }
+          for (int kk = 0; kk < P.k; ++kk) sidx[r * P.k + kk] = valid ? __ldg(P.idx + prow * P.k + kk) : -1;
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&in_full[st]);
+      }
+      if (!ok && lane == 0) {
+        latch_error(P.err, DELTAKV_ERR_DEVICE_TIMEOUT, 20);
+        *abort_flag = 1;
+      }
+    }
+  } else if (warp == dtc::PRODUCER && P.code4) {
     // -------------------------------------------- producer, 4-bit codes
     // lane 0 issues chunk it's copies (packed codes and scales into the
     // stage's staging area, slots into its slot area); then the warp expands
@@ -1028,7 +1078,8 @@ int decode_tc_grid(const Plan& p, int64_t N) {
 }
 
 cudaError_t launch_decode_tc(const Plan& p, const CacheView& cv, const SeqLens& sl, const int32_t* cho,
-                             const void* W3, const float* b3, void* ws, cudaStream_t st, int* grid_out) {
+                             const void* W3, const float* b3, void* ws, cudaStream_t st, int* grid_out,
+                             const int32_t* rowlist, const int32_t* ncode, int64_t rl_cap) {
   const auto& c = p.cfg;
   const int BH = c.batch * c.kv_heads;
   const int n_ch_all = (int)ceil_div64(n_code_of(sl.T_all, c.stride_s), dtc::CH);
@@ -1043,6 +1094,7 @@ cudaError_t launch_decode_tc(const Plan& p, const CacheView& cv, const SeqLens& 
   P.act = (int)c.act; P.H = c.kv_heads; P.BH = BH;
   P.n_ref_cap = p.n_ref_cap;
   P.cv = cv; P.sl = sl; P.n_ch_all = n_ch_all; P.cho = cho;
+  P.rowlist = rowlist; P.ncode = ncode; P.rl_cap = rl_cap;
   P.grid = grid; P.nslot_cap = p.nslot_cap;
   P.n_refblk = (int)ceil_div64(n_ref_of(sl.T_max, c.stride_s), 64);
   P.n_refblk_cap = (int)ceil_div64(p.n_ref_cap, 64);

@@ -39,7 +39,7 @@ constexpr size_t kErrBytes = 256;
 enum KernelId {
   KID_REFPACK = 0, KID_CAND_SIMT, KID_CAND_TC, KID_ENCODE_SIMT, KID_ENCODE_TC, KID_RECONSTRUCT, KID_DEC_REF,
   KID_DEC_PREP, KID_DEC_STREAM_SIMT, KID_DEC_STREAM_TC, KID_DEC_COMBINE, KID_DEC_FINAL,
-  KID_APPEND_REFS, KID_APPEND_ROWS, KID_SPARSE_ATTEND, KID_SPARSE_MERGE, KID_COUNT
+  KID_APPEND_REFS, KID_APPEND_ROWS, KID_SPARSE_ATTEND, KID_SPARSE_MERGE, KID_SPARSE_SELECT, KID_COUNT
 };
 const char* kernel_name(int id);
 
@@ -67,6 +67,10 @@ struct Plan {
   size_t ws_cho;         // sequences of different lengths: int32 chunk offsets [batch * kv_heads + 1], then the
                          // checked lengths [batch]
   size_t ws_decode_end;  // error word + the dense decode's regions (S .. cho)
+  // sparse decode on the tensor-core token loop: reference multiplicities
+  // [BH][n_ref_cap], listed compressed rows [BH][n_code_cap + n_ref_cap],
+  // row counts [BH]
+  size_t ws_mult, ws_rowlist, ws_ncode;
   size_t ws_bytes;
 };
 
@@ -188,8 +192,18 @@ bool decode_tc_supported(const Plan& p);
 int decode_tc_grid(const Plan& p, int64_t N);
 // The token loop on the tensor cores; cho: chunk offsets per (sequence,
 // kv-head) when the lengths differ (else null); the grid used goes to *grid.
+// rowlist / ncode / rl_cap: gathered rows (sparse decode), else null.
 cudaError_t launch_decode_tc(const Plan& p, const CacheView& cv, const SeqLens& sl, const int32_t* cho,
-                             const void* W3, const float* b3, void* ws, cudaStream_t st, int* grid);
+                             const void* W3, const float* b3, void* ws, cudaStream_t st, int* grid,
+                             const int32_t* rowlist = nullptr, const int32_t* ncode = nullptr, int64_t rl_cap = 0);
+// Sparse decode through the tensor-core token loop: the selected tokens'
+// compressed rows gathered chunk by chunk, the selected references counted
+// in the reference combine.  cudaErrorNotSupported when the plan or the
+// selection size does not fit it (the CUDA-core sparse kernels then run).
+cudaError_t launch_decode_sparse_tc(const Plan& p, int T, const void* q, int64_t qsb, int64_t qsh, const void* cache,
+                                    const void* W3, const float* b3, const void* W4, const float* b4,
+                                    const int32_t* tokens, int n_sel, float* out, int64_t osb, int64_t osh, void* ws,
+                                    cudaStream_t st);
 cudaError_t launch_decode(const Plan& p, const CacheView& cv, const SeqLens& sl, const void* q, int64_t qsb,
                           int64_t qsh, const void* W3, const float* b3, const void* W4, const float* b4, float* out,
                           int64_t osb, int64_t osh, void* ws, cudaStream_t st);

@@ -29,7 +29,7 @@ const char* kernel_name(int id) {
   static const char* names[KID_COUNT] = {
       "refpack", "candidates_simt", "candidates_tc", "encode_simt", "encode_tc", "reconstruct",
       "decode_ref", "decode_prep", "decode_stream_simt", "decode_stream_tc", "decode_combine", "decode_final",
-      "append_refs", "append_rows", "sparse_attend", "sparse_merge"};
+      "append_refs", "append_rows", "sparse_attend", "sparse_merge", "sparse_select"};
   return (id >= 0 && id < KID_COUNT) ? names[id] : "?";
 }
 

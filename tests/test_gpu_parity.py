@@ -69,6 +69,8 @@ BF16_CASES = [
                             act=dkv.ACT_GELU_TANH, biases=True)),
     ("identity_act_tc", Case(B=1, H=1, Hq=2, d_h=64, T=1800, s=4, k=2, d_c=32, hidden=128, dtype=dkv.BF16,
                              act=dkv.ACT_NONE, biases=True)),
+    # eight query heads per kv-head (the widest group the token loop lays out)
+    ("g8_tc", Case(B=2, H=2, Hq=16, d_h=128, T=3000, s=16, k=4, d_c=32, hidden=256, dtype=dkv.BF16, n_lat=8)),
     # points of the single-layer sweep (d_h 128, bf16, hidden 256, 8 latent
     # directions), two kv-heads each so that the oracle covers every row
     ("sweep_s4_k1_dc16", Case(B=1, H=2, Hq=8, d_h=128, T=4096, s=4, k=1, d_c=16, hidden=256, dtype=dkv.BF16,
@@ -89,6 +91,7 @@ TC_EXPECT = {
     "d_h64_tc": {"candidates_tc", "encode_tc", "decode_stream_tc"},
     "biases_tanh_tc": {"candidates_tc", "encode_tc", "decode_stream_tc"},
     "identity_act_tc": {"encode_tc", "decode_stream_simt"},
+    "g8_tc": {"candidates_tc", "encode_tc", "decode_stream_tc"},
     "sweep_s4_k1_dc16": {"candidates_tc", "encode_tc", "decode_stream_tc"},
     "sweep_s8_k2_dc64": {"candidates_tc", "encode_tc", "decode_stream_tc"},
     "sweep_s32_k8_dc32": {"candidates_tc", "encode_tc", "decode_stream_tc"},

@@ -33,6 +33,16 @@ def _selection(c: Case, n_sel: int, seed: int, repeats: bool = False):
     return sel.astype(np.int32)
 
 
+def _tc_path(c: Case, n_sel: int) -> bool:
+    """The sparse decode runs the tensor-core token loop over the gathered
+    rows when the plan has one (bf16 codes, hidden 128 or 256, a nonlinear
+    codec) and the selection fits its row list; else the CUDA-core kernels."""
+    n_ref_cap = max(128, -(-(-(-c.T // c.s)) // 128) * 128)
+    n_code_cap = max(128, -(-(c.T - -(-c.T // c.s)) // 128) * 128)
+    return (c.dtype == dkv.BF16 and c.hidden in (128, 256) and c.act != dkv.ACT_NONE
+            and n_sel <= n_ref_cap + n_code_cap)
+
+
 def _sparse(c, inp, p, W, bias, cache, ws, sel):
     out = torch.empty((c.B, c.Hq, c.d_h), dtype=torch.float32, device="cuda")
     dkv.set_profiling(p, True)
@@ -40,7 +50,11 @@ def _sparse(c, inp, p, W, bias, cache, ws, sel):
                                 torch.from_numpy(sel).cuda(), out, ws)
     status = dkv.device_status(p, ws)
     torch.cuda.synchronize()
-    assert "sparse_attend" in set(dkv.profile_collect(p))
+    kernels = set(dkv.profile_collect(p))
+    if _tc_path(c, sel.shape[-1]):
+        assert {"sparse_select", "decode_stream_tc", "decode_combine"} <= kernels, kernels
+    else:
+        assert "sparse_attend" in kernels, kernels
     return out.double().cpu().numpy(), status
 
 
@@ -55,6 +69,12 @@ def _sparse(c, inp, p, W, bias, cache, ws, sel):
     ("bf16_G1_repeats", Case(B=2, H=2, Hq=2, d_h=128, T=700, s=16, k=4, d_c=32, hidden=256, dtype=dkv.BF16), 1500,
      True),
     ("bf16_one_token", Case(B=1, H=2, Hq=4, d_h=64, T=300, s=8, k=2, d_c=16, hidden=64, dtype=dkv.BF16), 1, False),
+    # tensor-core token loop: one selected token; repeats; several chunks per
+    # (sequence, kv-head) with many sequences
+    ("tc_one_token", Case(B=1, H=2, Hq=4, d_h=64, T=300, s=8, k=2, d_c=16, hidden=128, dtype=dkv.BF16), 1, False),
+    ("tc_repeats", Case(B=2, H=2, Hq=4, d_h=128, T=900, s=8, k=4, d_c=32, hidden=256, dtype=dkv.BF16), 600, True),
+    ("tc_multi_chunk", Case(B=4, H=2, Hq=16, d_h=128, T=4000, s=16, k=4, d_c=32, hidden=256, dtype=dkv.BF16,
+                            n_lat=8), 1300, False),
 ])
 def test_sparse_matches_oracle(name, case, n_sel, repeats):
     c = case
@@ -87,8 +107,9 @@ def test_sparse_over_every_token_equals_dense_decode():
 
 
 @pytest.mark.gpu
-def test_sparse_reports_an_out_of_range_token():
-    c = Case(B=1, H=1, Hq=2, d_h=64, T=500, s=8, k=2, d_c=16, hidden=64, dtype=dkv.BF16)
+@pytest.mark.parametrize("hidden", [64, 128])  # CUDA-core kernels, tensor-core token loop
+def test_sparse_reports_an_out_of_range_token(hidden):
+    c = Case(B=1, H=1, Hq=2, d_h=64, T=500, s=8, k=2, d_c=16, hidden=hidden, dtype=dkv.BF16)
     inp, p, W, bias, cache, ws = _setup(c)
     sel = _selection(c, 40, 3)
     sel[0, 0, 5] = c.T + 17
