@@ -203,11 +203,16 @@ deltakv_status deltakv_decode_attention(deltakv_plan_t plan, int32_t T,
  *            occurrence; an index outside [0, T) is skipped and reported as
  *            DELTAKV_ERR_DEVICE_BOUNDS); n_sel >= 1; caller-owned, read only.
  *   every other argument as for deltakv_decode_attention.
- * Runs on CUDA cores in float32, 16 selected tokens per pass of a CTA: the
- * first decompressor layer per token, and the (linear) second layer folded
- * into the query and applied once per CTA to the softmax-weighted sum of its
- * activations, so no K_hat/V_hat row is formed; a second kernel merges the
- * CTAs' shares. */
+ * Plans that take the tensor-core token loop of deltakv_decode_attention
+ * (bf16 codes, hidden 128 or 256, a nonlinear codec), with n_sel at most the
+ * plan's reference plus compressed-row capacity, run that loop over the
+ * selected tokens' compressed rows (listed per (sequence, kv-head), gathered
+ * 128 at a time), with each selected reference counted in the reference
+ * combine.  Other plans run CUDA-core kernels in float32, 16 selected tokens
+ * per pass of a CTA: the first decompressor layer per token, and the
+ * (linear) second layer folded into the query and applied once per CTA to
+ * the softmax-weighted sum of its activations.  Neither forms a K_hat/V_hat
+ * row. */
 deltakv_status deltakv_decode_attention_sparse(deltakv_plan_t plan, int32_t T,
                                                const void* q, const int64_t q_strides[2],
                                                const void* cache,
