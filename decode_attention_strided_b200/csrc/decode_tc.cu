@@ -151,14 +151,6 @@ __device__ __forceinline__ uint32_t swz_off(int row, int bo, int swz) {
   return (uint32_t)(row * swz + (chunk << 4) + (bo & 15));
 }
 
-__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                   smem_u32(dst)),
-               "l"(src), "r"(bytes), "r"(smem_u32(bar))
-               : "memory");
-}
 
 __device__ __forceinline__ void tmem_ld16f(uint32_t taddr, float (&v)[16]) {
   uint32_t r[16];
