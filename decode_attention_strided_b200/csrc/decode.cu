@@ -25,6 +25,7 @@
 #include <cfloat>
 
 #include "common.cuh"
+#include "sm100.cuh"
 
 namespace dkv {
 
@@ -383,22 +384,43 @@ __device__ __forceinline__ int slots_of(const SlotInfo& si, int64_t bh) {
 // M_g = max(m_ref, split maxima).  For 256 slots: weights
 // w_j = 2^(S_j - M) + 2^(m_ref - M) sum_splits wtab, then sum_j w_j V_ref_j.
 // GP: heads per kv-head as laid out in registers (4 or 8, at least G).
+//
+// The CTA's V rows (at most 256 x d_h elements, two runs of up to 128
+// consecutive rows: a pool page holds 128) come into shared memory by bulk
+// copies issued first, so the copy overlaps the weight computation; the sum
+// then reads them from shared memory: thread (slot group, 4 consecutive
+// elements), every row segment used for all heads of the group.
 template <typename T, int GP>
 __global__ void __launch_bounds__(256)
     decode_combine_kernel(SeqLens sl, int s, int d_h, int H, int G, SlotInfo si, int64_t n_ref_cap,
                           int n_chunk_cap, CacheView cv, const float* __restrict__ S,
                           const float* __restrict__ mref, const float* __restrict__ wtab_g,
                           const float* __restrict__ part, float* __restrict__ ochunk,
-                          const int32_t* __restrict__ mult) {
-  __shared__ float wts[kCombineSlots][kMaxG];
+                          const int32_t* __restrict__ mult, uint32_t* __restrict__ err) {
+  extern __shared__ __align__(128) unsigned char vsm[];  // kCombineSlots x d_h elements of T
+  __shared__ __align__(16) float wts[kCombineSlots][GP];
   __shared__ float Mg[kMaxG], mrefg[kMaxG], lw[8][kMaxG];
-  __shared__ float red[8][kMaxG][128];
+  __shared__ __align__(16) float red[8 * kMaxG * 128];  // [slot group][head][element]
+  __shared__ __align__(8) uint64_t vbar;
   const int b = blockIdx.z, h = blockIdx.y, ch = blockIdx.x, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int64_t bh = (int64_t)b * H + h;
   const int64_t n_ref = n_ref_of(sl.T(b), s);
   const int64_t j0 = (int64_t)ch * kCombineSlots;
   if (j0 >= n_ref) return;  // past this sequence's references (its final reads n_chunk of its own)
+  const int nrows = (int)(n_ref - j0 < kCombineSlots ? n_ref - j0 : kCombineSlots);
+  const T* refv = reinterpret_cast<const T*>(cv.base + cv.off_refv);
+  if (tid == 0) {
+    const uint32_t row_bytes = (uint32_t)(d_h * sizeof(T));
+    sm100::mbar_init(&vbar, 1);
+    sm100::fence_mbar_init();
+    sm100::mbar_arrive_expect_tx(&vbar, (uint32_t)nrows * row_bytes);
+    for (int r0 = 0; r0 < nrows; r0 += 128) {
+      const int nr = nrows - r0 < 128 ? nrows - r0 : 128;
+      sm100::bulk_load(vsm + (size_t)r0 * row_bytes, refv + cv.ref_row(bh, j0 + r0) * d_h, (uint32_t)nr * row_bytes,
+                       &vbar);
+    }
+  }
   if (tid < G) {
     const float m = mref[bh * G + tid];
     mrefg[tid] = m;
@@ -415,18 +437,16 @@ __global__ void __launch_bounds__(256)
     const int64_t j = j0 + jj;
 #pragma unroll
     for (int g = 0; g < GP; ++g) {
-      if (g < G) {
-        float w = 0.f;
-        if (j < n_ref) {
-          // a reference's own term counts once per selection of it (sparse
-          // decode), once otherwise
-          float own = exp2f(S[(bh * n_ref_cap + j) * G + g] - Mg[g]);
-          if (mult) own *= (float)mult[bh * n_ref_cap + j];
-          w = own + wtab_g[(bh * n_ref_cap + j) * G + g] * exp2f(mrefg[g] - Mg[g]);
-          lsum[g] += own;
-        }
-        wts[jj][g] = w;
+      float w = 0.f;
+      if (g < G && j < n_ref) {
+        // a reference's own term counts once per selection of it (sparse
+        // decode), once otherwise
+        float own = exp2f(S[(bh * n_ref_cap + j) * G + g] - Mg[g]);
+        if (mult) own *= (float)mult[bh * n_ref_cap + j];
+        w = own + wtab_g[(bh * n_ref_cap + j) * G + g] * exp2f(mrefg[g] - Mg[g]);
+        lsum[g] += own;
       }
+      wts[jj][g] = w;
     }
   }
 #pragma unroll
@@ -434,63 +454,65 @@ __global__ void __launch_bounds__(256)
     const float ls = warp_sum(lsum[g]);
     if (lane == 0 && g < G) lw[warp][g] = ls;
   }
-  __syncthreads();
-  // sum_j w_j V_ref_j: thread = (slot group, 8 consecutive elements); every
-  // V row segment is loaded once (16 bytes of bf16) for all heads of the group
-  const T* refv = reinterpret_cast<const T*>(cv.base + cv.off_refv);
-  const int eg = d_h / 8, e8 = tid % eg, js = tid / eg, njs = blockDim.x / eg;
-  float acc[GP][8];
+  // the V rows have landed (bounded wait; every thread leaves together if
+  // it ran out)
+  if (!__syncthreads_and(sm100::mbar_wait_drain(&vbar, 0))) {
+    if (tid == 0) latch_error(err, DELTAKV_ERR_DEVICE_TIMEOUT, 31);
+    return;
+  }
+  // sum_j w_j V_ref_j: thread = (slot group, elements 4 e4 .. 4 e4 + 3)
+  const int e4n = d_h / 4, e4 = tid % e4n, grp = tid / e4n, ngrp = blockDim.x / e4n;
+  const int spg = kCombineSlots / ngrp;  // slots per group
+  float acc[GP][4];
 #pragma unroll
   for (int g = 0; g < GP; ++g)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[g][i] = 0.f;
-  // four rows' loads in flight at a time
-  for (int jj0 = js; jj0 < kCombineSlots; jj0 += 4 * njs) {
-    float v[4][8];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int jj = jj0 + u * njs;
-      const int64_t j = j0 + jj;
-      if (jj < kCombineSlots && j < n_ref) {
-        load8(refv + cv.ref_row(bh, j) * d_h + e8 * 8, v[u]);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[u][i] = 0.f;
-      }
+    for (int i = 0; i < 4; ++i) acc[g][i] = 0.f;
+  const int q_end = nrows - grp * spg < spg ? nrows - grp * spg : spg;  // rows past nrows were not copied
+#pragma unroll 4
+  for (int q = 0; q < q_end; ++q) {
+    const int jj = grp * spg + q;
+    float v[4];
+    const T* row = reinterpret_cast<const T*>(vsm) + (size_t)jj * d_h + e4 * 4;
+    if constexpr (sizeof(T) == 2) {
+      const uint2 r = *reinterpret_cast<const uint2*>(row);
+      const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.x));
+      const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.y));
+      v[0] = f0.x;
+      v[1] = f0.y;
+      v[2] = f1.x;
+      v[3] = f1.y;
+    } else {
+      const float4 r = *reinterpret_cast<const float4*>(row);
+      v[0] = r.x;
+      v[1] = r.y;
+      v[2] = r.z;
+      v[3] = r.w;
     }
+    float w[GP];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int jj = jj0 + u * njs;
-      if (jj < kCombineSlots) {
-#pragma unroll
-        for (int g = 0; g < GP; ++g) {
-          if (g < G) {
-            const float w = wts[jj][g];  // 0 past the sequence's references
-#pragma unroll
-            for (int i = 0; i < 8; ++i) acc[g][i] = fmaf(w, v[u][i], acc[g][i]);
-          }
-        }
-      }
+    for (int g4 = 0; g4 < GP; g4 += 4) {
+      const float4 w4 = *reinterpret_cast<const float4*>(&wts[jj][g4]);
+      w[g4] = w4.x;
+      w[g4 + 1] = w4.y;
+      w[g4 + 2] = w4.z;
+      w[g4 + 3] = w4.w;
     }
-  }
-  // lanes that share e8 hold different slot groups: fold them, then the warps
-  for (int o = eg; o < 32; o <<= 1)
 #pragma unroll
     for (int g = 0; g < GP; ++g)
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[g][i] += __shfl_xor_sync(0xffffffffu, acc[g][i], o);
-  if (lane < eg) {
-#pragma unroll
-    for (int g = 0; g < GP; ++g)
-      if (g < G)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) red[warp][g][e8 * 8 + i] = acc[g][i];
+      for (int i = 0; i < 4; ++i) acc[g][i] = fmaf(w[g], v[i], acc[g][i]);
   }
+#pragma unroll
+  for (int g = 0; g < GP; ++g)
+    if (g < G)
+      *reinterpret_cast<float4*>(&red[(grp * kMaxG + g) * d_h + e4 * 4]) =
+          make_float4(acc[g][0], acc[g][1], acc[g][2], acc[g][3]);
   __syncthreads();
   for (int o = tid; o < G * d_h; o += blockDim.x) {
     const int g = o / d_h, e = o - g * d_h;
     float sum = 0.f;
-    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) sum += red[w][g][e];
+    for (int w = 0; w < ngrp; ++w) sum += red[(w * kMaxG + g) * d_h + e];
     ochunk[((bh * n_chunk_cap + ch) * G + g) * (d_h + 1) + e] = sum;
   }
   if (tid < G) {
@@ -888,12 +910,12 @@ static cudaError_t decode_launch(const Plan& p, const CacheView& cv, const SeqLe
   if (e != cudaSuccess) return e;
   {
     ProfScope ps(p, st, KID_DEC_COMBINE);
-    if (G <= 4)
-      decode_combine_kernel<E, 4><<<dim3(n_chunk, H, B), 256, 0, st>>>(
-          sl, c.stride_s, c.d_h, H, G, si, p.n_ref_cap, p.n_chunk_cap, cv, S, mref, wtab, part, ochunk, mult);
-    else
-      decode_combine_kernel<E, 8><<<dim3(n_chunk, H, B), 256, 0, st>>>(
-          sl, c.stride_s, c.d_h, H, G, si, p.n_ref_cap, p.n_chunk_cap, cv, S, mref, wtab, part, ochunk, mult);
+    const size_t vbytes = (size_t)kCombineSlots * c.d_h * sizeof(E);
+    auto kc = G <= 4 ? decode_combine_kernel<E, 4> : decode_combine_kernel<E, 8>;
+    e = cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)vbytes);
+    if (e != cudaSuccess) return e;
+    kc<<<dim3(n_chunk, H, B), 256, vbytes, st>>>(sl, c.stride_s, c.d_h, H, G, si, p.n_ref_cap, p.n_chunk_cap, cv,
+                                                 S, mref, wtab, part, ochunk, mult, (uint32_t*)ws);
   }
   {
     ProfScope ps(p, st, KID_DEC_FINAL);
