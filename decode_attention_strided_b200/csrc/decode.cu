@@ -523,6 +523,10 @@ __global__ void __launch_bounds__(256)
 }
 
 // ---------------------------------------------------------- decode_final
+// kFinalSplit CTAs per (sequence, kv-head), each for d_h / kFinalSplit of
+// the output elements (the merge of the splits' maxima, sums and U is
+// repeated by each: it is small).
+constexpr int kFinalSplit = 4;
 template <typename T>
 __global__ void __launch_bounds__(256)
     decode_final_kernel(SeqLens sl, int s, int d_h, int H, int G, int hidden, SlotInfo si,
@@ -530,10 +534,12 @@ __global__ void __launch_bounds__(256)
                         const float* __restrict__ mref, const float* __restrict__ part,
                         const float* __restrict__ Upart, const float* __restrict__ ochunk,
                         float* __restrict__ out, int64_t osb, int64_t osh) {
-  __shared__ float Ut[kMaxG][kMaxHidden];
+  __shared__ __align__(16) float Ut[kMaxG][kMaxHidden];
   __shared__ float Mg[kMaxG], Lnr[kMaxG], Lall[kMaxG];
+  __shared__ float Oc[kMaxG][128 / kFinalSplit];
   const int b = blockIdx.z, h = blockIdx.y, tid = threadIdx.x;
   const int64_t bh = (int64_t)b * H + h;
+  const int nout = d_h / kFinalSplit, e_base = blockIdx.x * nout;  // this CTA's output elements
   const int ns = slots_of(si, bh);
   const int64_t pb0 = bh * si.nslot_cap;
   const int n_chunk = (int)((n_ref_of(sl.T(b), s) + kCombineSlots - 1) / kCombineSlots);
@@ -543,6 +549,7 @@ __global__ void __launch_bounds__(256)
     const int warp = tid >> 5, lane = tid & 31;
     for (int g = warp; g < G; g += (int)(blockDim.x >> 5)) {
       float M = mref[bh * G + g];
+#pragma unroll 4
       for (int sp = 0; sp < ns; ++sp) M = fmaxf(M, part[((pb0 + sp) * G + g) * 2]);
       float lnr = 0.f;
       for (int sp = lane; sp < ns; sp += 32) {
@@ -565,6 +572,7 @@ __global__ void __launch_bounds__(256)
   for (int i = tid; i < G * hidden; i += blockDim.x) {
     int g = i / hidden, n = i - g * hidden;
     float acc = 0.f;
+#pragma unroll 4
     for (int sp = 0; sp < ns; ++sp) {
       float m = part[((pb0 + sp) * G + g) * 2];
       if (m != -INFINITY) acc += Upart[((pb0 + sp) * G + g) * hidden + n] * exp2f(m - Mg[g]);
@@ -572,40 +580,56 @@ __global__ void __launch_bounds__(256)
     Ut[g][n] = acc;
   }
   __syncthreads();
-  // the reference chunks' sums: threads over (head, element), chunk loads
-  // independent of one another
-  __shared__ float Oc[kMaxG][128];
-  for (int o = tid; o < G * d_h; o += blockDim.x) {
-    const int g = o / d_h, e = o - g * d_h;
+  // the reference chunks' sums for this CTA's elements: threads over
+  // (head, element), chunk loads independent of one another
+  for (int o = tid; o < G * nout; o += blockDim.x) {
+    const int g = o / nout, el = o - g * nout;
     float acc = 0.f;
 #pragma unroll 8
-    for (int c = 0; c < n_chunk; ++c) acc += ochunk[((bh * n_chunk_cap + c) * G + g) * (d_h + 1) + e];
-    Oc[g][e] = acc;
+    for (int c = 0; c < n_chunk; ++c) acc += ochunk[((bh * n_chunk_cap + c) * G + g) * (d_h + 1) + e_base + el];
+    Oc[g][el] = acc;
   }
   __syncthreads();
   // W4_V . U: a warp per output element, its lanes over the hidden units
-  // (8 consecutive weights per 16-byte load), every head of the group at once
-  const int warp = tid >> 5, lane = tid & 31;
-  for (int e = warp; e < d_h; e += (int)(blockDim.x >> 5)) {
-    const T* w4 = W4 + (int64_t)(d_h + e) * hidden;
+  // (8 consecutive weights per 16-byte load; hidden <= 256, so one load a
+  // lane), every head of the group at once; the weight rows of all of a
+  // warp's elements are loaded before any is used
+  const int warp = tid >> 5, lane = tid & 31, nw = (int)(blockDim.x >> 5);
+  constexpr int kRows = 128 / kFinalSplit / 8;  // elements per warp at d_h = 128, 8 warps
+  float w[kRows][8];
+#pragma unroll
+  for (int r = 0; r < kRows; ++r) {
+    const int el = warp + r * nw;
+    if (el < nout && lane * 8 < hidden) {
+      load8(W4 + (int64_t)(d_h + e_base + el) * hidden + lane * 8, w[r]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) w[r][i] = 0.f;
+    }
+  }
+  const int n0 = lane * 8 < hidden ? lane * 8 : 0;  // lanes past hidden hold zero weights
+#pragma unroll
+  for (int r = 0; r < kRows; ++r) {
+    const int el = warp + r * nw;
+    if (el >= nout) break;
     float y[kMaxG];
 #pragma unroll
-    for (int g = 0; g < kMaxG; ++g) y[g] = 0.f;
-    for (int n0 = lane * 8; n0 < hidden; n0 += 256) {
-      float w[8];
-      load8(w4 + n0, w);
-#pragma unroll
-      for (int g = 0; g < kMaxG; ++g)
-        if (g < G)
-#pragma unroll
-          for (int i = 0; i < 8; ++i) y[g] = fmaf(w[i], Ut[g][n0 + i], y[g]);
+    for (int g = 0; g < kMaxG; ++g) {
+      y[g] = 0.f;
+      if (g < G) {
+        const float4 u0 = *reinterpret_cast<const float4*>(&Ut[g][n0]);
+        const float4 u1 = *reinterpret_cast<const float4*>(&Ut[g][n0 + 4]);
+        y[g] = fmaf(w[r][0], u0.x, fmaf(w[r][1], u0.y, fmaf(w[r][2], u0.z, fmaf(w[r][3], u0.w, y[g]))));
+        y[g] = fmaf(w[r][4], u1.x, fmaf(w[r][5], u1.y, fmaf(w[r][6], u1.z, fmaf(w[r][7], u1.w, y[g]))));
+      }
     }
 #pragma unroll
     for (int g = 0; g < kMaxG; ++g) {
       if (g < G) {
         const float yg = warp_sum(y[g]);
         if (lane == g) {
-          const float acc = Oc[g][e] + yg + (b4 ? b4[d_h + e] * Lnr[g] : 0.f);
+          const int e = e_base + el;
+          const float acc = Oc[g][el] + yg + (b4 ? b4[d_h + e] * Lnr[g] : 0.f);
           out[b * osb + (int64_t)(h * G + g) * osh + e] = acc / Lall[g];
         }
       }
@@ -919,7 +943,7 @@ static cudaError_t decode_launch(const Plan& p, const CacheView& cv, const SeqLe
   }
   {
     ProfScope ps(p, st, KID_DEC_FINAL);
-    decode_final_kernel<E><<<dim3(1, H, B), 256, 0, st>>>(
+    decode_final_kernel<E><<<dim3(kFinalSplit, H, B), 256, 0, st>>>(
         sl, c.stride_s, c.d_h, H, G, c.hidden, si, p.n_chunk_cap, (const E*)W4, b4, mref, part, Upart, ochunk,
         out, osb, osh);
   }
