@@ -48,41 +48,77 @@ __device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
   v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
   v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
+// the same from shared memory (16-byte aligned)
+__device__ __forceinline__ void load8s(const __nv_bfloat16* p, float (&v)[8]) {
+  const uint4 r = *reinterpret_cast<const uint4*>(p);
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&r);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+__device__ __forceinline__ void load8s(const float* p, float (&v)[8]) {
+  const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
 
 // ------------------------------------------------------------ decode_ref
 // One thread per reference row (64 rows per CTA): the row's d_h elements
 // with 16-byte loads, every head's dot product at once against the scaled
 // queries in shared memory (stored element-major, so one 16-byte shared load
 // gives four heads), S and the cleared slot weights written as one vector
-// per row.
+// per row.  Each thread's row comes into shared memory by a bulk copy of
+// its own, issued before the queries are staged; rows sit 16 bytes apart
+// beyond their length, so the threads' 16-byte reads at one offset fall on
+// different banks.
 template <typename T>
 __global__ void __launch_bounds__(kRefBlockSlots)
     decode_ref_kernel(SeqLens sl, int s_, int64_t n_ref_cap, int d_h, int H, int G, float c,
                       const T* __restrict__ q, int64_t qsb, int64_t qsh, CacheView cv,
                       float* __restrict__ S, float* __restrict__ Smax, int n_refblk_cap,
-                      float* __restrict__ wtab) {
+                      float* __restrict__ wtab, uint32_t* __restrict__ err) {
+  extern __shared__ __align__(16) unsigned char krow[];  // kRefBlockSlots rows of d_h T + 16 bytes
   __shared__ __align__(16) float qt[128][kMaxG];  // [element][head]
   __shared__ float wmax[kRefBlockSlots / 32][kMaxG];
+  __shared__ __align__(8) uint64_t kbar;
   const int b = blockIdx.z, h = blockIdx.y, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int64_t bh = (int64_t)b * H + h;
   const int64_t n_ref = n_ref_of(sl.T(b), s_);
   const T* refk = reinterpret_cast<const T*>(cv.base + cv.off_refk);
+  const int64_t j = (int64_t)blockIdx.x * kRefBlockSlots + tid;
+  const uint32_t row_bytes = (uint32_t)(d_h * sizeof(T)), row_pitch = row_bytes + 16;
+  if (tid == 0) {
+    const int64_t jb = (int64_t)blockIdx.x * kRefBlockSlots;
+    const int64_t nv = n_ref - jb < 0 ? 0 : (n_ref - jb < kRefBlockSlots ? n_ref - jb : kRefBlockSlots);
+    sm100::mbar_init(&kbar, 1);
+    sm100::fence_mbar_init();
+    sm100::mbar_arrive_expect_tx(&kbar, (uint32_t)nv * row_bytes);
+  }
+  __syncthreads();
+  if (j < n_ref) sm100::bulk_load(krow + tid * row_pitch, refk + cv.ref_row(bh, j) * d_h, row_bytes, &kbar);
   for (int i = tid; i < kMaxG * d_h; i += blockDim.x) {
     const int g = i % kMaxG, e = i / kMaxG;
     qt[e][g] = g < G ? c * to_f(q[b * qsb + (int64_t)(h * G + g) * qsh + e]) : 0.f;
   }
-  __syncthreads();
-  const int64_t j = (int64_t)blockIdx.x * kRefBlockSlots + tid;
+  // the rows have landed (bounded wait; every thread leaves together if it
+  // ran out)
+  if (!__syncthreads_and(sm100::mbar_wait_drain(&kbar, 0))) {
+    if (tid == 0) latch_error(err, DELTAKV_ERR_DEVICE_TIMEOUT, 32);
+    return;
+  }
   float acc[kMaxG];
 #pragma unroll
   for (int g = 0; g < kMaxG; ++g) acc[g] = 0.f;
   if (j < n_ref) {
-    const T* kr = refk + cv.ref_row(bh, j) * d_h;
+    const T* kr = reinterpret_cast<const T*>(krow + tid * row_pitch);
 #pragma unroll 4
     for (int e0 = 0; e0 < d_h; e0 += 8) {
       float v[8];
-      load8(kr + e0, v);
+      load8s(kr + e0, v);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const float4 qa = *reinterpret_cast<const float4*>(&qt[e0 + i][0]);
@@ -877,9 +913,10 @@ static cudaError_t decode_launch(const Plan& p, const CacheView& cv, const SeqLe
 
   {
     ProfScope ps(p, st, KID_DEC_REF);
-    decode_ref_kernel<E><<<dim3(n_refblk, H, B), kRefBlockSlots, 0, st>>>(sl, c.stride_s, p.n_ref_cap, c.d_h, H, G, cs,
-                                                               (const E*)q, qsb, qsh, cv, S, Smax, n_refblk_cap,
-                                                               wtab);
+    const size_t kbytes = (size_t)kRefBlockSlots * (c.d_h * sizeof(E) + 16);
+    decode_ref_kernel<E><<<dim3(n_refblk, H, B), kRefBlockSlots, kbytes, st>>>(
+        sl, c.stride_s, p.n_ref_cap, c.d_h, H, G, cs, (const E*)q, qsb, qsh, cv, S, Smax, n_refblk_cap, wtab,
+        (uint32_t*)ws);
   }
   {
     ProfScope ps(p, st, KID_DEC_PREP);
