@@ -433,10 +433,13 @@ __global__ void __launch_bounds__(256)
                           const float* __restrict__ mref, const float* __restrict__ wtab_g,
                           const float* __restrict__ part, float* __restrict__ ochunk,
                           const int32_t* __restrict__ mult, uint32_t* __restrict__ err) {
-  extern __shared__ __align__(128) unsigned char vsm[];  // kCombineSlots x d_h elements of T
+  // kCombineSlots x d_h elements of T; once every thread has read its rows,
+  // the partial sums [slot group][head][element] (8 kMaxG 128 floats, at
+  // most the rows' size)
+  extern __shared__ __align__(128) unsigned char vsm[];
+  float* red = reinterpret_cast<float*>(vsm);
   __shared__ __align__(16) float wts[kCombineSlots][GP];
   __shared__ float Mg[kMaxG], mrefg[kMaxG], lw[8][kMaxG];
-  __shared__ __align__(16) float red[8 * kMaxG * 128];  // [slot group][head][element]
   __shared__ __align__(8) uint64_t vbar;
   const int b = blockIdx.z, h = blockIdx.y, ch = blockIdx.x, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -539,6 +542,7 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[g][i] = fmaf(w[g], v[i], acc[g][i]);
   }
+  __syncthreads();  // every row read: the rows' space takes the partial sums
 #pragma unroll
   for (int g = 0; g < GP; ++g)
     if (g < G)
