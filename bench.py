@@ -94,6 +94,18 @@ class Shape:
         D = 2 * self.d_h
         return 2 * (D * self.hidden + self.hidden * self.d_c) * self.n_code * self.H * B
 
+    def append_bytes_per_layer(self, t):
+        """Algorithmic bytes of appending one non-reference token t to each of
+        the Bc compress sequences: the K and V rows of every earlier
+        reference (ceil(t / s) of them) and the token's own, once, per
+        (sequence, kv-head); the compressor weights once; the code and slot
+        rows written."""
+        es = 2
+        D = 2 * self.d_h
+        per_head = (math.ceil(t / self.s) + 1) * D * es + self.d_c * es + self.k * 4
+        weights = (D * self.hidden + self.hidden * self.d_c) * es
+        return per_head * self.Bc * self.H + weights
+
     def decode_bytes_per_layer(self):
         es = 2
         per_head = self.n_ref * 2 * self.d_h * es + self.n_code * (self.d_c * es + self.k * 4)
@@ -610,6 +622,11 @@ def main():
             n, ms = prof[k_]
             decode_attn["stream_kernel_ms_per_launch"] = ms / n
     decode_attn["bounds"] = decode_bounds(sh, peaks, clk.get("sm_mhz"))
+    if append:
+        ab = sh.append_bytes_per_layer(sh.T - 1)
+        agbs = ab / (append["us_per_layer"] * 1e-6) / 1e9
+        append.update({"bytes_per_layer": ab, "GBps": agbs, "peak": hbm, "peak_source": peak_kind,
+                       "hbm_frac": agbs / hbm})
     comp_fl = sh.cand_flops_per_layer(sh.Bc) + sh.mlp_flops_per_layer(sh.Bc)
     compress = {"value": sh.T * sh.Bc / (sc / a.steps / 1e3) / 1e6, "unit": "Mtok/s",
                 "ms": sc / a.steps,

@@ -74,3 +74,13 @@ def test_decode_bounds_of_the_128k_batch8_layer():
     flops = 2 * th * (32 * 256 + 2 * 256 * 8 + 2 * 256 * 8)
     assert math.isclose(b["tensor_ms"], flops / 1e15 * 1e3)
     assert b["binding"] in ("sfu_ms", "mma_issue_ms")
+
+
+def test_append_bytes_of_one_token_at_128k():
+    """t = T - 1 = 131071 searches ceil(t / 16) = 8192 references: their K
+    and V rows plus the token's own row per kv-head (8 heads, one sequence),
+    W1 and W2 once, and a 32-element code row and 4 slots written per head."""
+    sh = _shape()
+    per_head = (8192 + 1) * 256 * 2 + 32 * 2 + 4 * 4
+    want = per_head * 8 + (256 * 256 + 256 * 32) * 2
+    assert sh.append_bytes_per_layer(131071) == want == 33706624
