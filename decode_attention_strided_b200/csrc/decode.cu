@@ -732,61 +732,95 @@ __global__ void __launch_bounds__(1024)
 // ------------------------------------------------- sparse selection
 // One block per (sequence, kv-head): the selected reference tokens are
 // counted per slot (a token selected twice counts twice), the selected other
-// tokens' compressed rows listed (in any order) for the token loop, and their
-// number kept; an index outside [0, T) is reported and skipped.
+// tokens' compressed rows listed for the token loop in the order of the
+// selection (positions from a ballot prefix per 256 tokens, so the list, and
+// with it the token loop's summation order, is the same on every run), and
+// their number kept; an index outside [0, T) is reported and skipped.  A
+// thread's tokens of eight such groups are loaded before any is used.
 __global__ void __launch_bounds__(256)
     sparse_select_kernel(int T, int s, int64_t n_ref_cap, int64_t rl_cap, int n_sel,
                          const int32_t* __restrict__ tokens, int32_t* __restrict__ mult,
                          int32_t* __restrict__ rowlist, int32_t* __restrict__ ncode, uint32_t* __restrict__ err) {
-  __shared__ int cnt;
+  constexpr int kGroups = 8;
+  __shared__ int wsum[8];
   const int64_t bh = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t n_ref = n_ref_of(T, s);
   int32_t* m = mult + bh * n_ref_cap;
-  for (int64_t j = threadIdx.x; j < n_ref; j += blockDim.x) m[j] = 0;
-  if (threadIdx.x == 0) cnt = 0;
+  for (int64_t j = tid; j < n_ref; j += blockDim.x) m[j] = 0;
   __syncthreads();
-  for (int i = threadIdx.x; i < n_sel; i += blockDim.x) {
-    const int t = tokens[bh * n_sel + i];
-    if (t < 0 || t >= T) {
-      latch_error(err, DELTAKV_ERR_DEVICE_BOUNDS, (uint32_t)t);
-      continue;
+  int base = 0;
+  for (int c0 = 0; c0 < n_sel; c0 += kGroups * 256) {
+    int tv[kGroups];
+#pragma unroll
+    for (int u = 0; u < kGroups; ++u) {
+      const int i = c0 + u * 256 + tid;
+      tv[u] = i < n_sel ? tokens[bh * n_sel + i] : 0;
     }
-    if (t % s == 0) {
-      atomicAdd(&m[t / s], 1);
-    } else {
-      const int pos = atomicAdd(&cnt, 1);
-      rowlist[bh * rl_cap + pos] = t - t / s - 1;
+#pragma unroll
+    for (int u = 0; u < kGroups; ++u) {
+      if (c0 + u * 256 >= n_sel) break;  // the same for every thread
+      const int t = tv[u];
+      bool code = false;
+      if (c0 + u * 256 + tid < n_sel) {
+        if (t < 0 || t >= T) latch_error(err, DELTAKV_ERR_DEVICE_BOUNDS, (uint32_t)t);
+        else if (t % s == 0) atomicAdd(&m[t / s], 1);
+        else code = true;
+      }
+      const unsigned bal = __ballot_sync(0xffffffffu, code);
+      if (lane == 0) wsum[warp] = __popc(bal);
+      __syncthreads();
+      int off = base, total = 0;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) {
+        const int c = wsum[w];
+        off += w < warp ? c : 0;
+        total += c;
+      }
+      if (code) rowlist[bh * rl_cap + off + __popc(bal & ((1u << lane) - 1u))] = t - t / s - 1;
+      base += total;
+      __syncthreads();  // wsum is reused by the next group
     }
   }
-  __syncthreads();
-  if (threadIdx.x == 0) ncode[bh] = cnt;
+  if (tid == 0) ncode[bh] = base;
 }
 
 // Chunk offsets of the token loop over the listed rows: cho[bh] = sum over
-// earlier (sequence, kv-head) pairs of their 128-row chunk counts.  One block.
+// earlier (sequence, kv-head) pairs of their 128-row chunk counts.  One block
+// of 1024 threads, each over a contiguous run of pairs; the runs' sums are
+// scanned with warp shuffles.
 __global__ void __launch_bounds__(1024)
     sparse_cho_kernel(int BH, const int32_t* __restrict__ ncode, int32_t* __restrict__ cho) {
-  __shared__ int32_t part[1024];
-  const int tid = threadIdx.x;
+  __shared__ int32_t wtot[32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int per = (BH + blockDim.x - 1) / blockDim.x;
   int32_t sum = 0;
   for (int i = 0; i < per; ++i) {
     const int bh = tid * per + i;
     if (bh < BH) sum += (ncode[bh] + 127) / 128;
   }
-  part[tid] = sum;
+  // inclusive scan within the warp, then across the warps' totals
+  int32_t x = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t v = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += v;
+  }
+  if (lane == 31) wtot[warp] = x;
   __syncthreads();
-  if (tid == 0) {
-    int32_t run = 0;
-    for (int t = 0; t < (int)blockDim.x; ++t) {
-      const int32_t v = part[t];
-      part[t] = run;
-      run += v;
+  if (warp == 0) {
+    const int nw = (int)(blockDim.x >> 5);
+    int32_t w = lane < nw ? wtot[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t v = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += v;
     }
-    cho[BH] = run;
+    wtot[lane] = w;  // inclusive totals of warps 0 .. lane
   }
   __syncthreads();
-  int32_t run = part[tid];
+  int32_t run = x - sum + (warp > 0 ? wtot[warp - 1] : 0);
+  if (tid == (int)blockDim.x - 1) cho[BH] = run + sum;
   for (int i = 0; i < per; ++i) {
     const int bh = tid * per + i;
     if (bh < BH) {
@@ -817,32 +851,58 @@ __global__ void __launch_bounds__(256)
   float m[kMaxG];
 #pragma unroll
   for (int g = 0; g < kMaxG; ++g) m[g] = -INFINITY;
-  for (int64_t j = tid; j < n_ref; j += blockDim.x) {
-    if (mult[bh * n_ref_cap + j] > 0)
+  // eight slots' counts, then their S rows, in flight at a time
+  for (int64_t j0 = tid; j0 < n_ref; j0 += 8 * (int64_t)blockDim.x) {
+    int mv[8];
 #pragma unroll
-      for (int g = 0; g < kMaxG; ++g)
-        if (g < G) m[g] = fmaxf(m[g], Sb[j * G + g]);
-  }
-  const int nc = ncode[bh];
-  for (int i = tid; i < nc; i += blockDim.x) {
-    const int64_t r = rowlist[bh * rl_cap + i];
-    const int32_t* ir = idx + (bh * n_code_cap + r) * k;
-    float sum[kMaxG];
-#pragma unroll
-    for (int g = 0; g < kMaxG; ++g) sum[g] = 0.f;
-    int ke = 0;
-    for (int q = 0; q < k; ++q) {
-      const int j = ir[q];
-      if (j < 0 || j >= n_ref) continue;
-      ++ke;
-#pragma unroll
-      for (int g = 0; g < kMaxG; ++g)
-        if (g < G) sum[g] += Sb[(int64_t)j * G + g];
+    for (int u = 0; u < 8; ++u) {
+      const int64_t j = j0 + (int64_t)u * blockDim.x;
+      mv[u] = j < n_ref ? mult[bh * n_ref_cap + j] : 0;
     }
-    if (ke > 0)
 #pragma unroll
-      for (int g = 0; g < kMaxG; ++g)
-        if (g < G) m[g] = fmaxf(m[g], sum[g] / (float)ke);
+    for (int u = 0; u < 8; ++u) {
+      const int64_t j = j0 + (int64_t)u * blockDim.x;
+      if (mv[u] > 0)
+#pragma unroll
+        for (int g = 0; g < kMaxG; ++g)
+          if (g < G) m[g] = fmaxf(m[g], Sb[j * G + g]);
+    }
+  }
+  // four listed rows at a time: their rows of the list, then their slots,
+  // then the slots' S rows
+  const int nc = ncode[bh];
+  for (int i0 = tid; i0 < nc; i0 += 4 * (int)blockDim.x) {
+    int64_t r[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u * (int)blockDim.x;
+      r[u] = i < nc ? rowlist[bh * rl_cap + i] : -1;
+    }
+    int js[4][kMaxK];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int q = 0; q < kMaxK; ++q) js[u][q] = (r[u] >= 0 && q < k) ? idx[(bh * n_code_cap + r[u]) * k + q] : -1;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      float sum[kMaxG];
+#pragma unroll
+      for (int g = 0; g < kMaxG; ++g) sum[g] = 0.f;
+      int ke = 0;
+#pragma unroll
+      for (int q = 0; q < kMaxK; ++q) {
+        const int j = js[u][q];
+        if (j < 0 || j >= n_ref) continue;
+        ++ke;
+#pragma unroll
+        for (int g = 0; g < kMaxG; ++g)
+          if (g < G) sum[g] += Sb[(int64_t)j * G + g];
+      }
+      if (ke > 0)
+#pragma unroll
+        for (int g = 0; g < kMaxG; ++g)
+          if (g < G) m[g] = fmaxf(m[g], sum[g] / (float)ke);
+    }
   }
 #pragma unroll
   for (int g = 0; g < kMaxG; ++g) {
