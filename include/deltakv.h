@@ -164,8 +164,13 @@ deltakv_status deltakv_compress(deltakv_plan_t plan, int32_t T,
  *   K, V       : device, as for deltakv_compress; only tokens [T0, T1) are
  *                read.
  *   W1, b1, W2, b2, workspace, stream: as for deltakv_compress.
- * Runs on CUDA cores (a few tokens per call): one CTA per new token and
- * kv-head.  Errors: as for deltakv_compress. */
+ * Runs on CUDA cores (a few tokens per call): each new token's references
+ * are scanned by several CTAs, whose lists one CTA per (token, kv-head)
+ * merges before the MLP.  The two kernels are launched with programmatic
+ * stream serialisation: they may start while the work before them on the
+ * stream is still running, but read nothing until it has completed, so the
+ * call is stream-ordered like any other (and can be captured in a CUDA
+ * graph).  Errors: as for deltakv_compress. */
 deltakv_status deltakv_append(deltakv_plan_t plan, int32_t T0, int32_t T1,
                               const void* K, const void* V, const int64_t kv_strides[3],
                               const void* W1, const float* b1,
