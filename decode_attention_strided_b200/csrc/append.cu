@@ -44,19 +44,22 @@ struct Frag {
   static constexpr int kBytes = NV * (int)sizeof(E);
   static constexpr int kWords = kBytes / 4;
   uint32_t w[kWords];
-  // read-only global load
-  __device__ __forceinline__ void ldg(const E* p) {
+  // global load cached in L2 only: the append kernels start before the
+  // grid ahead of them on the stream has finished (programmatic launch), so
+  // they read nothing through the read-only path, which assumes data that
+  // no grid changes during the kernel's lifetime
+  __device__ __forceinline__ void ldcg(const E* p) {
     if constexpr (kBytes % 16 == 0) {
 #pragma unroll
       for (int c = 0; c < kBytes / 16; ++c) {
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(p) + c);
+        const uint4 v = __ldcg(reinterpret_cast<const uint4*>(p) + c);
         w[4 * c] = v.x;
         w[4 * c + 1] = v.y;
         w[4 * c + 2] = v.z;
         w[4 * c + 3] = v.w;
       }
     } else {
-      const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
+      const uint2 v = __ldcg(reinterpret_cast<const uint2*>(p));
       w[0] = v.x;
       w[1] = v.y;
     }
@@ -249,7 +252,7 @@ __global__ void __launch_bounds__(kScanThreads, 2)
   float x[NV];
   {
     Frag<E, NV> f;
-    f.ldg((inK ? K + e0 : V + (e0 - d_h)) + b * P.sb + h * P.sh + t * P.st);
+    f.ldcg((inK ? K + e0 : V + (e0 - d_h)) + b * P.sb + h * P.sh + t * P.st);
 #pragma unroll
     for (int i = 0; i < NV; ++i) x[i] = f[i];
   }
@@ -271,7 +274,7 @@ __global__ void __launch_bounds__(kScanThreads, 2)
   auto fetch = [&](int64_t g0) {
 #pragma unroll
     for (int u = 0; u < kAppendRows; ++u) {
-      if (g0 + u < jhi) nxt[u].ldg(rs + (g0 + u) * d_h);
+      if (g0 + u < jhi) nxt[u].ldcg(rs + (g0 + u) * d_h);
       else nxt[u].zero();
     }
   };
@@ -384,8 +387,8 @@ __global__ void __launch_bounds__(kFinishThreads, 1)
   const float* l = lists + ((int64_t)bh * gridDim.y + blockIdx.y) * nsplit * (2 * kAppendKMax);
   for (int i = tid; i < n; i += kFinishThreads) {
     const int sp = i / k, q = i - sp * k;
-    cd[i] = l[sp * 2 * kAppendKMax + q];
-    cj[i] = __float_as_int(l[sp * 2 * kAppendKMax + kAppendKMax + q]);
+    cd[i] = __ldcg(l + sp * 2 * kAppendKMax + q);
+    cj[i] = __float_as_int(__ldcg(l + sp * 2 * kAppendKMax + kAppendKMax + q));
   }
   __syncthreads();
   const int k_eff = select_k(cd, cj, n, k, k, sx, seld, sel);
@@ -395,7 +398,7 @@ __global__ void __launch_bounds__(kFinishThreads, 1)
     const bool inK = e0 < d_h;
     const E* rs = (inK ? refk + e0 : refv + (e0 - d_h)) + (int64_t)bh * P.n_ref_cap * d_h;
     Frag<E, NV> f;
-    f.ldg(rs + (int64_t)sel[warp] * d_h);
+    f.ldcg(rs + (int64_t)sel[warp] * d_h);
 #pragma unroll
     for (int i = 0; i < NV; ++i) md[warp][e0 + i] = f[i];
   }
